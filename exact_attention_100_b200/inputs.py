@@ -1,0 +1,56 @@
+"""Seeded synthetic inputs shared by the tests, the bench and the oracle checks.
+
+This module holds no attention, transform or quantisation arithmetic: it only draws random
+numbers and rounds them to the storage type (bf16, round to nearest even).
+
+Recipe (the same for every workload):
+
+* ``numpy.random.default_rng(seed)`` (seed 0 unless stated) draws ``standard_normal``
+  float32 arrays for Q, then K, then V, each of shape ``[B, H, N, d]``.
+* Outlier workloads then visit Q, K, V in that order: ``mask = rng.random(shape) < frac``
+  and the masked entries are replaced by ``rng.normal(0, outlier_std, mask.sum())``.
+* Every tensor is rounded to bf16 (round to nearest even) last.
+* The random-sign diagonal of the Hadamard transform is ``2 * (default_rng(seed).random(d)
+  < 0.5) - 1`` with seed 1, stored as int8 +-1.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """float32 array whose values are ``x`` rounded to bfloat16 (ties to even)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    bias = ((u >> np.uint32(16)) & np.uint32(1)) + np.uint32(0x7FFF)
+    r = ((u + bias) & np.uint32(0xFFFF0000)).astype(np.uint32)
+    return r.view(np.float32)
+
+
+def bf16_bits(x_bf16_values: np.ndarray) -> np.ndarray:
+    """uint16 bit patterns of float32 values that are exact bf16 numbers."""
+    u = np.ascontiguousarray(x_bf16_values, dtype=np.float32).view(np.uint32)
+    return (u >> np.uint32(16)).astype(np.uint16)
+
+
+def normal_qkv(B: int, H: int, N: int, d: int, seed: int = 0,
+               outlier_frac: float = 0.0, outlier_std: float = 10.0):
+    """(q, k, v): float32 arrays of bf16 values, shape [B, H, N, d], iid N(0, 1).
+
+    With ``outlier_frac > 0`` that fraction of entries (in expectation) of each tensor is
+    replaced by N(0, outlier_std^2) draws before rounding.
+    """
+    rng = np.random.default_rng(seed)
+    shape = (B, H, N, d)
+    ts = [rng.standard_normal(shape, dtype=np.float32) for _ in range(3)]
+    if outlier_frac > 0.0:
+        for t in ts:
+            mask = rng.random(shape) < outlier_frac
+            t[mask] = rng.normal(0.0, outlier_std, int(mask.sum())).astype(np.float32)
+    return tuple(round_to_bf16(t) for t in ts)
+
+
+def hadamard_signs(d: int, seed: int = 1) -> np.ndarray:
+    """int8 vector of +-1 of length d (the random-sign diagonal D)."""
+    rng = np.random.default_rng(seed)
+    return (2 * (rng.random(d) < 0.5).astype(np.int8) - 1).astype(np.int8)
