@@ -1,0 +1,158 @@
+"""Exact attention forward for NVIDIA B200 (sm_100a): Python binding of ``include/attn.h``.
+
+Argument marshalling only: every step of the computation runs in the CUDA kernels of
+``libattn_b200.so``; torch supplies device memory and the current stream.  There is no CPU
+fallback: if the library is missing or a call fails, an exception is raised.
+
+    import torch, exact_attention_100_b200 as ea
+    o, lse = ea.attn_fwd(q, k, v, causal=True)           # q, k, v: [B, H, N, d] bf16 on cuda
+    q8, qs = ea.attn_hadamard_quant(q, signs)             # E4M3 codes + per-block scales
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_CUDA = 3
+ATTN_ERR_TIMEOUT = 4
+
+ATTN_BF16 = 0
+ATTN_FP32 = 1
+ATTN_E4M3 = 2
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn_b200.so")
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {attn_status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m exact_attention_100_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
+        L.attn_fwd.restype = i
+        L.attn_hadamard_quant.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
+        L.attn_hadamard_quant.restype = i
+        L.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+        L.attn_fwd_fp8.restype = i
+        L.attn_device_status.argtypes = [vp]
+        L.attn_device_status.restype = i
+        L.attn_status_string.argtypes = [i]
+        L.attn_status_string.restype = ctypes.c_char_p
+        L.attn_num_kernel_launches.argtypes = []
+        L.attn_num_kernel_launches.restype = ctypes.c_ulonglong
+        L.attn_shutdown.argtypes = []
+        L.attn_shutdown.restype = None
+        _lib = L
+    return _lib
+
+
+def attn_status_string(status: int) -> str:
+    return lib().attn_status_string(int(status)).decode()
+
+
+def attn_num_kernel_launches() -> int:
+    return int(lib().attn_num_kernel_launches())
+
+
+def attn_shutdown() -> None:
+    lib().attn_shutdown()
+
+
+def _stream_ptr(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _check(status: int, what: str) -> None:
+    if status != ATTN_OK:
+        raise AttnError(status, what)
+
+
+def _dims(q):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d]")
+    return tuple(int(x) for x in q.shape)
+
+
+def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, o_dtype=None, stream=None,
+             want_lse=True):
+    """O = softmax(scale * Q K^T) V and LSE for contiguous [B, H, N, d] bf16 cuda tensors.
+
+    ``o`` / ``lse`` may be given (written in place) or are allocated; ``o_dtype`` is
+    torch.bfloat16 (default) or torch.float32; ``scale`` defaults to 1/sqrt(d).
+    Returns ``(o, lse)`` (lse is None when ``want_lse`` is False and none was given).
+    """
+    import torch
+    B, H, N, d = _dims(q)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError("q, k, v must be contiguous bf16 tensors of one shape")
+    if o is None:
+        o = torch.empty(q.shape, dtype=o_dtype or torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, s, int(bool(causal)),
+                          ATTN_BF16, od, _stream_ptr(stream)), "attn_fwd")
+    return o, lse
+
+
+def attn_hadamard_quant(x, signs=None, x8=None, scales=None, stream=None):
+    """Per-block E4M3 quantisation of a [B, H, N, d] bf16 tensor, after H_d D when ``signs``.
+
+    ``signs``: int8 cuda tensor of d entries +-1, or None.  Returns ``(x8 uint8, scales f32)``.
+    """
+    import torch
+    B, H, N, d = _dims(x)
+    nb = (N + 127) // 128
+    if x8 is None:
+        x8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((B, H, nb), dtype=torch.float32, device=x.device)
+    _check(lib().attn_hadamard_quant(_ptr(x), _ptr(x8), _ptr(scales), _ptr(signs), B, H, N, d,
+                                     _stream_ptr(stream)), "attn_hadamard_quant")
+    return x8, scales
+
+
+def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o=None, lse=None, scale=None, causal=False,
+                 o_dtype=None, stream=None):
+    """Attention on E4M3 inputs with per-block scales (from ``attn_hadamard_quant``)."""
+    import torch
+    B, H, N, d = _dims(q8)
+    if o is None:
+        o = torch.empty((B, H, N, d), dtype=o_dtype or torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
+                              _ptr(o), _ptr(lse), B, H, N, d, s, int(bool(causal)), od, _stream_ptr(stream)),
+           "attn_fwd_fp8")
+    return o, lse
+
+
+def attn_device_status(stream=None) -> int:
+    """Synchronises the stream; returns and clears the device status word (0 = ATTN_OK)."""
+    return int(lib().attn_device_status(_stream_ptr(stream)))

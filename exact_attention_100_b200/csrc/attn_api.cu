@@ -1,0 +1,236 @@
+// C ABI of the library (declared in include/attn.h): argument checks, per-device state,
+// TMA tensor-map encoding and kernel launches.  Every argument is checked before the first
+// CUDA call, so a bad call returns a status without touching the device.
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "attn_kernels.h"
+
+namespace ea {
+cudaError_t setup_fwd_bf16_kernels();
+cudaError_t setup_fwd_fp8_kernels();
+}  // namespace ea
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  int num_sms = 0;
+  int* status = nullptr;  // device status word (library-owned workspace)
+};
+
+std::mutex g_mutex;
+DeviceState g_dev[kMaxDevices];
+std::atomic<unsigned long long> g_launches{0};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Per-device set-up (under the mutex): device properties, the status word, kernel attributes.
+int device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (major != 10 || minor != 0) return ATTN_ERR_UNSUPPORTED;
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q{};
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return ATTN_ERR_CUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    if (st.status == nullptr) {
+      if (cudaMalloc(&st.status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+      if (cudaMemset(st.status, 0, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    }
+    if (ea::setup_fwd_bf16_kernels() != cudaSuccess) return ATTN_ERR_CUDA;
+    if (ea::setup_fwd_fp8_kernels() != cudaSuccess) return ATTN_ERR_CUDA;
+    st.num_sms = sms;
+    st.ready = true;
+  }
+  *out = &st;
+  return ATTN_OK;
+}
+
+// 3-D tiled map over a contiguous [BH, N, row_bytes/elem] tensor: box = 128 bytes x 128 rows
+// x 1 head, 128-byte swizzle, zero fill outside the tensor.
+bool encode_rows_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N,
+                     int BH) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem_bytes,
+                                 static_cast<cuuint64_t>(d) * elem_bytes * static_cast<cuuint64_t>(N)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes), 128u, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return g_encode(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int check_common(int B, int H, int N, float scale, int causal, int o_dtype) {
+  if (B <= 0 || H <= 0 || N <= 0) return ATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 0x7FFFFFFFLL) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (o_dtype != ATTN_BF16 && o_dtype != ATTN_FP32) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+void fill_params(ea::FwdParams& p, void* o, float* lse, int* status, int B, int H, int N, int q_tiles, float scale,
+                 int causal, int o_dtype) {
+  p.o = o;
+  p.lse = lse;
+  p.status = status;
+  p.q_scale = p.k_scale = p.v_scale = nullptr;
+  p.N = N;
+  p.BH = B * H;
+  p.n_blocks = (N + 127) / 128;
+  p.n_pairs = (p.n_blocks + q_tiles - 1) / q_tiles;
+  p.num_units = p.BH * p.n_pairs;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.causal = causal;
+  p.o_fp32 = o_dtype == ATTN_FP32 ? 1 : 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK:
+      return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG:
+      return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED:
+      return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_CUDA:
+      return "ATTN_ERR_CUDA";
+    case ATTN_ERR_TIMEOUT:
+      return "ATTN_ERR_TIMEOUT";
+    default:
+      return "ATTN_ERR_UNKNOWN";
+  }
+}
+
+unsigned long long attn_num_kernel_launches(void) { return g_launches.load(); }
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+             float scale, int causal, int dtype, int o_dtype, void* stream) {
+  if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+    return ATTN_ERR_INVALID_ARG;
+  int rc = check_common(B, H, N, scale, causal, o_dtype);
+  if (rc != ATTN_OK) return rc;
+  if (dtype != ATTN_BF16) return dtype == ATTN_E4M3 || dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  CUtensorMap mq, mk, mv;
+  if (!encode_rows_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H) ||
+      !encode_rows_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H) ||
+      !encode_rows_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H))
+    return ATTN_ERR_CUDA;
+  ea::FwdParams p;
+  fill_params(p, o, lse, st->status, B, H, N, ea::fwd_units_per_tile_pair(d), scale, causal, o_dtype);
+  if (ea::launch_attn_fwd_bf16(d, mq, mk, mv, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return ATTN_OK;
+}
+
+int attn_hadamard_quant(const void* x, void* x8, float* scales, const signed char* signs, int B, int H, int N, int d,
+                        void* stream) {
+  if (!x || !x8 || !scales) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x8) || !aligned16(scales) || (signs && !aligned16(signs)))
+    return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || N <= 0 || static_cast<long long>(B) * H > 0x7FFFFFFFLL) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  const float post = signs ? static_cast<float>(1.0 / std::sqrt(static_cast<double>(d))) : 1.0f;
+  if (ea::launch_hadamard_quant(x, x8, scales, signs, B * H, N, d, post, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return ATTN_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return ATTN_OK;
+}
+
+int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
+                 const float* v_scale, void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
+                 int o_dtype, void* stream) {
+  if (!q8 || !k8 || !v8 || !q_scale || !k_scale || !v_scale || !o) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || (lse && !aligned16(lse)) ||
+      !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(v_scale))
+    return ATTN_ERR_INVALID_ARG;
+  int rc = check_common(B, H, N, scale, causal, o_dtype);
+  if (rc != ATTN_OK) return rc;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  CUtensorMap mq, mk, mv;
+  if (!encode_rows_map(&mq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, B * H) ||
+      !encode_rows_map(&mk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, B * H) ||
+      !encode_rows_map(&mv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, B * H))
+    return ATTN_ERR_CUDA;
+  ea::FwdParams p;
+  fill_params(p, o, lse, st->status, B, H, N, 2, scale, causal, o_dtype);
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  if (ea::launch_attn_fwd_fp8(d, mq, mk, mv, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return ATTN_OK;
+}
+
+int attn_device_status(void* stream) {
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int host = 0;
+  if (cudaMemcpyAsync(&host, st->status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (host != 0) {
+    if (cudaMemsetAsync(st->status, 0, sizeof(int), s) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_ERR_TIMEOUT;
+  }
+  return ATTN_OK;
+}
+
+void attn_shutdown(void) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  int cur = 0;
+  const bool have_dev = cudaGetDevice(&cur) == cudaSuccess;
+  for (int dev = 0; dev < kMaxDevices; ++dev) {
+    DeviceState& st = g_dev[dev];
+    if (st.status != nullptr && cudaSetDevice(dev) == cudaSuccess) cudaFree(st.status);
+    st = DeviceState{};
+  }
+  if (have_dev) cudaSetDevice(cur);
+}
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// Internal interface between the C ABI (attn_api.cu) and the kernels.  Not installed.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace ea {
+
+// Parameters of the attention forward kernels (bf16 and E4M3).
+struct FwdParams {
+  void* o;          // [BH, N, d] bf16 or f32
+  float* lse;       // [BH, N] or nullptr
+  int* status;      // device status word
+  const float* q_scale;  // E4M3 only: [BH, n_blocks] block scales
+  const float* k_scale;
+  const float* v_scale;
+  int N;            // sequence length (queries = keys)
+  int BH;           // batch * heads
+  int n_blocks;     // ceil(N / 128)
+  int n_pairs;      // ceil(n_blocks / Q tiles per unit)
+  int num_units;    // BH * n_pairs
+  float scale_log2; // softmax scale * log2(e)
+  int causal;
+  int o_fp32;
+};
+
+// Q tiles of 128 rows handled together by one unit of the bf16 kernel for head dim d.
+int fwd_units_per_tile_pair(int d);
+
+// Sets the kernels' shared-memory attributes on the current device (once per device).
+cudaError_t setup_kernels_for_current_device();
+
+cudaError_t launch_attn_fwd_bf16(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                                 const FwdParams& p, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_attn_fwd_fp8(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                                const FwdParams& p, int num_sms, cudaStream_t stream);
+
+// Hadamard + per-block E4M3 quantisation: x [BH, N, d] bf16 -> x8 [BH, N, d] e4m3, scales
+// [BH, ceil(N/128)].  signs may be nullptr (no transform).  post_scale = float(1/sqrt(d)) with
+// the transform, 1 without.
+cudaError_t launch_hadamard_quant(const void* x, void* x8, float* scales, const signed char* signs, int BH,
+                                  int N, int d, float post_scale, cudaStream_t stream);
+
+}  // namespace ea

@@ -1,0 +1,143 @@
+/*
+ * exact_attention_100_b200 -- C ABI of the exact attention forward for NVIDIA B200 (sm_100a).
+ *
+ * What is computed (cited by page title and section):
+ *   O = softmax(scale * Q K^T) V per (batch, head)        "FlashAttention-3", intro formula and
+ *                                                           section "数学对象没变"
+ *   LSE_i = log sum_j exp(scale * q_i . k_j)              "Flash Attention V3 解析", section 2.2
+ *                                                           (only the logsumexp is kept per row)
+ *   tiled, with a running row max m and row sum l, never   "FlashAttention-2/3", sections
+ *   writing the N x N score matrix to memory               "在线 Softmax" and "技术原理"
+ *   causal masking with all-masked blocks skipped          "Flash Attention V3 解析", section 2.2
+ *   FP8 path: x~ = H D x (random-sign Hadamard) on Q, K    "FlashAttention-3", section
+ *   before E4M3 quantisation with per-block scales         "FP8 路径与低精度误差"; "FlashAttention-2/3",
+ *                                                           section "FA-3：拥抱 Hopper", features 2-3
+ *
+ * Conventions shared by every entry point
+ *   - Pointers to tensors are DEVICE pointers (cudaMalloc'd or equivalent) on the current CUDA
+ *     device, unless an argument says otherwise.  The caller owns every tensor.
+ *   - Tensors are contiguous [B, H, N, d] (row-major, d fastest); LSE is contiguous [B, H, N]
+ *     float32; per-block scales are contiguous [B, H, ceil(N/128)] float32.
+ *   - Every tensor pointer must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Work is
+ *     enqueued asynchronously; the call returns once it is enqueued.
+ *   - Arguments are checked before any CUDA call; a bad argument returns an error status and
+ *     enqueues nothing.  No entry point allocates memory per call.  The library keeps one small
+ *     per-device workspace (a device status word), created on first use and released by
+ *     attn_shutdown().
+ *   - Calls on the same device may come from several host threads; the library's per-device
+ *     set-up is guarded by a mutex.
+ *   - Errors of the device-side work itself (a bounded wait inside a kernel that ran out) are
+ *     reported by attn_device_status(), not by the launching call.
+ */
+#ifndef EXACT_ATTENTION_100_B200_ATTN_H
+#define EXACT_ATTENTION_100_B200_ATTN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every int-returning entry point. */
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* NULL or misaligned pointer, non-positive size, bad scale/flag   */
+  ATTN_ERR_UNSUPPORTED = 2, /* head dim / dtype combination not built, or device not sm_100  */
+  ATTN_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed (no device, launch error) */
+  ATTN_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (from attn_device_status)      */
+} attn_status;
+
+/* Element types. */
+typedef enum {
+  ATTN_BF16 = 0, /* bfloat16                       */
+  ATTN_FP32 = 1, /* float32                        */
+  ATTN_E4M3 = 2  /* OCP FP8 E4M3FN (max 448, no inf) */
+} attn_dtype;
+
+/*
+ * attn_fwd -- exact attention forward, bf16 inputs.
+ *
+ *   q, k, v  [B, H, N, d] bf16, device.  K and V have the same length N as Q.
+ *   o        [B, H, N, d] of o_dtype (ATTN_BF16 or ATTN_FP32), device, written.
+ *   lse      [B, H, N] float32, device, written: natural-log logsumexp of the scaled scores
+ *            of each row over its visible keys.  May be NULL (not written).
+ *   B, H, N  >= 1;  B*H < 2^31;  N < 2^31.
+ *   d        head dimension: 64, 128 or 256.
+ *   scale    score scale (softmax(scale * Q K^T)); finite and > 0; usually 1/sqrt(d).
+ *   causal   0: every key visible.  1: key j visible to query i iff j <= i (queries and keys
+ *            have equal length, so top-left and bottom-right alignment coincide).
+ *   dtype    must be ATTN_BF16.
+ *   o_dtype  ATTN_BF16 or ATTN_FP32.
+ *   stream   cudaStream_t.
+ * Arithmetic: bf16 products accumulated in float32 (tensor cores); softmax in float32 with
+ * exp2; P rounded to bf16 before the P.V product; the running sum l is summed from the float32
+ * values of P.  Returns ATTN_OK once the kernel is enqueued.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int H, int N, int d, float scale, int causal,
+             int dtype, int o_dtype, void* stream);
+
+/*
+ * attn_hadamard_quant -- random-sign Hadamard transform plus per-block E4M3 quantisation.
+ *
+ *   x       [B, H, N, d] bf16, device (read).
+ *   x8      [B, H, N, d] E4M3 bytes, device (written).
+ *   scales  [B, H, ceil(N/128)] float32, device (written): dequantisation scale per block of
+ *           128 rows of one (batch, head), so that x8 * scale approximates the transformed row.
+ *   signs   d int8 entries, each +1 or -1, device (read): the diagonal D of the transform.
+ *           NULL = no transform (plain per-block quantisation, as for V).
+ *   d       64, 128 or 256.
+ * Definition: with y = H_d (D x) (unnormalised Sylvester Hadamard, float32 butterflies of
+ * stride 1, 2, 4, ...; y = x when signs is NULL), per block s_u = max(max|y| / 448, 2^-126),
+ * x8 = E4M3(y * (1/s_u)) rounded to nearest even with saturation, and
+ * scale = s_u * (1/sqrt(d)) (or s_u without the transform), all in IEEE float32.  The
+ * normalised transform (1/sqrt(d)) H_d D is orthogonal, so scores computed from transformed Q
+ * and K are unchanged.  Entries of `signs` other than +-1 are not checked on the device; an
+ * entry that is not -1 counts as +1.
+ */
+int attn_hadamard_quant(const void* x, void* x8, float* scales, const signed char* signs,
+                        int B, int H, int N, int d, void* stream);
+
+/*
+ * attn_fwd_fp8 -- exact-attention forward on per-block E4M3 inputs (approximate: the inputs
+ * and P carry E4M3 rounding).
+ *
+ *   q8, k8, v8     [B, H, N, d] E4M3 bytes, device (from attn_hadamard_quant; Q and K with the
+ *                  same sign vector, V usually without the transform).
+ *   q_scale, k_scale, v_scale   [B, H, ceil(N/128)] float32 block scales, device.
+ *   o              [B, H, N, d] of o_dtype (ATTN_BF16 or ATTN_FP32), device, written.
+ *   lse            [B, H, N] float32 or NULL, as for attn_fwd.
+ *   d              must be 128.
+ *   scale, causal, stream   as for attn_fwd.
+ * Arithmetic: E4M3 products accumulated in float32; the Q/K block scales are folded into the
+ * softmax scale of each tile pair; P is scaled by 2^(8-tau) * s_v(block) / max_block s_v and
+ * rounded to E4M3 before the P.V product; O is divided by l and rescaled at the end.
+ */
+int attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
+                 const float* q_scale, const float* k_scale, const float* v_scale,
+                 void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
+                 int o_dtype, void* stream);
+
+/*
+ * attn_device_status -- synchronises `stream`, returns the current device's status word and
+ * clears it.  ATTN_OK if no kernel of this library reported a problem since the last call;
+ * ATTN_ERR_TIMEOUT if a bounded wait inside a kernel ran out (that kernel's outputs are then
+ * undefined, the CUDA context stays usable); ATTN_ERR_CUDA if synchronising failed.
+ */
+int attn_device_status(void* stream);
+
+/* attn_status_string -- static, human-readable name of a status code (never NULL). */
+const char* attn_status_string(int status);
+
+/* attn_num_kernel_launches -- number of kernels this library has launched in this process
+ * (all devices), for launch accounting in benchmarks. */
+unsigned long long attn_num_kernel_launches(void);
+
+/* attn_shutdown -- frees the library's per-device workspaces.  Call with no work of this
+ * library pending; later calls re-create what they need. */
+void attn_shutdown(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTENTION_100_B200_ATTN_H */

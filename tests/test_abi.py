@@ -1,0 +1,101 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point the public
+header declares, and rejects bad arguments before making any CUDA call."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_attention_100_b200 as ea
+from exact_attention_100_b200 import build as ea_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    ea_build.build()
+    return ea.lib()
+
+
+def _declared_functions():
+    with open(os.path.join(ROOT, "include", "attn.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|void|const char\*|unsigned long long)\s+(attn_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    assert names == sorted(["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status",
+                            "attn_status_string", "attn_num_kernel_launches", "attn_shutdown"])
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    assert ea.attn_status_string(0) == "ATTN_OK"
+    assert ea.attn_status_string(1) == "ATTN_ERR_INVALID_ARG"
+    assert ea.attn_status_string(4) == "ATTN_ERR_TIMEOUT"
+    assert ea.attn_status_string(99) == "ATTN_ERR_UNKNOWN"
+
+
+# fake, 16-byte-aligned addresses: the calls below must fail their argument checks before any
+# CUDA call, so these are never dereferenced
+P = ctypes.c_void_p(0x10000)
+P2 = ctypes.c_void_p(0x20000)
+NULL = ctypes.c_void_p(0)
+MIS = ctypes.c_void_p(0x10008)
+
+
+def _fwd(L, q=P, k=P, v=P, o=P2, lse=NULL, B=1, H=1, N=128, d=128, scale=0.1, causal=0, dtype=0, o_dtype=0):
+    return L.attn_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, o_dtype, NULL)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=NULL), dict(k=NULL), dict(v=NULL), dict(o=NULL), dict(q=MIS), dict(o=MIS), dict(lse=MIS),
+    dict(B=0), dict(H=-1), dict(N=0), dict(scale=0.0), dict(scale=-1.0), dict(scale=float("inf")),
+    dict(scale=float("nan")), dict(causal=2), dict(o_dtype=2), dict(dtype=7), dict(B=1 << 16, H=1 << 16),
+])
+def test_fwd_rejects_bad_arguments(L, kw):
+    assert _fwd(L, **kw) == ea.ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw", [dict(d=96), dict(d=32), dict(d=512), dict(dtype=ea.ATTN_E4M3), dict(dtype=ea.ATTN_FP32)])
+def test_fwd_reports_unsupported(L, kw):
+    assert _fwd(L, **kw) == ea.ATTN_ERR_UNSUPPORTED
+
+
+def test_hadamard_quant_rejects_bad_arguments(L):
+    f = L.attn_hadamard_quant
+    assert f(NULL, P, P2, NULL, 1, 1, 128, 128, NULL) == ea.ATTN_ERR_INVALID_ARG
+    assert f(P, NULL, P2, NULL, 1, 1, 128, 128, NULL) == ea.ATTN_ERR_INVALID_ARG
+    assert f(P, P, NULL, NULL, 1, 1, 128, 128, NULL) == ea.ATTN_ERR_INVALID_ARG
+    assert f(P, P, P2, MIS, 1, 1, 128, 128, NULL) == ea.ATTN_ERR_INVALID_ARG
+    assert f(P, P, P2, NULL, 1, 0, 128, 128, NULL) == ea.ATTN_ERR_INVALID_ARG
+    assert f(P, P, P2, NULL, 1, 1, 128, 48, NULL) == ea.ATTN_ERR_UNSUPPORTED
+
+
+def test_fwd_fp8_rejects_bad_arguments(L):
+    f = L.attn_fwd_fp8
+    ok = [P, P, P, P2, P2, P2, P2, NULL, 1, 1, 128, 128, 0.1, 0, 0, NULL]
+    for i in range(7):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    a = list(ok)
+    a[11] = 64
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+    a = list(ok)
+    a[12] = -0.5
+    assert f(*a) == ea.ATTN_ERR_INVALID_ARG
+
+
+def test_python_binding_has_same_names():
+    for name in ["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status", "attn_status_string",
+                 "attn_num_kernel_launches", "attn_shutdown"]:
+        assert callable(getattr(ea, name)), name

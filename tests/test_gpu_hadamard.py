@@ -1,0 +1,63 @@
+"""GPU parity of the Hadamard + per-block E4M3 pre-kernel against the oracle: codes and scales
+must be bit-identical (the quantisation decision is taken in float32 on both sides)."""
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import exact_attention_100_b200 as ea
+from exact_attention_100_b200 import build as ea_build
+from exact_attention_100_b200.inputs import hadamard_signs, normal_qkv, round_to_bf16
+from oracle import hadamard_quant_ref
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    ea_build.build()
+    ea.lib()
+
+
+def _run(x_np, signs_np):
+    x = torch.from_numpy(x_np).to(torch.bfloat16).cuda()
+    s = torch.from_numpy(signs_np).cuda() if signs_np is not None else None
+    x8, sc = ea.attn_hadamard_quant(x, s)
+    torch.cuda.synchronize()
+    return x8.cpu().numpy(), sc.cpu().numpy()
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("use_signs", [True, False])
+@pytest.mark.parametrize("shape", [(1, 1, 1), (1, 2, 127), (2, 3, 300), (1, 1, 1024)])
+def test_bit_exact_against_oracle(d, use_signs, shape):
+    B, H, N = shape
+    q, _, _ = normal_qkv(B, H, N, d, seed=N + d, outlier_frac=1e-3)
+    signs = hadamard_signs(d) if use_signs else None
+    codes, scales = _run(q, signs)
+    rc, rs = hadamard_quant_ref(q, signs)
+    np.testing.assert_array_equal(scales, rs)
+    np.testing.assert_array_equal(codes, rc)
+
+
+def test_fp8_config_q_tensor_bit_exact():
+    # B=2 H=16 N=8192 d=128 with 0.1% N(0, 10^2) outliers, seeded signs (the FP8 workload)
+    q, _, _ = normal_qkv(2, 16, 8192, 128, seed=0, outlier_frac=1e-3)
+    signs = hadamard_signs(128)
+    codes, scales = _run(q, signs)
+    rc, rs = hadamard_quant_ref(q, signs)
+    np.testing.assert_array_equal(scales, rs)
+    np.testing.assert_array_equal(codes, rc)
+
+
+def test_zero_block_and_large_values():
+    x = np.zeros((1, 1, 260, 128), dtype=np.float32)
+    x[0, 0, 128:256] = 3.0e4
+    x[0, 0, 256:, ::2] = -1.0e-30
+    x = round_to_bf16(x)
+    signs = hadamard_signs(128)
+    codes, scales = _run(x, signs)
+    rc, rs = hadamard_quant_ref(x.astype(np.float64), signs)
+    np.testing.assert_array_equal(scales, rs)
+    np.testing.assert_array_equal(codes, rc)
