@@ -50,6 +50,8 @@ def lib() -> ctypes.CDLL:
         L.attn_hadamard_quant.restype = i
         L.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
         L.attn_fwd_fp8.restype = i
+        L.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
+        L.attn_fwd_noalloc.restype = i
         L.attn_device_status.argtypes = [vp]
         L.attn_device_status.restype = i
         L.attn_status_string.argtypes = [i]
@@ -116,6 +118,19 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, o_dtype=None, 
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
     _check(lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, s, int(bool(causal)),
                           ATTN_BF16, od, _stream_ptr(stream)), "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_noalloc(q, k, v, o, lse=None, scale=None, causal=False, stream=None):
+    """``attn_fwd`` through the entry point that allocates no device memory (its scratch is a
+    static device array of the library).  ``o`` (bf16 or f32) must be given; ``lse`` may be
+    None.  The first call on a device does a one-time set-up."""
+    import torch
+    B, H, N, d = _dims(q)
+    od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, s,
+                                  int(bool(causal)), ATTN_BF16, od, _stream_ptr(stream)), "attn_fwd_noalloc")
     return o, lse
 
 

@@ -118,6 +118,30 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
                  int o_dtype, void* stream);
 
 /*
+ * attn_fwd_noalloc -- attn_fwd for callers that cannot allocate device memory.  The pages have
+ * no counterpart; it exists for this library's users.
+ *
+ * Same arguments, arithmetic and results as attn_fwd.  attn_fwd creates a small per-device
+ * workspace with cudaMalloc on its first call; runtimes that own all device memory through
+ * their own pool, hosts with a fixed memory budget and latency-critical loops that must never
+ * reach cudaMalloc (it can synchronise the device) cannot allow that.  This entry point calls
+ * no cudaMalloc, cudaFree or other allocating routine: the kernel's scratch (its device status
+ * word, 4 bytes) lives in a static device array of 256 bytes that every GPU loading this
+ * library holds until the process exits.  The scratch needed does not depend on B, H, N or d;
+ * a call needing more than the array holds would be refused with ATTN_ERR_INVALID_ARG.
+ *   - The first call on each device does a one-time set-up (device address of the array,
+ *     kernel attributes); make that first call before any stream capture.
+ *   - Every call shares the array: each call clears the status word on `stream` before its
+ *     kernel runs, and calls that overlap on the GPU (different streams) race on it.
+ *   - A bounded wait that runs out inside such a call is recorded only in that static word;
+ *     attn_device_status() does not report it (use attn_fwd when that report is needed).
+ *   - Calls through this entry point are not counted by attn_num_kernel_launches().
+ */
+int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int N, int d, float scale, int causal,
+                     int dtype, int o_dtype, void* stream);
+
+/*
  * attn_device_status -- synchronises `stream`, returns the current device's status word and
  * clears it.  ATTN_OK if no kernel of this library reported a problem since the last call;
  * ATTN_ERR_TIMEOUT if a bounded wait inside a kernel ran out (that kernel's outputs are then

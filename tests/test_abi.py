@@ -29,7 +29,8 @@ def _declared_functions():
 def test_header_declares_the_boundary():
     names = _declared_functions()
     assert names == sorted(["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status",
-                            "attn_status_string", "attn_num_kernel_launches", "attn_shutdown"])
+                            "attn_status_string", "attn_num_kernel_launches", "attn_shutdown",
+                            "attn_fwd_noalloc"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -97,5 +98,5 @@ def test_fwd_fp8_rejects_bad_arguments(L):
 
 def test_python_binding_has_same_names():
     for name in ["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status", "attn_status_string",
-                 "attn_num_kernel_launches", "attn_shutdown"]:
+                 "attn_num_kernel_launches", "attn_shutdown", "attn_fwd_noalloc"]:
         assert callable(getattr(ea, name)), name
