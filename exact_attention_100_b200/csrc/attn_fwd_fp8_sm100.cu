@@ -1,13 +1,14 @@
-// E4M3 attention forward for sm_100a.
-#include "attn_kernels.h"
+// E4M3 instantiation of the attention forward (kernel template in attn_fwd_kernel.cuh).
+#include "attn_fwd_kernel.cuh"
 
 namespace ea {
 
-cudaError_t setup_fwd_fp8_kernels() { return cudaSuccess; }
+cudaError_t setup_fwd_fp8_kernels() { return set_fwd_smem_attr<128, 2, ElemE4m3>(); }
 
-cudaError_t launch_attn_fwd_fp8(int, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&,
-                                int, cudaStream_t) {
-  return cudaErrorNotSupported;
+cudaError_t launch_attn_fwd_fp8(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                                const FwdParams& p, int num_sms, cudaStream_t stream) {
+  if (d != 128) return cudaErrorInvalidValue;
+  return launch_fwd<128, 2, ElemE4m3>(q, k, v, p, num_sms, stream);
 }
 
 }  // namespace ea

@@ -1,0 +1,758 @@
+// Exact attention forward for sm_100a (B200): persistent, warp-specialised, tcgen05 + TMEM.
+// One template serves the bf16 forward and the E4M3 forward (Elem = ElemBf16 / ElemE4m3).
+//
+// What one CTA computes: for a unit (one batch*head and NQ consecutive 128-row Q tiles) the
+// tiled recurrence of "FlashAttention-2/3", section "技术原理" (outer loop over Q blocks,
+// inner loop over K/V blocks, running row max m and row sum l), in the FA-2 form with the
+// normalisation deferred to the end ("FlashAttention-2/3", FA-2 improvement 1), writing O and
+// the per-row logsumexp ("Flash Attention V3 解析", section 2.2).  Causal units skip the K/V
+// blocks that are entirely masked (same section) and run longest first.
+//
+// Roles (warp specialisation, "FlashAttention-3", section "异步搬运与异步计算"):
+//   warps 0..4*NQ-1   softmax warpgroup q = warp/4: one thread per S row (= TMEM lane)
+//   next 4 warps      correction warpgroup: serves events from the MMA thread -- a lazy O
+//                     rescale before a P.V, or the epilogue of a finished Q tile
+//   next warp         MMA issuer (one thread issues every tcgen05.mma)
+//   next warp         TMA producer (one thread; Q tiles and a ring of K/V slots)
+//   remaining warps   idle (the CTA is a whole number of warpgroups)
+//
+// Overlap ("FlashAttention-3", sections "Ping-pong 调度" and "同一个 warpgroup 内部也能再叠一层";
+// "Flash Attention V3 解析", section 3.2.3):
+//   NQ = 2: per K/V block j the MMA order is PV0(j), S0(j+1), PV1(j), S1(j+1): the tensor core
+//           runs one tile's GEMMs while the other tile's softmax runs.
+//   NQ = 1: S is double-buffered in TMEM and S(j+1) is issued before PV(j), so the softmax of
+//           block j+1 overlaps P.V of block j.
+//
+// TMEM (512 columns x 128 lanes of 32 bit): S buffers of 128 columns at [0, 256); P (packed
+// bf16 or E4M3) overwrites the first columns of its S buffer; O_q at [256 + D*q, +D).
+//
+// Lazy rescale: a row's reference max m moves only when a block max exceeds it by more than
+// Elem::kTau (base-2 units).  The softmax thread rescales l itself and flags the rows whose O
+// must be multiplied by alpha = 2^(m_old - m_new); only then does the MMA thread ask the
+// correction warpgroup to rescale O before the next P.V.  O and l always refer to the same m,
+// so O / l is exact, and p <= 2^kTau.
+//
+// Softmax arithmetic per block: one TMEM load of the whole row, a tree of 3-input maxima,
+// x = s * c - m with packed f32x2 FMAs, p = 2^x on the special-function unit for most pairs
+// and, for a quarter of them, on the FMA pipe (2^x = 2^n * q(x - n) with n = round(x) and q a
+// cubic fitted on [-1/2, 1/2], relative error < 1e-4), packed f32x2 row sums.
+
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "attn_kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace ea {
+
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct ElemBf16 {
+  static constexpr int kBytes = 2;
+  static constexpr bool kFp8 = false;
+  static constexpr uint32_t kFmt = 1;   // bf16 in kind::f16
+  static constexpr int kKeysPerMma = 16;  // K of one P.V MMA
+  static constexpr float kTau = 8.0f;
+  static constexpr int kPCols = 64;     // TMEM columns of a 128-key P row
+};
+
+struct ElemE4m3 {
+  static constexpr int kBytes = 1;
+  static constexpr bool kFp8 = true;
+  static constexpr uint32_t kFmt = 0;   // e4m3 in kind::f8f6f4
+  static constexpr int kKeysPerMma = 32;
+  static constexpr float kTau = 4.0f;   // p <= 16, and p * 16 <= 256 < 448
+  static constexpr float kPScale = 16.0f;
+  static constexpr int kPCols = 32;
+};
+
+template <int D, int NQ, class E>
+struct FwdCfg {
+  static constexpr int kBoxBytes = 128 * 128;                 // one TMA box: 128 rows x 128 bytes
+  static constexpr int kBoxes = D * E::kBytes / 128;
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;       // 128 rows x D elements
+  static constexpr int kSlots = (NQ == 1) ? 2 : (196608 - NQ * kTileBytes) / kTileBytes > 8 ? 8
+                                                : (196608 - NQ * kTileBytes) / kTileBytes;
+  static constexpr int kSBufs = NQ == 1 ? 2 : NQ;             // S buffers in TMEM
+  static constexpr int kOCol = 256;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kCorrWarp0 = 4 * NQ;
+  static constexpr int kMmaWarp = 4 * NQ + 4;
+  static constexpr int kLoadWarp = 4 * NQ + 5;
+  static constexpr int kThreads = (4 * NQ + 8) * 32;
+  static constexpr int kEvents = 4;                           // correction event ring
+  static constexpr int kQOff = 0;
+  static constexpr int kRingOff = NQ * kTileBytes;
+  static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
+  // full[kSlots], empty[kSlots], q_full, q_empty, s_full[kSBufs], p_full[kSBufs], o_corr[NQ],
+  // o_done[NQ], o_free[NQ], ev_full[kEvents], ev_empty[kEvents], drain
+  static constexpr int kNumBars = 2 * kSlots + 2 + 2 * kSBufs + 3 * NQ + 2 * kEvents + 1;
+  static constexpr int kAlphaOff = kBarOff + ((kNumBars * 8 + 15) / 16) * 16;
+  static constexpr int kRowMOff = kAlphaOff + NQ * 2 * 128 * 4;
+  static constexpr int kRowLOff = kRowMOff + NQ * 2 * 128 * 4;
+  static constexpr int kFlagOff = kRowLOff + NQ * 2 * 128 * 4;  // [NQ][2][4] int
+  static constexpr int kEventOff = kFlagOff + NQ * 2 * 4 * 4;  // [kEvents][4] int
+  static constexpr int kMiscOff = kEventOff + kEvents * 16;
+  static constexpr int kSmemBytes = kMiscOff + 16;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;        // room to align the base to 1024 bytes
+  static_assert(kSlots >= 2, "K/V ring");
+  static_assert(kSmemAlloc <= 232448, "shared memory budget");
+  static_assert(kSBufs * 128 <= kOCol && kOCol + NQ * D <= kTmemCols, "TMEM budget");
+  // register split (setmaxnreg) for NQ = 2: 2 softmax warpgroups, 1 correction, 1 MMA/TMA
+  static constexpr uint32_t kRegSoftmax = 168, kRegCorr = 80, kRegOther = 96;
+  static_assert(NQ != 2 || (2 * kRegSoftmax + kRegCorr + kRegOther) * 128 == 65536, "register split");
+};
+
+enum : int { kEvRescale = 0, kEvEpilogue = 1, kEvEnd = 2 };
+
+struct Unit {
+  int bh;
+  int tile0;   // index of the first 128-row Q tile of the unit
+  int n[2];    // K/V blocks each Q tile visits (0: the tile lies past the sequence end)
+  int n_max;
+};
+
+template <int NQ>
+__device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
+  Unit U;
+  const int r = u / p.BH;
+  U.bh = u - r * p.BH;
+  const int pair = p.causal ? (p.n_pairs - 1 - r) : r;  // causal: longest units first
+  U.tile0 = pair * NQ;
+  U.n_max = 0;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int t = U.tile0 + q;
+    int n = 0;
+    if (q < NQ && t * 128 < p.N) n = p.causal ? min(t + 1, p.n_blocks) : p.n_blocks;
+    U.n[q] = n;
+    U.n_max = max(U.n_max, n);
+  }
+  return U;
+}
+
+// k-th unit of this CTA: round-robin over CTAs, alternating direction every round.
+__device__ __forceinline__ int unit_index(int k) {
+  const int g = gridDim.x;
+  return k * g + ((k & 1) ? (g - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+}
+
+// Bounded wait that ignores the abort flag: used at exit so that this thread's own async
+// copies and MMAs finish before shared memory and TMEM are released.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* status) {
+  const uint32_t a = smem_addr(bar);
+  const unsigned long long t0 = global_timer_ns();
+  while (!bar_try_wait(a, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(status, kDevStatusTimeout);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// (x0, x1) <- (s0 * c + nm, s1 * c + nm), one packed f32x2 FMA
+__device__ __forceinline__ void fma2_bcast(float& x0, float& x1, float s0, float s1, float c, float nm) {
+  asm("{\n\t.reg .b64 ra, rc, rm, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rc, {%4, %4};\n\t"
+      "mov.b64 rm, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rc, rm;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(x0), "=f"(x1)
+      : "f"(s0), "f"(s1), "f"(c), "f"(nm));
+}
+
+// (a0, a1) += (b0, b1), one packed f32x2 add
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%0, %1};\n\t"
+      "mov.b64 rb, {%2, %3};\n\t"
+      "add.rn.f32x2 ra, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+
+// 2^x for a pair, on the FMA pipe: n = round(x) by the 1.5*2^23 shift, f = x - n in [-1/2, 1/2],
+// 2^f by the cubic of fit_exp2_poly.py (relative error < 7.5e-5), 2^n added to the exponent.
+// x is clamped to >= -125 so the result stays a normal float (2^-125 stands in for 0).
+__device__ __forceinline__ void exp2_fma_pair(float& y0, float& y1, float x0, float x1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  float t0, t1, p0, p1;
+  asm("{\n\t.reg .b64 rx, rs, rt, rn, rf, rp, c3, c2, c1, c0;\n\t"
+      "mov.b64 rx, {%4, %5};\n\t"
+      "mov.b64 rs, {%6, %6};\n\t"
+      "add.rn.f32x2 rt, rx, rs;\n\t"      // t = x + shift: round(x) in the low mantissa bits
+      "sub.rn.f32x2 rn, rt, rs;\n\t"      // n = round(x) as a float
+      "sub.rn.f32x2 rf, rx, rn;\n\t"      // f = x - n
+      "mov.b64 c3, {%7, %7};\n\t"
+      "mov.b64 c2, {%8, %8};\n\t"
+      "mov.b64 c1, {%9, %9};\n\t"
+      "mov.b64 c0, {%10, %10};\n\t"
+      "fma.rn.f32x2 rp, c3, rf, c2;\n\t"
+      "fma.rn.f32x2 rp, rp, rf, c1;\n\t"
+      "fma.rn.f32x2 rp, rp, rf, c0;\n\t"
+      "mov.b64 {%0, %1}, rt;\n\t"
+      "mov.b64 {%2, %3}, rp;\n\t}"
+      : "=f"(t0), "=f"(t1), "=f"(p0), "=f"(p1)
+      : "f"(x0), "f"(x1), "f"(kShift), "f"(0.0551716648042202f), "f"(0.2426111251115799f),
+        "f"(0.6932609677314758f), "f"(0.9999280571937561f));
+  // the integer n sits in the low bits of t; shifting by 23 drops the shift's own bits
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+// Loads a 128-column row slice of S (this thread's lane) with four loads and one wait.
+__device__ __forceinline__ void tmem_ld_row128(uint32_t taddr, uint32_t (&r)[128]) {
+  uint32_t(&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
+  uint32_t(&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
+  uint32_t(&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[64]);
+  uint32_t(&d)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[96]);
+  tmem_ld_32cols(taddr, a);
+  tmem_ld_32cols(taddr + 32, b);
+  tmem_ld_32cols(taddr + 64, c);
+  tmem_ld_32cols(taddr + 96, d);
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 128; i += 8)
+    asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]),
+                 "+r"(r[i + 6]), "+r"(r[i + 7]));
+}
+
+// Softmax of one 128-key block for this thread's row.  r holds the raw scores; on return the
+// packed P of the block is in pk (kPCols words), and the function returns sum_j p_j (not yet
+// scaled back for E4M3).  c = softmax scale * log2 e (times the Q/K block scales for E4M3);
+// nm = -(reference max) (+ log2 of the P scale for E4M3).
+template <class E, bool kMasked>
+__device__ __forceinline__ float softmax_block(uint32_t (&r)[128], uint32_t* pk, float c, float nm) {
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  float pv[4];
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    float x0, x1, p0, p1;
+    fma2_bcast(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), c, nm);
+    if (!kMasked && (i & 3) == 3) {
+      exp2_fma_pair(p0, p1, x0, x1);
+    } else {
+      p0 = ex2_approx(x0);
+      p1 = ex2_approx(x1);
+    }
+    add2(acc[2 * (i & 3)], acc[2 * (i & 3) + 1], p0, p1);
+    if constexpr (E::kFp8) {
+      pv[2 * (i & 1)] = p0;
+      pv[2 * (i & 1) + 1] = p1;
+      if (i & 1) pk[i >> 1] = pack_e4m3x4(pv[0], pv[1], pv[2], pv[3]);
+    } else {
+      pk[i] = pack_bf16x2(p0, p1);
+    }
+  }
+  add2(acc[0], acc[1], acc[2], acc[3]);
+  add2(acc[4], acc[5], acc[6], acc[7]);
+  add2(acc[0], acc[1], acc[4], acc[5]);
+  return acc[0] + acc[1];
+}
+
+template <int D, int NQ, class E>
+__global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<D, NQ, E>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* full = bars;                   // [kSlots] K/V slot loaded
+  uint64_t* empty = full + C::kSlots;      // [kSlots] K/V slot released by the MMAs
+  uint64_t* q_full = empty + C::kSlots;
+  uint64_t* q_empty = q_full + 1;
+  uint64_t* s_full = q_empty + 1;          // [kSBufs] S ready in TMEM
+  uint64_t* p_full = s_full + C::kSBufs;   // [kSBufs] P ready in TMEM (softmax warps)
+  uint64_t* o_corr = p_full + C::kSBufs;   // [NQ] O rescaled (correction warps)
+  uint64_t* o_done = o_corr + NQ;          // [NQ] a P.V finished (commit)
+  uint64_t* o_free = o_done + NQ;          // [NQ] epilogue finished reading O (correction warps)
+  uint64_t* ev_full = o_free + NQ;         // [kEvents] event posted (MMA thread)
+  uint64_t* ev_empty = ev_full + C::kEvents;  // [kEvents] event taken (correction warps)
+  uint64_t* drain = ev_empty + C::kEvents;
+  float* alpha_s = reinterpret_cast<float*>(smem + C::kAlphaOff);  // [NQ][2][128]
+  // [NQ][2][128], slot = parity of the tile's unit count: a tile with a single K/V block writes
+  // the next unit's values before the previous epilogue has necessarily read its own
+  float* row_m = reinterpret_cast<float*>(smem + C::kRowMOff);     // base-2 LSE
+  float* row_l = reinterpret_cast<float*>(smem + C::kRowLOff);     // divisor of O
+  volatile int* flags = reinterpret_cast<volatile int*>(smem + C::kFlagOff);    // [NQ][2][4]
+  volatile int* events = reinterpret_cast<volatile int*>(smem + C::kEventOff);  // [kEvents][4]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kSlots; ++i) {
+      bar_init(&full[i], 1);
+      bar_init(&empty[i], 1);
+    }
+    bar_init(q_full, 1);
+    bar_init(q_empty, 1);
+    for (int b = 0; b < C::kSBufs; ++b) {
+      bar_init(&s_full[b], 1);
+      bar_init(&p_full[b], 4);  // one arrive per softmax warp
+    }
+    for (int q = 0; q < NQ; ++q) {
+      bar_init(&o_corr[q], 4);
+      bar_init(&o_done[q], 1);
+      bar_init(&o_free[q], 4);
+    }
+    for (int e = 0; e < C::kEvents; ++e) {
+      bar_init(&ev_full[e], 1);
+      bar_init(&ev_empty[e], 4);
+    }
+    bar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == C::kLoadWarp && lane == 0) {
+    prefetch_tensor_map(&tmQ);
+    prefetch_tensor_map(&tmK);
+    prefetch_tensor_map(&tmV);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const AbortState ab{abort_flag, p.status};
+  const int nb = p.n_blocks;
+
+  if (warp < 4 * NQ) {
+    // ==================================================================== softmax warpgroups
+    if constexpr (NQ == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kRegSoftmax));
+    const int q = warp >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    uint32_t sit = 0;  // S blocks consumed by this warpgroup so far
+    uint32_t uit = 0;  // units this warpgroup's tile took part in
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int u = unit_index(k);
+      if (u >= p.num_units) break;
+      const Unit U = decode_unit<NQ>(u, p);
+      const int n = U.n[q];
+      if (n == 0) continue;
+      const int tile_row0 = (U.tile0 + q) * 128;
+      const int row_g = tile_row0 + row;
+      int lim_row = p.N;  // keys [0, lim_row) are visible to this row
+      if (p.causal) lim_row = min(lim_row, row_g + 1);
+      float c_base = p.scale_log2;
+      float ps_log2_base = 0.f, l_div = 1.f;
+      const float* ks = nullptr;
+      const float* vs = nullptr;
+      float kj = 1.f, vj = 1.f;
+      if constexpr (E::kFp8) {
+        // the Q block scale folds into c; P is stored as p * 16 * s_v(j) / max_j s_v(j)
+        c_base *= __ldg(p.q_scale + static_cast<size_t>(U.bh) * nb + U.tile0 + q);
+        ks = p.k_scale + static_cast<size_t>(U.bh) * nb;
+        vs = p.v_scale + static_cast<size_t>(U.bh) * nb;
+        float vmax = 0.f;
+        for (int b = lane; b < nb; b += 32) vmax = fmaxf(vmax, __ldg(vs + b));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+        ps_log2_base = lg2_approx(E::kPScale / vmax);
+        l_div = E::kPScale / vmax;
+        kj = __ldg(ks);
+        vj = __ldg(vs);
+      }
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < n; ++j) {
+        float c = c_base, ps_log2 = 0.f;
+        if constexpr (E::kFp8) {
+          c *= kj;
+          ps_log2 = ps_log2_base + lg2_approx(vj);
+          if (j + 1 < n) {  // next block's scales, ahead of their use
+            kj = __ldg(ks + j + 1);
+            vj = __ldg(vs + j + 1);
+          }
+        }
+        const uint32_t sbuf = (C::kSBufs == NQ) ? static_cast<uint32_t>(q) : (sit & 1u);
+        const uint32_t sphase = (C::kSBufs == NQ) ? (sit & 1u) : ((sit >> 1) & 1u);
+        ok = warp_all(wait_bar(&s_full[sbuf], sphase, ab));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tS = lane_base + sbuf * 128;
+        uint32_t r[128];
+        tmem_ld_row128(tS, r);
+        const int key0 = j * 128;
+        const bool need_mask = (key0 + 128 > p.N) || (p.causal && key0 + 127 > tile_row0);
+        if (need_mask) {
+          const int lim = lim_row - key0;
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i >= lim) r[i] = __float_as_uint(-INFINITY);
+        }
+        // row max: eight independent two-input max chains.  (The three-input max.f32 gave
+        // wrong partial maxima on masked rows in this kernel on B200 and is not used.)
+        float mx[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) mx[t] = __uint_as_float(r[t]);
+#pragma unroll
+        for (int i = 8; i < 128; i += 8)
+#pragma unroll
+          for (int t = 0; t < 8; ++t) mx[t] = fmaxf(mx[t], __uint_as_float(r[i + t]));
+        const float mb =
+            fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
+        float alpha = 1.f;
+        if (mb > m + E::kTau) {
+          alpha = ex2_approx(m - mb);
+          m = mb;
+          l *= alpha;
+        }
+        uint32_t pk[E::kPCols];
+        float lb = need_mask ? softmax_block<E, true>(r, pk, c, ps_log2 - m)
+                             : softmax_block<E, false>(r, pk, c, ps_log2 - m);
+        if constexpr (E::kFp8) lb *= ex2_approx(-ps_log2);
+        l += lb;
+        tmem_st_32cols(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        if constexpr (!E::kFp8) tmem_st_32cols(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        tmem_st_wait();
+        const uint32_t slot = sit & 1u;
+        alpha_s[(q * 2 + slot) * 128 + row] = alpha;
+        const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && j > 0;
+        if (j == n - 1) {
+          row_m[(q * 2 + (uit & 1u)) * 128 + row] = m + lg2_approx(l);
+          row_l[(q * 2 + (uit & 1u)) * 128 + row] = l * l_div;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          flags[(q * 2 + slot) * 4 + quarter] = need_rescale ? 1 : 0;
+          bar_arrive(&p_full[sbuf]);
+        }
+        ++sit;
+      }
+      ++uit;
+    }
+  } else if (warp < C::kCorrWarp0 + 4) {
+    // ========================================= correction warpgroup: rescale and epilogue events
+    if constexpr (NQ == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegCorr));
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    uint32_t eit = 0;
+    bool ok = true;
+    while (ok) {
+      const uint32_t es = eit % C::kEvents;
+      ok = warp_all(wait_bar(&ev_full[es], (eit / C::kEvents) & 1u, ab));
+      if (!ok) break;
+      const int kq = events[es * 4 + 0];
+      const uint32_t c = static_cast<uint32_t>(events[es * 4 + 1]);
+      const int bh = events[es * 4 + 2];
+      const int tile = events[es * 4 + 3];
+      __syncwarp();
+      if (lane == 0) bar_arrive(&ev_empty[es]);
+      ++eit;
+      const int kind = kq & 0xff;
+      const int q = (kq >> 8) & 0xff;
+      const int uslot = kq >> 16;
+      if (kind == kEvEnd) break;
+      const uint32_t tO = tmem + lane_off + C::kOCol + q * D;
+      if (kind == kEvRescale) {
+        // P.V number c-1 of this tile must have landed before O is rescaled for number c
+        ok = warp_all(wait_bar(&o_done[q], (c - 1u) & 1u, ab));
+        if (!ok) break;
+        tc_fence_after();
+        const float alpha = alpha_s[(q * 2 + (c & 1u)) * 128 + row];
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t r[32];
+            tmem_ld_32cols(tO + 32 * cc, r);
+            tmem_ld_wait(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st_32cols(tO + 32 * cc, r);
+          }
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(&o_corr[q]);
+      } else {
+        // epilogue after P.V number c, the tile's last: O / l and the LSE to global memory
+        ok = warp_all(wait_bar(&o_done[q], c & 1u, ab));
+        if (!ok) break;
+        tc_fence_after();
+        const float lse2 = row_m[(q * 2 + uslot) * 128 + row];
+        const float inv = 1.f / row_l[(q * 2 + uslot) * 128 + row];
+        const int row_g = tile * 128 + row;
+        const bool valid = row_g < p.N;
+        const size_t orow = (static_cast<size_t>(bh) * p.N + row_g) * D;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld_32cols(tO + 32 * cc, r);
+          tmem_ld_wait(r);
+          if (!valid) continue;
+          if (p.o_fp32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + 32 * cc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
+                                   __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + orow + 32 * cc);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv, __uint_as_float(r[8 * i + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv);
+              dst[i] = w;
+            }
+          }
+        }
+        if (valid && p.lse != nullptr) p.lse[static_cast<size_t>(bh) * p.N + row_g] = lse2 * kLn2;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(&o_free[q]);
+      }
+    }
+  } else {
+    if constexpr (NQ == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegOther));
+    if (warp == C::kMmaWarp && lane == 0) {
+      // ======================================================================= MMA issuer
+      constexpr uint32_t kIdS = make_idesc(128, 128, E::kFmt, false);  // S = Q K^T, both K-major
+      constexpr uint32_t kIdPV = make_idesc(128, D, E::kFmt, true);    // O += P V, V MN-major
+      const uint32_t q_base = smem_addr(smem + C::kQOff);
+      const uint32_t ring_base = smem_addr(smem + C::kRingOff);
+      uint32_t it = 0, qit = 0, sc = 0, ev = 0;
+      uint32_t pc[NQ], rc[NQ], uc[NQ];
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) pc[q] = rc[q] = uc[q] = 0;
+
+      auto slot_of = [&](uint32_t idx) { return idx % C::kSlots; };
+      auto wait_loaded = [&](uint32_t idx) {
+        const bool r = wait_bar(&full[idx % C::kSlots], (idx / C::kSlots) & 1u, ab);
+        tc_fence_after();
+        return r;
+      };
+      auto issue_s = [&](int q, uint32_t slot, uint32_t buf) {
+        const uint32_t d = tmem + buf * 128;
+#pragma unroll
+        for (int kk = 0; kk < D * E::kBytes / 32; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+          const uint64_t a = make_sdesc_sw128(q_base + q * C::kTileBytes + off, 16, 1024);
+          const uint64_t b = make_sdesc_sw128(ring_base + slot * C::kTileBytes + off, 16, 1024);
+          if constexpr (E::kFp8)
+            mma_f8_ss(d, a, b, kIdS, kk > 0 ? 1u : 0u);
+          else
+            mma_f16_ss(d, a, b, kIdS, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int q, uint32_t slot, uint32_t buf, bool acc) {
+        const uint32_t d = tmem + C::kOCol + q * D;
+#pragma unroll
+        for (int kk = 0; kk < 128 / E::kKeysPerMma; ++kk) {
+          const uint32_t a = tmem + buf * 128 + kk * 8;  // kKeysPerMma keys of P = 8 columns
+          const uint64_t b =
+              make_sdesc_sw128(ring_base + slot * C::kTileBytes + kk * E::kKeysPerMma * 128, C::kBoxBytes, 1024);
+          if constexpr (E::kFp8)
+            mma_f8_ts(d, a, b, kIdPV, (acc || kk > 0) ? 1u : 0u);
+          else
+            mma_f16_ts(d, a, b, kIdPV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto push_event = [&](int kind, int q, uint32_t c, int bh, int tile, uint32_t uslot) {
+        const uint32_t es = ev % C::kEvents;
+        if (!wait_bar(&ev_empty[es], ((ev / C::kEvents) & 1u) ^ 1u, ab)) return false;
+        events[es * 4 + 0] = kind | (q << 8) | static_cast<int>(uslot << 16);
+        events[es * 4 + 1] = static_cast<int>(c);
+        events[es * 4 + 2] = bh;
+        events[es * 4 + 3] = tile;
+        bar_arrive(&ev_full[es]);
+        ++ev;
+        return true;
+      };
+      // P.V of tile q for block j: wait for P, keep O safe (epilogue / lazy rescale), issue.
+      auto pv_step = [&](int q, int j, const Unit& U, uint32_t vslot, uint32_t buf) {
+        // P of this block sits in S buffer `buf`; that buffer's p_full completes once per use
+        const uint32_t pphase = (C::kSBufs == NQ) ? (pc[q] & 1u) : ((pc[q] >> 1) & 1u);
+        if (!wait_bar(&p_full[buf], pphase, ab)) return false;
+        tc_fence_after();
+        if (j == 0) {
+          // P.V 0 overwrites O: the previous unit's epilogue of this tile must be done with it
+          if (!wait_bar(&o_free[q], (uc[q] & 1u) ^ 1u, ab)) return false;
+          ++uc[q];
+        } else {
+          const uint32_t fs = (q * 2 + (pc[q] & 1u)) * 4;
+          if (flags[fs] | flags[fs + 1] | flags[fs + 2] | flags[fs + 3]) {
+            if (!push_event(kEvRescale, q, pc[q], 0, 0, 0)) return false;
+            if (!wait_bar(&o_corr[q], rc[q] & 1u, ab)) return false;
+            ++rc[q];
+          }
+        }
+        tc_fence_after();
+        issue_pv(q, vslot, buf, j > 0);
+        tc_commit(&o_done[q]);
+        // uc[q] was counted at j == 0 of this unit: the softmax wrote slot (uc[q] - 1) & 1
+        if (j == U.n[q] - 1 && !push_event(kEvEpilogue, q, pc[q], U.bh, U.tile0 + q, (uc[q] - 1u) & 1u)) return false;
+        ++pc[q];
+        return true;
+      };
+
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int u = unit_index(k);
+        if (u >= p.num_units) break;
+        const Unit U = decode_unit<NQ>(u, p);
+        const uint32_t base = it;  // ring index of K_0; K_j = base + 2j, V_j = base + 2j + 1
+        it += 2u * U.n_max;
+        ok = wait_bar(q_full, qit & 1u, ab);
+        ++qit;
+        if (!ok) break;
+        if (!(ok = wait_loaded(base))) break;
+        if constexpr (NQ == 2) {
+#pragma unroll
+          for (int q = 0; q < NQ; ++q)
+            if (U.n[q] > 0) {
+              issue_s(q, slot_of(base), q);
+              tc_commit(&s_full[q]);
+            }
+          tc_commit(&empty[slot_of(base)]);
+          if (U.n_max == 1) tc_commit(q_empty);
+          for (int j = 0; j < U.n_max && ok; ++j) {
+            const uint32_t vi = base + 2 * j + 1, ki = base + 2 * j + 2;
+            const bool more = j + 1 < U.n_max;
+            if (!(ok = wait_loaded(vi))) break;
+            if (j < U.n[0] && !(ok = pv_step(0, j, U, slot_of(vi), 0))) break;
+            if (more) {
+              if (!(ok = wait_loaded(ki))) break;
+              if (j + 1 < U.n[0]) {
+                issue_s(0, slot_of(ki), 0);
+                tc_commit(&s_full[0]);
+              }
+            }
+            if (j < U.n[1] && !(ok = pv_step(1, j, U, slot_of(vi), 1))) break;
+            tc_commit(&empty[slot_of(vi)]);
+            if (more) {
+              if (j + 1 < U.n[1]) {
+                issue_s(1, slot_of(ki), 1);
+                tc_commit(&s_full[1]);
+              }
+              tc_commit(&empty[slot_of(ki)]);
+              if (j + 2 == U.n_max) tc_commit(q_empty);
+            }
+          }
+        } else {
+          // one Q tile, S double-buffered: S(j+1) goes in before P.V(j)
+          issue_s(0, slot_of(base), sc & 1u);
+          tc_commit(&s_full[sc & 1u]);
+          ++sc;
+          tc_commit(&empty[slot_of(base)]);
+          if (U.n_max == 1) tc_commit(q_empty);
+          for (int j = 0; j < U.n_max && ok; ++j) {
+            const uint32_t vi = base + 2 * j + 1, ki = base + 2 * j + 2;
+            const uint32_t pbuf = (sc - 1u) & 1u;  // buffer holding P(j)
+            if (j + 1 < U.n_max) {
+              if (!(ok = wait_loaded(ki))) break;
+              issue_s(0, slot_of(ki), sc & 1u);
+              tc_commit(&s_full[sc & 1u]);
+              ++sc;
+              tc_commit(&empty[slot_of(ki)]);
+              if (j + 2 == U.n_max) tc_commit(q_empty);
+            }
+            if (!(ok = wait_loaded(vi))) break;
+            if (!(ok = pv_step(0, j, U, slot_of(vi), pbuf))) break;
+            tc_commit(&empty[slot_of(vi)]);
+          }
+        }
+      }
+      if (ok) push_event(kEvEnd, 0, 0, 0, 0, 0);
+      // every MMA issued so far must complete before TMEM is released
+      tc_commit(drain);
+      drain_wait(drain, 0, p.status);
+    } else if (warp == C::kLoadWarp && lane == 0) {
+      // ====================================================================== TMA producer
+      uint32_t it = 0, qit = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int u = unit_index(k);
+        if (u >= p.num_units) break;
+        const Unit U = decode_unit<NQ>(u, p);
+        if (qit > 0 && !(ok = wait_bar(q_empty, (qit - 1u) & 1u, ab))) break;
+        bar_arrive_expect_tx(q_full, NQ * C::kTileBytes);
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+#pragma unroll
+          for (int b = 0; b < C::kBoxes; ++b)
+            tma_load_3d(smem + C::kQOff + q * C::kTileBytes + b * C::kBoxBytes, &tmQ, q_full,
+                        b * (128 / E::kBytes), (U.tile0 + q) * 128, U.bh);
+        ++qit;
+        for (int j = 0; j < U.n_max && ok; ++j) {
+#pragma unroll
+          for (int kv = 0; kv < 2; ++kv) {
+            const uint32_t s = it % C::kSlots;
+            if (!(ok = wait_bar(&empty[s], ((it / C::kSlots) & 1u) ^ 1u, ab))) break;
+            bar_arrive_expect_tx(&full[s], C::kTileBytes);
+            uint8_t* dst = smem + C::kRingOff + s * C::kTileBytes;
+#pragma unroll
+            for (int b = 0; b < C::kBoxes; ++b)
+              tma_load_3d(dst + b * C::kBoxBytes, kv ? &tmV : &tmK, &full[s], b * (128 / E::kBytes), j * 128,
+                          U.bh);
+            ++it;
+          }
+        }
+      }
+      // let every issued copy land before the CTA can exit
+      const uint32_t first = it > static_cast<uint32_t>(C::kSlots) ? it - C::kSlots : 0u;
+      for (uint32_t i = first; i < it; ++i) drain_wait(&full[i % C::kSlots], (i / C::kSlots) & 1u, p.status);
+      if (qit > 0) drain_wait(q_full, (qit - 1u) & 1u, p.status);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D, int NQ, class E>
+cudaError_t set_fwd_smem_attr() {
+  return cudaFuncSetAttribute(attn_fwd_kernel<D, NQ, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              FwdCfg<D, NQ, E>::kSmemAlloc);
+}
+
+template <int D, int NQ, class E>
+cudaError_t launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const FwdParams& p,
+                       int num_sms, cudaStream_t stream) {
+  using C = FwdCfg<D, NQ, E>;
+  const int grid = p.num_units < num_sms ? p.num_units : num_sms;
+  attn_fwd_kernel<D, NQ, E><<<grid, C::kThreads, C::kSmemAlloc, stream>>>(q, k, v, p);
+  return cudaGetLastError();
+}
+
+}  // namespace ea

@@ -146,3 +146,25 @@ def test_lse_optional_and_launch_count():
     assert torch.equal(o1, o2)
     assert ea.attn_num_kernel_launches() - n0 == 2
     assert ea.attn_device_status() == ea.ATTN_OK
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_growing_scores_exercise_lazy_rescale(d, causal):
+    # key magnitudes ramp up along the sequence, so the running max of late rows climbs by far
+    # more than the lazy threshold several times: O must be rescaled in TMEM on the way
+    B, H, N = 1, 2, 1100
+    (q, k, v), _ = device_qkv(B, H, N, d, seed=11)
+    ramp = (1.0 + 6.0 * np.arange(N) / N).astype(np.float32)[None, None, :, None]
+    from exact_attention_100_b200.inputs import round_to_bf16
+    k = round_to_bf16(k * ramp)
+    qd, kd, vd = (torch.from_numpy(a).to(torch.bfloat16).cuda() for a in (q, k, v))
+    o, lse = ea.attn_fwd(qd, kd, vd, scale=1.0 / math.sqrt(d), causal=causal, o_dtype=torch.float32)
+    torch.cuda.synchronize()
+    res = compare_full(o, lse, q, k, v, 1.0 / math.sqrt(d), causal)
+    # These scores are far from iid N(0,1): the weights are peaked, so the bf16 rounding of P no
+    # longer averages out.  With P = bf16(p) = p (1 + e), |e| <= 2^-8, and l summed from f32 p,
+    # |O_kernel - O| <= 2^-8 * sum_j w_j |v_j| <= 2^-8 max|v| (plus ~1e-4 relative from exp2).
+    bound = (2.0 ** -8 + 2e-4) * float(np.abs(v).max())
+    assert res["finite"] and res["o_max_abs"] <= bound and res["o_mean_abs"] <= 1e-3, (d, causal, res, bound)
+    assert res["lse_max_rel"] <= 1e-3, (d, causal, res)

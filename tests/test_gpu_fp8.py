@@ -1,0 +1,87 @@
+"""GPU checks of the E4M3 forward (attn_fwd_fp8) fed by the Hadamard/E4M3 pre-kernel.
+
+Two references:
+* the float64 oracle on the dequantised inputs (codes x block scales): the only difference
+  left is the E4M3 rounding of P, so the RMSE must be small (<= 1e-2) and LSE, which is summed
+  from float32 p, must match to 1e-3 relative;
+* the float64 oracle on the original bf16 inputs (the spec's reference): RMSE <= 3e-2 with and
+  without the Hadamard transform on the FP8 workload (B=2 H=16 N=8192 d=128, 0.1% N(0, 10^2)
+  outliers), sampled rows.  The transform must lower the error ("FlashAttention-3", section
+  "FP8 路径与低精度误差": incoherent processing reduces the FP8 error).
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import exact_attention_100_b200 as ea
+from exact_attention_100_b200 import build as ea_build
+from exact_attention_100_b200.inputs import hadamard_signs, normal_qkv
+from oracle import attention_ref, dequant_ref, hadamard_rotate_ref
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    ea_build.build()
+    ea.lib()
+    yield
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+
+
+def _quantise(q, k, v, signs):
+    dev = lambda a: torch.from_numpy(a).to(torch.bfloat16).cuda()
+    s = torch.from_numpy(signs).cuda() if signs is not None else None
+    q8, qs = ea.attn_hadamard_quant(dev(q), s)
+    k8, ks = ea.attn_hadamard_quant(dev(k), s)
+    v8, vs = ea.attn_hadamard_quant(dev(v), None)
+    return q8, qs, k8, ks, v8, vs
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n", [1, 127, 300, 1024])
+@pytest.mark.parametrize("use_signs", [True, False])
+def test_against_oracle_on_dequantised_inputs(causal, n, use_signs):
+    d = 128
+    q, k, v = normal_qkv(1, 2, n, d, seed=n, outlier_frac=1e-3)
+    signs = hadamard_signs(d) if use_signs else None
+    q8, qs, k8, ks, v8, vs = _quantise(q, k, v, signs)
+    o, lse = ea.attn_fwd_fp8(q8, k8, v8, qs, ks, vs, causal=causal, o_dtype=torch.float32)
+    torch.cuda.synchronize()
+    qd = dequant_ref(q8.cpu().numpy(), qs.cpu().numpy())
+    kd = dequant_ref(k8.cpu().numpy(), ks.cpu().numpy())
+    vd = dequant_ref(v8.cpu().numpy(), vs.cpu().numpy())
+    o_ref, lse_ref = attention_ref(qd, kd, vd, 1 / math.sqrt(d), causal)
+    og = o.cpu().numpy().astype(np.float64)
+    assert np.isfinite(og).all()
+    rmse = float(np.sqrt(np.mean((og - o_ref) ** 2)))
+    assert rmse <= 1e-2, rmse
+    # element bound: E4M3 keeps 3 fraction bits, so each P entry carries a relative rounding of
+    # at most 2^-4 (normal range), i.e. |O_kernel - O| <= 2^-4 max|v| (+ the subnormal floor)
+    assert np.abs(og - o_ref).max() <= (2.0 ** -4 + 1e-2) * np.abs(vd).max()
+    lrel = np.abs(lse.cpu().numpy() - lse_ref) / np.abs(lse_ref)
+    assert lrel.max() <= 1e-3, lrel.max()
+
+
+def test_fp8_workload_rmse_with_and_without_hadamard():
+    B, H, N, d = 2, 16, 8192, 128
+    q, k, v = normal_qkv(B, H, N, d, seed=0, outlier_frac=1e-3)
+    rng = np.random.default_rng(3)
+    rows = [(int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(N))) for _ in range(48)]
+    rmse = {}
+    for use in (True, False):
+        q8, qs, k8, ks, v8, vs = _quantise(q, k, v, hadamard_signs(d) if use else None)
+        o, _ = ea.attn_fwd_fp8(q8, k8, v8, qs, ks, vs, causal=False, o_dtype=torch.float32)
+        torch.cuda.synchronize()
+        err = []
+        for (b, h, i) in rows:
+            o_ref, _ = attention_ref(q[b, h, i:i + 1], k[b, h], v[b, h], 1 / math.sqrt(d), False)
+            err.append(o[b, h, i].cpu().numpy().astype(np.float64) - o_ref[0])
+        rmse[use] = float(np.sqrt(np.mean(np.square(err))))
+    assert rmse[True] <= 3e-2 and rmse[False] <= 3e-2, rmse
+    assert rmse[True] < rmse[False], rmse
