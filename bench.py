@@ -367,10 +367,10 @@ def fp8_section(args, dev, rank):
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
-    def pre():
-        ea.attn_hadamard_quant(q, signs, x8[0], sc[0], stream=stream)
-        ea.attn_hadamard_quant(k, signs, x8[1], sc[1], stream=stream)
-        ea.attn_hadamard_quant(v, None, x8[2], sc[2], stream=stream)
+    outs = (x8[0], x8[1], x8[2], sc[0], sc[1], sc[2])
+
+    def pre():  # one launch for the three tensors (Q, K transformed; V not)
+        ea.attn_hadamard_quant_qkv(q, k, v, signs, outs=outs, stream=stream)
 
     steps = max(3, min(args.steps, 50))
     for _ in range(3):

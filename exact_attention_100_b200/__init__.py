@@ -48,6 +48,8 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd.restype = i
         L.attn_hadamard_quant.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
         L.attn_hadamard_quant.restype = i
+        L.attn_hadamard_quant_qkv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
+        L.attn_hadamard_quant_qkv.restype = i
         L.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
         L.attn_fwd_fp8.restype = i
         L.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
@@ -149,6 +151,24 @@ def attn_hadamard_quant(x, signs=None, x8=None, scales=None, stream=None):
     _check(lib().attn_hadamard_quant(_ptr(x), _ptr(x8), _ptr(scales), _ptr(signs), B, H, N, d,
                                      _stream_ptr(stream)), "attn_hadamard_quant")
     return x8, scales
+
+
+def attn_hadamard_quant_qkv(q, k, v, signs, outs=None, stream=None):
+    """One launch: Q and K through H_d D then E4M3, V straight to E4M3 (per-block scales).
+
+    Returns ``(q8, k8, v8, q_scale, k_scale, v_scale)``; ``outs`` may supply them.
+    """
+    import torch
+    B, H, N, d = _dims(q)
+    nb = (N + 127) // 128
+    if outs is None:
+        outs = tuple(torch.empty(q.shape, dtype=torch.uint8, device=q.device) for _ in range(3)) + \
+            tuple(torch.empty((B, H, nb), dtype=torch.float32, device=q.device) for _ in range(3))
+    q8, k8, v8, qs, ks, vs = outs
+    _check(lib().attn_hadamard_quant_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs), _ptr(ks),
+                                         _ptr(vs), _ptr(signs), B, H, N, d, _stream_ptr(stream)),
+           "attn_hadamard_quant_qkv")
+    return outs
 
 
 def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o=None, lse=None, scale=None, causal=False,

@@ -63,6 +63,7 @@ int device_state(DeviceState** out) {
     }
     if (ea::setup_fwd_bf16_kernels() != cudaSuccess) return ATTN_ERR_CUDA;
     if (ea::setup_fwd_fp8_kernels() != cudaSuccess) return ATTN_ERR_CUDA;
+    if (ea::setup_hadamard_quant_kernels() != cudaSuccess) return ATTN_ERR_CUDA;
     st.num_sms = sms;
     st.ready = true;
   }
@@ -169,8 +170,42 @@ int attn_hadamard_quant(const void* x, void* x8, float* scales, const signed cha
   int rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
   const float post = signs ? static_cast<float>(1.0 / std::sqrt(static_cast<double>(d))) : 1.0f;
-  if (ea::launch_hadamard_quant(x, x8, scales, signs, B * H, N, d, post, static_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
+  CUtensorMap mx;
+  if (!encode_rows_map(&mx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H)) return ATTN_ERR_CUDA;
+  uint8_t* out = static_cast<uint8_t*>(x8);
+  const int transform = signs != nullptr ? 1 : 0;
+  if (ea::launch_hadamard_quant(&mx, 1, &out, &scales, &post, &transform, signs, B * H, N, d, st->num_sms, st->status,
+                               static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return ATTN_OK;
+}
+
+int attn_hadamard_quant_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8,
+                            float* q_scale, float* k_scale, float* v_scale, const signed char* signs, int B, int H,
+                            int N, int d, void* stream) {
+  const void* in[3] = {q, k, v};
+  void* out[3] = {q8, k8, v8};
+  float* sc[3] = {q_scale, k_scale, v_scale};
+  for (int t = 0; t < 3; ++t) {
+    if (!in[t] || !out[t] || !sc[t]) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(in[t]) || !aligned16(out[t]) || !aligned16(sc[t])) return ATTN_ERR_INVALID_ARG;
+  }
+  if (!signs || !aligned16(signs)) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || N <= 0 || static_cast<long long>(B) * H > 0x7FFFFFFFLL) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  CUtensorMap maps[3];
+  for (int t = 0; t < 3; ++t)
+    if (!encode_rows_map(&maps[t], in[t], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H)) return ATTN_ERR_CUDA;
+  const float rsd = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  uint8_t* o8[3] = {static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8), static_cast<uint8_t*>(v8)};
+  const float post[3] = {rsd, rsd, 1.0f};
+  const int transform[3] = {1, 1, 0};
+  if (ea::launch_hadamard_quant(maps, 3, o8, sc, post, transform, signs, B * H, N, d, st->num_sms, st->status,
+                               static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
   return ATTN_OK;

@@ -92,8 +92,8 @@ struct FwdCfg {
   static constexpr int kAlphaOff = kBarOff + ((kNumBars * 8 + 15) / 16) * 16;
   static constexpr int kRowMOff = kAlphaOff + NQ * 2 * 128 * 4;
   static constexpr int kRowLOff = kRowMOff + NQ * 2 * 128 * 4;
-  static constexpr int kFlagOff = kRowLOff + NQ * 2 * 128 * 4;  // [NQ][2][4] int
-  static constexpr int kEventOff = kFlagOff + NQ * 2 * 4 * 4;  // [kEvents][4] int
+  static constexpr int kFlagOff = kRowLOff + NQ * 2 * 128 * 4;  // [NQ][2] int, one byte per warp
+  static constexpr int kEventOff = kFlagOff + 16;               // [kEvents][4] int
   static constexpr int kMiscOff = kEventOff + kEvents * 16;
   static constexpr int kSmemBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;        // room to align the base to 1024 bytes
@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
   // the next unit's values before the previous epilogue has necessarily read its own
   float* row_m = reinterpret_cast<float*>(smem + C::kRowMOff);     // base-2 LSE
   float* row_l = reinterpret_cast<float*>(smem + C::kRowLOff);     // divisor of O
-  volatile int* flags = reinterpret_cast<volatile int*>(smem + C::kFlagOff);    // [NQ][2][4]
+  volatile int* flags = reinterpret_cast<volatile int*>(smem + C::kFlagOff);    // [NQ][2]
   volatile int* events = reinterpret_cast<volatile int*>(smem + C::kEventOff);  // [kEvents][4]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
@@ -445,7 +445,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          flags[(q * 2 + slot) * 4 + quarter] = need_rescale ? 1 : 0;
+          reinterpret_cast<volatile uint8_t*>(flags + q * 2 + slot)[quarter] = need_rescale ? 1 : 0;
           bar_arrive(&p_full[sbuf]);
         }
         ++sit;
@@ -477,11 +477,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       if (kind == kEvEnd) break;
       const uint32_t tO = tmem + lane_off + C::kOCol + q * D;
       if (kind == kEvRescale) {
-        // P.V number c-1 of this tile must have landed before O is rescaled for number c
-        ok = warp_all(wait_bar(&o_done[q], (c - 1u) & 1u, ab));
+        // the MMA thread committed o_done (phase c) after issuing P.V number `tile` - 1 (for a
+        // rescale the event's last field carries the P.V number): that P.V must land first
+        ok = warp_all(wait_bar(&o_done[q], c & 1u, ab));
         if (!ok) break;
         tc_fence_after();
-        const float alpha = alpha_s[(q * 2 + (c & 1u)) * 128 + row];
+        const float alpha = alpha_s[(q * 2 + (static_cast<uint32_t>(tile) & 1u)) * 128 + row];
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
@@ -498,7 +499,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         __syncwarp();
         if (lane == 0) bar_arrive(&o_corr[q]);
       } else {
-        // epilogue after P.V number c, the tile's last: O / l and the LSE to global memory
+        // epilogue: the MMA thread committed o_done (phase c) after the tile's last P.V
         ok = warp_all(wait_bar(&o_done[q], c & 1u, ab));
         if (!ok) break;
         tc_fence_after();
@@ -547,15 +548,16 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       const uint32_t q_base = smem_addr(smem + C::kQOff);
       const uint32_t ring_base = smem_addr(smem + C::kRingOff);
       uint32_t it = 0, qit = 0, sc = 0, ev = 0;
-      uint32_t pc[NQ], rc[NQ], uc[NQ];
+      // per tile: P.V issued, rescale requests (o_corr phases), units (o_free phases), o_done commits
+      uint32_t pc[NQ], rc[NQ], uc[NQ], od[NQ];
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) pc[q] = rc[q] = uc[q] = 0;
+      for (int q = 0; q < NQ; ++q) pc[q] = rc[q] = uc[q] = od[q] = 0;
 
       auto slot_of = [&](uint32_t idx) { return idx % C::kSlots; };
+      // TMA-filled shared memory read by the tensor core stays in the async proxy: the wait alone
+      // orders it (no tcgen05 fence)
       auto wait_loaded = [&](uint32_t idx) {
-        const bool r = wait_bar(&full[idx % C::kSlots], (idx / C::kSlots) & 1u, ab);
-        tc_fence_after();
-        return r;
+        return wait_bar(&full[idx % C::kSlots], (idx / C::kSlots) & 1u, ab);
       };
       auto issue_s = [&](int q, uint32_t slot, uint32_t buf) {
         const uint32_t d = tmem + buf * 128;
@@ -604,19 +606,21 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
           // P.V 0 overwrites O: the previous unit's epilogue of this tile must be done with it
           if (!wait_bar(&o_free[q], (uc[q] & 1u) ^ 1u, ab)) return false;
           ++uc[q];
-        } else {
-          const uint32_t fs = (q * 2 + (pc[q] & 1u)) * 4;
-          if (flags[fs] | flags[fs + 1] | flags[fs + 2] | flags[fs + 3]) {
-            if (!push_event(kEvRescale, q, pc[q], 0, 0, 0)) return false;
-            if (!wait_bar(&o_corr[q], rc[q] & 1u, ab)) return false;
-            ++rc[q];
-          }
+        } else if (flags[q * 2 + (pc[q] & 1u)] != 0) {
+          // o_done is committed only when the correction warpgroup needs it: the commit covers
+          // every MMA issued so far, P.V number pc[q]-1 included
+          tc_commit(&o_done[q]);
+          if (!push_event(kEvRescale, q, od[q]++, 0, static_cast<int>(pc[q]), 0)) return false;
+          if (!wait_bar(&o_corr[q], rc[q] & 1u, ab)) return false;
+          ++rc[q];
         }
         tc_fence_after();
         issue_pv(q, vslot, buf, j > 0);
-        tc_commit(&o_done[q]);
-        // uc[q] was counted at j == 0 of this unit: the softmax wrote slot (uc[q] - 1) & 1
-        if (j == U.n[q] - 1 && !push_event(kEvEpilogue, q, pc[q], U.bh, U.tile0 + q, (uc[q] - 1u) & 1u)) return false;
+        if (j == U.n[q] - 1) {
+          // uc[q] was counted at j == 0 of this unit: the softmax wrote slot (uc[q] - 1) & 1
+          tc_commit(&o_done[q]);
+          if (!push_event(kEvEpilogue, q, od[q]++, U.bh, U.tile0 + q, (uc[q] - 1u) & 1u)) return false;
+        }
         ++pc[q];
         return true;
       };

@@ -36,10 +36,15 @@ cudaError_t launch_attn_fwd_bf16(int d, const CUtensorMap& q, const CUtensorMap&
 cudaError_t launch_attn_fwd_fp8(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                                 const FwdParams& p, int num_sms, cudaStream_t stream);
 
-// Hadamard + per-block E4M3 quantisation: x [BH, N, d] bf16 -> x8 [BH, N, d] e4m3, scales
-// [BH, ceil(N/128)].  signs may be nullptr (no transform).  post_scale = float(1/sqrt(d)) with
-// the transform, 1 without.
-cudaError_t launch_hadamard_quant(const void* x, void* x8, float* scales, const signed char* signs, int BH,
-                                  int N, int d, float post_scale, cudaStream_t stream);
+// Hadamard + per-block E4M3 quantisation of 1..3 tensors of one shape [BH, N, d] in one launch:
+// tm[t] is a 3-D tiled map over tensor t (bf16, box 64 x 128 x 1, 128-byte swizzle); x8[t] its
+// E4M3 output, scales[t] its [BH, ceil(N/128)] block scales, post[t] the factor on the stored
+// scale, transform[t] != 0 to apply H_d D (signs: d entries +-1).
+cudaError_t launch_hadamard_quant(const CUtensorMap* tm, int ntensors, uint8_t* const* x8, float* const* scales,
+                                  const float* post, const int* transform, const signed char* signs, int BH, int N,
+                                  int d, int num_sms, int* status, cudaStream_t stream);
+
+// Sets the pre-kernel's shared-memory attributes on the current device.
+cudaError_t setup_hadamard_quant_kernels();
 
 }  // namespace ea

@@ -5,146 +5,327 @@
 // O(d log d) and is memory-bound.  "FlashAttention-2/3", section "FA-3：拥抱 Hopper",
 // feature 3: the FP8 scales are per block, not global.
 //
-// One CTA per (batch*head, 128-row block).  A row of d bf16 is spread over d/8 lanes, 8
-// consecutive elements (16 bytes) per lane, so one warp-wide load covers 32*16 contiguous
-// bytes.  The unnormalised transform y = H_d (D x) is computed in float32 with butterfly
-// stages of stride 1, 2, 4 inside each lane's 8 values and 8, 16, ... across lanes by warp
-// shuffles -- the textbook stage order, so every element sees the same float32 additions in
-// the same order as a plain sequential transform.  The block's largest |y| sets
-// s_u = max(amax / 448, 2^-126); codes are E4M3(y * (1/s_u)) (round to nearest even,
-// saturating); the stored dequantisation scale is s_u * post_scale (post_scale = 1/sqrt(d)
-// with the transform, 1 without).
+// Persistent grid: each CTA walks over (batch*head, 128-row block) units.  The block is brought
+// into shared memory by TMA (128-byte swizzle, rows past the sequence end read as zero),
+// double-buffered so the next block streams in while the current one is transformed.  A row
+// is split over d/64 adjacent lanes, 64 consecutive elements each: the unnormalised transform
+// y = H_d (D x) runs in float32 registers with butterfly stages of stride 1, 2, ..., 32 inside
+// a thread and 64, 128 between the lanes of a row (shuffles) -- the textbook stage order, so
+// every element sees the same float32 additions in the same order as a plain sequential
+// transform.  The block's largest |y| sets s_u = max(amax / 448, 2^-126); codes are
+// E4M3(y * (1/s_u)) (round to nearest even, saturating); the stored dequantisation scale is
+// s_u * post_scale (post_scale = 1/sqrt(d) with the transform, 1 without).
 
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
 #include "attn_kernels.h"
+#include "sm100_ptx.cuh"
 
 namespace ea {
 
-template <int D, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32)
-    hadamard_quant_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ x8, float* __restrict__ scales,
-                          const signed char* __restrict__ signs, int N, int n_blocks, float post_scale) {
-  constexpr int kLanesPerRow = D / 8;
-  constexpr int kRowsPerStep = 32 / kLanesPerRow;
-  constexpr int kRowsPerWarp = 128 / WARPS;
-  constexpr int kSteps = kRowsPerWarp / kRowsPerStep;
-  static_assert(kSteps * kRowsPerStep * WARPS == 128, "row split");
+// (a0, a1) += (b0, b1) and (a0, a1) -= (b0, b1) as packed f32x2 operations
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb;\n\tmov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %3};\n\t"
+      "add.rn.f32x2 ra, ra, rb;\n\tmov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1) : "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void sub2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb;\n\tmov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %3};\n\t"
+      "sub.rn.f32x2 ra, ra, rb;\n\tmov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1) : "f"(b0), "f"(b1));
+}
+// (v0, v1) <- (s * v0 + o0, s * v1 + o1), one packed f32x2 fma; with s = +-1 the product is
+// exact and the result is the correctly rounded o +- v
+__device__ __forceinline__ void fma2_rn(float& v0, float& v1, float s, float o0, float o1) {
+  asm("{\n\t.reg .b64 rv, rs, ro;\n\tmov.b64 rv, {%0, %1};\n\tmov.b64 rs, {%2, %2};\n\t"
+      "mov.b64 ro, {%3, %4};\n\tfma.rn.f32x2 rv, rs, rv, ro;\n\tmov.b64 {%0, %1}, rv;\n\t}"
+      : "+f"(v0), "+f"(v1) : "f"(s), "f"(o0), "f"(o1));
+}
 
-  __shared__ float warp_max[WARPS];
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int blk = blockIdx.x % n_blocks;
-  const int bh = blockIdx.x / n_blocks;
-  const int sub_row = lane / kLanesPerRow;
-  const int col0 = (lane % kLanesPerRow) * 8;
-  const size_t head_base = static_cast<size_t>(bh) * N * D;
-  const int row_base = blk * 128 + warp * kRowsPerWarp + sub_row;
-
-  float v[kSteps][8];
-  // load (rows past the sequence end are zero and do not raise the block max)
-#pragma unroll
-  for (int s = 0; s < kSteps; ++s) {
-    const int row = row_base + s * kRowsPerStep;
-    uint4 w = make_uint4(0u, 0u, 0u, 0u);
-    if (row < N) w = __ldg(reinterpret_cast<const uint4*>(x + head_base + static_cast<size_t>(row) * D + col0));
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      v[s][2 * e] = __uint_as_float(ws[e] << 16);
-      v[s][2 * e + 1] = __uint_as_float(ws[e] & 0xFFFF0000u);
+// Bounded wait of every thread of the CTA on `bar`; flags `abort_s` if it ran out.  Callers
+// follow it with __syncthreads() and a CTA-uniform check of `abort_s`.
+__device__ __forceinline__ void cta_wait(uint64_t* bar, uint32_t parity, volatile int* abort_s, int* status) {
+  const uint32_t a = smem_addr(bar);
+  if (bar_try_wait(a, parity)) return;
+  const unsigned long long t0 = global_timer_ns();
+  while (!bar_try_wait(a, parity)) {
+    if (*abort_s || global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_s = 1;
+      atomicOr(status, kDevStatusTimeout);
+      return;
     }
-  }
-
-  if (signs != nullptr) {
-    float sg[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) sg[e] = (__ldg(signs + col0 + e) == -1) ? -1.f : 1.f;
-#pragma unroll
-    for (int s = 0; s < kSteps; ++s) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[s][e] *= sg[e];
-      // strides 1, 2, 4: inside the lane
-#pragma unroll
-      for (int h = 1; h < 8; h <<= 1) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if ((e & h) == 0) {
-            const float a = v[s][e], b = v[s][e + h];
-            v[s][e] = __fadd_rn(a, b);
-            v[s][e + h] = __fsub_rn(a, b);
-          }
-        }
-      }
-      // strides 8 .. D/2: partner lane differs in bit (h/8) of the lane index within the row
-#pragma unroll
-      for (int hl = 1; hl < kLanesPerRow; hl <<= 1) {
-        const bool upper = (lane & hl) != 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float other = __shfl_xor_sync(0xffffffffu, v[s][e], hl);
-          v[s][e] = upper ? __fsub_rn(other, v[s][e]) : __fadd_rn(v[s][e], other);
-        }
-      }
-    }
-  }
-
-  float amax = 0.f;
-#pragma unroll
-  for (int s = 0; s < kSteps; ++s)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[s][e]));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if (lane == 0) warp_max[warp] = amax;
-  __syncthreads();
-  amax = warp_max[0];
-#pragma unroll
-  for (int w = 1; w < WARPS; ++w) amax = fmaxf(amax, warp_max[w]);
-
-  const float s_u = fmaxf(__fdiv_rn(amax, 448.f), 1.17549435e-38f);
-  const float rcp = __frcp_rn(s_u);
-  if (threadIdx.x == 0) scales[static_cast<size_t>(bh) * n_blocks + blk] = __fmul_rn(s_u, post_scale);
-
-#pragma unroll
-  for (int s = 0; s < kSteps; ++s) {
-    const int row = row_base + s * kRowsPerStep;
-    if (row >= N) continue;
-    uint32_t packed[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
-          make_float2(__fmul_rn(v[s][4 * h], rcp), __fmul_rn(v[s][4 * h + 1], rcp)), __NV_SATFINITE, __NV_E4M3);
-      const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
-          make_float2(__fmul_rn(v[s][4 * h + 2], rcp), __fmul_rn(v[s][4 * h + 3], rcp)), __NV_SATFINITE, __NV_E4M3);
-      packed[h] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
-    }
-    *reinterpret_cast<uint2*>(x8 + head_base + static_cast<size_t>(row) * D + col0) = make_uint2(packed[0], packed[1]);
   }
 }
 
-cudaError_t launch_hadamard_quant(const void* x, void* x8, float* scales, const signed char* signs, int BH, int N,
-                                  int d, float post_scale, cudaStream_t stream) {
+template <int D>
+struct HqCfg {
+  static constexpr int kThreadsPerRow = D / 64;
+  static constexpr int kThreads = 128 * kThreadsPerRow;
+  static constexpr int kElems = 64;                 // elements of a row held by one thread
+  static constexpr int kBoxes = D / 64;             // 128-byte TMA boxes per row (one per thread)
+  static constexpr int kBufBytes = 128 * D * 2;
+  static constexpr int kCtasPerSm = D == 256 ? 1 : (D == 128 ? 3 : 4);
+};
+
+// Up to three tensors of one shape in one launch (Q and K with the transform, V without).
+struct HqJob {
+  uint8_t* x8[3];
+  float* scales[3];
+  float post[3];
+  int transform[3];
+  int ntensors;
+};
+
+template <int D>
+__global__ void __launch_bounds__(HqCfg<D>::kThreads, HqCfg<D>::kCtasPerSm)
+    hadamard_quant_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
+                          const __grid_constant__ CUtensorMap tm2, const HqJob job,
+                          const signed char* __restrict__ signs, int N, int n_blocks, int total_blocks, int* status) {
+  using C = HqCfg<D>;
+  constexpr int kE = C::kElems;
+  constexpr int kWarps = C::kThreads / 32;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ float warp_max[2][kWarps];
+  __shared__ int abort_s;
+  __shared__ __align__(16) uint32_t smask[D / 2];  // bf16x2 sign-bit masks of D (bits 15 and 31)
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int row = tid / C::kThreadsPerRow;   // row of the block
+  const int half = tid % C::kThreadsPerRow;  // which 64-element part of the row
+
+  if (tid == 0) {
+    bar_init(&bar[0], 1);
+    bar_init(&bar[1], 1);
+    abort_s = 0;
+    fence_barrier_init();
+    prefetch_tensor_map(&tm0);
+    prefetch_tensor_map(&tm1);
+    prefetch_tensor_map(&tm2);
+  }
+  for (int i = tid; i < D / 2; i += C::kThreads) {
+    uint32_t m = 0u;
+    if (signs != nullptr) {
+      if (__ldg(signs + 2 * i) == -1) m |= 0x00008000u;
+      if (__ldg(signs + 2 * i + 1) == -1) m |= 0x80000000u;
+    }
+    smask[i] = m;
+  }
+  __syncthreads();
+
+  // units interleave the tensors (u -> tensor u % ntensors) so that every SM mixes blocks that
+  // run the transform with blocks that only quantise
+  auto issue = [&](int u, int buf) {
+    const int t = u % job.ntensors;
+    const int b = u / job.ntensors;
+    const int blk = b % n_blocks;
+    const int bh = b / n_blocks;
+    const CUtensorMap* tm = t == 0 ? &tm0 : (t == 1 ? &tm1 : &tm2);
+    bar_arrive_expect_tx(&bar[buf], C::kBufBytes);
+#pragma unroll
+    for (int bx = 0; bx < C::kBoxes; ++bx)
+      tma_load_3d(smem + buf * C::kBufBytes + bx * 16384, tm, &bar[buf], bx * 64, blk * 128, bh);
+  };
+
+  if (tid == 0 && blockIdx.x < total_blocks) issue(blockIdx.x, 0);
+  int it = 0;
+  for (int u = blockIdx.x; u < total_blocks; u += gridDim.x, ++it) {
+    const int buf = it & 1;
+    // the other buffer was released by the __syncthreads() that ended the previous iteration
+    if (tid == 0 && u + static_cast<int>(gridDim.x) < total_blocks) issue(u + gridDim.x, buf ^ 1);
+    cta_wait(&bar[buf], (it >> 1) & 1, &abort_s, status);
+    __syncthreads();
+    if (abort_s) break;
+
+    const int t = u % job.ntensors;
+    const int b = u / job.ntensors;
+    const int blk = b % n_blocks;
+    const int bh = b / n_blocks;
+    // explicit selects keep the parameter block out of local memory
+    const bool transform = (t == 0 ? job.transform[0] : (t == 1 ? job.transform[1] : job.transform[2])) != 0;
+    uint8_t* const x8 = t == 0 ? job.x8[0] : (t == 1 ? job.x8[1] : job.x8[2]);
+    float* const scales = t == 0 ? job.scales[0] : (t == 1 ? job.scales[1] : job.scales[2]);
+    const float post = t == 0 ? job.post[0] : (t == 1 ? job.post[1] : job.post[2]);
+    const uint8_t* sb = smem + buf * C::kBufBytes;
+
+    // this thread's kE elements of its row: box (half*kE + e)/64, 16-byte chunk c of the
+    // 128-byte box row lives at chunk c ^ (row % 8) (128-byte swizzle)
+    float v[kE];
+#pragma unroll
+    for (int c = 0; c < kE / 8; ++c) {
+      const int e0 = half * kE + c * 8;
+      const int bx = e0 >> 6;
+      const int ch = (e0 & 63) >> 3;
+      uint4 w = *reinterpret_cast<const uint4*>(sb + bx * 16384 + row * 128 + ((ch ^ (row & 7)) << 4));
+      if (transform) {  // D x: flipping the bf16 sign bits is exact
+        const uint4 mk = *reinterpret_cast<const uint4*>(&smask[e0 / 2]);
+        w.x ^= mk.x;
+        w.y ^= mk.y;
+        w.z ^= mk.z;
+        w.w ^= mk.w;
+      }
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[c * 8 + 2 * k] = __uint_as_float(ws[k] << 16);
+        v[c * 8 + 2 * k + 1] = __uint_as_float(ws[k] & 0xFFFF0000u);
+      }
+    }
+
+    if (transform) {
+      // in-thread stages, two butterflies per packed f32x2 add/sub (each lane rounds on its own,
+      // exactly like two scalar operations): stride 1 pairs (e, e+2) with (e+1, e+3)
+#pragma unroll
+      for (int e = 0; e < kE; e += 4) {
+        float s0 = v[e], s1 = v[e + 2], d0 = v[e], d1 = v[e + 2];
+        add2(s0, s1, v[e + 1], v[e + 3]);
+        sub2(d0, d1, v[e + 1], v[e + 3]);
+        v[e] = s0;
+        v[e + 2] = s1;
+        v[e + 1] = d0;
+        v[e + 3] = d1;
+      }
+#pragma unroll
+      for (int h = 2; h < kE; h <<= 1) {
+#pragma unroll
+        for (int e = 0; e < kE; e += 2) {
+          if ((e & h) == 0) {
+            float s0 = v[e], s1 = v[e + 1], d0 = v[e], d1 = v[e + 1];
+            add2(s0, s1, v[e + h], v[e + h + 1]);
+            sub2(d0, d1, v[e + h], v[e + h + 1]);
+            v[e] = s0;
+            v[e + 1] = s1;
+            v[e + h] = d0;
+            v[e + h + 1] = d1;
+          }
+        }
+      }
+      // strides 64, 128: the partner lane holds another 64-element part of the row; the lower
+      // part keeps v + other, the upper other - v, i.e. other + sgn * v with sgn = +-1 (exact)
+#pragma unroll
+      for (int hl = 1; hl < C::kThreadsPerRow; hl <<= 1) {
+        const float sgn = (half & hl) != 0 ? -1.f : 1.f;
+#pragma unroll
+        for (int e = 0; e < kE; e += 2) {
+          const float o0 = __shfl_xor_sync(0xffffffffu, v[e], hl);
+          const float o1 = __shfl_xor_sync(0xffffffffu, v[e + 1], hl);
+          fma2_rn(v[e], v[e + 1], sgn, o0, o1);
+        }
+      }
+    }
+
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < kE; ++e) amax = fmaxf(amax, fabsf(v[e]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (lane == 0) warp_max[buf][warp] = amax;
+    __syncthreads();
+    amax = warp_max[buf][0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) amax = fmaxf(amax, warp_max[buf][w]);
+
+    const float s_u = fmaxf(__fdiv_rn(amax, 448.f), 1.17549435e-38f);
+    const float rcp = __frcp_rn(s_u);
+    if (tid == 0) scales[static_cast<size_t>(bh) * n_blocks + blk] = __fmul_rn(s_u, post);
+
+    const int grow = blk * 128 + row;
+    if (grow < N) {
+      uint8_t* out = x8 + (static_cast<size_t>(bh) * N + grow) * D + half * kE;
+#pragma unroll
+      for (int c = 0; c < kE / 16; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int e = c * 16 + 4 * k;
+          const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+              make_float2(__fmul_rn(v[e], rcp), __fmul_rn(v[e + 1], rcp)), __NV_SATFINITE, __NV_E4M3);
+          const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+              make_float2(__fmul_rn(v[e + 2], rcp), __fmul_rn(v[e + 3], rcp)), __NV_SATFINITE, __NV_E4M3);
+          w[k] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+        }
+        *reinterpret_cast<uint4*>(out + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    // every thread is done with this buffer (and with warp_max[buf]) before it is refilled
+    __syncthreads();
+  }
+  // no TMA copy may still be in flight when the CTA exits
+  if (tid == 0) {
+    const int issued = total_blocks > static_cast<int>(blockIdx.x)
+                           ? (total_blocks - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                                 static_cast<int>(gridDim.x)
+                           : 0;
+    for (int i = it; i < issued && i < it + 2; ++i) {
+      const uint32_t a = smem_addr(&bar[i & 1]);
+      const unsigned long long t0 = global_timer_ns();
+      while (!bar_try_wait(a, (i >> 1) & 1)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          atomicOr(status, kDevStatusTimeout);
+          break;
+        }
+      }
+    }
+  }
+}
+
+template <int D>
+static cudaError_t launch_hq(const CUtensorMap* tm, int ntensors, const HqJob& job0, const signed char* signs, int BH,
+                             int N, int num_sms, int* status, cudaStream_t stream) {
+  using C = HqCfg<D>;
   const int n_blocks = (N + 127) / 128;
-  const long long grid = static_cast<long long>(BH) * n_blocks;
-  if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  const auto* xb = static_cast<const __nv_bfloat16*>(x);
-  auto* out = static_cast<uint8_t*>(x8);
+  const long long per = static_cast<long long>(BH) * n_blocks;
+  const long long total = per * ntensors;
+  if (total > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  HqJob job = job0;
+  job.ntensors = ntensors;
+  const long long cap = static_cast<long long>(num_sms) * C::kCtasPerSm;
+  const int grid = static_cast<int>(total < cap ? total : cap);
+  hadamard_quant_kernel<D><<<grid, C::kThreads, 2 * C::kBufBytes + 1024, stream>>>(
+      tm[0], tm[ntensors > 1 ? 1 : 0], tm[ntensors > 2 ? 2 : 0], job, signs, N, n_blocks, static_cast<int>(total),
+      status);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t set_hq_attr() {
+  return cudaFuncSetAttribute(hadamard_quant_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              2 * HqCfg<D>::kBufBytes + 1024);
+}
+
+cudaError_t setup_hadamard_quant_kernels() {
+  cudaError_t e = set_hq_attr<64>();
+  if (e == cudaSuccess) e = set_hq_attr<128>();
+  if (e == cudaSuccess) e = set_hq_attr<256>();
+  return e;
+}
+
+cudaError_t launch_hadamard_quant(const CUtensorMap* tm, int ntensors, uint8_t* const* x8, float* const* scales,
+                                  const float* post, const int* transform, const signed char* signs, int BH, int N,
+                                  int d, int num_sms, int* status, cudaStream_t stream) {
+  if (ntensors < 1 || ntensors > 3) return cudaErrorInvalidValue;
+  HqJob job{};
+  for (int t = 0; t < 3; ++t) {
+    const int s = t < ntensors ? t : 0;
+    job.x8[t] = x8[s];
+    job.scales[t] = scales[s];
+    job.post[t] = post[s];
+    job.transform[t] = transform[s];
+  }
   switch (d) {
     case 64:
-      hadamard_quant_kernel<64, 8><<<(unsigned)grid, 256, 0, stream>>>(xb, out, scales, signs, N, n_blocks, post_scale);
-      break;
+      return launch_hq<64>(tm, ntensors, job, signs, BH, N, num_sms, status, stream);
     case 128:
-      hadamard_quant_kernel<128, 8><<<(unsigned)grid, 256, 0, stream>>>(xb, out, scales, signs, N, n_blocks, post_scale);
-      break;
+      return launch_hq<128>(tm, ntensors, job, signs, BH, N, num_sms, status, stream);
     case 256:
-      hadamard_quant_kernel<256, 16><<<(unsigned)grid, 512, 0, stream>>>(xb, out, scales, signs, N, n_blocks, post_scale);
-      break;
+      return launch_hq<256>(tm, ntensors, job, signs, BH, N, num_sms, status, stream);
     default:
       return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace ea

@@ -98,6 +98,22 @@ int attn_hadamard_quant(const void* x, void* x8, float* scales, const signed cha
                         int B, int H, int N, int d, void* stream);
 
 /*
+ * attn_hadamard_quant_qkv -- attn_hadamard_quant of Q and K (with the transform) and of V
+ * (without it) in one launch: the pre-processing of the FP8 path in one call.
+ *
+ *   q, k, v                     [B, H, N, d] bf16, device (read).
+ *   q8, k8, v8                  [B, H, N, d] E4M3 bytes, device (written).
+ *   q_scale, k_scale, v_scale   [B, H, ceil(N/128)] float32, device (written).
+ *   signs                       d int8 entries +-1, device (read); must not be NULL.
+ *   d                           64, 128 or 256.
+ * Each output is bit-identical to the corresponding attn_hadamard_quant call (signs for Q and
+ * K, NULL for V).
+ */
+int attn_hadamard_quant_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8,
+                            float* q_scale, float* k_scale, float* v_scale, const signed char* signs,
+                            int B, int H, int N, int d, void* stream);
+
+/*
  * attn_fwd_fp8 -- exact-attention forward on per-block E4M3 inputs (approximate: the inputs
  * and P carry E4M3 rounding).
  *

@@ -30,7 +30,7 @@ def test_header_declares_the_boundary():
     names = _declared_functions()
     assert names == sorted(["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status",
                             "attn_status_string", "attn_num_kernel_launches", "attn_shutdown",
-                            "attn_fwd_noalloc"])
+                            "attn_fwd_noalloc", "attn_hadamard_quant_qkv"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -81,6 +81,21 @@ def test_hadamard_quant_rejects_bad_arguments(L):
     assert f(P, P, P2, NULL, 1, 1, 128, 48, NULL) == ea.ATTN_ERR_UNSUPPORTED
 
 
+def test_hadamard_quant_qkv_rejects_bad_arguments(L):
+    f = L.attn_hadamard_quant_qkv
+    ok = [P, P, P, P2, P2, P2, P2, P2, P2, P, 1, 1, 128, 128, NULL]
+    for i in range(10):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    a = list(ok)
+    a[0] = MIS
+    assert f(*a) == ea.ATTN_ERR_INVALID_ARG
+    a = list(ok)
+    a[13] = 32
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+
+
 def test_fwd_fp8_rejects_bad_arguments(L):
     f = L.attn_fwd_fp8
     ok = [P, P, P, P2, P2, P2, P2, NULL, 1, 1, 128, 128, 0.1, 0, 0, NULL]
@@ -98,5 +113,5 @@ def test_fwd_fp8_rejects_bad_arguments(L):
 
 def test_python_binding_has_same_names():
     for name in ["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status", "attn_status_string",
-                 "attn_num_kernel_launches", "attn_shutdown", "attn_fwd_noalloc"]:
+                 "attn_num_kernel_launches", "attn_shutdown", "attn_fwd_noalloc", "attn_hadamard_quant_qkv"]:
         assert callable(getattr(ea, name)), name

@@ -61,3 +61,17 @@ def test_zero_block_and_large_values():
     rc, rs = hadamard_quant_ref(x.astype(np.float64), signs)
     np.testing.assert_array_equal(scales, rs)
     np.testing.assert_array_equal(codes, rc)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("n", [1, 300, 1024])
+def test_qkv_launch_matches_oracle(d, n):
+    q, k, v = normal_qkv(2, 3, n, d, seed=n + 7 * d, outlier_frac=1e-3)
+    signs = hadamard_signs(d)
+    dev = lambda a: torch.from_numpy(a).to(torch.bfloat16).cuda()
+    outs = ea.attn_hadamard_quant_qkv(dev(q), dev(k), dev(v), torch.from_numpy(signs).cuda())
+    torch.cuda.synchronize()
+    for x, s, c8, sc in ((q, signs, outs[0], outs[3]), (k, signs, outs[1], outs[4]), (v, None, outs[2], outs[5])):
+        rc, rs = hadamard_quant_ref(x, s)
+        np.testing.assert_array_equal(sc.cpu().numpy(), rs)
+        np.testing.assert_array_equal(c8.cpu().numpy(), rc)
