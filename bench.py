@@ -452,6 +452,32 @@ def run_sweep(args):
                       flush=True)
 
 
+def run_profile_case(args):
+    """A few untimed calls of one entry point on a small case, for an ncu capture (no JSON line)."""
+    import torch
+    import exact_attention_100_b200 as ea
+    from exact_attention_100_b200.inputs import hadamard_signs
+    B, H, N, d, causal = args.shape
+    dev = torch.device("cuda", 0)
+    torch.manual_seed(0)
+    q, k, v = (torch.randn(B, H, N, d, device=dev).to(torch.bfloat16) for _ in range(3))
+    signs = torch.from_numpy(hadamard_signs(d)).to(dev)
+    if args.profile_case == "fwd":
+        for _ in range(args.reps):
+            ea.attn_fwd(q, k, v, causal=bool(causal))
+    else:
+        outs = None
+        for _ in range(args.reps):
+            outs = ea.attn_hadamard_quant_qkv(q, k, v, signs, outs=outs)
+        if args.profile_case == "fwd_fp8":
+            for _ in range(args.reps):
+                ea.attn_fwd_fp8(*outs, causal=bool(causal))
+    torch.cuda.synchronize()
+    if ea.attn_device_status() != 0:
+        raise SystemExit("device status set")
+    print("ok", args.profile_case, B, H, N, d, causal, flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -462,7 +488,14 @@ def main():
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv"], default=None,
+                    help="run --reps untimed calls of one entry point (for an ncu capture) and exit")
+    ap.add_argument("--shape", type=int, nargs=5, default=[2, 16, 8192, 128, 1], metavar=("B", "H", "N", "d", "CAUSAL"))
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
+    if args.profile_case is not None:
+        run_profile_case(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

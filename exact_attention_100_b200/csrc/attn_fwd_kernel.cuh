@@ -32,7 +32,7 @@
 // correction warpgroup to rescale O before the next P.V.  O and l always refer to the same m,
 // so O / l is exact, and p <= 2^kTau.
 //
-// Softmax arithmetic per block: one TMEM load of the whole row, a tree of 3-input maxima,
+// Softmax arithmetic per block: one TMEM load of the whole row, eight independent max chains,
 // x = s * c - m with packed f32x2 FMAs, p = 2^x on the special-function unit for most pairs
 // and, for a quarter of them, on the FMA pipe (2^x = 2^n * q(x - n) with n = round(x) and q a
 // cubic fitted on [-1/2, 1/2], relative error < 1e-4), packed f32x2 row sums.

@@ -5,16 +5,17 @@
 // O(d log d) and is memory-bound.  "FlashAttention-2/3", section "FA-3：拥抱 Hopper",
 // feature 3: the FP8 scales are per block, not global.
 //
-// Persistent grid: each CTA walks over (batch*head, 128-row block) units.  The block is brought
-// into shared memory by TMA (128-byte swizzle, rows past the sequence end read as zero),
-// double-buffered so the next block streams in while the current one is transformed.  A row
-// is split over d/64 adjacent lanes, 64 consecutive elements each: the unnormalised transform
-// y = H_d (D x) runs in float32 registers with butterfly stages of stride 1, 2, ..., 32 inside
-// a thread and 64, 128 between the lanes of a row (shuffles) -- the textbook stage order, so
-// every element sees the same float32 additions in the same order as a plain sequential
-// transform.  The block's largest |y| sets s_u = max(amax / 448, 2^-126); codes are
-// E4M3(y * (1/s_u)) (round to nearest even, saturating); the stored dequantisation scale is
-// s_u * post_scale (post_scale = 1/sqrt(d) with the transform, 1 without).
+// Persistent grid: each CTA walks over (tensor, batch*head, 128-row block) units.  A block is
+// brought into shared memory by TMA (128-byte swizzle, rows past the sequence end read as
+// zero); two blocks are in flight per CTA, the next load being issued as soon as every thread
+// has copied the current block into registers.  One thread holds a whole row (d = 64, 128) or
+// a quarter of it (d = 256, 64 elements each, four adjacent lanes): the unnormalised transform
+// y = H_d (D x) runs in float32 registers with butterfly stages of stride 1, 2, ..., 32/64
+// inside a thread and, for d = 256, 64 and 128 between the lanes of a row (shuffles) -- the
+// textbook stage order, so every element sees the same float32 additions in the same order
+// as a plain sequential transform.  The block's largest |y| sets s_u = max(amax / 448, 2^-126);
+// codes are E4M3(y * (1/s_u)) (round to nearest even, saturating); the stored dequantisation
+// scale is s_u * post_scale (post_scale = 1/sqrt(d) with the transform, 1 without).
 
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -43,9 +44,16 @@ __device__ __forceinline__ void fma2_rn(float& v0, float& v1, float s, float o0,
       : "+f"(v0), "+f"(v1) : "f"(s), "f"(o0), "f"(o1));
 }
 
-// Bounded wait of every thread of the CTA on `bar`; flags `abort_s` if it ran out.  Callers
-// follow it with __syncthreads() and a CTA-uniform check of `abort_s`.
-__device__ __forceinline__ void cta_wait(uint64_t* bar, uint32_t parity, volatile int* abort_s, int* status) {
+// (a0, a1) *= (b, b) as one packed f32x2 multiply (each lane rounds like a scalar multiply)
+__device__ __forceinline__ void mul2(float& a0, float& a1, float b) {
+  asm("{\n\t.reg .b64 ra, rb;\n\tmov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %2};\n\t"
+      "mul.rn.f32x2 ra, ra, rb;\n\tmov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1) : "f"(b));
+}
+
+// Bounded wait of this thread on `bar`; on running out it flags `abort_s` and the status word.
+// Callers reach a __syncthreads() before they act on `abort_s`, so the CTA leaves together.
+__device__ __forceinline__ void thread_wait(uint64_t* bar, uint32_t parity, volatile int* abort_s, int* status) {
   const uint32_t a = smem_addr(bar);
   if (bar_try_wait(a, parity)) return;
   const unsigned long long t0 = global_timer_ns();
@@ -60,12 +68,12 @@ __device__ __forceinline__ void cta_wait(uint64_t* bar, uint32_t parity, volatil
 
 template <int D>
 struct HqCfg {
-  static constexpr int kThreadsPerRow = D / 64;
+  static constexpr int kElems = D == 256 ? 64 : D;  // elements of a row held by one thread
+  static constexpr int kThreadsPerRow = D / kElems;
   static constexpr int kThreads = 128 * kThreadsPerRow;
-  static constexpr int kElems = 64;                 // elements of a row held by one thread
-  static constexpr int kBoxes = D / 64;             // 128-byte TMA boxes per row (one per thread)
+  static constexpr int kBoxes = D / 64;             // 128-byte TMA boxes per row
   static constexpr int kBufBytes = 128 * D * 2;
-  static constexpr int kCtasPerSm = D == 256 ? 1 : (D == 128 ? 3 : 4);
+  static constexpr int kCtasPerSm = D == 256 ? 1 : (D == 128 ? 3 : 5);
 };
 
 // Up to three tensors of one shape in one launch (Q and K with the transform, V without).
@@ -74,7 +82,7 @@ struct HqJob {
   float* scales[3];
   float post[3];
   int transform[3];
-  int ntensors;
+  int blocks_per_tensor;
 };
 
 template <int D>
@@ -96,7 +104,7 @@ __global__ void __launch_bounds__(HqCfg<D>::kThreads, HqCfg<D>::kCtasPerSm)
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int row = tid / C::kThreadsPerRow;   // row of the block
-  const int half = tid % C::kThreadsPerRow;  // which 64-element part of the row
+  const int part = tid % C::kThreadsPerRow;  // which kE-element part of the row
 
   if (tid == 0) {
     bar_init(&bar[0], 1);
@@ -117,11 +125,9 @@ __global__ void __launch_bounds__(HqCfg<D>::kThreads, HqCfg<D>::kCtasPerSm)
   }
   __syncthreads();
 
-  // units interleave the tensors (u -> tensor u % ntensors) so that every SM mixes blocks that
-  // run the transform with blocks that only quantise
   auto issue = [&](int u, int buf) {
-    const int t = u % job.ntensors;
-    const int b = u / job.ntensors;
+    const int t = u / job.blocks_per_tensor;
+    const int b = u - t * job.blocks_per_tensor;
     const int blk = b % n_blocks;
     const int bh = b / n_blocks;
     const CUtensorMap* tm = t == 0 ? &tm0 : (t == 1 ? &tm1 : &tm2);
@@ -131,64 +137,47 @@ __global__ void __launch_bounds__(HqCfg<D>::kThreads, HqCfg<D>::kCtasPerSm)
       tma_load_3d(smem + buf * C::kBufBytes + bx * 16384, tm, &bar[buf], bx * 64, blk * 128, bh);
   };
 
-  if (tid == 0 && blockIdx.x < total_blocks) issue(blockIdx.x, 0);
+  // two blocks in flight: block i of this CTA goes to buffer i % 2, and the load of block i + 2
+  // is issued as soon as every thread has read block i into registers
+  if (tid == 0) {
+    if (static_cast<int>(blockIdx.x) < total_blocks) issue(blockIdx.x, 0);
+    if (static_cast<int>(blockIdx.x + gridDim.x) < total_blocks) issue(blockIdx.x + gridDim.x, 1);
+  }
   int it = 0;
   for (int u = blockIdx.x; u < total_blocks; u += gridDim.x, ++it) {
     const int buf = it & 1;
-    // the other buffer was released by the __syncthreads() that ended the previous iteration
-    if (tid == 0 && u + static_cast<int>(gridDim.x) < total_blocks) issue(u + gridDim.x, buf ^ 1);
-    cta_wait(&bar[buf], (it >> 1) & 1, &abort_s, status);
-    __syncthreads();
-    if (abort_s) break;
+    thread_wait(&bar[buf], (it >> 1) & 1, &abort_s, status);
 
-    const int t = u % job.ntensors;
-    const int b = u / job.ntensors;
+    const int t = u / job.blocks_per_tensor;
+    const int b = u - t * job.blocks_per_tensor;
     const int blk = b % n_blocks;
     const int bh = b / n_blocks;
     // explicit selects keep the parameter block out of local memory
     const bool transform = (t == 0 ? job.transform[0] : (t == 1 ? job.transform[1] : job.transform[2])) != 0;
-    uint8_t* const x8 = t == 0 ? job.x8[0] : (t == 1 ? job.x8[1] : job.x8[2]);
-    float* const scales = t == 0 ? job.scales[0] : (t == 1 ? job.scales[1] : job.scales[2]);
-    const float post = t == 0 ? job.post[0] : (t == 1 ? job.post[1] : job.post[2]);
     const uint8_t* sb = smem + buf * C::kBufBytes;
 
-    // this thread's kE elements of its row: box (half*kE + e)/64, 16-byte chunk c of the
-    // 128-byte box row lives at chunk c ^ (row % 8) (128-byte swizzle)
+    // this thread's kE elements of its row: element e0 = part*kE + 8c.. lives in box e0/64 at
+    // 16-byte chunk ((e0 % 64) / 8) ^ (row % 8) of the row (128-byte swizzle).  With the
+    // transform, D x is a flip of bf16 sign bits, and the stride-1 butterflies of H run here.
     float v[kE];
-#pragma unroll
-    for (int c = 0; c < kE / 8; ++c) {
-      const int e0 = half * kE + c * 8;
-      const int bx = e0 >> 6;
-      const int ch = (e0 & 63) >> 3;
-      uint4 w = *reinterpret_cast<const uint4*>(sb + bx * 16384 + row * 128 + ((ch ^ (row & 7)) << 4));
-      if (transform) {  // D x: flipping the bf16 sign bits is exact
-        const uint4 mk = *reinterpret_cast<const uint4*>(&smask[e0 / 2]);
-        w.x ^= mk.x;
-        w.y ^= mk.y;
-        w.z ^= mk.z;
-        w.w ^= mk.w;
-      }
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        v[c * 8 + 2 * k] = __uint_as_float(ws[k] << 16);
-        v[c * 8 + 2 * k + 1] = __uint_as_float(ws[k] & 0xFFFF0000u);
-      }
-    }
-
     if (transform) {
-      // in-thread stages, two butterflies per packed f32x2 add/sub (each lane rounds on its own,
-      // exactly like two scalar operations): stride 1 pairs (e, e+2) with (e+1, e+3)
 #pragma unroll
-      for (int e = 0; e < kE; e += 4) {
-        float s0 = v[e], s1 = v[e + 2], d0 = v[e], d1 = v[e + 2];
-        add2(s0, s1, v[e + 1], v[e + 3]);
-        sub2(d0, d1, v[e + 1], v[e + 3]);
-        v[e] = s0;
-        v[e + 2] = s1;
-        v[e + 1] = d0;
-        v[e + 3] = d1;
+      for (int c = 0; c < kE / 8; ++c) {
+        const int e0 = part * kE + c * 8;
+        uint4 w = *reinterpret_cast<const uint4*>(sb + (e0 >> 6) * 16384 + row * 128 +
+                                                  ((((e0 & 63) >> 3) ^ (row & 7)) << 4));
+        const uint4 mk = *reinterpret_cast<const uint4*>(&smask[e0 / 2]);
+        const uint32_t ws[4] = {w.x ^ mk.x, w.y ^ mk.y, w.z ^ mk.z, w.w ^ mk.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float lo = __uint_as_float(ws[k] << 16);
+          const float hi = __uint_as_float(ws[k] & 0xFFFF0000u);
+          v[c * 8 + 2 * k] = lo + hi;
+          v[c * 8 + 2 * k + 1] = lo - hi;
+        }
       }
+      // strides 2 .. kE/2 inside the thread, on register pairs (e, e+1): one packed add and one
+      // packed sub make two butterflies, each lane rounding like a scalar operation
 #pragma unroll
       for (int h = 2; h < kE; h <<= 1) {
 #pragma unroll
@@ -204,11 +193,11 @@ __global__ void __launch_bounds__(HqCfg<D>::kThreads, HqCfg<D>::kCtasPerSm)
           }
         }
       }
-      // strides 64, 128: the partner lane holds another 64-element part of the row; the lower
-      // part keeps v + other, the upper other - v, i.e. other + sgn * v with sgn = +-1 (exact)
+      // strides kE .. D/2: the partner lane holds another part of the row; the lower part keeps
+      // v + other, the upper other - v, i.e. other + sgn * v with sgn = +-1 (exact)
 #pragma unroll
       for (int hl = 1; hl < C::kThreadsPerRow; hl <<= 1) {
-        const float sgn = (half & hl) != 0 ? -1.f : 1.f;
+        const float sgn = (part & hl) != 0 ? -1.f : 1.f;
 #pragma unroll
         for (int e = 0; e < kE; e += 2) {
           const float o0 = __shfl_xor_sync(0xffffffffu, v[e], hl);
@@ -216,45 +205,66 @@ __global__ void __launch_bounds__(HqCfg<D>::kThreads, HqCfg<D>::kCtasPerSm)
           fma2_rn(v[e], v[e + 1], sgn, o0, o1);
         }
       }
+    } else {
+#pragma unroll
+      for (int c = 0; c < kE / 8; ++c) {
+        const int e0 = part * kE + c * 8;
+        const uint4 w = *reinterpret_cast<const uint4*>(sb + (e0 >> 6) * 16384 + row * 128 +
+                                                        ((((e0 & 63) >> 3) ^ (row & 7)) << 4));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          v[c * 8 + 2 * k] = __uint_as_float(ws[k] << 16);
+          v[c * 8 + 2 * k + 1] = __uint_as_float(ws[k] & 0xFFFF0000u);
+        }
+      }
     }
 
-    float amax = 0.f;
+    // block amax: four chains in the thread, then the lanes, then the warps
+    float am[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int e = 0; e < kE; ++e) amax = fmaxf(amax, fabsf(v[e]));
+    for (int e = 0; e < kE; ++e) am[e & 3] = fmaxf(am[e & 3], fabsf(v[e]));
+    float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if (lane == 0) warp_max[buf][warp] = amax;
+    // every thread has read buffer `buf` and posted its warp maximum
     __syncthreads();
+    if (abort_s) break;
+    if (tid == 0 && u + 2 * static_cast<int>(gridDim.x) < total_blocks) issue(u + 2 * gridDim.x, buf);
     amax = warp_max[buf][0];
 #pragma unroll
     for (int w = 1; w < kWarps; ++w) amax = fmaxf(amax, warp_max[buf][w]);
 
+    uint8_t* const x8 = t == 0 ? job.x8[0] : (t == 1 ? job.x8[1] : job.x8[2]);
+    float* const scales = t == 0 ? job.scales[0] : (t == 1 ? job.scales[1] : job.scales[2]);
+    const float post = t == 0 ? job.post[0] : (t == 1 ? job.post[1] : job.post[2]);
     const float s_u = fmaxf(__fdiv_rn(amax, 448.f), 1.17549435e-38f);
     const float rcp = __frcp_rn(s_u);
     if (tid == 0) scales[static_cast<size_t>(bh) * n_blocks + blk] = __fmul_rn(s_u, post);
 
     const int grow = blk * 128 + row;
     if (grow < N) {
-      uint8_t* out = x8 + (static_cast<size_t>(bh) * N + grow) * D + half * kE;
+      uint8_t* out = x8 + (static_cast<size_t>(bh) * N + grow) * D + part * kE;
 #pragma unroll
       for (int c = 0; c < kE / 16; ++c) {
         uint32_t w[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int e = c * 16 + 4 * k;
-          const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
-              make_float2(__fmul_rn(v[e], rcp), __fmul_rn(v[e + 1], rcp)), __NV_SATFINITE, __NV_E4M3);
-          const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
-              make_float2(__fmul_rn(v[e + 2], rcp), __fmul_rn(v[e + 3], rcp)), __NV_SATFINITE, __NV_E4M3);
+          float a0 = v[e], a1 = v[e + 1], a2 = v[e + 2], a3 = v[e + 3];
+          mul2(a0, a1, rcp);
+          mul2(a2, a3, rcp);
+          const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a0, a1), __NV_SATFINITE, __NV_E4M3);
+          const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(a2, a3), __NV_SATFINITE, __NV_E4M3);
           w[k] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
         }
         *reinterpret_cast<uint4*>(out + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
-    // every thread is done with this buffer (and with warp_max[buf]) before it is refilled
-    __syncthreads();
   }
-  // no TMA copy may still be in flight when the CTA exits
+  // no TMA copy may still be in flight when the CTA exits: after an abort at block `it`, blocks
+  // it and it + 1 may have been issued and not waited for
   if (tid == 0) {
     const int issued = total_blocks > static_cast<int>(blockIdx.x)
                            ? (total_blocks - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
@@ -280,9 +290,9 @@ static cudaError_t launch_hq(const CUtensorMap* tm, int ntensors, const HqJob& j
   const int n_blocks = (N + 127) / 128;
   const long long per = static_cast<long long>(BH) * n_blocks;
   const long long total = per * ntensors;
-  if (total > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  if (total > 0x7FFFFFFFLL - 65536) return cudaErrorInvalidValue;  // u + 2 * grid stays an int
   HqJob job = job0;
-  job.ntensors = ntensors;
+  job.blocks_per_tensor = static_cast<int>(per);
   const long long cap = static_cast<long long>(num_sms) * C::kCtasPerSm;
   const int grid = static_cast<int>(total < cap ? total : cap);
   hadamard_quant_kernel<D><<<grid, C::kThreads, 2 * C::kBufBytes + 1024, stream>>>(
