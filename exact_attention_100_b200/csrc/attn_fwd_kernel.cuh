@@ -648,10 +648,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
           for (int j = 0; j < U.n_max && ok; ++j) {
             const uint32_t vi = base + 2 * j + 1, ki = base + 2 * j + 2;
             const bool more = j + 1 < U.n_max;
+            // both waits come before the wait for P: a completed barrier still costs a round
+            // trip, which here overlaps the softmax instead of sitting between P.V and S
             if (!(ok = wait_loaded(vi))) break;
+            if (more && !(ok = wait_loaded(ki))) break;
             if (j < U.n[0] && !(ok = pv_step(0, j, U, slot_of(vi), 0))) break;
             if (more) {
-              if (!(ok = wait_loaded(ki))) break;
               if (j + 1 < U.n[0]) {
                 issue_s(0, slot_of(ki), 0);
                 tc_commit(&s_full[0]);
