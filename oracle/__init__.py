@@ -23,10 +23,14 @@ Modules
                       recurrence, and a lazy-rescale blockwise variant in base 2.
 ``oracle.fp8``        Sylvester Hadamard matrix, fast Walsh-Hadamard transform in float32,
                       E4M3 (OCP E4M3FN) rounding/encoding, per-block quantisation.
+``oracle.attention_bwd``  the backward pass (dQ, dK, dV) from the chain rule on whole score
+                      matrices; the pages only state that it exists and recomputes the softmax
+                      ("FlashAttention-3", "适用范围和工程限制"; "Flash Attention V3 解析" 2.1).
 
 Every function is pinned by ``tests/test_oracle_*.py`` against closed forms, invariants,
-library routines (torch SDPA in float64, scipy's Hadamard, ml_dtypes/torch float8) and
-hand-derived fixtures in ``tests/golden/``.
+library routines (torch SDPA in float64, scipy's Hadamard, ml_dtypes/torch float8), central
+finite differences of the forward oracle (for the backward) and hand-derived fixtures in
+``tests/golden/``.
 """
 
 from .attention import (  # noqa: F401
@@ -34,6 +38,12 @@ from .attention import (  # noqa: F401
     attention_blockwise_ref,
     attention_blockwise_lazy_ref,
     visible_mask,
+)
+from .attention_bwd import (  # noqa: F401
+    attention_bwd_ref,
+    attention_bwd_terms,
+    softmax_bwd_delta,
+    softmax_probs,
 )
 from .fp8 import (  # noqa: F401
     E4M3_MAX,

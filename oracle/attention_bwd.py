@@ -1,0 +1,85 @@
+"""float64 oracle of the attention backward pass (TEST INFRASTRUCTURE ONLY; see ``oracle/__init__.py``).
+
+The pages state that the backward pass exists for FP16/BF16 ("FlashAttention-3", section
+"适用范围和工程限制"), that it recomputes the softmax instead of storing it ("Flash
+Attention V3 解析", section 2.1, "反向重计算"), and that dQ is accumulated across K/V blocks
+(section 4.2, "dQ更新时").  They do not write the gradient out; it is the chain rule applied
+to the forward definition, which is what this module evaluates, on whole score matrices:
+
+    S = scale * Q K^T          P = softmax(S) over the visible keys of each row
+    O = P V
+    dV = P^T dO                dP = dO V^T
+    dS = P * (dP - rowsum(P * dP))            (the softmax Jacobian applied row by row)
+    dQ = scale * dS K          dK = scale * dS^T Q
+
+``rowsum(P * dP)`` equals ``rowsum(dO * O)`` (both are sum_j P_ij sum_c dO_ic V_jc); the
+second form is the one a tiled kernel can compute before its loops, from O alone.
+
+All arrays are float64 ``[..., N, d]``; leading dimensions are independent problems.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .attention import visible_mask
+
+
+def _as_3d(x: np.ndarray):
+    lead = x.shape[:-2]
+    return x.reshape((-1,) + x.shape[-2:]), lead
+
+
+def softmax_probs(q, k, scale: float, causal: bool = False) -> np.ndarray:
+    """P = softmax(scale * Q K^T) over the visible keys, float64 ``[..., N_q, N_k]``."""
+    q3, lead = _as_3d(np.asarray(q, dtype=np.float64))
+    k3, _ = _as_3d(np.asarray(k, dtype=np.float64))
+    s = scale * np.einsum("bid,bjd->bij", q3, k3)
+    vis = visible_mask(q3.shape[1], k3.shape[1], causal)
+    s = np.where(vis[None], s, -np.inf)
+    m = s.max(axis=-1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    e = np.where(vis[None], np.exp(s - m), 0.0)
+    den = e.sum(axis=-1, keepdims=True)
+    p = np.divide(e, den, out=np.zeros_like(e), where=den > 0)
+    return p.reshape(lead + p.shape[-2:])
+
+
+def softmax_bwd_delta(o, do) -> np.ndarray:
+    """D_i = sum_c dO_ic O_ic, float64 ``[..., N]`` (equal to rowsum(P * dP))."""
+    return np.einsum("...ic,...ic->...i", np.asarray(do, dtype=np.float64), np.asarray(o, dtype=np.float64))
+
+
+def attention_bwd_ref(q, k, v, do, scale: float, causal: bool = False):
+    """(dQ, dK, dV) of ``O = softmax(scale Q K^T) V`` for the upstream gradient ``dO``, float64.
+
+    Straight from the definition above: P is formed in full, dS uses rowsum(P * dP).
+    """
+    q3, lead = _as_3d(np.asarray(q, dtype=np.float64))
+    k3, _ = _as_3d(np.asarray(k, dtype=np.float64))
+    v3, _ = _as_3d(np.asarray(v, dtype=np.float64))
+    do3, _ = _as_3d(np.asarray(do, dtype=np.float64))
+    p = softmax_probs(q3, k3, scale, causal)
+    dv = np.einsum("bij,bic->bjc", p, do3)
+    dp = np.einsum("bic,bjc->bij", do3, v3)
+    ds = p * (dp - (p * dp).sum(axis=-1, keepdims=True))
+    dq = scale * np.einsum("bij,bjc->bic", ds, k3)
+    dk = scale * np.einsum("bij,bic->bjc", ds, q3)
+    return dq.reshape(q.shape), dk.reshape(k.shape), dv.reshape(v.shape)
+
+
+def attention_bwd_terms(q, k, v, do, scale: float, causal: bool = False):
+    """Elementwise magnitudes that bound the rounding error of a kernel that rounds P and dS
+    to bf16 before the three products (used by the GPU tests to state their tolerance):
+    ``|P|^T |dO|`` for dV, ``scale |dS| |K|`` for dQ and ``scale |dS|^T |Q|`` for dK."""
+    q3, lead = _as_3d(np.asarray(q, dtype=np.float64))
+    k3, _ = _as_3d(np.asarray(k, dtype=np.float64))
+    v3, _ = _as_3d(np.asarray(v, dtype=np.float64))
+    do3, _ = _as_3d(np.asarray(do, dtype=np.float64))
+    p = softmax_probs(q3, k3, scale, causal)
+    dp = np.einsum("bic,bjc->bij", do3, v3)
+    ds = p * (dp - (p * dp).sum(axis=-1, keepdims=True))
+    tv = np.einsum("bij,bic->bjc", np.abs(p), np.abs(do3))
+    tq = scale * np.einsum("bij,bjc->bic", np.abs(ds), np.abs(k3))
+    tk = scale * np.einsum("bij,bic->bjc", np.abs(ds), np.abs(q3))
+    return tq.reshape(q.shape), tk.reshape(k.shape), tv.reshape(v.shape)
