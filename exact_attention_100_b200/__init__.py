@@ -7,6 +7,7 @@ fallback: if the library is missing or a call fails, an exception is raised.
     import torch, exact_attention_100_b200 as ea
     o, lse = ea.attn_fwd(q, k, v, causal=True)           # q, k, v: [B, H, N, d] bf16 on cuda
     q8, qs = ea.attn_hadamard_quant(q, signs)             # E4M3 codes + per-block scales
+    dq, dk, dv = ea.attn_bwd(q, k, v, o, lse, do, causal=True)  # backward (bf16 O from attn_fwd)
 """
 
 from __future__ import annotations
@@ -54,6 +55,10 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_fp8.restype = i
         L.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
         L.attn_fwd_noalloc.restype = i
+        L.attn_bwd_workspace_bytes.argtypes = [i, i, i]
+        L.attn_bwd_workspace_bytes.restype = ctypes.c_ulonglong
+        L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+        L.attn_bwd.restype = i
         L.attn_device_status.argtypes = [vp]
         L.attn_device_status.restype = i
         L.attn_status_string.argtypes = [i]
@@ -121,6 +126,38 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, o_dtype=None, 
     _check(lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, s, int(bool(causal)),
                           ATTN_BF16, od, _stream_ptr(stream)), "attn_fwd")
     return o, lse
+
+
+def attn_bwd_workspace_bytes(B: int, H: int, N: int) -> int:
+    return int(lib().attn_bwd_workspace_bytes(int(B), int(H), int(N)))
+
+
+def attn_bwd(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None, scale=None, causal=False,
+             g_dtype=None, stream=None):
+    """(dQ, dK, dV) of attn_fwd for the upstream gradient ``dout``.
+
+    q, k, v, o, dout: contiguous [B, H, N, d] bf16 cuda tensors (o from attn_fwd with bf16 O);
+    lse: the forward's [B, H, N] float32 LSE.  dq/dk/dv may be given (written in place) or are
+    allocated with ``g_dtype`` (torch.bfloat16 default, or torch.float32); ``workspace`` (a
+    float32 tensor of at least attn_bwd_workspace_bytes bytes) likewise.
+    """
+    import torch
+    B, H, N, d = _dims(q)
+    for t in (q, k, v, o, dout):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError("q, k, v, o, dout must be contiguous bf16 tensors of one shape")
+    gd = g_dtype or (dq.dtype if dq is not None else torch.bfloat16)
+    dq = dq if dq is not None else torch.empty(q.shape, dtype=gd, device=q.device)
+    dk = dk if dk is not None else torch.empty(q.shape, dtype=gd, device=q.device)
+    dv = dv if dv is not None else torch.empty(q.shape, dtype=gd, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device=q.device)
+    gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                          _ptr(workspace), B, H, N, d, s, int(bool(causal)), gcode, _stream_ptr(stream)),
+           "attn_bwd")
+    return dq, dk, dv
 
 
 def attn_fwd_noalloc(q, k, v, o, lse=None, scale=None, causal=False, stream=None):

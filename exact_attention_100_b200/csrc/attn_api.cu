@@ -64,6 +64,7 @@ int device_state(DeviceState** out) {
     if (ea::setup_fwd_bf16_kernels() != cudaSuccess) return ATTN_ERR_CUDA;
     if (ea::setup_fwd_fp8_kernels() != cudaSuccess) return ATTN_ERR_CUDA;
     if (ea::setup_hadamard_quant_kernels() != cudaSuccess) return ATTN_ERR_CUDA;
+    if (ea::setup_bwd_kernels() != cudaSuccess) return ATTN_ERR_CUDA;
     st.num_sms = sms;
     st.ready = true;
   }
@@ -237,6 +238,59 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_
   if (ea::launch_attn_fwd_fp8(d, mq, mk, mv, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
+  return ATTN_OK;
+}
+
+unsigned long long attn_bwd_workspace_bytes(int B, int H, int N) {
+  if (B <= 0 || H <= 0 || N <= 0) return 0ull;
+  const unsigned long long n_pad = (static_cast<unsigned long long>(N) + 127ull) / 128ull * 128ull;
+  return 2ull * static_cast<unsigned long long>(B) * static_cast<unsigned long long>(H) * n_pad * 4ull;
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+             void* dq, void* dk, void* dv, void* workspace, int B, int H, int N, int d, float scale, int causal,
+             int g_dtype, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+    return ATTN_ERR_INVALID_ARG;
+  int rc = check_common(B, H, N, scale, causal, g_dtype);
+  if (rc != ATTN_OK) return rc;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  const long long n_blocks = (static_cast<long long>(N) + 127) / 128;
+  if (static_cast<long long>(B) * H * n_blocks > 0x7FFFFFFFLL || n_blocks * 128 > 0x7FFFFFFFLL)
+    return ATTN_ERR_INVALID_ARG;
+
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!encode_rows_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H) ||
+      !encode_rows_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H) ||
+      !encode_rows_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H) ||
+      !encode_rows_map(&mdo, dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H))
+    return ATTN_ERR_CUDA;
+  ea::BwdParams p;
+  p.lse = lse;
+  p.o = o;
+  p.dout = dout;
+  p.BH = B * H;
+  p.N = N;
+  p.n_blocks = static_cast<int>(n_blocks);
+  p.n_pad = static_cast<int>(n_blocks * 128);
+  p.delta = static_cast<float*>(workspace);
+  p.lse2 = static_cast<float*>(workspace) + static_cast<size_t>(p.BH) * p.n_pad;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.status = st->status;
+  p.scale = scale;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.causal = causal;
+  p.g_fp32 = g_dtype == ATTN_FP32 ? 1 : 0;
+  if (ea::launch_attn_bwd(d, mq, mk, mv, mdo, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  g_launches.fetch_add(3);
   return ATTN_OK;
 }
 

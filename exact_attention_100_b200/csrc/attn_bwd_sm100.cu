@@ -1,0 +1,678 @@
+// Backward pass of the exact attention forward, sm_100a (B200): tcgen05 + TMEM + TMA.
+//
+// The pages state that the backward exists and recomputes the softmax from what the forward
+// kept ("FlashAttention-3", section "适用范围和工程限制"; "Flash Attention V3 解析", section
+// 2.1, "反向重计算").  With P = softmax(scale Q K^T) rebuilt from the forward's LSE:
+//     dV = P^T dO,   dP = dO V^T,   dS = P * (dP - D),   D_i = sum_c dO_ic O_ic,
+//     dQ = scale dS K,   dK = scale dS^T Q.
+//
+// Three launches:
+//   bwd_prep_kernel   D and LSE * log2 e per row into a padded workspace (bandwidth-bound).
+//   bwd_dkdv_kernel   one CTA per (batch*head, 128-key block): S^T = K Q^T and dP^T = V dO^T per
+//                     128-query block, P^T and dS^T back into TMEM, dV += P^T dO, dK += dS^T Q.
+//   bwd_dq_kernel     one CTA per (batch*head, 128-query block): S = Q K^T and dP = dO V^T per
+//                     128-key block, dS into TMEM, dQ += dS K.
+// dQ gets its own pass (recomputing S and dP) instead of atomic additions from the dK/dV
+// kernel ("Flash Attention V3 解析", section 4.2): no float atomics, deterministic results.
+//
+// Roles (both main kernels, 192 threads): warps 0-3 one thread per TMEM lane (a row of S or
+// S^T: the softmax backward and the epilogue), warp 4 lane 0 issues every tcgen05.mma, warp 5
+// lane 0 is the TMA producer.  Every mbarrier wait is bounded (wait_bar).
+
+#include <cuda_bf16.h>
+
+#include "attn_kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace ea {
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------------------------ preparation
+// One row per group of d/16 lanes: D = sum_c dO * O (f32), lse2 = LSE * log2 e; rows past N get
+// D = 0 and lse2 = +inf, so that their P (= 2^(s - lse2)) is exactly zero in the main kernels.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
+  constexpr int kLanes = D / 16;
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = t / kLanes;  // over BH * n_pad
+  const int part = static_cast<int>(t % kLanes);
+  const long long total = static_cast<long long>(p.BH) * p.n_pad;
+  const bool in_range = row < total;
+  const int bh = in_range ? static_cast<int>(row / p.n_pad) : 0;
+  const int r = in_range ? static_cast<int>(row % p.n_pad) : 0;
+  const bool valid = in_range && r < p.N;
+  float acc = 0.f;
+  if (valid) {
+    const size_t off = (static_cast<size_t>(bh) * p.N + r) * D + part * 16;
+    const uint4* po = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.o) + off);
+    const uint4* pd = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dout) + off);
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const uint4 a = __ldg(po + c), b = __ldg(pd + c);
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc = fmaf(__uint_as_float(wa[k] << 16), __uint_as_float(wb[k] << 16), acc);
+        acc = fmaf(__uint_as_float(wa[k] & 0xFFFF0000u), __uint_as_float(wb[k] & 0xFFFF0000u), acc);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = kLanes / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (in_range && part == 0) {
+    p.delta[row] = valid ? acc : 0.f;
+    p.lse2[row] = valid ? p.lse[static_cast<size_t>(bh) * p.N + r] * kLog2e : INFINITY;
+  }
+}
+
+// --------------------------------------------------------------------------- shared pieces
+template <int D>
+struct BwdCfg {
+  static constexpr int kBoxBytes = 128 * 128;            // a 128-row x 128-byte column box
+  static constexpr int kBoxes = D * 2 / 128;             // column boxes of a bf16 row
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;  // 128 rows x D bf16
+  static constexpr int kThreads = 192;
+  static constexpr int kMmaWarp = 4;
+  static constexpr int kLoadWarp = 5;
+  static constexpr uint32_t kIdS = make_idesc(128, 128, 1, false);  // S-type products, both K-major
+  static constexpr uint32_t kIdD = make_idesc(128, D, 1, true);     // accumulations, B MN-major
+};
+
+// Loads a 128-row tile at rows [row0, row0 + 128) of head bh: one 128-row x 128-byte TMA box
+// per column box (the maps the forward uses).
+template <int D>
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row0, int bh) {
+  using C = BwdCfg<D>;
+#pragma unroll
+  for (int b = 0; b < C::kBoxes; ++b) tma_load_3d(dst + b * C::kBoxBytes, map, bar, b * 64, row0, bh);
+}
+
+// X[tmem, 128 x 128] = A B^T with A and B 128 x D tiles in shared memory, both K-major.
+template <int D>
+__device__ __forceinline__ void mma_abt(uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
+  using C = BwdCfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+    mma_f16_ss(d_tmem, make_sdesc_sw128(a_base + off, 16, 1024), make_sdesc_sw128(b_base + off, 16, 1024),
+               C::kIdS, kk > 0 ? 1u : 0u);
+  }
+}
+
+// Acc[tmem, 128 x D] (+)= X B with X 128 x 128 bf16 in TMEM (packed pairs, 64 columns) and B a
+// 128 x D tile in shared memory read MN-major (its rows are the contraction index).
+template <int D>
+__device__ __forceinline__ void mma_xb(uint32_t d_tmem, uint32_t x_tmem, uint32_t b_base, bool acc) {
+  using C = BwdCfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_f16_ts(d_tmem, x_tmem + kk * 8, make_sdesc_sw128(b_base + kk * 16 * 128, C::kBoxBytes, 1024), C::kIdD,
+               (acc || kk > 0) ? 1u : 0u);
+}
+
+// Stores one row of a 128 x D f32 TMEM accumulator (this thread's lane), times `mul`, as bf16
+// or f32.
+template <int D>
+__device__ __forceinline__ void store_row(uint32_t t_acc, void* out, size_t row_off, float mul, bool fp32,
+                                          bool valid) {
+#pragma unroll 1
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t r[32];
+    tmem_ld_32cols(t_acc + 32 * cc, r);
+    tmem_ld_wait(r);
+    if (!valid) continue;
+    if (fp32) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + row_off + 32 * cc);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        dst[i] = make_float4(__uint_as_float(r[4 * i]) * mul, __uint_as_float(r[4 * i + 1]) * mul,
+                             __uint_as_float(r[4 * i + 2]) * mul, __uint_as_float(r[4 * i + 3]) * mul);
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + row_off + 32 * cc);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * mul, __uint_as_float(r[8 * i + 1]) * mul);
+        w.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * mul, __uint_as_float(r[8 * i + 3]) * mul);
+        w.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * mul, __uint_as_float(r[8 * i + 5]) * mul);
+        w.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * mul, __uint_as_float(r[8 * i + 7]) * mul);
+        dst[i] = w;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ int unit_of(int k) {
+  const int g = gridDim.x;
+  return k * g + ((k & 1) ? (g - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x));
+}
+
+__device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity, int* status) {
+  const uint32_t a = smem_addr(bar);
+  const unsigned long long t0 = global_timer_ns();
+  while (!bar_try_wait(a, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(status, kDevStatusTimeout);
+      return;
+    }
+  }
+}
+
+// --------------------------------------------------------------------------- dK / dV kernel
+// Unit u: bh = u % BH, key block kb = u / BH (causal: longest first, kb = 0 visits every query
+// block).  Query blocks i = (causal ? kb : 0) .. n_blocks - 1 stream through two stages of
+// shared memory (Q_i, dO_i, and the workspace rows of lse2 and D).
+// TMEM columns: S^T [0,128) (then P^T as bf16 pairs in [0,64)), dP^T [128,256) (then dS^T in
+// [128,192)), dV [256, 256+D), dK [256+D, 256+2D).
+template <int D>
+struct DkdvCfg : BwdCfg<D> {
+  static constexpr int kStages = 2;
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = BwdCfg<D>::kTileBytes;
+  static constexpr int kStageOff = 2 * BwdCfg<D>::kTileBytes;
+  static constexpr int kStageBytes = 2 * BwdCfg<D>::kTileBytes + 1024;  // Q, dO, lse2[128], D[128]
+  static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
+  // kv_full, kv_empty, st_full[2], st_empty[2], s_full, p_full, dkv_done, dkv_free, drain
+  static constexpr int kNumBars = 2 + 2 * kStages + 5;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kMiscOff + 16;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;
+  static_assert(kSmemAlloc <= 232448, "shared memory budget");
+  static_assert(256 + 2 * D <= 512, "TMEM budget");
+};
+
+template <int D>
+__global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                    const BwdParams p) {
+  using C = DkdvCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + 1;
+  uint64_t* st_full = bars + 2;
+  uint64_t* st_empty = st_full + C::kStages;
+  uint64_t* s_full = st_empty + C::kStages;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* dkv_done = p_full + 1;
+  uint64_t* dkv_free = dkv_done + 1;
+  uint64_t* drain_bar = dkv_free + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+  if (threadIdx.x == 0) {
+    bar_init(kv_full, 1);
+    bar_init(kv_empty, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      bar_init(&st_full[s], 1);
+      bar_init(&st_empty[s], 1);
+    }
+    bar_init(s_full, 1);
+    bar_init(p_full, 4);
+    bar_init(dkv_done, 1);
+    bar_init(dkv_free, 4);
+    bar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == C::kLoadWarp && lane == 0) {
+    prefetch_tensor_map(&tmQ);
+    prefetch_tensor_map(&tmK);
+    prefetch_tensor_map(&tmV);
+    prefetch_tensor_map(&tmdO);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const AbortState ab{abort_flag, p.status};
+  const int nb = p.n_blocks;
+  const int num_units = p.BH * nb;
+
+  if (warp < 4) {
+    // ===================================================== softmax backward: one key row each
+    const int row = warp * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    uint32_t qc = 0, uit = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int u = unit_of(k);
+      if (u >= num_units) break;
+      const int bh = u % p.BH, kb = u / p.BH;
+      const int key_g = kb * 128 + row;
+      const int i0 = p.causal ? kb : 0;
+      for (int i = i0; i < nb && ok; ++i, ++qc) {
+        const uint32_t st = qc % C::kStages;
+        // the stage's lse2 / D rows arrived with its TMA transaction count
+        ok = warp_all(wait_bar(&st_full[st], (qc / C::kStages) & 1u, ab));
+        if (!ok) break;
+        ok = warp_all(wait_bar(s_full, qc & 1u, ab));
+        if (!ok) break;
+        tc_fence_after();
+        const float* lse2 = reinterpret_cast<const float*>(smem + C::kStageOff + st * C::kStageBytes +
+                                                           2 * C::kTileBytes);
+        const float* dlt = lse2 + 128;
+        const bool diag = p.causal && i == kb;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t s[32], dp[32];
+          tmem_ld_32cols(lane_base + 32 * c, s);
+          tmem_ld_32cols(lane_base + 128 + 32 * c, dp);
+          tmem_ld_wait(s);
+          tmem_ld_wait(dp);
+          uint32_t pk[16], dk[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            float pv[2], dv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int qq = 32 * c + 2 * t + e;  // query within the block
+              float pe = ex2_approx(fmaf(__uint_as_float(s[2 * t + e]), p.scale_log2, -lse2[qq]));
+              if (diag && i * 128 + qq < key_g) pe = 0.f;  // query before the key: masked
+              pv[e] = pe;
+              dv[e] = pe * (__uint_as_float(dp[2 * t + e]) - dlt[qq]);
+            }
+            pk[t] = pack_bf16x2(pv[0], pv[1]);
+            dk[t] = pack_bf16x2(dv[0], dv[1]);
+          }
+          // P^T over S^T columns [16c, 16c+16), dS^T over dP^T columns [16c, 16c+16): both already
+          // read by this thread
+          tmem_st_16cols(lane_base + 16 * c, pk);
+          tmem_st_16cols(lane_base + 128 + 16 * c, dk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(p_full);
+      }
+      if (!ok) break;
+      // epilogue: dV and scale * dK of this key block
+      ok = warp_all(wait_bar(dkv_done, uit & 1u, ab));
+      if (!ok) break;
+      tc_fence_after();
+      const bool valid = key_g < p.N;
+      const size_t off = (static_cast<size_t>(bh) * p.N + key_g) * D;
+      store_row<D>(lane_base + 256, p.dv, off, 1.f, p.g_fp32 != 0, valid);
+      store_row<D>(lane_base + 256 + D, p.dk, off, p.scale, p.g_fp32 != 0, valid);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) bar_arrive(dkv_free);
+      ++uit;
+    }
+  } else if (warp == C::kMmaWarp) {
+    if (lane == 0) {
+      // ================================================================== MMA issuer
+      const uint32_t k_base = smem_addr(smem + C::kKOff);
+      const uint32_t v_base = smem_addr(smem + C::kVOff);
+      uint32_t qc = 0, uc = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int u = unit_of(k);
+        if (u >= num_units) break;
+        const int kb = u / p.BH;
+        const int i0 = p.causal ? kb : 0;
+        if (!(ok = wait_bar(kv_full, uc & 1u, ab))) break;
+        for (int i = i0; i < nb && ok; ++i, ++qc) {
+          const uint32_t st = qc % C::kStages;
+          if (!(ok = wait_bar(&st_full[st], (qc / C::kStages) & 1u, ab))) break;
+          const uint32_t q_base = smem_addr(smem + C::kStageOff + st * C::kStageBytes);
+          const uint32_t do_base = q_base + C::kTileBytes;
+          mma_abt<D>(tmem, k_base, q_base);          // S^T = K Q^T
+          mma_abt<D>(tmem + 128, v_base, do_base);   // dP^T = V dO^T
+          tc_commit(s_full);
+          if (!(ok = wait_bar(p_full, qc & 1u, ab))) break;
+          tc_fence_after();
+          if (i == i0) {
+            // the previous unit's epilogue must be done reading dV / dK
+            if (!(ok = wait_bar(dkv_free, (uc & 1u) ^ 1u, ab))) break;
+            tc_fence_after();
+          }
+          mma_xb<D>(tmem + 256, tmem, do_base, i > i0);           // dV += P^T dO
+          mma_xb<D>(tmem + 256 + D, tmem + 128, q_base, i > i0);  // dK += dS^T Q
+          tc_commit(&st_empty[st]);
+        }
+        if (!ok) break;
+        tc_commit(dkv_done);
+        tc_commit(kv_empty);
+        ++uc;
+      }
+      tc_commit(drain_bar);
+      drain(drain_bar, 0, p.status);
+    }
+  } else {
+    if (lane == 0) {
+      // =============================================================== TMA producer
+      uint32_t qc = 0, uc = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int u = unit_of(k);
+        if (u >= num_units) break;
+        const int bh = u % p.BH, kb = u / p.BH;
+        const int i0 = p.causal ? kb : 0;
+        if (uc > 0 && !(ok = wait_bar(kv_empty, (uc - 1u) & 1u, ab))) break;
+        bar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
+        load_tile<D>(smem + C::kKOff, &tmK, kv_full, kb * 128, bh);
+        load_tile<D>(smem + C::kVOff, &tmV, kv_full, kb * 128, bh);
+        ++uc;
+        for (int i = i0; i < nb && ok; ++i, ++qc) {
+          const uint32_t st = qc % C::kStages;
+          if (!(ok = wait_bar(&st_empty[st], ((qc / C::kStages) & 1u) ^ 1u, ab))) break;
+          uint8_t* base = smem + C::kStageOff + st * C::kStageBytes;
+          bar_arrive_expect_tx(&st_full[st], 2 * C::kTileBytes + 1024);
+          load_tile<D>(base, &tmQ, &st_full[st], i * 128, bh);
+          load_tile<D>(base + C::kTileBytes, &tmdO, &st_full[st], i * 128, bh);
+          const size_t w = static_cast<size_t>(bh) * p.n_pad + static_cast<size_t>(i) * 128;
+          bulk_load_g2s(base + 2 * C::kTileBytes, p.lse2 + w, 512, &st_full[st]);
+          bulk_load_g2s(base + 2 * C::kTileBytes + 512, p.delta + w, 512, &st_full[st]);
+        }
+      }
+      // every issued copy lands before the CTA can exit
+      if (uc > 0) drain(kv_full, (uc - 1u) & 1u, p.status);
+      const uint32_t first = qc > static_cast<uint32_t>(C::kStages) ? qc - C::kStages : 0u;
+      for (uint32_t i = first; i < qc; ++i) drain(&st_full[i % C::kStages], (i / C::kStages) & 1u, p.status);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------ dQ kernel
+// Unit u: bh = u % BH, query block qb (causal: longest first).  K_j, V_j stream through a ring
+// of slots.  TMEM columns: S [0,128), dP [128,256), dQ [256, 256+D), dS double buffer
+// [384, 448) and [448, 512) (bf16 pairs), so that S(j+1) and dP(j+1) run while dS(j) is formed.
+template <int D>
+struct DqCfg : BwdCfg<D> {
+  static constexpr int kQOff = 0;
+  static constexpr int kDoOff = BwdCfg<D>::kTileBytes;
+  static constexpr int kRingOff = 2 * BwdCfg<D>::kTileBytes;
+  static constexpr int kSlotsFit = (196608 - kRingOff) / BwdCfg<D>::kTileBytes;
+  static constexpr int kSlots = kSlotsFit > 8 ? 8 : kSlotsFit;
+  static constexpr int kBarOff = kRingOff + kSlots * BwdCfg<D>::kTileBytes;
+  // full[kSlots], empty[kSlots], qdo_full, qdo_empty, s_full, ds_full[2], dq_done, dq_free, drain
+  static constexpr int kNumBars = 2 * kSlots + 8;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kMiscOff + 16;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;
+  static_assert(kSlots >= 4, "K/V ring");
+  static_assert(kSmemAlloc <= 232448, "shared memory budget");
+  static_assert(256 + D <= 384, "TMEM budget");
+};
+
+template <int D>
+__global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                  const BwdParams p) {
+  using C = DqCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* full = bars;
+  uint64_t* empty = full + C::kSlots;
+  uint64_t* qdo_full = empty + C::kSlots;
+  uint64_t* qdo_empty = qdo_full + 1;
+  uint64_t* s_full = qdo_empty + 1;
+  uint64_t* ds_full = s_full + 1;  // [2]
+  uint64_t* dq_done = ds_full + 2;
+  uint64_t* dq_free = dq_done + 1;
+  uint64_t* drain_bar = dq_free + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kSlots; ++i) {
+      bar_init(&full[i], 1);
+      bar_init(&empty[i], 1);
+    }
+    bar_init(qdo_full, 1);
+    bar_init(qdo_empty, 1);
+    bar_init(s_full, 1);
+    bar_init(&ds_full[0], 4);
+    bar_init(&ds_full[1], 4);
+    bar_init(dq_done, 1);
+    bar_init(dq_free, 4);
+    bar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == C::kLoadWarp && lane == 0) {
+    prefetch_tensor_map(&tmQ);
+    prefetch_tensor_map(&tmK);
+    prefetch_tensor_map(&tmV);
+    prefetch_tensor_map(&tmdO);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const AbortState ab{abort_flag, p.status};
+  const int nb = p.n_blocks;
+  const int num_units = p.BH * nb;
+
+  if (warp < 4) {
+    // ===================================================== softmax backward: one query row each
+    const int row = warp * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    uint32_t sc = 0, uit = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int u = unit_of(k);
+      if (u >= num_units) break;
+      const int bh = u % p.BH;
+      const int qb = p.causal ? nb - 1 - u / p.BH : u / p.BH;
+      const int q_g = qb * 128 + row;
+      const int n = p.causal ? qb + 1 : nb;
+      const size_t w = static_cast<size_t>(bh) * p.n_pad + q_g;
+      const float lse2 = p.lse2[w];  // +inf on padded rows: P = 0 there
+      const float dlt = p.delta[w];
+      for (int j = 0; j < n && ok; ++j, ++sc) {
+        ok = warp_all(wait_bar(s_full, sc & 1u, ab));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t t_ds = lane_base + 384 + (sc & 1u) * 64;
+        const bool mask = (j * 128 + 128 > p.N) || (p.causal && j == qb);
+        const int lim = min(p.N, p.causal ? q_g + 1 : p.N) - j * 128;  // visible keys of this block
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t s[32], dp[32];
+          tmem_ld_32cols(lane_base + 32 * c, s);
+          tmem_ld_32cols(lane_base + 128 + 32 * c, dp);
+          tmem_ld_wait(s);
+          tmem_ld_wait(dp);
+          uint32_t dk[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            float dv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int kk = 32 * c + 2 * t + e;
+              float pe = ex2_approx(fmaf(__uint_as_float(s[2 * t + e]), p.scale_log2, -lse2));
+              if (mask && kk >= lim) pe = 0.f;
+              dv[e] = pe * (__uint_as_float(dp[2 * t + e]) - dlt);
+            }
+            dk[t] = pack_bf16x2(dv[0], dv[1]);
+          }
+          tmem_st_16cols(t_ds + 16 * c, dk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(&ds_full[sc & 1u]);
+      }
+      if (!ok) break;
+      ok = warp_all(wait_bar(dq_done, uit & 1u, ab));
+      if (!ok) break;
+      tc_fence_after();
+      store_row<D>(lane_base + 256, p.dq, (static_cast<size_t>(bh) * p.N + q_g) * D, p.scale, p.g_fp32 != 0,
+                   q_g < p.N);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) bar_arrive(dq_free);
+      ++uit;
+    }
+  } else if (warp == C::kMmaWarp) {
+    if (lane == 0) {
+      // ================================================================== MMA issuer
+      const uint32_t q_base = smem_addr(smem + C::kQOff);
+      const uint32_t do_base = smem_addr(smem + C::kDoOff);
+      const uint32_t ring_base = smem_addr(smem + C::kRingOff);
+      uint32_t it = 0, qit = 0, sc = 0, uc = 0;
+      bool ok = true;
+      auto slot_addr = [&](uint32_t idx) { return ring_base + (idx % C::kSlots) * C::kTileBytes; };
+      auto wait_loaded = [&](uint32_t idx) { return wait_bar(&full[idx % C::kSlots], (idx / C::kSlots) & 1u, ab); };
+      for (int k = 0; ok; ++k) {
+        const int u = unit_of(k);
+        if (u >= num_units) break;
+        const int qb = p.causal ? nb - 1 - u / p.BH : u / p.BH;
+        const int n = p.causal ? qb + 1 : nb;
+        const uint32_t base = it;  // K_j = base + 2j, V_j = base + 2j + 1
+        it += 2u * n;
+        if (!(ok = wait_bar(qdo_full, qit & 1u, ab))) break;
+        ++qit;
+        // S(0), dP(0)
+        if (!(ok = wait_loaded(base)) || !(ok = wait_loaded(base + 1))) break;
+        mma_abt<D>(tmem, q_base, slot_addr(base));
+        mma_abt<D>(tmem + 128, do_base, slot_addr(base + 1));
+        tc_commit(s_full);
+        tc_commit(&empty[(base + 1) % C::kSlots]);
+        for (int j = 0; j < n && ok; ++j, ++sc) {
+          const uint32_t ki = base + 2 * j;
+          if (j + 1 < n && (!(ok = wait_loaded(ki + 2)) || !(ok = wait_loaded(ki + 3)))) break;
+          if (!(ok = wait_bar(&ds_full[sc & 1u], (sc >> 1) & 1u, ab))) break;
+          tc_fence_after();
+          if (j + 1 < n) {
+            // the softmax has read S(j) and dP(j): the next pair can overwrite them
+            mma_abt<D>(tmem, q_base, slot_addr(ki + 2));
+            mma_abt<D>(tmem + 128, do_base, slot_addr(ki + 3));
+            tc_commit(s_full);
+            tc_commit(&empty[(ki + 3) % C::kSlots]);
+          }
+          if (j == 0) {
+            if (!(ok = wait_bar(dq_free, (uc & 1u) ^ 1u, ab))) break;
+            tc_fence_after();
+          }
+          mma_xb<D>(tmem + 256, tmem + 384 + (sc & 1u) * 64, slot_addr(ki), j > 0);  // dQ += dS K
+          tc_commit(&empty[ki % C::kSlots]);
+        }
+        if (!ok) break;
+        tc_commit(dq_done);
+        tc_commit(qdo_empty);
+        ++uc;
+      }
+      tc_commit(drain_bar);
+      drain(drain_bar, 0, p.status);
+    }
+  } else {
+    if (lane == 0) {
+      // =============================================================== TMA producer
+      uint32_t it = 0, qit = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int u = unit_of(k);
+        if (u >= num_units) break;
+        const int bh = u % p.BH;
+        const int qb = p.causal ? nb - 1 - u / p.BH : u / p.BH;
+        const int n = p.causal ? qb + 1 : nb;
+        if (qit > 0 && !(ok = wait_bar(qdo_empty, (qit - 1u) & 1u, ab))) break;
+        bar_arrive_expect_tx(qdo_full, 2 * C::kTileBytes);
+        load_tile<D>(smem + C::kQOff, &tmQ, qdo_full, qb * 128, bh);
+        load_tile<D>(smem + C::kDoOff, &tmdO, qdo_full, qb * 128, bh);
+        ++qit;
+        for (int j = 0; j < n && ok; ++j) {
+#pragma unroll
+          for (int kv = 0; kv < 2; ++kv) {
+            const uint32_t s = it % C::kSlots;
+            if (!(ok = wait_bar(&empty[s], ((it / C::kSlots) & 1u) ^ 1u, ab))) break;
+            bar_arrive_expect_tx(&full[s], C::kTileBytes);
+            load_tile<D>(smem + C::kRingOff + s * C::kTileBytes, kv ? &tmV : &tmK, &full[s], j * 128, bh);
+            ++it;
+          }
+        }
+      }
+      const uint32_t first = it > static_cast<uint32_t>(C::kSlots) ? it - C::kSlots : 0u;
+      for (uint32_t i = first; i < it; ++i) drain(&full[i % C::kSlots], (i / C::kSlots) & 1u, p.status);
+      if (qit > 0) drain(qdo_full, (qit - 1u) & 1u, p.status);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t setup_d() {
+  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       DkdvCfg<D>::kSmemAlloc);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DqCfg<D>::kSmemAlloc);
+  return e;
+}
+
+template <int D>
+cudaError_t launch_d(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& dout,
+                     const BwdParams& p, int num_sms, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(p.BH) * p.n_pad;
+  const long long threads = rows * (D / 16);
+  const long long blocks = (threads + 255) / 256;
+  if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  bwd_prep_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int units = p.BH * p.n_blocks;
+  const int grid = units < num_sms ? units : num_sms;
+  bwd_dkdv_kernel<D><<<grid, BwdCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(q, k, v, dout, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bwd_dq_kernel<D><<<grid, BwdCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(q, k, v, dout, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t setup_bwd_kernels() {
+  cudaError_t e = setup_d<64>();
+  if (e == cudaSuccess) e = setup_d<128>();
+  return e;
+}
+
+cudaError_t launch_attn_bwd(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                            const CUtensorMap& dout, const BwdParams& p, int num_sms, cudaStream_t stream) {
+  switch (d) {
+    case 64:
+      return launch_d<64>(q, k, v, dout, p, num_sms, stream);
+    case 128:
+      return launch_d<128>(q, k, v, dout, p, num_sms, stream);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace ea

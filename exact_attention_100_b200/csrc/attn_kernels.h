@@ -36,6 +36,32 @@ cudaError_t launch_attn_fwd_bf16(int d, const CUtensorMap& q, const CUtensorMap&
 cudaError_t launch_attn_fwd_fp8(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                                 const FwdParams& p, int num_sms, cudaStream_t stream);
 
+// Parameters of the backward kernels (bf16 inputs, d = 64 or 128).
+struct BwdParams {
+  const float* lse;       // forward LSE [BH, N] (natural log), read by the preparation kernel
+  const void* o;          // forward O [BH, N, d] bf16 (preparation kernel)
+  const void* dout;       // dO [BH, N, d] bf16 (preparation kernel)
+  float* delta;           // workspace [BH, n_pad]: rowsum(dO * O), 0 on padded rows
+  float* lse2;            // workspace [BH, n_pad]: LSE * log2 e, +inf on padded rows
+  void* dq;               // [BH, N, d] bf16 or f32
+  void* dk;
+  void* dv;
+  int* status;
+  int N;
+  int BH;
+  int n_blocks;           // ceil(N / 128)
+  int n_pad;              // n_blocks * 128
+  float scale;
+  float scale_log2;       // scale * log2 e
+  int causal;
+  int g_fp32;             // gradients stored as f32 (else bf16)
+};
+
+cudaError_t setup_bwd_kernels();
+// D and LSE*log2e into the workspace, then dK/dV and dQ; q/k/v/dout maps as for the forward.
+cudaError_t launch_attn_bwd(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                            const CUtensorMap& dout, const BwdParams& p, int num_sms, cudaStream_t stream);
+
 // Hadamard + per-block E4M3 quantisation of 1..3 tensors of one shape [BH, N, d] in one launch:
 // tm[t] is a 3-D tiled map over tensor t (bf16, box 64 x 128 x 1, 128-byte swizzle); x8[t] its
 // E4M3 output, scales[t] its [BH, ceil(N/128)] block scales, post[t] the factor on the stored

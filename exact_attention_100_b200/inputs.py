@@ -12,6 +12,8 @@ Recipe (the same for every workload):
 * Every tensor is rounded to bf16 (round to nearest even) last.
 * The random-sign diagonal of the Hadamard transform is ``2 * (default_rng(seed).random(d)
   < 0.5) - 1`` with seed 1, stored as int8 +-1.
+* The upstream gradient dO of the backward workloads is ``default_rng(seed).standard_normal``
+  float32 of shape ``[B, H, N, d]`` with seed 7 unless stated, rounded to bf16.
 """
 
 from __future__ import annotations
@@ -54,3 +56,9 @@ def hadamard_signs(d: int, seed: int = 1) -> np.ndarray:
     """int8 vector of +-1 of length d (the random-sign diagonal D)."""
     rng = np.random.default_rng(seed)
     return (2 * (rng.random(d) < 0.5).astype(np.int8) - 1).astype(np.int8)
+
+
+def normal_dout(B: int, H: int, N: int, d: int, seed: int = 7) -> np.ndarray:
+    """dO for the backward workloads: float32 array of bf16 values, [B, H, N, d], iid N(0, 1)."""
+    rng = np.random.default_rng(seed)
+    return round_to_bf16(rng.standard_normal((B, H, N, d), dtype=np.float32))

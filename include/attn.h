@@ -134,6 +134,38 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
                  int o_dtype, void* stream);
 
 /*
+ * attn_bwd_workspace_bytes -- size of the float32 workspace attn_bwd needs:
+ * 2 * B * H * ceil(N / 128) * 128 * 4 bytes (per row, padded to whole 128-row blocks: the
+ * rowsum D of dO * O and LSE * log2 e).  Returns 0 if a size is not positive.
+ */
+unsigned long long attn_bwd_workspace_bytes(int B, int H, int N);
+
+/*
+ * attn_bwd -- backward pass of attn_fwd, bf16.  "FlashAttention-3" (section on scope and
+ * limits) has the backward for FP16/BF16; "Flash Attention V3 解析" (section 2.1) recomputes
+ * the softmax in it instead of storing P.  With S = scale Q K^T and P = exp(S - LSE):
+ *     dV = P^T dO,  dP = dO V^T,  dS = P (dP - D) with D_i = sum_c dO_ic O_ic,
+ *     dQ = scale dS K,  dK = scale dS^T Q.
+ *
+ *   q, k, v     [B, H, N, d] bf16, device: the forward's inputs.
+ *   o           [B, H, N, d] bf16, device: the forward's output (attn_fwd with o_dtype bf16).
+ *   dout        [B, H, N, d] bf16, device: gradient of the loss with respect to O.
+ *   lse         [B, H, N] float32, device: the forward's LSE.
+ *   dq, dk, dv  [B, H, N, d] of g_dtype (ATTN_BF16 or ATTN_FP32), device, written.
+ *   workspace   device, 16-byte aligned, attn_bwd_workspace_bytes(B, H, N) bytes; owned by the
+ *               caller and overwritten.
+ *   d           64 or 128 (256: ATTN_ERR_UNSUPPORTED, dK and dV alone would fill TMEM).
+ *   scale, causal, stream   as for attn_fwd; the same values as the forward call.
+ * Arithmetic: S and dP recomputed by tensor cores (bf16 products, float32 accumulation); P and
+ * dS in float32, rounded to bf16 before the three accumulating products (float32 accumulation).
+ * No atomics: the result does not depend on scheduling.  Three kernel launches.  Returns
+ * ATTN_OK once they are enqueued.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, void* workspace,
+             int B, int H, int N, int d, float scale, int causal, int g_dtype, void* stream);
+
+/*
  * attn_fwd_noalloc -- attn_fwd for callers that cannot allocate device memory.  The pages have
  * no counterpart; it exists for this library's users.
  *

@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
     names = _declared_functions()
     assert names == sorted(["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status",
                             "attn_status_string", "attn_num_kernel_launches", "attn_shutdown",
-                            "attn_fwd_noalloc", "attn_hadamard_quant_qkv"])
+                            "attn_fwd_noalloc", "attn_hadamard_quant_qkv", "attn_bwd",
+                            "attn_bwd_workspace_bytes"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -111,7 +112,37 @@ def test_fwd_fp8_rejects_bad_arguments(L):
     assert f(*a) == ea.ATTN_ERR_INVALID_ARG
 
 
+def test_bwd_workspace_bytes(L):
+    assert L.attn_bwd_workspace_bytes(1, 1, 1) == 2 * 128 * 4
+    assert L.attn_bwd_workspace_bytes(2, 16, 8192) == 2 * 32 * 8192 * 4
+    assert L.attn_bwd_workspace_bytes(1, 3, 129) == 2 * 3 * 256 * 4
+    assert L.attn_bwd_workspace_bytes(0, 1, 1) == 0
+    assert L.attn_bwd_workspace_bytes(1, 1, -5) == 0
+
+
+def test_bwd_rejects_bad_arguments(L):
+    f = L.attn_bwd
+    ok = [P, P, P, P, P, P2, P2, P2, P2, P2, 1, 1, 128, 128, 0.1, 0, 0, NULL]
+    for i in range(10):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for i in range(10):
+        a = list(ok)
+        a[i] = MIS
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for idx, val in [(10, 0), (12, 0), (14, float("nan")), (14, -1.0), (15, 2), (16, 7)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+    for dd in (32, 256):
+        a = list(ok)
+        a[13] = dd
+        assert f(*a) == ea.ATTN_ERR_UNSUPPORTED, dd
+
+
 def test_python_binding_has_same_names():
     for name in ["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status", "attn_status_string",
-                 "attn_num_kernel_launches", "attn_shutdown", "attn_fwd_noalloc", "attn_hadamard_quant_qkv"]:
+                 "attn_num_kernel_launches", "attn_shutdown", "attn_fwd_noalloc", "attn_hadamard_quant_qkv",
+                 "attn_bwd", "attn_bwd_workspace_bytes"]:
         assert callable(getattr(ea, name)), name

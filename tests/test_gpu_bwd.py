@@ -1,0 +1,126 @@
+"""Parity of the backward pass (attn_bwd, through the C ABI) with the float64 oracle.
+
+Tolerance, derived from the arithmetic rather than fitted (u = 2^-9, the bf16 unit roundoff;
+all products elementwise in absolute value, everything from the oracle in float64):
+
+* P is recomputed in float32 from the forward's LSE (relative error < 1e-4: scores summed in
+  float32, ex2.approx) and rounded to bf16 (u):           dP_err  <= (u + 1e-4) |P|
+* D = rowsum(dO * O) is formed from the forward's bf16 O, whose own error is at most
+  u |O| + 2u (|P| |V|) (bf16 rounding of O and of P in the forward):
+                                                          D_err   <= sum_c |dO| (u |O| + 2u |P||V|)
+* dP is a float32 sum of d exact products:                dP_err  <= d 2^-23 (|dO| |V|^T)
+* dS = P (dP - D) is rounded to bf16:                     dS_err  <= (u + 1e-4) |dS| + |P| (D_err + dP_err)
+* the three products accumulate n terms in float32:       n 2^-23 times the same sums of magnitudes
+so  |dV - dV_ref| <= dP_err^T |dO| + n 2^-23 |P|^T |dO|, and likewise scale (dS_err |K| + ...) for
+dQ and scale (dS_err^T |Q| + ...) for dK.  The tests allow twice that bound, plus u |g| when the
+gradients are stored as bf16.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_100_b200 as ea
+from exact_attention_100_b200.inputs import normal_dout
+from oracle import attention_bwd_ref, softmax_probs
+
+from gpu_util import device_qkv
+
+pytestmark = pytest.mark.gpu
+
+U = 2.0 ** -9
+
+
+def _bounds(q, k, v, do, o_ref, scale, causal):
+    p = softmax_probs(q, k, scale, causal)
+    dp = np.einsum("bhic,bhjc->bhij", do, v)
+    ds = p * (dp - (p * dp).sum(-1, keepdims=True))
+    ap, ads = np.abs(p), np.abs(ds)
+    n, d = q.shape[-2], q.shape[-1]
+    pv = np.einsum("bhij,bhjc->bhic", ap, np.abs(v))
+    d_err = np.einsum("bhic,bhic->bhi", np.abs(do), U * np.abs(o_ref) + 2 * U * pv)
+    dp_err = d * 2.0 ** -23 * np.einsum("bhic,bhjc->bhij", np.abs(do), np.abs(v))
+    ds_err = (U + 1e-4) * ads + ap * (d_err[..., None] + dp_err)
+    acc = n * 2.0 ** -23
+    bv = np.einsum("bhij,bhic->bhjc", (U + 1e-4 + acc) * ap, np.abs(do))
+    bq = scale * (np.einsum("bhij,bhjc->bhic", ds_err + acc * ads, np.abs(k)))
+    bk = scale * (np.einsum("bhij,bhic->bhjc", ds_err + acc * ads, np.abs(q)))
+    return bq, bk, bv
+
+
+def _run(B, H, N, d, causal, g_dtype=torch.float32, seed=0):
+    (q, k, v), (tq, tk, tv) = device_qkv(B, H, N, d, seed=seed)
+    do = normal_dout(B, H, N, d, seed=seed + 7)
+    tdo = torch.from_numpy(do).to(torch.bfloat16).cuda()
+    scale = 1.0 / math.sqrt(d)
+    o, lse = ea.attn_fwd(tq, tk, tv, causal=causal)  # bf16 O, as the backward expects
+    dq, dk, dv = ea.attn_bwd(tq, tk, tv, o, lse, tdo, causal=causal, g_dtype=g_dtype)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+    return (q, k, v, do, scale), (dq, dk, dv)
+
+
+def _check(inputs, grads, causal, bf16_out=False):
+    q, k, v, do, scale = inputs
+    refs = attention_bwd_ref(q, k, v, do, scale, causal)
+    from oracle import attention_ref
+    o_ref, _ = attention_ref(q, k, v, scale, causal)
+    bounds = _bounds(q, k, v, do, o_ref, scale, causal)
+    for name, g, r, b in zip(("dq", "dk", "dv"), grads, refs, bounds):
+        g = g.float().cpu().numpy().astype(np.float64)
+        assert np.isfinite(g).all(), name
+        tol = 2.0 * b + 1e-6 * np.abs(r).max() + (U * np.abs(r) if bf16_out else 0.0)
+        err = np.abs(g - r)
+        worst = float((err / tol).max())
+        assert worst <= 1.0, (name, worst, float(err.max()), float(np.abs(r).max()))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,H,N,d", [
+    (1, 1, 128, 64), (1, 2, 256, 128), (2, 1, 384, 64), (1, 1, 1, 128), (1, 1, 7, 64),
+    (1, 2, 129, 128), (1, 1, 200, 64), (2, 2, 300, 128), (1, 1, 513, 128),
+])
+def test_bwd_matches_oracle(B, H, N, d, causal):
+    inputs, grads = _run(B, H, N, d, causal)
+    _check(inputs, grads, causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_bf16_gradients(causal):
+    inputs, grads = _run(1, 2, 256, 128, causal, g_dtype=torch.bfloat16, seed=3)
+    assert all(g.dtype == torch.bfloat16 for g in grads)
+    _check(inputs, grads, causal, bf16_out=True)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_larger_problem(causal):
+    inputs, grads = _run(1, 2, 1024, 128, causal, seed=5)
+    _check(inputs, grads, causal)
+
+
+def test_bwd_key_gradients_sum_to_zero():
+    """sum_j dK_j = 0 in exact arithmetic; on the GPU it is small against sum_j |dK_j|."""
+    inputs, (dq, dk, dv) = _run(1, 2, 512, 128, True, seed=9)
+    g = dk.double().cpu().numpy()
+    assert np.all(np.abs(g.sum(axis=2)) <= 0.05 * np.abs(g).sum(axis=2) + 1e-6)
+
+
+def test_bwd_is_deterministic():
+    """No atomics: two calls give identical bits."""
+    (q, k, v), (tq, tk, tv) = device_qkv(1, 2, 640, 128, seed=11)
+    tdo = torch.from_numpy(normal_dout(1, 2, 640, 128, seed=12)).to(torch.bfloat16).cuda()
+    o, lse = ea.attn_fwd(tq, tk, tv, causal=True)
+    a = ea.attn_bwd(tq, tk, tv, o, lse, tdo, causal=True)
+    b = ea.attn_bwd(tq, tk, tv, o, lse, tdo, causal=True)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_bwd_rejects_head_dim_256():
+    (q, k, v), (tq, tk, tv) = device_qkv(1, 1, 128, 256)
+    o, lse = ea.attn_fwd(tq, tk, tv)
+    with pytest.raises(ea.AttnError):
+        ea.attn_bwd(tq, tk, tv, o, lse, torch.zeros_like(tq))
