@@ -316,6 +316,7 @@ def run_ours(args):
     d2h = pin_o.numel() * pin_o.element_size() + pin_l.numel() * pin_l.element_size()
 
     fp8 = fp8_section(args, dev, rank) if not args.no_fp8 else None
+    bwd = bwd_section(args, dev, rank) if not args.no_bwd else None
     barrier()
     if rank == 0:
         peaks = load_peaks()
@@ -348,6 +349,8 @@ def run_ours(args):
         }
         if fp8 is not None:
             line["fp8"] = fp8
+        if bwd is not None:
+            line["bwd"] = bwd
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -420,6 +423,48 @@ def fp8_section(args, dev, rank):
     return out
 
 
+def bwd_section(args, dev, rank):
+    """Times attn_bwd on the headline workload (device-resident inputs, bf16 gradients)."""
+    import torch
+    import exact_attention_100_b200 as ea
+    from exact_attention_100_b200.inputs import normal_qkv, normal_dout
+    w = WORKLOAD
+    B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
+    qn, kn, vn = normal_qkv(B, H, N, d, seed=rank)
+    q, k, v = (torch.from_numpy(a).to(torch.bfloat16).to(dev) for a in (qn, kn, vn))
+    do = torch.from_numpy(normal_dout(B, H, N, d, seed=7 + rank)).to(torch.bfloat16).to(dev)
+    stream = torch.cuda.current_stream()
+    o, lse = ea.attn_fwd(q, k, v, causal=causal, stream=stream)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    ws = torch.empty(ea.attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal=causal, stream=stream)
+
+    for _ in range(3):
+        step()
+    steps = max(3, min(args.steps, 50))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    flops = 2.5 * attn_flops(B, H, N, d, causal)  # dV, dP, dS-recompute S, dK, dQ: five N x N x d products
+    peaks = load_peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": "bf16 attention bwd B=2 H=16 N=8192 d=128 causal (dQ, dK, dV from O, LSE, dO)",
+            "ms": ms, "achieved_tflops": tf, "peak_tflops": float(peaks["bf16_tflops"]),
+            "frac": tf / float(peaks["bf16_tflops"]), "bound": "tensor",
+            "flops_per_call": flops, "flops_note": "algorithmic 2.5 x forward (five products); the kernels "
+                                                 "recompute S and dP a second time for dQ",
+            "launches_per_call": 3, "peak_source": peaks["source"]}
+
+
 def run_sweep(args):
     """Head-dim / length sweep at 16K tokens per head-batch: one JSON line per point (rank 0)."""
     import torch
@@ -467,6 +512,11 @@ def run_profile_case(args):
     if args.profile_case == "fwd":
         for _ in range(args.reps):
             ea.attn_fwd(q, k, v, causal=bool(causal))
+    elif args.profile_case == "bwd":
+        o, lse = ea.attn_fwd(q, k, v, causal=bool(causal))
+        do = torch.randn_like(q)
+        for _ in range(args.reps):
+            ea.attn_bwd(q, k, v, o, lse, do, causal=bool(causal))
     else:
         outs = None
         for _ in range(args.reps):
@@ -489,8 +539,9 @@ def main():
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv"], default=None,
+    ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv", "bwd"], default=None,
                     help="run --reps untimed calls of one entry point (for an ncu capture) and exit")
     ap.add_argument("--shape", type=int, nargs=5, default=[2, 16, 8192, 128, 1], metavar=("B", "H", "N", "d", "CAUSAL"))
     ap.add_argument("--reps", type=int, default=3)

@@ -175,8 +175,9 @@ struct DkdvCfg : BwdCfg<D> {
   static constexpr int kStageOff = 2 * BwdCfg<D>::kTileBytes;
   static constexpr int kStageBytes = 2 * BwdCfg<D>::kTileBytes + 1024;  // Q, dO, lse2[128], D[128]
   static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
-  // kv_full, kv_empty, st_full[2], st_empty[2], s_full, p_full, dkv_done, dkv_free, drain
-  static constexpr int kNumBars = 2 + 2 * kStages + 5;
+  // kv_full, kv_empty, st_full[2], st_empty[2], st_s (S^T in TMEM), st_dp (dP^T in TMEM),
+  // pt_full (P^T written), dst_full (dS^T written), dkv_done, dkv_free, drain
+  static constexpr int kNumBars = 2 + 2 * kStages + 7;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;
@@ -199,9 +200,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   uint64_t* kv_empty = bars + 1;
   uint64_t* st_full = bars + 2;
   uint64_t* st_empty = st_full + C::kStages;
-  uint64_t* s_full = st_empty + C::kStages;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* dkv_done = p_full + 1;
+  uint64_t* st_s = st_empty + C::kStages;
+  uint64_t* st_dp = st_s + 1;
+  uint64_t* pt_full = st_dp + 1;
+  uint64_t* dst_full = pt_full + 1;
+  uint64_t* dkv_done = dst_full + 1;
   uint64_t* dkv_free = dkv_done + 1;
   uint64_t* drain_bar = dkv_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
@@ -214,8 +217,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       bar_init(&st_full[s], 1);
       bar_init(&st_empty[s], 1);
     }
-    bar_init(s_full, 1);
-    bar_init(p_full, 4);
+    bar_init(st_s, 1);
+    bar_init(st_dp, 1);
+    bar_init(pt_full, 4);
+    bar_init(dst_full, 4);
     bar_init(dkv_done, 1);
     bar_init(dkv_free, 4);
     bar_init(drain_bar, 1);
@@ -257,44 +262,58 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         // the stage's lse2 / D rows arrived with its TMA transaction count
         ok = warp_all(wait_bar(&st_full[st], (qc / C::kStages) & 1u, ab));
         if (!ok) break;
-        ok = warp_all(wait_bar(s_full, qc & 1u, ab));
-        if (!ok) break;
-        tc_fence_after();
         const float* lse2 = reinterpret_cast<const float*>(smem + C::kStageOff + st * C::kStageBytes +
                                                            2 * C::kTileBytes);
         const float* dlt = lse2 + 128;
         const bool diag = p.causal && i == kb;
-#pragma unroll 1
+        // pass 1, from S^T alone: P^T (kept in registers, and as bf16 over S^T columns [0, 64))
+        ok = warp_all(wait_bar(st_s, qc & 1u, ab));
+        if (!ok) break;
+        tc_fence_after();
+        float pr[128];
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t s[32], dp[32];
-          tmem_ld_32cols(lane_base + 32 * c, s);
+          uint32_t sv[32];
+          tmem_ld_32cols(lane_base + 32 * c, sv);
+          tmem_ld_wait(sv);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int qq = 32 * c + e;  // query within the block
+            float pe = ex2_approx(fmaf(__uint_as_float(sv[e]), p.scale_log2, -lse2[qq]));
+            if (diag && i * 128 + qq < key_g) pe = 0.f;  // query before the key: masked
+            pr[qq] = pe;
+          }
+#pragma unroll
+          for (int t = 0; t < 16; ++t) pk[t] = pack_bf16x2(pr[32 * c + 2 * t], pr[32 * c + 2 * t + 1]);
+          tmem_st_16cols(lane_base + 16 * c, pk);  // S^T columns [16c, 16c+16): already read
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(pt_full);
+        // pass 2, from dP^T: dS^T = P^T (dP^T - D) as bf16 over dP^T columns [0, 64)
+        ok = warp_all(wait_bar(st_dp, qc & 1u, ab));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t dp[32];
           tmem_ld_32cols(lane_base + 128 + 32 * c, dp);
-          tmem_ld_wait(s);
           tmem_ld_wait(dp);
-          uint32_t pk[16], dk[16];
+          uint32_t dk[16];
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
-            float pv[2], dv[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int qq = 32 * c + 2 * t + e;  // query within the block
-              float pe = ex2_approx(fmaf(__uint_as_float(s[2 * t + e]), p.scale_log2, -lse2[qq]));
-              if (diag && i * 128 + qq < key_g) pe = 0.f;  // query before the key: masked
-              pv[e] = pe;
-              dv[e] = pe * (__uint_as_float(dp[2 * t + e]) - dlt[qq]);
-            }
-            pk[t] = pack_bf16x2(pv[0], pv[1]);
-            dk[t] = pack_bf16x2(dv[0], dv[1]);
+            const int q0 = 32 * c + 2 * t;
+            dk[t] = pack_bf16x2(pr[q0] * (__uint_as_float(dp[2 * t]) - dlt[q0]),
+                                pr[q0 + 1] * (__uint_as_float(dp[2 * t + 1]) - dlt[q0 + 1]));
           }
-          // P^T over S^T columns [16c, 16c+16), dS^T over dP^T columns [16c, 16c+16): both already
-          // read by this thread
-          tmem_st_16cols(lane_base + 16 * c, pk);
           tmem_st_16cols(lane_base + 128 + 16 * c, dk);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) bar_arrive(p_full);
+        if (lane == 0) bar_arrive(dst_full);
       }
       if (!ok) break;
       // epilogue: dV and scale * dK of this key block
@@ -323,24 +342,39 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         const int kb = u / p.BH;
         const int i0 = p.causal ? kb : 0;
         if (!(ok = wait_bar(kv_full, uc & 1u, ab))) break;
+        auto q_at = [&](uint32_t c) { return smem_addr(smem + C::kStageOff + (c % C::kStages) * C::kStageBytes); };
+        // S^T and dP^T of the unit's first query block
+        if (!(ok = wait_bar(&st_full[qc % C::kStages], (qc / C::kStages) & 1u, ab))) break;
+        mma_abt<D>(tmem, k_base, q_at(qc));                              // S^T = K Q^T
+        tc_commit(st_s);
+        mma_abt<D>(tmem + 128, v_base, q_at(qc) + C::kTileBytes);       // dP^T = V dO^T
+        tc_commit(st_dp);
         for (int i = i0; i < nb && ok; ++i, ++qc) {
-          const uint32_t st = qc % C::kStages;
-          if (!(ok = wait_bar(&st_full[st], (qc / C::kStages) & 1u, ab))) break;
-          const uint32_t q_base = smem_addr(smem + C::kStageOff + st * C::kStageBytes);
+          const uint32_t q_base = q_at(qc);
           const uint32_t do_base = q_base + C::kTileBytes;
-          mma_abt<D>(tmem, k_base, q_base);          // S^T = K Q^T
-          mma_abt<D>(tmem + 128, v_base, do_base);   // dP^T = V dO^T
-          tc_commit(s_full);
-          if (!(ok = wait_bar(p_full, qc & 1u, ab))) break;
+          const bool next = i + 1 < nb;
+          if (!(ok = wait_bar(pt_full, qc & 1u, ab))) break;
           tc_fence_after();
           if (i == i0) {
             // the previous unit's epilogue must be done reading dV / dK
             if (!(ok = wait_bar(dkv_free, (uc & 1u) ^ 1u, ab))) break;
             tc_fence_after();
           }
-          mma_xb<D>(tmem + 256, tmem, do_base, i > i0);           // dV += P^T dO
+          mma_xb<D>(tmem + 256, tmem, do_base, i > i0);  // dV += P^T dO
+          if (next) {
+            // S^T of the next block replaces P^T, which dV (issued first) has read
+            if (!(ok = wait_bar(&st_full[(qc + 1) % C::kStages], ((qc + 1) / C::kStages) & 1u, ab))) break;
+            mma_abt<D>(tmem, k_base, q_at(qc + 1));
+            tc_commit(st_s);
+          }
+          if (!(ok = wait_bar(dst_full, qc & 1u, ab))) break;
+          tc_fence_after();
           mma_xb<D>(tmem + 256 + D, tmem + 128, q_base, i > i0);  // dK += dS^T Q
-          tc_commit(&st_empty[st]);
+          tc_commit(&st_empty[qc % C::kStages]);
+          if (next) {
+            mma_abt<D>(tmem + 128, v_base, q_at(qc + 1) + C::kTileBytes);
+            tc_commit(st_dp);
+          }
         }
         if (!ok) break;
         tc_commit(dkv_done);
@@ -405,8 +439,9 @@ struct DqCfg : BwdCfg<D> {
   static constexpr int kSlotsFit = (196608 - kRingOff) / BwdCfg<D>::kTileBytes;
   static constexpr int kSlots = kSlotsFit > 8 ? 8 : kSlotsFit;
   static constexpr int kBarOff = kRingOff + kSlots * BwdCfg<D>::kTileBytes;
-  // full[kSlots], empty[kSlots], qdo_full, qdo_empty, s_full, ds_full[2], dq_done, dq_free, drain
-  static constexpr int kNumBars = 2 * kSlots + 8;
+  // full[kSlots], empty[kSlots], qdo_full, qdo_empty, s_full, dp_full, s_free, ds_full[2], dq_done,
+  // dq_free, drain
+  static constexpr int kNumBars = 2 * kSlots + 10;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;
@@ -430,8 +465,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   uint64_t* empty = full + C::kSlots;
   uint64_t* qdo_full = empty + C::kSlots;
   uint64_t* qdo_empty = qdo_full + 1;
-  uint64_t* s_full = qdo_empty + 1;
-  uint64_t* ds_full = s_full + 1;  // [2]
+  uint64_t* s_full = qdo_empty + 1;  // S in TMEM
+  uint64_t* dp_full = s_full + 1;    // dP in TMEM
+  uint64_t* s_free = dp_full + 1;    // the softmax has read S (pass 1 done)
+  uint64_t* ds_full = s_free + 1;    // [2] dS written
   uint64_t* dq_done = ds_full + 2;
   uint64_t* dq_free = dq_done + 1;
   uint64_t* drain_bar = dq_free + 1;
@@ -446,6 +483,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     bar_init(qdo_full, 1);
     bar_init(qdo_empty, 1);
     bar_init(s_full, 1);
+    bar_init(dp_full, 1);
+    bar_init(s_free, 4);
     bar_init(&ds_full[0], 4);
     bar_init(&ds_full[1], 4);
     bar_init(dq_done, 1);
@@ -489,31 +528,43 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       const float lse2 = p.lse2[w];  // +inf on padded rows: P = 0 there
       const float dlt = p.delta[w];
       for (int j = 0; j < n && ok; ++j, ++sc) {
-        ok = warp_all(wait_bar(s_full, sc & 1u, ab));
-        if (!ok) break;
-        tc_fence_after();
         const uint32_t t_ds = lane_base + 384 + (sc & 1u) * 64;
         const bool mask = (j * 128 + 128 > p.N) || (p.causal && j == qb);
         const int lim = min(p.N, p.causal ? q_g + 1 : p.N) - j * 128;  // visible keys of this block
-#pragma unroll 1
+        // pass 1, from S alone: P in registers; then S's columns may take the next block
+        ok = warp_all(wait_bar(s_full, sc & 1u, ab));
+        if (!ok) break;
+        tc_fence_after();
+        float pr[128];
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t s[32], dp[32];
-          tmem_ld_32cols(lane_base + 32 * c, s);
+          uint32_t sv[32];
+          tmem_ld_32cols(lane_base + 32 * c, sv);
+          tmem_ld_wait(sv);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float pe = ex2_approx(fmaf(__uint_as_float(sv[e]), p.scale_log2, -lse2));
+            if (mask && 32 * c + e >= lim) pe = 0.f;
+            pr[32 * c + e] = pe;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(s_free);
+        // pass 2, from dP: dS = P (dP - D) as bf16 into the dS buffer of this block
+        ok = warp_all(wait_bar(dp_full, sc & 1u, ab));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t dp[32];
           tmem_ld_32cols(lane_base + 128 + 32 * c, dp);
-          tmem_ld_wait(s);
           tmem_ld_wait(dp);
           uint32_t dk[16];
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
-            float dv[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int kk = 32 * c + 2 * t + e;
-              float pe = ex2_approx(fmaf(__uint_as_float(s[2 * t + e]), p.scale_log2, -lse2));
-              if (mask && kk >= lim) pe = 0.f;
-              dv[e] = pe * (__uint_as_float(dp[2 * t + e]) - dlt);
-            }
-            dk[t] = pack_bf16x2(dv[0], dv[1]);
+            const int k0 = 32 * c + 2 * t;
+            dk[t] = pack_bf16x2(pr[k0] * (__uint_as_float(dp[2 * t]) - dlt), pr[k0 + 1] * (__uint_as_float(dp[2 * t + 1]) - dlt));
           }
           tmem_st_16cols(t_ds + 16 * c, dk);
         }
@@ -555,19 +606,28 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         // S(0), dP(0)
         if (!(ok = wait_loaded(base)) || !(ok = wait_loaded(base + 1))) break;
         mma_abt<D>(tmem, q_base, slot_addr(base));
-        mma_abt<D>(tmem + 128, do_base, slot_addr(base + 1));
         tc_commit(s_full);
+        mma_abt<D>(tmem + 128, do_base, slot_addr(base + 1));
+        tc_commit(dp_full);
         tc_commit(&empty[(base + 1) % C::kSlots]);
         for (int j = 0; j < n && ok; ++j, ++sc) {
           const uint32_t ki = base + 2 * j;
-          if (j + 1 < n && (!(ok = wait_loaded(ki + 2)) || !(ok = wait_loaded(ki + 3)))) break;
+          const bool next = j + 1 < n;
+          if (next) {
+            // S(j+1) as soon as the softmax has read S(j) (its pass 1)
+            if (!(ok = wait_loaded(ki + 2))) break;
+            if (!(ok = wait_bar(s_free, sc & 1u, ab))) break;
+            tc_fence_after();
+            mma_abt<D>(tmem, q_base, slot_addr(ki + 2));
+            tc_commit(s_full);
+          }
+          // dP(j+1) once dS(j) is written (pass 2 has read dP(j))
           if (!(ok = wait_bar(&ds_full[sc & 1u], (sc >> 1) & 1u, ab))) break;
           tc_fence_after();
-          if (j + 1 < n) {
-            // the softmax has read S(j) and dP(j): the next pair can overwrite them
-            mma_abt<D>(tmem, q_base, slot_addr(ki + 2));
+          if (next) {
+            if (!(ok = wait_loaded(ki + 3))) break;
             mma_abt<D>(tmem + 128, do_base, slot_addr(ki + 3));
-            tc_commit(s_full);
+            tc_commit(dp_full);
             tc_commit(&empty[(ki + 3) % C::kSlots]);
           }
           if (j == 0) {
