@@ -61,13 +61,16 @@ def load_peaks():
         return dict(FALLBACK_PEAKS)
 
 
-def kernel_source_hash():
+FWD_SOURCES = ("attn_fwd_kernel.cuh", "attn_fwd_sm100.cu", "attn_kernels.h", "sm100_ptx.cuh")
+
+
+def kernel_source_hash(names=FWD_SOURCES):
+    """Hash of the sources a kernel is built from (the bf16 forward by default)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_attention_100_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in sorted(names):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 

@@ -181,37 +181,6 @@ __device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
       : "f"(b0), "f"(b1));
 }
 
-// 2^x for a pair, on the FMA pipe: n = round(x) by the 1.5*2^23 shift, f = x - n in [-1/2, 1/2],
-// 2^f by the cubic of fit_exp2_poly.py (relative error < 7.5e-5), 2^n added to the exponent.
-// x is clamped to >= -125 so the result stays a normal float (2^-125 stands in for 0).
-__device__ __forceinline__ void exp2_fma_pair(float& y0, float& y1, float x0, float x1) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
-  float t0, t1, p0, p1;
-  asm("{\n\t.reg .b64 rx, rs, rt, rn, rf, rp, c3, c2, c1, c0;\n\t"
-      "mov.b64 rx, {%4, %5};\n\t"
-      "mov.b64 rs, {%6, %6};\n\t"
-      "add.rn.f32x2 rt, rx, rs;\n\t"      // t = x + shift: round(x) in the low mantissa bits
-      "sub.rn.f32x2 rn, rt, rs;\n\t"      // n = round(x) as a float
-      "sub.rn.f32x2 rf, rx, rn;\n\t"      // f = x - n
-      "mov.b64 c3, {%7, %7};\n\t"
-      "mov.b64 c2, {%8, %8};\n\t"
-      "mov.b64 c1, {%9, %9};\n\t"
-      "mov.b64 c0, {%10, %10};\n\t"
-      "fma.rn.f32x2 rp, c3, rf, c2;\n\t"
-      "fma.rn.f32x2 rp, rp, rf, c1;\n\t"
-      "fma.rn.f32x2 rp, rp, rf, c0;\n\t"
-      "mov.b64 {%0, %1}, rt;\n\t"
-      "mov.b64 {%2, %3}, rp;\n\t}"
-      : "=f"(t0), "=f"(t1), "=f"(p0), "=f"(p1)
-      : "f"(x0), "f"(x1), "f"(kShift), "f"(0.0551716648042202f), "f"(0.2426111251115799f),
-        "f"(0.6932609677314758f), "f"(0.9999280571937561f));
-  // the integer n sits in the low bits of t; shifting by 23 drops the shift's own bits
-  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
   const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
   const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);

@@ -4,7 +4,8 @@ Tolerance, derived from the arithmetic rather than fitted (u = 2^-9, the bf16 un
 all products elementwise in absolute value, everything from the oracle in float64):
 
 * P is recomputed in float32 from the forward's LSE (relative error < 1e-4: scores summed in
-  float32, ex2.approx) and rounded to bf16 (u):           dP_err  <= (u + 1e-4) |P|
+  float32, ex2.approx or a cubic with relative error < 7.5e-5) and rounded to bf16 (u):
+                                                          dP_err  <= (u + 1e-4) |P|
 * D = rowsum(dO * O) is formed from the forward's bf16 O, whose own error is at most
   u |O| + 2u (|P| |V|) (bf16 rounding of O and of P in the forward):
                                                           D_err   <= sum_c |dO| (u |O| + 2u |P||V|)
