@@ -458,24 +458,27 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
 }
 
 // ------------------------------------------------------------------------------ dQ kernel
-// Unit u: bh = u % BH, query block qb (causal: longest first).  K_j, V_j stream through a ring
-// of slots.  TMEM columns: S [0,128), dP [128,256), dQ [256, 256+D), dS double buffer
-// [384, 448) and [448, 512) (bf16 pairs), so that S(j+1) and dP(j+1) run while dS(j) is formed.
+// Unit u: bh = u % BH, query block qb (causal: longest first).  K_j and V_j stream through two
+// rings (K: 3 slots, since dQ(j) is issued a block late and holds K_j; V: 2).  TMEM columns:
+// S [0,128), dP [128,256), dQ [256, 256+D), dS double buffer [384, 448) and [448, 512) (bf16
+// pairs).  The single MMA thread is the tensor pipe's timeline (an issue returns about when the
+// pipe has taken it), so it issues in order of urgency: S(j+1) as soon as the softmax has read
+// S(j), then dQ(j-1), then dP(j+1) once dS(j) is written.
 template <int D>
 struct DqCfg : BwdCfg<D> {
   static constexpr int kQOff = 0;
   static constexpr int kDoOff = BwdCfg<D>::kTileBytes;
-  static constexpr int kRingOff = 2 * BwdCfg<D>::kTileBytes;
-  static constexpr int kSlotsFit = (196608 - kRingOff) / BwdCfg<D>::kTileBytes;
-  static constexpr int kSlots = kSlotsFit > 8 ? 8 : kSlotsFit;
-  static constexpr int kBarOff = kRingOff + kSlots * BwdCfg<D>::kTileBytes;
-  // full[kSlots], empty[kSlots], qdo_full, qdo_empty, s_full, dp_full, s_free, ds_full[2], dq_done,
-  // dq_free, drain
-  static constexpr int kNumBars = 2 * kSlots + 10;
+  static constexpr int kKSlots = 3;
+  static constexpr int kVSlots = 2;
+  static constexpr int kKOff = 2 * BwdCfg<D>::kTileBytes;
+  static constexpr int kVOff = kKOff + kKSlots * BwdCfg<D>::kTileBytes;
+  static constexpr int kBarOff = kVOff + kVSlots * BwdCfg<D>::kTileBytes;
+  // kfull[3], kempty[3], vfull[2], vempty[2], qdo_full, qdo_empty, s_full, dp_full, s_free,
+  // ds_full[2], dq_done, dq_free, drain
+  static constexpr int kNumBars = 2 * (kKSlots + kVSlots) + 10;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;
-  static_assert(kSlots >= 4, "K/V ring");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
   static_assert(256 + D <= 384, "TMEM budget");
 };
@@ -491,9 +494,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-  uint64_t* full = bars;
-  uint64_t* empty = full + C::kSlots;
-  uint64_t* qdo_full = empty + C::kSlots;
+  uint64_t* kfull = bars;
+  uint64_t* kempty = kfull + C::kKSlots;
+  uint64_t* vfull = kempty + C::kKSlots;
+  uint64_t* vempty = vfull + C::kVSlots;
+  uint64_t* qdo_full = vempty + C::kVSlots;
   uint64_t* qdo_empty = qdo_full + 1;
   uint64_t* s_full = qdo_empty + 1;  // S in TMEM
   uint64_t* dp_full = s_full + 1;    // dP in TMEM
@@ -506,9 +511,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kSlots; ++i) {
-      bar_init(&full[i], 1);
-      bar_init(&empty[i], 1);
+    for (int i = 0; i < C::kKSlots; ++i) {
+      bar_init(&kfull[i], 1);
+      bar_init(&kempty[i], 1);
+    }
+    for (int i = 0; i < C::kVSlots; ++i) {
+      bar_init(&vfull[i], 1);
+      bar_init(&vempty[i], 1);
     }
     bar_init(qdo_full, 1);
     bar_init(qdo_empty, 1);
@@ -628,54 +637,67 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       // ================================================================== MMA issuer
       const uint32_t q_base = smem_addr(smem + C::kQOff);
       const uint32_t do_base = smem_addr(smem + C::kDoOff);
-      const uint32_t ring_base = smem_addr(smem + C::kRingOff);
-      uint32_t it = 0, qit = 0, sc = 0, uc = 0;
+      const uint32_t k_ring = smem_addr(smem + C::kKOff);
+      const uint32_t v_ring = smem_addr(smem + C::kVOff);
+      uint32_t kit = 0, vit = 0, qit = 0, sc = 0, uc = 0;
       bool ok = true;
-      auto slot_addr = [&](uint32_t idx) { return ring_base + (idx % C::kSlots) * C::kTileBytes; };
-      auto wait_loaded = [&](uint32_t idx) { return wait_bar(&full[idx % C::kSlots], (idx / C::kSlots) & 1u, ab); };
+      auto k_addr = [&](uint32_t idx) { return k_ring + (idx % C::kKSlots) * C::kTileBytes; };
+      auto v_addr = [&](uint32_t idx) { return v_ring + (idx % C::kVSlots) * C::kTileBytes; };
+      auto k_wait = [&](uint32_t idx) { return wait_bar(&kfull[idx % C::kKSlots], (idx / C::kKSlots) & 1u, ab); };
+      auto v_wait = [&](uint32_t idx) { return wait_bar(&vfull[idx % C::kVSlots], (idx / C::kVSlots) & 1u, ab); };
       for (int k = 0; ok; ++k) {
         const int u = unit_of(k);
         if (u >= num_units) break;
         const int qb = p.causal ? nb - 1 - u / p.BH : u / p.BH;
         const int n = p.causal ? qb + 1 : nb;
-        const uint32_t base = it;  // K_j = base + 2j, V_j = base + 2j + 1
-        it += 2u * n;
+        const uint32_t kb0 = kit, vb0 = vit;  // K_j = kb0 + j, V_j = vb0 + j
+        kit += n;
+        vit += n;
         if (!(ok = wait_bar(qdo_full, qit & 1u, ab))) break;
         ++qit;
+        bool dq_started = false;
+        // dQ(j) += dS(j) K_j, from the dS buffer of global block number `blk`
+        auto issue_dq = [&](int j, uint32_t blk) {
+          if (!dq_started) {
+            // the previous unit's epilogue must be done reading dQ
+            if (!wait_bar(dq_free, (uc & 1u) ^ 1u, ab)) return false;
+            tc_fence_after();
+            dq_started = true;
+          }
+          mma_xb<D>(tmem + 256, tmem + 384 + (blk & 1u) * 64, k_addr(kb0 + j), j > 0);
+          tc_commit(&kempty[(kb0 + j) % C::kKSlots]);
+          return true;
+        };
         // S(0), dP(0)
-        if (!(ok = wait_loaded(base)) || !(ok = wait_loaded(base + 1))) break;
-        mma_abt<D>(tmem, q_base, slot_addr(base));
+        if (!(ok = k_wait(kb0)) || !(ok = v_wait(vb0))) break;
+        mma_abt<D>(tmem, q_base, k_addr(kb0));
         tc_commit(s_full);
-        mma_abt<D>(tmem + 128, do_base, slot_addr(base + 1));
+        mma_abt<D>(tmem + 128, do_base, v_addr(vb0));
         tc_commit(dp_full);
-        tc_commit(&empty[(base + 1) % C::kSlots]);
+        tc_commit(&vempty[vb0 % C::kVSlots]);
         for (int j = 0; j < n && ok; ++j, ++sc) {
-          const uint32_t ki = base + 2 * j;
           const bool next = j + 1 < n;
           if (next) {
             // S(j+1) as soon as the softmax has read S(j) (its pass 1)
-            if (!(ok = wait_loaded(ki + 2))) break;
+            if (!(ok = k_wait(kb0 + j + 1))) break;
             if (!(ok = wait_bar(s_free, sc & 1u, ab))) break;
             tc_fence_after();
-            mma_abt<D>(tmem, q_base, slot_addr(ki + 2));
+            mma_abt<D>(tmem, q_base, k_addr(kb0 + j + 1));
             tc_commit(s_full);
           }
+          if (j > 0 && !(ok = issue_dq(j - 1, sc - 1))) break;
           // dP(j+1) once dS(j) is written (pass 2 has read dP(j))
           if (!(ok = wait_bar(&ds_full[sc & 1u], (sc >> 1) & 1u, ab))) break;
           tc_fence_after();
           if (next) {
-            if (!(ok = wait_loaded(ki + 3))) break;
-            mma_abt<D>(tmem + 128, do_base, slot_addr(ki + 3));
+            if (!(ok = v_wait(vb0 + j + 1))) break;
+            mma_abt<D>(tmem + 128, do_base, v_addr(vb0 + j + 1));
             tc_commit(dp_full);
-            tc_commit(&empty[(ki + 3) % C::kSlots]);
+            tc_commit(&vempty[(vb0 + j + 1) % C::kVSlots]);
           }
-          if (j == 0) {
-            if (!(ok = wait_bar(dq_free, (uc & 1u) ^ 1u, ab))) break;
-            tc_fence_after();
-          }
-          mma_xb<D>(tmem + 256, tmem + 384 + (sc & 1u) * 64, slot_addr(ki), j > 0);  // dQ += dS K
-          tc_commit(&empty[ki % C::kSlots]);
         }
+        if (!ok) break;
+        if (!(ok = issue_dq(n - 1, sc - 1))) break;
         if (!ok) break;
         tc_commit(dq_done);
         tc_commit(qdo_empty);
@@ -687,7 +709,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   } else {
     if (lane == 0) {
       // =============================================================== TMA producer
-      uint32_t it = 0, qit = 0;
+      uint32_t kit = 0, vit = 0, qit = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int u = unit_of(k);
@@ -701,18 +723,23 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         load_tile<D>(smem + C::kDoOff, &tmdO, qdo_full, qb * 128, bh);
         ++qit;
         for (int j = 0; j < n && ok; ++j) {
-#pragma unroll
-          for (int kv = 0; kv < 2; ++kv) {
-            const uint32_t s = it % C::kSlots;
-            if (!(ok = wait_bar(&empty[s], ((it / C::kSlots) & 1u) ^ 1u, ab))) break;
-            bar_arrive_expect_tx(&full[s], C::kTileBytes);
-            load_tile<D>(smem + C::kRingOff + s * C::kTileBytes, kv ? &tmV : &tmK, &full[s], j * 128, bh);
-            ++it;
-          }
+          const uint32_t ks = kit % C::kKSlots;
+          if (!(ok = wait_bar(&kempty[ks], ((kit / C::kKSlots) & 1u) ^ 1u, ab))) break;
+          bar_arrive_expect_tx(&kfull[ks], C::kTileBytes);
+          load_tile<D>(smem + C::kKOff + ks * C::kTileBytes, &tmK, &kfull[ks], j * 128, bh);
+          ++kit;
+          const uint32_t vs = vit % C::kVSlots;
+          if (!(ok = wait_bar(&vempty[vs], ((vit / C::kVSlots) & 1u) ^ 1u, ab))) break;
+          bar_arrive_expect_tx(&vfull[vs], C::kTileBytes);
+          load_tile<D>(smem + C::kVOff + vs * C::kTileBytes, &tmV, &vfull[vs], j * 128, bh);
+          ++vit;
         }
       }
-      const uint32_t first = it > static_cast<uint32_t>(C::kSlots) ? it - C::kSlots : 0u;
-      for (uint32_t i = first; i < it; ++i) drain(&full[i % C::kSlots], (i / C::kSlots) & 1u, p.status);
+      // every issued copy lands before the CTA can exit
+      const uint32_t kf = kit > static_cast<uint32_t>(C::kKSlots) ? kit - C::kKSlots : 0u;
+      for (uint32_t i = kf; i < kit; ++i) drain(&kfull[i % C::kKSlots], (i / C::kKSlots) & 1u, p.status);
+      const uint32_t vf = vit > static_cast<uint32_t>(C::kVSlots) ? vit - C::kVSlots : 0u;
+      for (uint32_t i = vf; i < vit; ++i) drain(&vfull[i % C::kVSlots], (i / C::kVSlots) & 1u, p.status);
       if (qit > 0) drain(qdo_full, (qit - 1u) & 1u, p.status);
     }
   }
