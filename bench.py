@@ -84,9 +84,9 @@ def profiled_traffic(kind):
                 if ":" in line:
                     k, v = line.split(":", 1)
                     fields[k.strip()] = v.strip()
-        if fields.get("source_sha256_16") != kernel_source_hash():
+        if fields.get("source_sha256_16", "").split(" ")[0] != kernel_source_hash():
             return None
-        return float(fields["dram_bytes_per_launch_full_size"])
+        return float(fields["dram_bytes_per_launch_full_size"].split(" ")[0])
     except (OSError, KeyError, ValueError):
         return None
 

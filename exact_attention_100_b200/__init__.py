@@ -47,6 +47,8 @@ def lib() -> ctypes.CDLL:
         vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
         L.attn_fwd.restype = i
+        L.attn_fwd_qk.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp]
+        L.attn_fwd_qk.restype = i
         L.attn_hadamard_quant.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
         L.attn_hadamard_quant.restype = i
         L.attn_hadamard_quant_qkv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
@@ -158,6 +160,29 @@ def attn_bwd(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None, s
                           _ptr(workspace), B, H, N, d, s, int(bool(causal)), gcode, _stream_ptr(stream)),
            "attn_bwd")
     return dq, dk, dv
+
+
+def attn_fwd_qk(q, k, v, o=None, lse=None, scale=None, causal=False, o_dtype=None, stream=None):
+    """attn_fwd with keys/values [B, H, Nk, d] whose length may differ from the queries'
+    [B, H, Nq, d].  Causal masking is bottom-right aligned (key j visible to query i iff
+    j <= i + Nk - Nq); rows that see no key get O = 0 and LSE = -inf.  Returns ``(o, lse)``."""
+    import torch
+    B, H, Nq, d = _dims(q)
+    Bk, Hk, Nk, dk = _dims(k)
+    if (Bk, Hk, dk) != (B, H, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H, Nk, d] with q's B, H, d")
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 tensors")
+    if o is None:
+        o = torch.empty(q.shape, dtype=o_dtype or torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_fwd_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d, s,
+                             int(bool(causal)), ATTN_BF16, od, _stream_ptr(stream)), "attn_fwd_qk")
+    return o, lse
 
 
 def attn_fwd_noalloc(q, k, v, o, lse=None, scale=None, causal=False, stream=None):

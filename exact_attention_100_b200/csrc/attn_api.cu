@@ -95,8 +95,8 @@ int check_common(int B, int H, int N, float scale, int causal, int o_dtype) {
   return ATTN_OK;
 }
 
-void fill_params(ea::FwdParams& p, void* o, float* lse, int* status, int B, int H, int N, int q_tiles, float scale,
-                 int causal, int o_dtype) {
+void fill_params(ea::FwdParams& p, void* o, float* lse, int* status, int B, int H, int N, int Nk, int q_tiles,
+                 float scale, int causal, int o_dtype) {
   p.o = o;
   p.lse = lse;
   p.status = status;
@@ -104,6 +104,9 @@ void fill_params(ea::FwdParams& p, void* o, float* lse, int* status, int B, int 
   p.N = N;
   p.BH = B * H;
   p.n_blocks = (N + 127) / 128;
+  p.Nk = Nk;
+  p.nbk = (Nk + 127) / 128;
+  p.off = Nk - N;
   p.n_pairs = (p.n_blocks + q_tiles - 1) / q_tiles;
   p.num_units = p.BH * p.n_pairs;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
@@ -134,13 +137,19 @@ const char* attn_status_string(int status) {
 
 unsigned long long attn_num_kernel_launches(void) { return g_launches.load(); }
 
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+}  // extern "C"
+
+namespace {
+
+// attn_fwd and attn_fwd_qk: queries [BH, Nq, d], keys and values [BH, Nk, d].
+int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk, int d,
              float scale, int causal, int dtype, int o_dtype, void* stream) {
   if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
     return ATTN_ERR_INVALID_ARG;
-  int rc = check_common(B, H, N, scale, causal, o_dtype);
+  int rc = check_common(B, H, Nq, scale, causal, o_dtype);
   if (rc != ATTN_OK) return rc;
+  if (Nk <= 0) return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_BF16) return dtype == ATTN_E4M3 || dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
 
@@ -148,16 +157,30 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
   CUtensorMap mq, mk, mv;
-  if (!encode_rows_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H) ||
-      !encode_rows_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H) ||
-      !encode_rows_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H))
+  if (!encode_rows_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nq, B * H) ||
+      !encode_rows_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nk, B * H) ||
+      !encode_rows_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nk, B * H))
     return ATTN_ERR_CUDA;
   ea::FwdParams p;
-  fill_params(p, o, lse, st->status, B, H, N, ea::fwd_units_per_tile_pair(d), scale, causal, o_dtype);
+  fill_params(p, o, lse, st->status, B, H, Nq, Nk, ea::fwd_units_per_tile_pair(d), scale, causal, o_dtype);
   if (ea::launch_attn_fwd_bf16(d, mq, mk, mv, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
   return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+             float scale, int causal, int dtype, int o_dtype, void* stream) {
+  return fwd_bf16(q, k, v, o, lse, B, H, N, N, d, scale, causal, dtype, o_dtype, stream);
+}
+
+int attn_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                int d, float scale, int causal, int dtype, int o_dtype, void* stream) {
+  return fwd_bf16(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, o_dtype, stream);
 }
 
 int attn_hadamard_quant(const void* x, void* x8, float* scales, const signed char* signs, int B, int H, int N, int d,
@@ -231,7 +254,7 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_
       !encode_rows_map(&mv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, B * H))
     return ATTN_ERR_CUDA;
   ea::FwdParams p;
-  fill_params(p, o, lse, st->status, B, H, N, 2, scale, causal, o_dtype);
+  fill_params(p, o, lse, st->status, B, H, N, N, 2, scale, causal, o_dtype);
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.v_scale = v_scale;

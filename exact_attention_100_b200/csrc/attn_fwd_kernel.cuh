@@ -126,7 +126,15 @@ __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
   for (int q = 0; q < 2; ++q) {
     const int t = U.tile0 + q;
     int n = 0;
-    if (q < NQ && t * 128 < p.N) n = p.causal ? min(t + 1, p.n_blocks) : p.n_blocks;
+    if (q < NQ && t * 128 < p.N) {
+      if (!p.causal) {
+        n = p.nbk;
+      } else {
+        // keys up to the tile's last row + off (bottom-right alignment); 0 if even it sees none
+        const int last = min(t * 128 + 127, p.N - 1) + p.off;
+        n = last < 0 ? 0 : min(last / 128 + 1, p.nbk);
+      }
+    }
     U.n[q] = n;
     U.n_max = max(U.n_max, n);
   }
@@ -328,11 +336,27 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       if (u >= p.num_units) break;
       const Unit U = decode_unit<NQ>(u, p);
       const int n = U.n[q];
-      if (n == 0) continue;
       const int tile_row0 = (U.tile0 + q) * 128;
       const int row_g = tile_row0 + row;
-      int lim_row = p.N;  // keys [0, lim_row) are visible to this row
-      if (p.causal) lim_row = min(lim_row, row_g + 1);
+      if (n == 0) {
+        // a tile inside the sequence whose rows see no key (causal, more queries than keys):
+        // O = 0 and LSE = -inf, written here; no MMA or epilogue event concerns it
+        if (tile_row0 < p.N) {
+          if (row_g < p.N) {
+            const size_t orow = (static_cast<size_t>(U.bh) * p.N + row_g) * D;
+            for (int c = 0; c < D; c += 4) {
+              if (p.o_fp32)
+                *reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+              else
+                *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.o) + orow + c) = make_uint2(0u, 0u);
+            }
+            if (p.lse != nullptr) p.lse[static_cast<size_t>(U.bh) * p.N + row_g] = -INFINITY;
+          }
+        }
+        continue;
+      }
+      int lim_row = p.Nk;  // keys [0, lim_row) are visible to this row (<= 0: none)
+      if (p.causal) lim_row = min(lim_row, row_g + p.off + 1);
       float c_base = p.scale_log2;
       float ps_log2_base = 0.f, l_div = 1.f;
       const float* ks = nullptr;
@@ -341,10 +365,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       if constexpr (E::kFp8) {
         // the Q block scale folds into c; P is stored as p * 16 * s_v(j) / max_j s_v(j)
         c_base *= __ldg(p.q_scale + static_cast<size_t>(U.bh) * nb + U.tile0 + q);
-        ks = p.k_scale + static_cast<size_t>(U.bh) * nb;
-        vs = p.v_scale + static_cast<size_t>(U.bh) * nb;
+        ks = p.k_scale + static_cast<size_t>(U.bh) * p.nbk;
+        vs = p.v_scale + static_cast<size_t>(U.bh) * p.nbk;
         float vmax = 0.f;
-        for (int b = lane; b < nb; b += 32) vmax = fmaxf(vmax, __ldg(vs + b));
+        for (int b = lane; b < p.nbk; b += 32) vmax = fmaxf(vmax, __ldg(vs + b));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
         ps_log2_base = lg2_approx(E::kPScale / vmax);
@@ -372,7 +396,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         uint32_t r[128];
         tmem_ld_row128(tS, r);
         const int key0 = j * 128;
-        const bool need_mask = (key0 + 128 > p.N) || (p.causal && key0 + 127 > tile_row0);
+        const bool need_mask = (key0 + 128 > p.Nk) || (p.causal && key0 + 127 > tile_row0 + p.off);
         if (need_mask) {
           const int lim = lim_row - key0;
 #pragma unroll
@@ -397,8 +421,14 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
           l *= alpha;
         }
         uint32_t pk[E::kPCols];
-        float lb = need_mask ? softmax_block<E, true>(r, pk, c, ps_log2 - m)
-                             : softmax_block<E, false>(r, pk, c, ps_log2 - m);
+        float lb;
+        if (need_mask) {
+          // only a masked block can leave a row without any visible key so far (m = -inf,
+          // possible when there are more queries than keys): its p must come out 0, not NaN
+          lb = softmax_block<E, true>(r, pk, c, ps_log2 - (m == -INFINITY ? 0.f : m));
+        } else {
+          lb = softmax_block<E, false>(r, pk, c, ps_log2 - m);
+        }
         if constexpr (E::kFp8) lb *= ex2_approx(-ps_log2);
         l += lb;
         tmem_st_32cols(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
@@ -473,7 +503,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const float lse2 = row_m[(q * 2 + uslot) * 128 + row];
-        const float inv = 1.f / row_l[(q * 2 + uslot) * 128 + row];
+        const float ls = row_l[(q * 2 + uslot) * 128 + row];
+        const float inv = ls > 0.f ? 1.f / ls : 0.f;  // a row with no visible key: O = 0
         const int row_g = tile * 128 + row;
         const bool valid = row_g < p.N;
         const size_t orow = (static_cast<size_t>(bh) * p.N + row_g) * D;
@@ -604,6 +635,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         ok = wait_bar(q_full, qit & 1u, ab);
         ++qit;
         if (!ok) break;
+        if (U.n_max == 0) {  // no tile of the unit sees a key: nothing to compute, Q is free again
+          tc_commit(q_empty);
+          continue;
+        }
         if (!(ok = wait_loaded(base))) break;
         if constexpr (NQ == 2) {
 #pragma unroll

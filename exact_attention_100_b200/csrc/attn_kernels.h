@@ -14,9 +14,12 @@ struct FwdParams {
   const float* q_scale;  // E4M3 only: [BH, n_blocks] block scales
   const float* k_scale;
   const float* v_scale;
-  int N;            // sequence length (queries = keys)
+  int N;            // query length (rows of Q, O, LSE)
   int BH;           // batch * heads
-  int n_blocks;     // ceil(N / 128)
+  int n_blocks;     // ceil(N / 128): Q tiles
+  int Nk;           // key length (rows of K, V)
+  int nbk;          // ceil(Nk / 128): K/V blocks
+  int off;          // Nk - N: causal key j is visible to query i iff j <= i + off (bottom-right)
   int n_pairs;      // ceil(n_blocks / Q tiles per unit)
   int num_units;    // BH * n_pairs
   float scale_log2; // softmax scale * log2(e)

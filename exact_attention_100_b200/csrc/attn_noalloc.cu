@@ -136,6 +136,9 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
   p.N = N;
   p.BH = B * H;
   p.n_blocks = (N + 127) / 128;
+  p.Nk = N;
+  p.nbk = p.n_blocks;
+  p.off = 0;
   const int tiles = ea::fwd_units_per_tile_pair(d);
   p.n_pairs = (p.n_blocks + tiles - 1) / tiles;
   p.num_units = p.BH * p.n_pairs;

@@ -12,6 +12,8 @@ Recipe (the same for every workload):
 * Every tensor is rounded to bf16 (round to nearest even) last.
 * The random-sign diagonal of the Hadamard transform is ``2 * (default_rng(seed).random(d)
   < 0.5) - 1`` with seed 1, stored as int8 +-1.
+* Workloads whose keys differ in length from the queries draw Q ``[B, H, Nq, d]``, then K and
+  V ``[B, H, Nk, d]``, in that order, from the same generator.
 * The upstream gradient dO of the backward workloads is ``default_rng(seed).standard_normal``
   float32 of shape ``[B, H, N, d]`` with seed 7 unless stated, rounded to bf16.
 """
@@ -62,3 +64,13 @@ def normal_dout(B: int, H: int, N: int, d: int, seed: int = 7) -> np.ndarray:
     """dO for the backward workloads: float32 array of bf16 values, [B, H, N, d], iid N(0, 1)."""
     rng = np.random.default_rng(seed)
     return round_to_bf16(rng.standard_normal((B, H, N, d), dtype=np.float32))
+
+
+def normal_qkv_lengths(B: int, H: int, Nq: int, Nk: int, d: int, seed: int = 0):
+    """(q, k, v) with q [B, H, Nq, d] and k, v [B, H, Nk, d]: float32 arrays of bf16 values,
+    iid N(0, 1), drawn in the order Q, K, V."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, H, Nq, d), dtype=np.float32)
+    k = rng.standard_normal((B, H, Nk, d), dtype=np.float32)
+    v = rng.standard_normal((B, H, Nk, d), dtype=np.float32)
+    return round_to_bf16(q), round_to_bf16(k), round_to_bf16(v)

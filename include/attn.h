@@ -77,6 +77,22 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int dtype, int o_dtype, void* stream);
 
 /*
+ * attn_fwd_qk -- attn_fwd with a key/value length Nk that may differ from the query length Nq.
+ *
+ *   q           [B, H, Nq, d] bf16, device.     k, v   [B, H, Nk, d] bf16, device.
+ *   o           [B, H, Nq, d] of o_dtype, written.   lse [B, H, Nq] float32 or NULL, written.
+ *   Nq, Nk      >= 1.
+ *   causal      1: key j is visible to query i iff j <= i + (Nk - Nq) (bottom-right alignment,
+ *               the reading taken where the pages are silent); a query row with no visible key
+ *               (only when Nq > Nk) gets O = 0 and LSE = -inf.
+ * Other arguments, arithmetic and errors as for attn_fwd, which is attn_fwd_qk with
+ * Nq = Nk = N.
+ */
+int attn_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse,
+                int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                int dtype, int o_dtype, void* stream);
+
+/*
  * attn_hadamard_quant -- random-sign Hadamard transform plus per-block E4M3 quantisation.
  *
  *   x       [B, H, N, d] bf16, device (read).

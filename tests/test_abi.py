@@ -31,7 +31,7 @@ def test_header_declares_the_boundary():
     assert names == sorted(["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status",
                             "attn_status_string", "attn_num_kernel_launches", "attn_shutdown",
                             "attn_fwd_noalloc", "attn_hadamard_quant_qkv", "attn_bwd",
-                            "attn_bwd_workspace_bytes"])
+                            "attn_bwd_workspace_bytes", "attn_fwd_qk"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -112,6 +112,22 @@ def test_fwd_fp8_rejects_bad_arguments(L):
     assert f(*a) == ea.ATTN_ERR_INVALID_ARG
 
 
+def test_fwd_qk_rejects_bad_arguments(L):
+    f = L.attn_fwd_qk
+    ok = [P, P, P, P2, NULL, 1, 1, 128, 300, 128, 0.1, 1, 0, 0, NULL]
+    for i in range(4):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for idx, val in [(7, 0), (8, 0), (8, -3), (10, 0.0), (11, 3), (13, 5)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+    a = list(ok)
+    a[9] = 96
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+
+
 def test_bwd_workspace_bytes(L):
     assert L.attn_bwd_workspace_bytes(1, 1, 1) == 2 * 128 * 4
     assert L.attn_bwd_workspace_bytes(2, 16, 8192) == 2 * 32 * 8192 * 4
@@ -144,5 +160,5 @@ def test_bwd_rejects_bad_arguments(L):
 def test_python_binding_has_same_names():
     for name in ["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status", "attn_status_string",
                  "attn_num_kernel_launches", "attn_shutdown", "attn_fwd_noalloc", "attn_hadamard_quant_qkv",
-                 "attn_bwd", "attn_bwd_workspace_bytes"]:
+                 "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_qk"]:
         assert callable(getattr(ea, name)), name
