@@ -15,9 +15,11 @@
 // dQ gets its own pass (recomputing S and dP) instead of atomic additions from the dK/dV
 // kernel ("Flash Attention V3 解析", section 4.2): no float atomics, deterministic results.
 //
-// Roles (both main kernels, 192 threads): warps 0-3 one thread per TMEM lane (a row of S or
-// S^T: the softmax backward and the epilogue), warp 4 lane 0 issues every tcgen05.mma, warp 5
-// lane 0 is the TMA producer.  Every mbarrier wait is bounded (wait_bar).
+// Roles (both main kernels, 320 threads): warps 0-7 form the softmax backward and the epilogue,
+// one TMEM lane (a row of S or S^T) per thread of warps w and w + 4, which take the first and
+// the second 64 columns of each block (no exchange between them: LSE and D are given); warp 8
+// lane 0 issues every tcgen05.mma, warp 9 lane 0 is the TMA producer.  Every mbarrier wait is
+// bounded (wait_bar).
 
 #include <cuda_bf16.h>
 
@@ -96,9 +98,10 @@ struct BwdCfg {
   static constexpr int kBoxBytes = 128 * 128;            // a 128-row x 128-byte column box
   static constexpr int kBoxes = D * 2 / 128;             // column boxes of a bf16 row
   static constexpr int kTileBytes = kBoxes * kBoxBytes;  // 128 rows x D bf16
-  static constexpr int kThreads = 192;
-  static constexpr int kMmaWarp = 4;
-  static constexpr int kLoadWarp = 5;
+  static constexpr int kThreads = 320;
+  static constexpr int kComputeWarps = 8;   // two per TMEM lane quarter, one per column half
+  static constexpr int kMmaWarp = 8;
+  static constexpr int kLoadWarp = 9;
   static constexpr uint32_t kIdS = make_idesc(128, 128, 1, false);  // S-type products, both K-major
   static constexpr uint32_t kIdD = make_idesc(128, D, 1, true);     // accumulations, B MN-major
 };
@@ -124,24 +127,27 @@ __device__ __forceinline__ void mma_abt(uint32_t d_tmem, uint32_t a_base, uint32
   }
 }
 
-// Acc[tmem, 128 x D] (+)= X B with X 128 x 128 bf16 in TMEM (packed pairs, 64 columns) and B a
-// 128 x D tile in shared memory read MN-major (its rows are the contraction index).
+// Acc[tmem, 128 x D] (+)= X B with X 128 x 128 bf16 in TMEM (packed pairs) and B a 128 x D tile
+// in shared memory read MN-major (its rows are the contraction index).  X's contraction index
+// 16 kk .. 16 kk + 15 sits at TMEM column x_tmem + (kk / 4) * half_stride + (kk % 4) * 8: the two
+// 64-wide halves of X are 32 columns each, half_stride apart.
 template <int D>
-__device__ __forceinline__ void mma_xb(uint32_t d_tmem, uint32_t x_tmem, uint32_t b_base, bool acc) {
+__device__ __forceinline__ void mma_xb(uint32_t d_tmem, uint32_t x_tmem, uint32_t half_stride, uint32_t b_base,
+                                       bool acc) {
   using C = BwdCfg<D>;
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
-    mma_f16_ts(d_tmem, x_tmem + kk * 8, make_sdesc_sw128(b_base + kk * 16 * 128, C::kBoxBytes, 1024), C::kIdD,
-               (acc || kk > 0) ? 1u : 0u);
+    mma_f16_ts(d_tmem, x_tmem + (kk >> 2) * half_stride + (kk & 3) * 8,
+               make_sdesc_sw128(b_base + kk * 16 * 128, C::kBoxBytes, 1024), C::kIdD, (acc || kk > 0) ? 1u : 0u);
 }
 
-// Stores one row of a 128 x D f32 TMEM accumulator (this thread's lane), times `mul`, as bf16
-// or f32.
-template <int D>
+// Stores kCols columns of one row of an f32 TMEM accumulator (this thread's lane), times `mul`,
+// as bf16 or f32 at out + row_off.
+template <int kCols>
 __device__ __forceinline__ void store_row(uint32_t t_acc, void* out, size_t row_off, float mul, bool fp32,
                                           bool valid) {
 #pragma unroll 1
-  for (int cc = 0; cc < D / 32; ++cc) {
+  for (int cc = 0; cc < kCols / 32; ++cc) {
     uint32_t r[32];
     tmem_ld_32cols(t_acc + 32 * cc, r);
     tmem_ld_wait(r);
@@ -241,10 +247,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     }
     bar_init(st_s, 1);
     bar_init(st_dp, 1);
-    bar_init(pt_full, 4);
-    bar_init(dst_full, 4);
+    bar_init(pt_full, C::kComputeWarps);
+    bar_init(dst_full, C::kComputeWarps);
     bar_init(dkv_done, 1);
-    bar_init(dkv_free, 4);
+    bar_init(dkv_free, C::kComputeWarps);
     bar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -267,10 +273,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   const int nb = p.n_blocks;
   const int num_units = p.BH * nb;
 
-  if (warp < 4) {
-    // ===================================================== softmax backward: one key row each
-    const int row = warp * 32 + lane;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  if (warp < C::kComputeWarps) {
+    // ===================================== softmax backward: one key row, one half of the queries
+    const int row = (warp & 3) * 32 + lane;
+    const int h = warp >> 2;  // queries [64h, 64h + 64) of each block
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     uint32_t qc = 0, uit = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
@@ -288,20 +295,22 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                                                            2 * C::kTileBytes);
         const float* dlt = lse2 + 128;
         const bool diag = p.causal && i == kb;
-        // pass 1, from S^T alone: P^T (kept in registers, and as bf16 over S^T columns [0, 64))
+        // pass 1, from S^T alone: P^T, kept in registers and stored as bf16 over this half's first
+        // 32 S^T columns [64h, 64h + 32) (already read by this thread)
         ok = warp_all(wait_bar(st_s, qc & 1u, ab));
         if (!ok) break;
         tc_fence_after();
-        float pr[128];
+        float pr[64];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t sv[32];
-          tmem_ld_32cols(lane_base + 32 * c, sv);
+          tmem_ld_32cols(lane_base + 64 * h + 32 * c, sv);
           tmem_ld_wait(sv);
           uint32_t pk[16];
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
-            const int qq = 32 * c + 2 * t;  // query pair within the block
+            const int ql = 32 * c + 2 * t;  // query pair within this half
+            const int qq = 64 * h + ql;     // ... within the block
             float p0, p1;
             float x0, x1;
             f2_fma(x0, x1, __uint_as_float(sv[2 * t]), __uint_as_float(sv[2 * t + 1]), p.scale_log2, p.scale_log2,
@@ -309,36 +318,37 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
             exp2_pair(p0, p1, x0, x1);
             if (diag && i * 128 + qq < key_g) p0 = 0.f;  // query before the key: masked
             if (diag && i * 128 + qq + 1 < key_g) p1 = 0.f;
-            pr[qq] = p0;
-            pr[qq + 1] = p1;
+            pr[ql] = p0;
+            pr[ql + 1] = p1;
           }
 #pragma unroll
           for (int t = 0; t < 16; ++t) pk[t] = pack_bf16x2(pr[32 * c + 2 * t], pr[32 * c + 2 * t + 1]);
-          tmem_st_16cols(lane_base + 16 * c, pk);  // S^T columns [16c, 16c+16): already read
+          tmem_st_16cols(lane_base + 64 * h + 16 * c, pk);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) bar_arrive(pt_full);
-        // pass 2, from dP^T: dS^T = P^T (dP^T - D) as bf16 over dP^T columns [0, 64)
+        // pass 2, from dP^T: dS^T = P^T (dP^T - D) as bf16 over dP^T columns [128 + 64h, +32)
         ok = warp_all(wait_bar(st_dp, qc & 1u, ab));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t dp[32];
-          tmem_ld_32cols(lane_base + 128 + 32 * c, dp);
+          tmem_ld_32cols(lane_base + 128 + 64 * h + 32 * c, dp);
           tmem_ld_wait(dp);
           uint32_t dk[16];
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
-            const int q0 = 32 * c + 2 * t;
+            const int ql = 32 * c + 2 * t;
+            const int q0 = 64 * h + ql;
             float y0, y1;
-            f2_sub_mul(y0, y1, __uint_as_float(dp[2 * t]), __uint_as_float(dp[2 * t + 1]), dlt[q0], dlt[q0 + 1], pr[q0],
-                       pr[q0 + 1]);
+            f2_sub_mul(y0, y1, __uint_as_float(dp[2 * t]), __uint_as_float(dp[2 * t + 1]), dlt[q0], dlt[q0 + 1], pr[ql],
+                       pr[ql + 1]);
             dk[t] = pack_bf16x2(y0, y1);
           }
-          tmem_st_16cols(lane_base + 128 + 16 * c, dk);
+          tmem_st_16cols(lane_base + 128 + 64 * h + 16 * c, dk);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -351,9 +361,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const bool valid = key_g < p.N;
-      const size_t off = (static_cast<size_t>(bh) * p.N + key_g) * D;
-      store_row<D>(lane_base + 256, p.dv, off, 1.f, p.g_fp32 != 0, valid);
-      store_row<D>(lane_base + 256 + D, p.dk, off, p.scale, p.g_fp32 != 0, valid);
+      const size_t off = (static_cast<size_t>(bh) * p.N + key_g) * D + h * (D / 2);  // this half's columns
+      store_row<D / 2>(lane_base + 256 + h * (D / 2), p.dv, off, 1.f, p.g_fp32 != 0, valid);
+      store_row<D / 2>(lane_base + 256 + D + h * (D / 2), p.dk, off, p.scale, p.g_fp32 != 0, valid);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) bar_arrive(dkv_free);
@@ -390,7 +400,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
             if (!(ok = wait_bar(dkv_free, (uc & 1u) ^ 1u, ab))) break;
             tc_fence_after();
           }
-          mma_xb<D>(tmem + 256, tmem, do_base, i > i0);  // dV += P^T dO
+          mma_xb<D>(tmem + 256, tmem, 64, do_base, i > i0);  // dV += P^T dO
           if (next) {
             // S^T of the next block replaces P^T, which dV (issued first) has read
             if (!(ok = wait_bar(&st_full[(qc + 1) % C::kStages], ((qc + 1) / C::kStages) & 1u, ab))) break;
@@ -399,7 +409,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           }
           if (!(ok = wait_bar(dst_full, qc & 1u, ab))) break;
           tc_fence_after();
-          mma_xb<D>(tmem + 256 + D, tmem + 128, q_base, i > i0);  // dK += dS^T Q
+          mma_xb<D>(tmem + 256 + D, tmem + 128, 64, q_base, i > i0);  // dK += dS^T Q
           tc_commit(&st_empty[qc % C::kStages]);
           if (next) {
             mma_abt<D>(tmem + 128, v_base, q_at(qc + 1) + C::kTileBytes);
@@ -523,11 +533,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     bar_init(qdo_empty, 1);
     bar_init(s_full, 1);
     bar_init(dp_full, 1);
-    bar_init(s_free, 4);
-    bar_init(&ds_full[0], 4);
-    bar_init(&ds_full[1], 4);
+    bar_init(s_free, C::kComputeWarps);
+    bar_init(&ds_full[0], C::kComputeWarps);
+    bar_init(&ds_full[1], C::kComputeWarps);
     bar_init(dq_done, 1);
-    bar_init(dq_free, 4);
+    bar_init(dq_free, C::kComputeWarps);
     bar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -550,10 +560,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   const int nb = p.n_blocks;
   const int num_units = p.BH * nb;
 
-  if (warp < 4) {
-    // ===================================================== softmax backward: one query row each
-    const int row = warp * 32 + lane;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  if (warp < C::kComputeWarps) {
+    // ===================================== softmax backward: one query row, one half of the keys
+    const int row = (warp & 3) * 32 + lane;
+    const int h = warp >> 2;  // keys [64h, 64h + 64) of each block
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     uint32_t sc = 0, uit = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
@@ -574,15 +585,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         ok = warp_all(wait_bar(s_full, sc & 1u, ab));
         if (!ok) break;
         tc_fence_after();
-        float pr[128];
+        float pr[64];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t sv[32];
-          tmem_ld_32cols(lane_base + 32 * c, sv);
+          tmem_ld_32cols(lane_base + 64 * h + 32 * c, sv);
           tmem_ld_wait(sv);
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
-            const int kk = 32 * c + 2 * t;
+            const int kl = 32 * c + 2 * t;  // key pair within this half
+            const int kk = 64 * h + kl;     // ... within the block
             float p0, p1;
             float x0, x1;
             f2_fma(x0, x1, __uint_as_float(sv[2 * t]), __uint_as_float(sv[2 * t + 1]), p.scale_log2, p.scale_log2,
@@ -590,8 +602,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
             exp2_pair(p0, p1, x0, x1);
             if (mask && kk >= lim) p0 = 0.f;
             if (mask && kk + 1 >= lim) p1 = 0.f;
-            pr[kk] = p0;
-            pr[kk + 1] = p1;
+            pr[kl] = p0;
+            pr[kl + 1] = p1;
           }
         }
         tc_fence_before();
@@ -602,9 +614,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t dp[32];
-          tmem_ld_32cols(lane_base + 128 + 32 * c, dp);
+          tmem_ld_32cols(lane_base + 128 + 64 * h + 32 * c, dp);
           tmem_ld_wait(dp);
           uint32_t dk[16];
 #pragma unroll
@@ -614,7 +626,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
             f2_sub_mul(y0, y1, __uint_as_float(dp[2 * t]), __uint_as_float(dp[2 * t + 1]), dlt, dlt, pr[k0], pr[k0 + 1]);
             dk[t] = pack_bf16x2(y0, y1);
           }
-          tmem_st_16cols(t_ds + 16 * c, dk);
+          tmem_st_16cols(t_ds + 32 * h + 16 * c, dk);  // the buffer holds the 128 keys in order
         }
         tmem_st_wait();
         tc_fence_before();
@@ -625,8 +637,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       ok = warp_all(wait_bar(dq_done, uit & 1u, ab));
       if (!ok) break;
       tc_fence_after();
-      store_row<D>(lane_base + 256, p.dq, (static_cast<size_t>(bh) * p.N + q_g) * D, p.scale, p.g_fp32 != 0,
-                   q_g < p.N);
+      store_row<D / 2>(lane_base + 256 + h * (D / 2), p.dq, (static_cast<size_t>(bh) * p.N + q_g) * D + h * (D / 2),
+                       p.scale, p.g_fp32 != 0, q_g < p.N);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) bar_arrive(dq_free);
@@ -664,7 +676,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
             tc_fence_after();
             dq_started = true;
           }
-          mma_xb<D>(tmem + 256, tmem + 384 + (blk & 1u) * 64, k_addr(kb0 + j), j > 0);
+          mma_xb<D>(tmem + 256, tmem + 384 + (blk & 1u) * 64, 32, k_addr(kb0 + j), j > 0);
           tc_commit(&kempty[(kb0 + j) % C::kKSlots]);
           return true;
         };
