@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
         L.attn_bwd_workspace_bytes.restype = ctypes.c_ulonglong
         L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
         L.attn_bwd.restype = i
+        L.attn_bwd_qk.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+        L.attn_bwd_qk.restype = i
         L.attn_device_status.argtypes = [vp]
         L.attn_device_status.restype = i
         L.attn_status_string.argtypes = [i]
@@ -183,6 +185,32 @@ def attn_fwd_qk(q, k, v, o=None, lse=None, scale=None, causal=False, o_dtype=Non
     _check(lib().attn_fwd_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d, s,
                              int(bool(causal)), ATTN_BF16, od, _stream_ptr(stream)), "attn_fwd_qk")
     return o, lse
+
+
+def attn_bwd_qk(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None, scale=None, causal=False,
+                g_dtype=None, stream=None):
+    """attn_bwd for attn_fwd_qk: q, o, dout [B, H, Nq, d], k, v [B, H, Nk, d] (bf16); returns
+    (dq [B, H, Nq, d], dk, dv [B, H, Nk, d])."""
+    import torch
+    B, H, Nq, d = _dims(q)
+    Nk = int(k.shape[2])
+    if k.shape != v.shape or tuple(k.shape) != (B, H, Nk, d) or o.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("expected q, o, dout [B, H, Nq, d] and k, v [B, H, Nk, d]")
+    for t in (q, k, v, o, dout):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("q, k, v, o, dout must be contiguous bf16 tensors")
+    gd = g_dtype or (dq.dtype if dq is not None else torch.bfloat16)
+    dq = dq if dq is not None else torch.empty(q.shape, dtype=gd, device=q.device)
+    dk = dk if dk is not None else torch.empty(k.shape, dtype=gd, device=q.device)
+    dv = dv if dv is not None else torch.empty(k.shape, dtype=gd, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(attn_bwd_workspace_bytes(B, H, Nq) // 4, dtype=torch.float32, device=q.device)
+    gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_bwd_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                             _ptr(workspace), B, H, Nq, Nk, d, s, int(bool(causal)), gcode, _stream_ptr(stream)),
+           "attn_bwd_qk")
+    return dq, dk, dv
 
 
 def attn_fwd_noalloc(q, k, v, o, lse=None, scale=None, causal=False, stream=None):

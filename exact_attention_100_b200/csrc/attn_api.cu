@@ -270,37 +270,47 @@ unsigned long long attn_bwd_workspace_bytes(int B, int H, int N) {
   return 2ull * static_cast<unsigned long long>(B) * static_cast<unsigned long long>(H) * n_pad * 4ull;
 }
 
-int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-             void* dq, void* dk, void* dv, void* workspace, int B, int H, int N, int d, float scale, int causal,
-             int g_dtype, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+             void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
+             int causal, int g_dtype, void* stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
     return ATTN_ERR_INVALID_ARG;
-  int rc = check_common(B, H, N, scale, causal, g_dtype);
+  int rc = check_common(B, H, Nq, scale, causal, g_dtype);
   if (rc != ATTN_OK) return rc;
+  if (Nk <= 0) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  const long long n_blocks = (static_cast<long long>(N) + 127) / 128;
-  if (static_cast<long long>(B) * H * n_blocks > 0x7FFFFFFFLL || n_blocks * 128 > 0x7FFFFFFFLL)
+  const long long n_blocks = (static_cast<long long>(Nq) + 127) / 128;
+  const long long nbk = (static_cast<long long>(Nk) + 127) / 128;
+  if (static_cast<long long>(B) * H * n_blocks > 0x7FFFFFFFLL || static_cast<long long>(B) * H * nbk > 0x7FFFFFFFLL ||
+      n_blocks * 128 > 0x7FFFFFFFLL)
     return ATTN_ERR_INVALID_ARG;
 
   DeviceState* st = nullptr;
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
   CUtensorMap mq, mk, mv, mdo;
-  if (!encode_rows_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H) ||
-      !encode_rows_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H) ||
-      !encode_rows_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H) ||
-      !encode_rows_map(&mdo, dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H))
+  if (!encode_rows_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nq, B * H) ||
+      !encode_rows_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nk, B * H) ||
+      !encode_rows_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nk, B * H) ||
+      !encode_rows_map(&mdo, dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nq, B * H))
     return ATTN_ERR_CUDA;
   ea::BwdParams p;
   p.lse = lse;
   p.o = o;
   p.dout = dout;
   p.BH = B * H;
-  p.N = N;
+  p.N = Nq;
   p.n_blocks = static_cast<int>(n_blocks);
   p.n_pad = static_cast<int>(n_blocks * 128);
+  p.Nk = Nk;
+  p.nbk = static_cast<int>(nbk);
+  p.off = Nk - Nq;
   p.delta = static_cast<float*>(workspace);
   p.lse2 = static_cast<float*>(workspace) + static_cast<size_t>(p.BH) * p.n_pad;
   p.dq = dq;
@@ -315,6 +325,22 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(3);
   return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+             void* dq, void* dk, void* dv, void* workspace, int B, int H, int N, int d, float scale, int causal,
+             int g_dtype, void* stream) {
+  return bwd_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, N, N, d, scale, causal, g_dtype, stream);
+}
+
+int attn_bwd_qk(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
+                int causal, int g_dtype, void* stream) {
+  return bwd_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale, causal, g_dtype, stream);
 }
 
 int attn_device_status(void* stream) {

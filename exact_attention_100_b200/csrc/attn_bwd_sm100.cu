@@ -178,6 +178,49 @@ __device__ __forceinline__ int unit_of(int k) {
   return k * g + ((k & 1) ? (g - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x));
 }
 
+// dK/dV unit u: key block kb of head bh and the first query block i0 that sees any of its keys
+// (causal, bottom-right: query r sees key c iff c <= r + off); i0 >= n_blocks: no query does.
+struct KvUnit {
+  int bh, kb, i0;
+};
+__device__ __forceinline__ KvUnit kv_unit(int u, const BwdParams& p) {
+  KvUnit U;
+  U.bh = u % p.BH;
+  U.kb = u / p.BH;
+  const int first_q = U.kb * 128 - p.off;  // the smallest query that sees the block's first key
+  U.i0 = (!p.causal || first_q <= 0) ? 0 : first_q / 128;
+  return U;
+}
+
+// dQ unit u: query block qb of head bh (causal: longest first) and its number n of visible key
+// blocks (0: its rows see no key).
+struct QUnit {
+  int bh, qb, n;
+};
+__device__ __forceinline__ QUnit q_unit(int u, const BwdParams& p) {
+  QUnit U;
+  U.bh = u % p.BH;
+  U.qb = p.causal ? p.n_blocks - 1 - u / p.BH : u / p.BH;
+  if (!p.causal) {
+    U.n = p.nbk;
+  } else {
+    const int last = min(U.qb * 128 + 127, p.N - 1) + p.off;
+    U.n = last < 0 ? 0 : min(last / 128 + 1, p.nbk);
+  }
+  return U;
+}
+
+// Zero rows [row_off, +cols) of a bf16 or f32 gradient (rows that no query or no key reaches).
+template <int kCols>
+__device__ __forceinline__ void zero_row(void* out, size_t row_off, bool fp32) {
+  for (int c = 0; c < kCols; c += 4) {
+    if (fp32)
+      *reinterpret_cast<float4*>(static_cast<float*>(out) + row_off + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+    else
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + row_off + c) = make_uint2(0u, 0u);
+  }
+}
+
 __device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity, int* status) {
   const uint32_t a = smem_addr(bar);
   const unsigned long long t0 = global_timer_ns();
@@ -271,7 +314,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const AbortState ab{abort_flag, p.status};
   const int nb = p.n_blocks;
-  const int num_units = p.BH * nb;
+  const int num_units = p.BH * p.nbk;
 
   if (warp < C::kComputeWarps) {
     // ===================================== softmax backward: one key row, one half of the queries
@@ -283,9 +326,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     for (int k = 0; ok; ++k) {
       const int u = unit_of(k);
       if (u >= num_units) break;
-      const int bh = u % p.BH, kb = u / p.BH;
+      const KvUnit U = kv_unit(u, p);
+      const int bh = U.bh, kb = U.kb, i0 = U.i0;
       const int key_g = kb * 128 + row;
-      const int i0 = p.causal ? kb : 0;
+      if (i0 >= nb) {
+        // no query sees these keys (causal, more keys than queries): dK = dV = 0
+        if (key_g < p.Nk) {
+          const size_t off = (static_cast<size_t>(bh) * p.Nk + key_g) * D + h * (D / 2);
+          zero_row<D / 2>(p.dv, off, p.g_fp32 != 0);
+          zero_row<D / 2>(p.dk, off, p.g_fp32 != 0);
+        }
+        continue;
+      }
       for (int i = i0; i < nb && ok; ++i, ++qc) {
         const uint32_t st = qc % C::kStages;
         // the stage's lse2 / D rows arrived with its TMA transaction count
@@ -294,7 +346,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         const float* lse2 = reinterpret_cast<const float*>(smem + C::kStageOff + st * C::kStageBytes +
                                                            2 * C::kTileBytes);
         const float* dlt = lse2 + 128;
-        const bool diag = p.causal && i == kb;
+        // some query of block i misses some key of block kb (bottom-right causal mask)
+        const bool diag = p.causal && kb * 128 + 127 > i * 128 + p.off;
         // pass 1, from S^T alone: P^T, kept in registers and stored as bf16 over this half's first
         // 32 S^T columns [64h, 64h + 32) (already read by this thread)
         ok = warp_all(wait_bar(st_s, qc & 1u, ab));
@@ -316,8 +369,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
             f2_fma(x0, x1, __uint_as_float(sv[2 * t]), __uint_as_float(sv[2 * t + 1]), p.scale_log2, p.scale_log2,
                    -lse2[qq], -lse2[qq + 1]);
             exp2_pair(p0, p1, x0, x1);
-            if (diag && i * 128 + qq < key_g) p0 = 0.f;  // query before the key: masked
-            if (diag && i * 128 + qq + 1 < key_g) p1 = 0.f;
+            if (diag && i * 128 + qq + p.off < key_g) p0 = 0.f;  // key after the query's diagonal
+            if (diag && i * 128 + qq + 1 + p.off < key_g) p1 = 0.f;
             pr[ql] = p0;
             pr[ql + 1] = p1;
           }
@@ -360,8 +413,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       ok = warp_all(wait_bar(dkv_done, uit & 1u, ab));
       if (!ok) break;
       tc_fence_after();
-      const bool valid = key_g < p.N;
-      const size_t off = (static_cast<size_t>(bh) * p.N + key_g) * D + h * (D / 2);  // this half's columns
+      const bool valid = key_g < p.Nk;
+      const size_t off = (static_cast<size_t>(bh) * p.Nk + key_g) * D + h * (D / 2);  // this half's columns
       store_row<D / 2>(lane_base + 256 + h * (D / 2), p.dv, off, 1.f, p.g_fp32 != 0, valid);
       store_row<D / 2>(lane_base + 256 + D + h * (D / 2), p.dk, off, p.scale, p.g_fp32 != 0, valid);
       tc_fence_before();
@@ -379,8 +432,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int u = unit_of(k);
         if (u >= num_units) break;
-        const int kb = u / p.BH;
-        const int i0 = p.causal ? kb : 0;
+        const KvUnit U = kv_unit(u, p);
+        const int i0 = U.i0;
+        if (i0 >= nb) continue;  // no query sees the block: nothing loaded, nothing to compute
         if (!(ok = wait_bar(kv_full, uc & 1u, ab))) break;
         auto q_at = [&](uint32_t c) { return smem_addr(smem + C::kStageOff + (c % C::kStages) * C::kStageBytes); };
         // S^T and dP^T of the unit's first query block
@@ -432,8 +486,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int u = unit_of(k);
         if (u >= num_units) break;
-        const int bh = u % p.BH, kb = u / p.BH;
-        const int i0 = p.causal ? kb : 0;
+        const KvUnit U = kv_unit(u, p);
+        const int bh = U.bh, kb = U.kb, i0 = U.i0;
+        if (i0 >= nb) continue;
         if (uc > 0 && !(ok = wait_bar(kv_empty, (uc - 1u) & 1u, ab))) break;
         bar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
         load_tile<D>(smem + C::kKOff, &tmK, kv_full, kb * 128, bh);
@@ -557,8 +612,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const AbortState ab{abort_flag, p.status};
-  const int nb = p.n_blocks;
-  const int num_units = p.BH * nb;
+  const int num_units = p.BH * p.n_blocks;
 
   if (warp < C::kComputeWarps) {
     // ===================================== softmax backward: one query row, one half of the keys
@@ -570,17 +624,21 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     for (int k = 0; ok; ++k) {
       const int u = unit_of(k);
       if (u >= num_units) break;
-      const int bh = u % p.BH;
-      const int qb = p.causal ? nb - 1 - u / p.BH : u / p.BH;
+      const QUnit U = q_unit(u, p);
+      const int bh = U.bh, qb = U.qb, n = U.n;
       const int q_g = qb * 128 + row;
-      const int n = p.causal ? qb + 1 : nb;
+      if (n == 0) {
+        // these queries see no key (causal, more queries than keys): dQ = 0
+        if (q_g < p.N) zero_row<D / 2>(p.dq, (static_cast<size_t>(bh) * p.N + q_g) * D + h * (D / 2), p.g_fp32 != 0);
+        continue;
+      }
       const size_t w = static_cast<size_t>(bh) * p.n_pad + q_g;
       const float lse2 = p.lse2[w];  // +inf on padded rows: P = 0 there
       const float dlt = p.delta[w];
       for (int j = 0; j < n && ok; ++j, ++sc) {
         const uint32_t t_ds = lane_base + 384 + (sc & 1u) * 64;
-        const bool mask = (j * 128 + 128 > p.N) || (p.causal && j == qb);
-        const int lim = min(p.N, p.causal ? q_g + 1 : p.N) - j * 128;  // visible keys of this block
+        const bool mask = (j * 128 + 128 > p.Nk) || (p.causal && j * 128 + 127 > qb * 128 + p.off);
+        const int lim = min(p.Nk, p.causal ? q_g + p.off + 1 : p.Nk) - j * 128;  // visible keys of this block
         // pass 1, from S alone: P in registers; then S's columns may take the next block
         ok = warp_all(wait_bar(s_full, sc & 1u, ab));
         if (!ok) break;
@@ -660,13 +718,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int u = unit_of(k);
         if (u >= num_units) break;
-        const int qb = p.causal ? nb - 1 - u / p.BH : u / p.BH;
-        const int n = p.causal ? qb + 1 : nb;
+        const int n = q_unit(u, p).n;
         const uint32_t kb0 = kit, vb0 = vit;  // K_j = kb0 + j, V_j = vb0 + j
         kit += n;
         vit += n;
         if (!(ok = wait_bar(qdo_full, qit & 1u, ab))) break;
         ++qit;
+        if (n == 0) {  // the unit's queries see no key: release Q, dO; no dQ
+          tc_commit(qdo_empty);
+          continue;
+        }
         bool dq_started = false;
         // dQ(j) += dS(j) K_j, from the dS buffer of global block number `blk`
         auto issue_dq = [&](int j, uint32_t blk) {
@@ -726,9 +787,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int u = unit_of(k);
         if (u >= num_units) break;
-        const int bh = u % p.BH;
-        const int qb = p.causal ? nb - 1 - u / p.BH : u / p.BH;
-        const int n = p.causal ? qb + 1 : nb;
+        const QUnit U = q_unit(u, p);
+        const int bh = U.bh, qb = U.qb, n = U.n;
         if (qit > 0 && !(ok = wait_bar(qdo_empty, (qit - 1u) & 1u, ab))) break;
         bar_arrive_expect_tx(qdo_full, 2 * C::kTileBytes);
         load_tile<D>(smem + C::kQOff, &tmQ, qdo_full, qb * 128, bh);
@@ -784,12 +844,14 @@ cudaError_t launch_d(const CUtensorMap& q, const CUtensorMap& k, const CUtensorM
   bwd_prep_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int units = p.BH * p.n_blocks;
-  const int grid = units < num_sms ? units : num_sms;
-  bwd_dkdv_kernel<D><<<grid, BwdCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(q, k, v, dout, p);
+  const int kv_units = p.BH * p.nbk;
+  const int kv_grid = kv_units < num_sms ? kv_units : num_sms;
+  bwd_dkdv_kernel<D><<<kv_grid, BwdCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(q, k, v, dout, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dq_kernel<D><<<grid, BwdCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(q, k, v, dout, p);
+  const int q_units = p.BH * p.n_blocks;
+  const int q_grid = q_units < num_sms ? q_units : num_sms;
+  bwd_dq_kernel<D><<<q_grid, BwdCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(q, k, v, dout, p);
   return cudaGetLastError();
 }
 

@@ -50,10 +50,13 @@ struct BwdParams {
   void* dk;
   void* dv;
   int* status;
-  int N;
+  int N;                  // query length (rows of Q, O, dO, LSE, dQ)
   int BH;
-  int n_blocks;           // ceil(N / 128)
+  int n_blocks;           // ceil(N / 128): query blocks
   int n_pad;              // n_blocks * 128
+  int Nk;                 // key length (rows of K, V, dK, dV)
+  int nbk;                // ceil(Nk / 128)
+  int off;                // Nk - N: causal key j is visible to query i iff j <= i + off
   float scale;
   float scale_log2;       // scale * log2 e
   int causal;

@@ -182,6 +182,17 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              int B, int H, int N, int d, float scale, int causal, int g_dtype, void* stream);
 
 /*
+ * attn_bwd_qk -- attn_bwd for attn_fwd_qk: queries (q, o, dout, lse, dq) of length Nq, keys and
+ * values (k, v, dk, dv) of length Nk; causal masking bottom-right aligned as in attn_fwd_qk.
+ * Keys that no query sees get dK = dV = 0; queries that see no key get dQ = 0.  The workspace
+ * is attn_bwd_workspace_bytes(B, H, Nq) bytes.  attn_bwd is attn_bwd_qk with Nq = Nk = N.
+ */
+int attn_bwd_qk(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                int B, int H, int Nq, int Nk, int d, float scale, int causal, int g_dtype,
+                void* stream);
+
+/*
  * attn_fwd_noalloc -- attn_fwd for callers that cannot allocate device memory.  The pages have
  * no counterpart; it exists for this library's users.
  *

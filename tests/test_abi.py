@@ -31,7 +31,7 @@ def test_header_declares_the_boundary():
     assert names == sorted(["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status",
                             "attn_status_string", "attn_num_kernel_launches", "attn_shutdown",
                             "attn_fwd_noalloc", "attn_hadamard_quant_qkv", "attn_bwd",
-                            "attn_bwd_workspace_bytes", "attn_fwd_qk"])
+                            "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -157,8 +157,24 @@ def test_bwd_rejects_bad_arguments(L):
         assert f(*a) == ea.ATTN_ERR_UNSUPPORTED, dd
 
 
+def test_bwd_qk_rejects_bad_arguments(L):
+    f = L.attn_bwd_qk
+    ok = [P, P, P, P, P, P2, P2, P2, P2, P2, 1, 1, 128, 300, 128, 0.1, 1, 0, NULL]
+    for i in range(10):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for idx, val in [(12, 0), (13, 0), (13, -1), (15, 0.0), (16, 2), (17, 9)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+    a = list(ok)
+    a[14] = 256
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+
+
 def test_python_binding_has_same_names():
     for name in ["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status", "attn_status_string",
                  "attn_num_kernel_launches", "attn_shutdown", "attn_fwd_noalloc", "attn_hadamard_quant_qkv",
-                 "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_qk"]:
+                 "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk"]:
         assert callable(getattr(ea, name)), name
