@@ -49,6 +49,8 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd.restype = i
         L.attn_fwd_qk.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp]
         L.attn_fwd_qk.restype = i
+        L.attn_fwd_strided.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, vp, f, i, i, i, vp]
+        L.attn_fwd_strided.restype = i
         L.attn_hadamard_quant.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
         L.attn_hadamard_quant.restype = i
         L.attn_hadamard_quant_qkv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
@@ -184,6 +186,33 @@ def attn_fwd_qk(q, k, v, o=None, lse=None, scale=None, causal=False, o_dtype=Non
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
     _check(lib().attn_fwd_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d, s,
                              int(bool(causal)), ATTN_BF16, od, _stream_ptr(stream)), "attn_fwd_qk")
+    return o, lse
+
+
+def attn_fwd_strided(q, k, v, o=None, lse=None, scale=None, causal=False, o_dtype=None, stream=None):
+    """attn_fwd_qk on logical [B, H, N, d] bf16 views with any strides whose last one is 1, e.g.
+    ``x.view(B, N, H, d).transpose(1, 2)`` of a sequence-major projection; no copy is made.  ``o``
+    defaults to a tensor with q's memory order.  Returns ``(o, lse)``."""
+    import torch
+    B, H, Nq, d = _dims(q)
+    Bk, Hk, Nk, dk = _dims(k)
+    if (Bk, Hk, dk) != (B, H, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H, Nk, d] with q's B, H, d")
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or t.stride(-1) != 1:
+            raise ValueError("q, k, v must be bf16 with a contiguous last dimension")
+    if o is None:
+        o = torch.empty_like(q, dtype=o_dtype or torch.bfloat16)
+    if o.shape != q.shape or o.stride(-1) != 1:
+        raise ValueError("o must be [B, H, Nq, d] with a contiguous last dimension")
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    strides = (ctypes.c_longlong * 12)(*[int(x) for t in (q, k, v, o) for x in t.stride()[:3]])
+    od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_fwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
+                                  ctypes.cast(strides, ctypes.c_void_p), s, int(bool(causal)), ATTN_BF16, od,
+                                  _stream_ptr(stream)), "attn_fwd_strided")
     return o, lse
 
 

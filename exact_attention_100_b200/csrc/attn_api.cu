@@ -86,6 +86,45 @@ bool encode_rows_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D tiled map for the forward kernels: dims (d, rows, heads, batch) with the caller's element
+// strides of a row, a head and a batch entry (d contiguous); box = 128 bytes x 128 rows x 1 x 1,
+// 128-byte swizzle, zero fill past the last row.
+bool encode_fwd_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N, int H,
+                    int B, long long sn, long long sh, long long sb) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(sn) * elem_bytes, static_cast<cuuint64_t>(sh) * elem_bytes,
+                                 static_cast<cuuint64_t>(sb) * elem_bytes};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), 128u, 1u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return g_encode(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Element strides (batch, head, row) of one [B, H, N, d] tensor; the forward's maps and its O
+// stores take any strides that are positive multiples of 8 elements below 2^36.  A stride of a
+// dimension of extent 1 is never used to address anything and is replaced by 8.
+struct Strides {
+  long long sb, sh, sn;
+};
+
+Strides contiguous_strides(int H, int N, int d) {
+  const long long sn = d, sh = sn * N;
+  return {sh * H, sh, sn};
+}
+
+bool canonical_strides(const long long* s, int B, int H, int N, Strides* out) {
+  long long v[3] = {s[0], s[1], s[2]};
+  const int ext[3] = {B, H, N};
+  for (int i = 0; i < 3; ++i) {
+    if (ext[i] == 1) v[i] = 8;
+    if (v[i] <= 0 || (v[i] & 7) != 0 || v[i] >= (1ll << 36)) return false;
+  }
+  *out = {v[0], v[1], v[2]};
+  return true;
+}
+
 int check_common(int B, int H, int N, float scale, int causal, int o_dtype) {
   if (B <= 0 || H <= 0 || N <= 0) return ATTN_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > 0x7FFFFFFFLL) return ATTN_ERR_INVALID_ARG;
@@ -103,6 +142,10 @@ void fill_params(ea::FwdParams& p, void* o, float* lse, int* status, int B, int 
   p.q_scale = p.k_scale = p.v_scale = nullptr;
   p.N = N;
   p.BH = B * H;
+  p.H = H;
+  p.o_sn = 0;  // set by the caller
+  p.o_sh = 0;
+  p.o_sb = 0;
   p.n_blocks = (N + 127) / 128;
   p.Nk = Nk;
   p.nbk = (Nk + 127) / 128;
@@ -141,9 +184,10 @@ unsigned long long attn_num_kernel_launches(void) { return g_launches.load(); }
 
 namespace {
 
-// attn_fwd and attn_fwd_qk: queries [BH, Nq, d], keys and values [BH, Nk, d].
+// attn_fwd, attn_fwd_qk and attn_fwd_strided: queries [B, H, Nq, d], keys and values
+// [B, H, Nk, d], output [B, H, Nq, d], each with element strides st[0..3] (q, k, v, o).
 int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk, int d,
-             float scale, int causal, int dtype, int o_dtype, void* stream) {
+             const Strides* st4, float scale, int causal, int dtype, int o_dtype, void* stream) {
   if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
     return ATTN_ERR_INVALID_ARG;
@@ -156,13 +200,17 @@ int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, i
   DeviceState* st = nullptr;
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
+  const Strides &sq = st4[0], &sk = st4[1], &sv = st4[2], &so = st4[3];
   CUtensorMap mq, mk, mv;
-  if (!encode_rows_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nq, B * H) ||
-      !encode_rows_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nk, B * H) ||
-      !encode_rows_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nk, B * H))
+  if (!encode_fwd_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nq, H, B, sq.sn, sq.sh, sq.sb) ||
+      !encode_fwd_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nk, H, B, sk.sn, sk.sh, sk.sb) ||
+      !encode_fwd_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nk, H, B, sv.sn, sv.sh, sv.sb))
     return ATTN_ERR_CUDA;
   ea::FwdParams p;
   fill_params(p, o, lse, st->status, B, H, Nq, Nk, ea::fwd_units_per_tile_pair(d), scale, causal, o_dtype);
+  p.o_sb = so.sb;
+  p.o_sh = so.sh;
+  p.o_sn = so.sn;
   if (ea::launch_attn_fwd_bf16(d, mq, mk, mv, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
@@ -175,12 +223,26 @@ extern "C" {
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
              float scale, int causal, int dtype, int o_dtype, void* stream) {
-  return fwd_bf16(q, k, v, o, lse, B, H, N, N, d, scale, causal, dtype, o_dtype, stream);
+  const Strides s = contiguous_strides(H, N, d);
+  const Strides st4[4] = {s, s, s, s};
+  return fwd_bf16(q, k, v, o, lse, B, H, N, N, d, st4, scale, causal, dtype, o_dtype, stream);
 }
 
 int attn_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
                 int d, float scale, int causal, int dtype, int o_dtype, void* stream) {
-  return fwd_bf16(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, o_dtype, stream);
+  const Strides sq = contiguous_strides(H, Nq, d), sk = contiguous_strides(H, Nk, d);
+  const Strides st4[4] = {sq, sk, sk, sq};
+  return fwd_bf16(q, k, v, o, lse, B, H, Nq, Nk, d, st4, scale, causal, dtype, o_dtype, stream);
+}
+
+int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                     int d, const long long* strides, float scale, int causal, int dtype, int o_dtype,
+                     void* stream) {
+  if (strides == nullptr || B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0) return ATTN_ERR_INVALID_ARG;
+  Strides st4[4];
+  for (int t = 0; t < 4; ++t)
+    if (!canonical_strides(strides + 3 * t, B, H, t == 1 || t == 2 ? Nk : Nq, &st4[t])) return ATTN_ERR_INVALID_ARG;
+  return fwd_bf16(q, k, v, o, lse, B, H, Nq, Nk, d, st4, scale, causal, dtype, o_dtype, stream);
 }
 
 int attn_hadamard_quant(const void* x, void* x8, float* scales, const signed char* signs, int B, int H, int N, int d,
@@ -248,13 +310,17 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_
   DeviceState* st = nullptr;
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
+  const Strides s = contiguous_strides(H, N, d);
   CUtensorMap mq, mk, mv;
-  if (!encode_rows_map(&mq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, B * H) ||
-      !encode_rows_map(&mk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, B * H) ||
-      !encode_rows_map(&mv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, B * H))
+  if (!encode_fwd_map(&mq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, H, B, s.sn, s.sh, s.sb) ||
+      !encode_fwd_map(&mk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, H, B, s.sn, s.sh, s.sb) ||
+      !encode_fwd_map(&mv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, H, B, s.sn, s.sh, s.sb))
     return ATTN_ERR_CUDA;
   ea::FwdParams p;
   fill_params(p, o, lse, st->status, B, H, N, N, 2, scale, causal, o_dtype);
+  p.o_sb = s.sb;
+  p.o_sh = s.sh;
+  p.o_sn = s.sn;
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.v_scale = v_scale;

@@ -343,7 +343,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         // O = 0 and LSE = -inf, written here; no MMA or epilogue event concerns it
         if (tile_row0 < p.N) {
           if (row_g < p.N) {
-            const size_t orow = (static_cast<size_t>(U.bh) * p.N + row_g) * D;
+            const long long orow =
+                (U.bh / p.H) * p.o_sb + (U.bh % p.H) * p.o_sh + static_cast<long long>(row_g) * p.o_sn;
             for (int c = 0; c < D; c += 4) {
               if (p.o_fp32)
                 *reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -507,7 +508,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         const float inv = ls > 0.f ? 1.f / ls : 0.f;  // a row with no visible key: O = 0
         const int row_g = tile * 128 + row;
         const bool valid = row_g < p.N;
-        const size_t orow = (static_cast<size_t>(bh) * p.N + row_g) * D;
+        const long long orow = (bh / p.H) * p.o_sb + (bh % p.H) * p.o_sh + static_cast<long long>(row_g) * p.o_sn;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t r[32];
@@ -716,8 +717,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         for (int q = 0; q < NQ; ++q)
 #pragma unroll
           for (int b = 0; b < C::kBoxes; ++b)
-            tma_load_3d(smem + C::kQOff + q * C::kTileBytes + b * C::kBoxBytes, &tmQ, q_full,
-                        b * (128 / E::kBytes), (U.tile0 + q) * 128, U.bh);
+            tma_load_4d(smem + C::kQOff + q * C::kTileBytes + b * C::kBoxBytes, &tmQ, q_full,
+                        b * (128 / E::kBytes), (U.tile0 + q) * 128, U.bh % p.H, U.bh / p.H);
         ++qit;
         for (int j = 0; j < U.n_max && ok; ++j) {
 #pragma unroll
@@ -728,8 +729,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
             uint8_t* dst = smem + C::kRingOff + s * C::kTileBytes;
 #pragma unroll
             for (int b = 0; b < C::kBoxes; ++b)
-              tma_load_3d(dst + b * C::kBoxBytes, kv ? &tmV : &tmK, &full[s], b * (128 / E::kBytes), j * 128,
-                          U.bh);
+              tma_load_4d(dst + b * C::kBoxBytes, kv ? &tmV : &tmK, &full[s], b * (128 / E::kBytes), j * 128,
+                          U.bh % p.H, U.bh / p.H);
             ++it;
           }
         }

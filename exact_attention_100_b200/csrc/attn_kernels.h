@@ -20,6 +20,10 @@ struct FwdParams {
   int Nk;           // key length (rows of K, V)
   int nbk;          // ceil(Nk / 128): K/V blocks
   int off;          // Nk - N: causal key j is visible to query i iff j <= i + off (bottom-right)
+  int H;            // heads (bh = b * H + h)
+  long long o_sb;   // element strides of O for batch, head and row (d is contiguous)
+  long long o_sh;
+  long long o_sn;
   int n_pairs;      // ceil(n_blocks / Q tiles per unit)
   int num_units;    // BH * n_pairs
   float scale_log2; // softmax scale * log2(e)
@@ -33,6 +37,8 @@ int fwd_units_per_tile_pair(int d);
 // Sets the kernels' shared-memory attributes on the current device (once per device).
 cudaError_t setup_kernels_for_current_device();
 
+// The forward kernels read Q, K and V through 4-D maps (d, rows, heads, batch) with a box of
+// 128 bytes x 128 rows x 1 x 1: any layout with d contiguous and 16-byte-aligned strides.
 cudaError_t launch_attn_fwd_bf16(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                                  const FwdParams& p, int num_sms, cudaStream_t stream);
 

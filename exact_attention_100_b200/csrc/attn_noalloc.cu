@@ -91,13 +91,16 @@ int noalloc_setup(NoAllocDevice** out) {
   return ATTN_OK;
 }
 
-bool encode_bf16_rows(CUtensorMap* map, const void* base, int d, int N, int BH) {
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                                 static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(N)};
-  const cuuint32_t box[3] = {64u, 128u, 1u};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  return g_encode_fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+// Contiguous [B, H, N, d] bf16 as the forward kernel's 4-D map (d, rows, heads, batch).
+bool encode_bf16_rows(CUtensorMap* map, const void* base, int d, int N, int H, int B) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t row = static_cast<cuuint64_t>(d) * 2;
+  const cuuint64_t strides[3] = {row, row * static_cast<cuuint64_t>(N),
+                                 row * static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(H)};
+  const cuuint32_t box[4] = {64u, 128u, 1u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return g_encode_fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -121,8 +124,8 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
   int rc = noalloc_setup(&st);
   if (rc != ATTN_OK) return rc;
   CUtensorMap mq, mk, mv;
-  if (!encode_bf16_rows(&mq, q, d, N, B * H) || !encode_bf16_rows(&mk, k, d, N, B * H) ||
-      !encode_bf16_rows(&mv, v, d, N, B * H))
+  if (!encode_bf16_rows(&mq, q, d, N, H, B) || !encode_bf16_rows(&mk, k, d, N, H, B) ||
+      !encode_bf16_rows(&mv, v, d, N, H, B))
     return ATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the status word must start at zero: the array keeps whatever the previous call left
@@ -135,6 +138,10 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
   p.q_scale = p.k_scale = p.v_scale = nullptr;
   p.N = N;
   p.BH = B * H;
+  p.H = H;
+  p.o_sn = d;
+  p.o_sh = static_cast<long long>(d) * N;
+  p.o_sb = p.o_sh * H;
   p.n_blocks = (N + 127) / 128;
   p.Nk = N;
   p.nbk = p.n_blocks;

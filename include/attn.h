@@ -93,6 +93,26 @@ int attn_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse
                 int dtype, int o_dtype, void* stream);
 
 /*
+ * attn_fwd_strided -- attn_fwd_qk on tensors laid out with arbitrary strides, e.g. the
+ * [B, N, H, d] (sequence-major) layout of a fused QKV projection, without a transpose copy.
+ *
+ *   q, k, v, o  logical [B, H, N, d] tensors (N = Nq for q and o, Nk for k and v); element
+ *               (b, h, n, c) of tensor t sits at  base_t + b*sb_t + h*sh_t + n*sn_t + c
+ *               elements: the head dimension is contiguous.
+ *   strides     HOST pointer to 12 int64 values, read during the call and not kept:
+ *               {sb, sh, sn} for q, then k, v and o, in elements.  Each stride of a dimension
+ *               of extent > 1 must be a positive multiple of 8 below 2^36 (16-byte rows for the
+ *               tensor-memory-access unit); the stride of an extent-1 dimension is ignored.
+ *               Outputs must not overlap the inputs or one another.
+ *   lse         [B, H, Nq] float32, contiguous, or NULL.
+ * Other arguments, causal alignment, arithmetic and errors as for attn_fwd_qk, which is
+ * attn_fwd_strided with contiguous strides; a bad stride returns ATTN_ERR_INVALID_ARG.
+ */
+int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int Nq, int Nk, int d, const long long* strides,
+                     float scale, int causal, int dtype, int o_dtype, void* stream);
+
+/*
  * attn_hadamard_quant -- random-sign Hadamard transform plus per-block E4M3 quantisation.
  *
  *   x       [B, H, N, d] bf16, device (read).

@@ -31,7 +31,7 @@ def test_header_declares_the_boundary():
     assert names == sorted(["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status",
                             "attn_status_string", "attn_num_kernel_launches", "attn_shutdown",
                             "attn_fwd_noalloc", "attn_hadamard_quant_qkv", "attn_bwd",
-                            "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk"])
+                            "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -128,6 +128,43 @@ def test_fwd_qk_rejects_bad_arguments(L):
     assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
 
 
+def test_fwd_strided_rejects_bad_arguments(L):
+    f = L.attn_fwd_strided
+    B, H, Nq, Nk, d = 2, 4, 128, 300, 128
+
+    def strides(vals):
+        return ctypes.cast((ctypes.c_longlong * 12)(*vals), ctypes.c_void_p)
+
+    # [B, N, H, d] sequence-major strides for all four tensors
+    good = [Nq * H * d, d, H * d, Nk * H * d, d, H * d, Nk * H * d, d, H * d, Nq * H * d, d, H * d]
+    ok = [P, P, P, P2, NULL, B, H, Nq, Nk, d, strides(good), 0.1, 1, 0, 0, NULL]
+    a = list(ok)
+    a[10] = NULL
+    assert f(*a) == ea.ATTN_ERR_INVALID_ARG
+    for i in range(4):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    # strides that are not positive multiples of 8 elements, or too large
+    for pos, val in [(0, 0), (1, 4), (2, -8), (5, 12), (11, 1), (9, 1 << 36)]:
+        bad = list(good)
+        bad[pos] = val
+        a = list(ok)
+        a[10] = strides(bad)
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (pos, val)
+    # a stride of an extent-1 dimension is ignored: with H = 1 the head strides may be anything,
+    # so the call reaches the head-dimension check
+    bad = list(good)
+    bad[1] = bad[4] = bad[7] = bad[10] = 3
+    a = list(ok)
+    a[6], a[9], a[10] = 1, 96, strides(bad)
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+    for idx, val in [(7, 0), (8, 0), (11, 0.0), (12, 3), (14, 5)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+
+
 def test_bwd_workspace_bytes(L):
     assert L.attn_bwd_workspace_bytes(1, 1, 1) == 2 * 128 * 4
     assert L.attn_bwd_workspace_bytes(2, 16, 8192) == 2 * 32 * 8192 * 4
@@ -176,5 +213,5 @@ def test_bwd_qk_rejects_bad_arguments(L):
 def test_python_binding_has_same_names():
     for name in ["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status", "attn_status_string",
                  "attn_num_kernel_launches", "attn_shutdown", "attn_fwd_noalloc", "attn_hadamard_quant_qkv",
-                 "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk"]:
+                 "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided"]:
         assert callable(getattr(ea, name)), name
