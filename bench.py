@@ -320,6 +320,7 @@ def run_ours(args):
 
     fp8 = fp8_section(args, dev, rank) if not args.no_fp8 else None
     bwd = bwd_section(args, dev, rank) if not args.no_bwd else None
+    varlen = varlen_section(args, dev, rank) if not args.no_varlen else None
     barrier()
     if rank == 0:
         peaks = load_peaks()
@@ -354,6 +355,8 @@ def run_ours(args):
             line["fp8"] = fp8
         if bwd is not None:
             line["bwd"] = bwd
+        if varlen is not None:
+            line["varlen"] = varlen
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -424,6 +427,67 @@ def fp8_section(args, dev, rank):
     except Exception as e:  # the E4M3 forward reports unsupported until it is built
         out["forward"] = {"unavailable": str(e)}
     return out
+
+
+VARLEN_WORKLOAD = dict(total=16384, lo=512, hi=4096, H=16, d=128, causal=True, seed=11)
+
+
+def varlen_lengths(total, lo, hi, seed):
+    """Sequence lengths drawn uniformly from [lo, hi] until they hold `total` tokens (the last one
+    cut to fit)."""
+    from exact_attention_100_b200.inputs import uniform_lengths
+    pool = [int(x) for x in uniform_lengths(4 * total // lo + 1, lo, hi, seed=seed)]
+    out, acc = [], 0
+    for n in pool:
+        n = min(n, total - acc)
+        out.append(n)
+        acc += n
+        if acc == total:
+            break
+    return out
+
+
+def varlen_section(args, dev, rank):
+    """Times attn_fwd_varlen on a packed batch holding as many query tokens as the headline
+    (2 x 8192), in sequences of 512..4096 tokens; FLOPs are counted per sequence."""
+    import torch
+    import exact_attention_100_b200 as ea
+    from exact_attention_100_b200.inputs import normal_qkv_packed
+    w = VARLEN_WORKLOAD
+    lens = varlen_lengths(w["total"], w["lo"], w["hi"], w["seed"])
+    H, d, causal = w["H"], w["d"], w["causal"]
+    qn, kn, vn, cq, ck = normal_qkv_packed(lens, lens, H, d, seed=w["seed"] + rank)
+    q, k, v = (torch.from_numpy(a).to(torch.bfloat16).to(dev) for a in (qn, kn, vn))
+    cu_q, cu_k = (torch.from_numpy(a).to(dev) for a in (cq, ck))
+    stream = torch.cuda.current_stream()
+    o = torch.empty_like(q)
+    lse = torch.empty((H, q.shape[0]), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        ea.attn_fwd_varlen(q, k, v, cu_q, cu_k, max(lens), o=o, lse=lse, causal=causal, stream=stream)
+
+    for _ in range(3):
+        step()
+    steps = max(3, min(args.steps, 50))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    flops = sum(attn_flops(1, H, n, d, causal) for n in lens)
+    peaks = load_peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": f"bf16 packed varlen fwd, {len(lens)} sequences of {w['lo']}..{w['hi']} tokens "
+                        f"(total {w['total']}), H={H} d={d} causal",
+            "lengths": lens, "ms": ms, "achieved_tflops": tf, "peak_tflops": float(peaks["bf16_tflops"]),
+            "frac": tf / float(peaks["bf16_tflops"]), "bound": "tensor", "flops_per_call": flops,
+            "flops_note": "sum over sequences of 4 H d N^2 / 2 (causal), as the headline counts",
+            "peak_source": peaks["source"]}
 
 
 def bwd_section(args, dev, rank):
@@ -543,6 +607,7 @@ def main():
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv", "bwd"], default=None,
                     help="run --reps untimed calls of one entry point (for an ncu capture) and exit")

@@ -51,6 +51,8 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_qk.restype = i
         L.attn_fwd_strided.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, vp, f, i, i, i, vp]
         L.attn_fwd_strided.restype = i
+        L.attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, f, i, i, i, vp]
+        L.attn_fwd_varlen.restype = i
         L.attn_hadamard_quant.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
         L.attn_hadamard_quant.restype = i
         L.attn_hadamard_quant_qkv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
@@ -213,6 +215,46 @@ def attn_fwd_strided(q, k, v, o=None, lse=None, scale=None, causal=False, o_dtyp
     _check(lib().attn_fwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
                                   ctypes.cast(strides, ctypes.c_void_p), s, int(bool(causal)), ATTN_BF16, od,
                                   _stream_ptr(stream)), "attn_fwd_strided")
+    return o, lse
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, o=None, lse=None, scale=None,
+                    causal=False, o_dtype=None, stream=None):
+    """Packed variable-length batch: ``q`` [total_q, H, d], ``k``, ``v`` [total_k, H, d] bf16 (any
+    row and head strides, last dimension contiguous); sequence b owns query rows
+    ``cu_seqlens_q[b]:cu_seqlens_q[b+1]`` and key rows ``cu_seqlens_k[b]:cu_seqlens_k[b+1]``
+    (int32 cuda tensors of B + 1 offsets); ``max_seqlen_q`` bounds every query length.
+    Returns ``(o [total_q, H, d], lse [H, total_q])``.  Offsets that break their rules are
+    reported by the next :func:`attn_device_status`."""
+    import torch
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape:
+        raise ValueError("q must be [total_q, H, d], k and v [total_k, H, d]")
+    total_q, H, d = (int(x) for x in q.shape)
+    total_k = int(k.shape[0])
+    if (int(k.shape[1]), int(k.shape[2])) != (H, d):
+        raise ValueError("k and v must have q's H and d")
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or t.stride(-1) != 1:
+            raise ValueError("q, k, v must be bf16 with a contiguous last dimension")
+    for c in (cu_seqlens_q, cu_seqlens_k):
+        if c.dtype != torch.int32 or c.dim() != 1 or not c.is_contiguous() or not c.is_cuda:
+            raise ValueError("cu_seqlens must be contiguous int32 cuda tensors")
+    if cu_seqlens_k.shape != cu_seqlens_q.shape:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B + 1 entries")
+    B = int(cu_seqlens_q.shape[0]) - 1
+    if o is None:
+        o = torch.empty_like(q, dtype=o_dtype or torch.bfloat16)
+    if o.shape != q.shape or o.stride(-1) != 1:
+        raise ValueError("o must be [total_q, H, d] with a contiguous last dimension")
+    if lse is None:
+        lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    strides = (ctypes.c_longlong * 8)(*[int(x) for t in (q, k, v, o) for x in t.stride()[:2]])
+    od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q),
+                                 _ptr(cu_seqlens_k), B, H, total_q, total_k, int(max_seqlen_q), d,
+                                 ctypes.cast(strides, ctypes.c_void_p), s, int(bool(causal)), ATTN_BF16, od,
+                                 _stream_ptr(stream)), "attn_fwd_varlen")
     return o, lse
 
 

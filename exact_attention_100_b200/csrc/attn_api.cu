@@ -125,6 +125,11 @@ bool canonical_strides(const long long* s, int B, int H, int N, Strides* out) {
   return true;
 }
 
+// The persistent kernels index their work units with int: B * H * ceil(N / 128) must fit.
+bool units_fit(int B, int H, int N) {
+  return static_cast<long long>(B) * H * ((static_cast<long long>(N) + 127) / 128) < 0x7FFFFFFFLL;
+}
+
 int check_common(int B, int H, int N, float scale, int causal, int o_dtype) {
   if (B <= 0 || H <= 0 || N <= 0) return ATTN_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > 0x7FFFFFFFLL) return ATTN_ERR_INVALID_ARG;
@@ -140,6 +145,8 @@ void fill_params(ea::FwdParams& p, void* o, float* lse, int* status, int B, int 
   p.lse = lse;
   p.status = status;
   p.q_scale = p.k_scale = p.v_scale = nullptr;
+  p.cu_q = p.cu_k = nullptr;
+  p.total_q = p.total_k = 0;
   p.N = N;
   p.BH = B * H;
   p.H = H;
@@ -193,7 +200,7 @@ int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, i
     return ATTN_ERR_INVALID_ARG;
   int rc = check_common(B, H, Nq, scale, causal, o_dtype);
   if (rc != ATTN_OK) return rc;
-  if (Nk <= 0) return ATTN_ERR_INVALID_ARG;
+  if (Nk <= 0 || !units_fit(B, H, Nq)) return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_BF16) return dtype == ATTN_E4M3 || dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
 
@@ -243,6 +250,55 @@ int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float
   for (int t = 0; t < 4; ++t)
     if (!canonical_strides(strides + 3 * t, B, H, t == 1 || t == 2 ? Nk : Nq, &st4[t])) return ATTN_ERR_INVALID_ARG;
   return fwd_bf16(q, k, v, o, lse, B, H, Nq, Nk, d, st4, scale, causal, dtype, o_dtype, stream);
+}
+
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
+                    const int* cu_seqlens_k, int B, int H, int total_q, int total_k, int max_seqlen_q, int d,
+                    const long long* strides, float scale, int causal, int dtype, int o_dtype, void* stream) {
+  if (!q || !k || !v || !o || !cu_seqlens_q || !cu_seqlens_k || !strides) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
+    return ATTN_ERR_INVALID_ARG;
+  int rc = check_common(B, H, max_seqlen_q, scale, causal, o_dtype);
+  if (rc != ATTN_OK) return rc;
+  // row coordinates (offset + 128 * tile) stay inside int
+  constexpr int kMaxRows = 0x7FFFFFFF - (1 << 20);
+  if (total_q <= 0 || total_k <= 0 || total_q > kMaxRows || total_k > kMaxRows || max_seqlen_q > kMaxRows)
+    return ATTN_ERR_INVALID_ARG;
+  if (max_seqlen_q > total_q) max_seqlen_q = total_q;  // no sequence is longer than the tensor
+  if (!units_fit(B, H, max_seqlen_q)) return ATTN_ERR_INVALID_ARG;
+  Strides st4[4];
+  for (int t = 0; t < 4; ++t) {
+    const long long s3[3] = {8, strides[2 * t + 1], strides[2 * t]};  // {batch (unused), head, row}
+    if (!canonical_strides(s3, 1, H, t == 1 || t == 2 ? total_k : total_q, &st4[t])) return ATTN_ERR_INVALID_ARG;
+  }
+  if (dtype != ATTN_BF16) return dtype == ATTN_E4M3 || dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  const Strides &sq = st4[0], &sk = st4[1], &sv = st4[2], &so = st4[3];
+  CUtensorMap mq, mk, mv;
+  if (!encode_fwd_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, total_q, H, 1, sq.sn, sq.sh, sq.sb) ||
+      !encode_fwd_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, total_k, H, 1, sk.sn, sk.sh, sk.sb) ||
+      !encode_fwd_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, total_k, H, 1, sv.sn, sv.sh, sv.sb))
+    return ATTN_ERR_CUDA;
+  ea::FwdParams p;
+  // sized for B sequences of max_seqlen_q queries each; shorter ones skip the surplus units
+  fill_params(p, o, lse, st->status, B, H, max_seqlen_q, total_k, ea::fwd_units_per_tile_pair(d), scale, causal,
+              o_dtype);
+  p.o_sb = 0;
+  p.o_sh = so.sh;
+  p.o_sn = so.sn;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  if (ea::launch_attn_fwd_bf16(d, mq, mk, mv, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return ATTN_OK;
 }
 
 int attn_hadamard_quant(const void* x, void* x8, float* scales, const signed char* signs, int B, int H, int N, int d,
@@ -420,7 +476,7 @@ int attn_device_status(void* stream) {
   if (host != 0) {
     if (cudaMemsetAsync(st->status, 0, sizeof(int), s) != cudaSuccess) return ATTN_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
-    return ATTN_ERR_TIMEOUT;
+    return (host & ea::kDevStatusTimeout) ? ATTN_ERR_TIMEOUT : ATTN_ERR_INVALID_ARG;
   }
   return ATTN_OK;
 }

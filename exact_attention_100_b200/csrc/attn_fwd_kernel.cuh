@@ -107,32 +107,84 @@ struct FwdCfg {
 
 enum : int { kEvRescale = 0, kEvEpilogue = 1, kEvEnd = 2 };
 
-struct Unit {
-  int bh;
-  int tile0;   // index of the first 128-row Q tile of the unit
-  int n[2];    // K/V blocks each Q tile visits (0: the tile lies past the sequence end)
-  int n_max;
+// The sequence of one (batch entry, head) pair.  Fixed-length batches take every field from
+// the parameters; packed variable-length batches (VL) read the sequence's row range from the
+// offset arrays.
+struct Seq {
+  int h, bc;        // head; batch coordinate of Q, K, V and O (0 for packed sequences)
+  int N, Nk;        // query and key lengths
+  int nbk;          // ceil(Nk / 128)
+  int off;          // Nk - N: key j is visible to query i iff j <= i + off (causal)
+  int q0, k0;       // first row of the sequence in Q/O and in K/V (0 unless packed)
+  long long lse0;   // LSE index of the sequence's row 0 for this head
+  bool bad;         // packed offsets out of order, outside the tensors or too long
 };
 
-template <int NQ>
+template <bool VL>
+__device__ __forceinline__ Seq seq_of(int bh, const FwdParams& p) {
+  Seq s;
+  const int b = bh / p.H;
+  s.h = bh - b * p.H;
+  s.bad = false;
+  if constexpr (!VL) {
+    s.bc = b;
+    s.N = p.N;
+    s.Nk = p.Nk;
+    s.nbk = p.nbk;
+    s.off = p.off;
+    s.q0 = s.k0 = 0;
+    s.lse0 = static_cast<long long>(bh) * p.N;
+  } else {
+    int q0 = __ldg(p.cu_q + b), q1 = __ldg(p.cu_q + b + 1);
+    int k0 = __ldg(p.cu_k + b), k1 = __ldg(p.cu_k + b + 1);
+    // p.N is the longest query length the launch was sized for; a sequence that breaks a
+    // bound is treated as empty (nothing read or written for it) and reported
+    if (!(0 <= q0 && q0 <= q1 && q1 <= p.total_q && q1 - q0 <= p.N && 0 <= k0 && k0 <= k1 && k1 <= p.total_k)) {
+      s.bad = true;
+      q0 = q1 = k0 = k1 = 0;
+    }
+    s.bc = 0;
+    s.N = q1 - q0;
+    s.Nk = k1 - k0;
+    s.nbk = (s.Nk + 127) / 128;
+    s.off = s.Nk - s.N;
+    s.q0 = q0;
+    s.k0 = k0;
+    s.lse0 = static_cast<long long>(s.h) * p.total_q + q0;
+  }
+  return s;
+}
+
+struct Unit {
+  int bh;
+  int tile0;     // index of the first 128-row Q tile of the unit
+  int n[2];      // K/V blocks each Q tile visits (0: no visible key, or past the sequence end)
+  int n_max;
+  bool present;  // the unit's first tile starts inside its sequence (always, unless packed)
+  Seq s;
+};
+
+template <int NQ, bool VL>
 __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
   Unit U;
   const int r = u / p.BH;
   U.bh = u - r * p.BH;
+  U.s = seq_of<VL>(U.bh, p);
   const int pair = p.causal ? (p.n_pairs - 1 - r) : r;  // causal: longest units first
   U.tile0 = pair * NQ;
+  U.present = U.tile0 * 128 < U.s.N;
   U.n_max = 0;
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     const int t = U.tile0 + q;
     int n = 0;
-    if (q < NQ && t * 128 < p.N) {
+    if (q < NQ && t * 128 < U.s.N) {
       if (!p.causal) {
-        n = p.nbk;
+        n = U.s.nbk;
       } else {
         // keys up to the tile's last row + off (bottom-right alignment); 0 if even it sees none
-        const int last = min(t * 128 + 127, p.N - 1) + p.off;
-        n = last < 0 ? 0 : min(last / 128 + 1, p.nbk);
+        const int last = min(t * 128 + 127, U.s.N - 1) + U.s.off;
+        n = last < 0 ? 0 : min(last / 128 + 1, U.s.nbk);
       }
     }
     U.n[q] = n;
@@ -247,7 +299,7 @@ __device__ __forceinline__ float softmax_block(uint32_t (&r)[128], uint32_t* pk,
   return acc[0] + acc[1];
 }
 
-template <int D, int NQ, class E>
+template <int D, int NQ, class E, bool VL>
 __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -334,30 +386,31 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
     for (int k = 0; ok; ++k) {
       const int u = unit_index(k);
       if (u >= p.num_units) break;
-      const Unit U = decode_unit<NQ>(u, p);
+      const Unit U = decode_unit<NQ, VL>(u, p);
+      const Seq& S = U.s;
       const int n = U.n[q];
       const int tile_row0 = (U.tile0 + q) * 128;
       const int row_g = tile_row0 + row;
       if (n == 0) {
-        // a tile inside the sequence whose rows see no key (causal, more queries than keys):
-        // O = 0 and LSE = -inf, written here; no MMA or epilogue event concerns it
-        if (tile_row0 < p.N) {
-          if (row_g < p.N) {
-            const long long orow =
-                (U.bh / p.H) * p.o_sb + (U.bh % p.H) * p.o_sh + static_cast<long long>(row_g) * p.o_sn;
+        // a tile inside the sequence whose rows see no key (causal, more queries than keys, or
+        // an empty key sequence): O = 0 and LSE = -inf, written here; no MMA or epilogue event
+        // concerns it.  A tile past the sequence end is skipped by every role.
+        if (tile_row0 < S.N) {
+          if (row_g < S.N) {
+            const long long orow = S.bc * p.o_sb + S.h * p.o_sh + static_cast<long long>(S.q0 + row_g) * p.o_sn;
             for (int c = 0; c < D; c += 4) {
               if (p.o_fp32)
                 *reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
               else
                 *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.o) + orow + c) = make_uint2(0u, 0u);
             }
-            if (p.lse != nullptr) p.lse[static_cast<size_t>(U.bh) * p.N + row_g] = -INFINITY;
+            if (p.lse != nullptr) p.lse[S.lse0 + row_g] = -INFINITY;
           }
         }
         continue;
       }
-      int lim_row = p.Nk;  // keys [0, lim_row) are visible to this row (<= 0: none)
-      if (p.causal) lim_row = min(lim_row, row_g + p.off + 1);
+      int lim_row = S.Nk;  // keys [0, lim_row) are visible to this row (<= 0: none)
+      if (p.causal) lim_row = min(lim_row, row_g + S.off + 1);
       float c_base = p.scale_log2;
       float ps_log2_base = 0.f, l_div = 1.f;
       const float* ks = nullptr;
@@ -397,7 +450,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         uint32_t r[128];
         tmem_ld_row128(tS, r);
         const int key0 = j * 128;
-        const bool need_mask = (key0 + 128 > p.Nk) || (p.causal && key0 + 127 > tile_row0 + p.off);
+        const bool need_mask = (key0 + 128 > S.Nk) || (p.causal && key0 + 127 > tile_row0 + S.off);
         if (need_mask) {
           const int lim = lim_row - key0;
 #pragma unroll
@@ -507,8 +560,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         const float ls = row_l[(q * 2 + uslot) * 128 + row];
         const float inv = ls > 0.f ? 1.f / ls : 0.f;  // a row with no visible key: O = 0
         const int row_g = tile * 128 + row;
-        const bool valid = row_g < p.N;
-        const long long orow = (bh / p.H) * p.o_sb + (bh % p.H) * p.o_sh + static_cast<long long>(row_g) * p.o_sn;
+        const Seq S = seq_of<VL>(bh, p);
+        const bool valid = row_g < S.N;
+        const long long orow = S.bc * p.o_sb + S.h * p.o_sh + static_cast<long long>(S.q0 + row_g) * p.o_sn;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t r[32];
@@ -534,7 +588,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
             }
           }
         }
-        if (valid && p.lse != nullptr) p.lse[static_cast<size_t>(bh) * p.N + row_g] = lse2 * kLn2;
+        if (valid && p.lse != nullptr) p.lse[S.lse0 + row_g] = lse2 * kLn2;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) bar_arrive(&o_free[q]);
@@ -598,7 +652,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         return true;
       };
       // P.V of tile q for block j: wait for P, keep O safe (epilogue / lazy rescale), issue.
-      auto pv_step = [&](int q, int j, const Unit& U, uint32_t vslot, uint32_t buf) {
+      // n_q: K/V blocks of tile q in this unit; bh and tile0 identify the unit for its epilogue
+      auto pv_step = [&](int q, int j, int n_q, int bh, int tile0, uint32_t vslot, uint32_t buf) {
         // P of this block sits in S buffer `buf`; that buffer's p_full completes once per use
         const uint32_t pphase = (C::kSBufs == NQ) ? (pc[q] & 1u) : ((pc[q] >> 1) & 1u);
         if (!wait_bar(&p_full[buf], pphase, ab)) return false;
@@ -617,10 +672,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         }
         tc_fence_after();
         issue_pv(q, vslot, buf, j > 0);
-        if (j == U.n[q] - 1) {
+        if (j == n_q - 1) {
           // uc[q] was counted at j == 0 of this unit: the softmax wrote slot (uc[q] - 1) & 1
           tc_commit(&o_done[q]);
-          if (!push_event(kEvEpilogue, q, od[q]++, U.bh, U.tile0 + q, (uc[q] - 1u) & 1u)) return false;
+          if (!push_event(kEvEpilogue, q, od[q]++, bh, tile0 + q, (uc[q] - 1u) & 1u)) return false;
         }
         ++pc[q];
         return true;
@@ -630,7 +685,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int u = unit_index(k);
         if (u >= p.num_units) break;
-        const Unit U = decode_unit<NQ>(u, p);
+        const Unit U = decode_unit<NQ, VL>(u, p);
+        if constexpr (VL) {
+          if (!U.present) continue;  // past its sequence's end: the producer skips it too
+        }
         const uint32_t base = it;  // ring index of K_0; K_j = base + 2j, V_j = base + 2j + 1
         it += 2u * U.n_max;
         ok = wait_bar(q_full, qit & 1u, ab);
@@ -657,14 +715,14 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
             // trip, which here overlaps the softmax instead of sitting between P.V and S
             if (!(ok = wait_loaded(vi))) break;
             if (more && !(ok = wait_loaded(ki))) break;
-            if (j < U.n[0] && !(ok = pv_step(0, j, U, slot_of(vi), 0))) break;
+            if (j < U.n[0] && !(ok = pv_step(0, j, U.n[0], U.bh, U.tile0, slot_of(vi), 0))) break;
             if (more) {
               if (j + 1 < U.n[0]) {
                 issue_s(0, slot_of(ki), 0);
                 tc_commit(&s_full[0]);
               }
             }
-            if (j < U.n[1] && !(ok = pv_step(1, j, U, slot_of(vi), 1))) break;
+            if (j < U.n[1] && !(ok = pv_step(1, j, U.n[1], U.bh, U.tile0, slot_of(vi), 1))) break;
             tc_commit(&empty[slot_of(vi)]);
             if (more) {
               if (j + 1 < U.n[1]) {
@@ -694,7 +752,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
               if (j + 2 == U.n_max) tc_commit(q_empty);
             }
             if (!(ok = wait_loaded(vi))) break;
-            if (!(ok = pv_step(0, j, U, slot_of(vi), pbuf))) break;
+            if (!(ok = pv_step(0, j, U.n[0], U.bh, U.tile0, slot_of(vi), pbuf))) break;
             tc_commit(&empty[slot_of(vi)]);
           }
         }
@@ -710,7 +768,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int u = unit_index(k);
         if (u >= p.num_units) break;
-        const Unit U = decode_unit<NQ>(u, p);
+        const Unit U = decode_unit<NQ, VL>(u, p);
+        const Seq& S = U.s;
+        if constexpr (VL) {
+          if (S.bad && U.tile0 == 0) atomicOr(p.status, kDevStatusBadSeqlens);
+          if (!U.present) continue;
+        }
         if (qit > 0 && !(ok = wait_bar(q_empty, (qit - 1u) & 1u, ab))) break;
         bar_arrive_expect_tx(q_full, NQ * C::kTileBytes);
 #pragma unroll
@@ -718,7 +781,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
 #pragma unroll
           for (int b = 0; b < C::kBoxes; ++b)
             tma_load_4d(smem + C::kQOff + q * C::kTileBytes + b * C::kBoxBytes, &tmQ, q_full,
-                        b * (128 / E::kBytes), (U.tile0 + q) * 128, U.bh % p.H, U.bh / p.H);
+                        b * (128 / E::kBytes), S.q0 + (U.tile0 + q) * 128, S.h, S.bc);
         ++qit;
         for (int j = 0; j < U.n_max && ok; ++j) {
 #pragma unroll
@@ -729,8 +792,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
             uint8_t* dst = smem + C::kRingOff + s * C::kTileBytes;
 #pragma unroll
             for (int b = 0; b < C::kBoxes; ++b)
-              tma_load_4d(dst + b * C::kBoxBytes, kv ? &tmV : &tmK, &full[s], b * (128 / E::kBytes), j * 128,
-                          U.bh % p.H, U.bh / p.H);
+              tma_load_4d(dst + b * C::kBoxBytes, kv ? &tmV : &tmK, &full[s], b * (128 / E::kBytes), S.k0 + j * 128,
+                          S.h, S.bc);
             ++it;
           }
         }
@@ -751,18 +814,18 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
   }
 }
 
-template <int D, int NQ, class E>
+template <int D, int NQ, class E, bool VL = false>
 cudaError_t set_fwd_smem_attr() {
-  return cudaFuncSetAttribute(attn_fwd_kernel<D, NQ, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(attn_fwd_kernel<D, NQ, E, VL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               FwdCfg<D, NQ, E>::kSmemAlloc);
 }
 
-template <int D, int NQ, class E>
+template <int D, int NQ, class E, bool VL = false>
 cudaError_t launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const FwdParams& p,
                        int num_sms, cudaStream_t stream) {
   using C = FwdCfg<D, NQ, E>;
   const int grid = p.num_units < num_sms ? p.num_units : num_sms;
-  attn_fwd_kernel<D, NQ, E><<<grid, C::kThreads, C::kSmemAlloc, stream>>>(q, k, v, p);
+  attn_fwd_kernel<D, NQ, E, VL><<<grid, C::kThreads, C::kSmemAlloc, stream>>>(q, k, v, p);
   return cudaGetLastError();
 }
 

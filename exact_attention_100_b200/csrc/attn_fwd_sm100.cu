@@ -9,18 +9,25 @@ cudaError_t setup_fwd_bf16_kernels() {
   cudaError_t e = set_fwd_smem_attr<64, 2, ElemBf16>();
   if (e == cudaSuccess) e = set_fwd_smem_attr<128, 2, ElemBf16>();
   if (e == cudaSuccess) e = set_fwd_smem_attr<256, 1, ElemBf16>();
+  if (e == cudaSuccess) e = set_fwd_smem_attr<64, 2, ElemBf16, true>();
+  if (e == cudaSuccess) e = set_fwd_smem_attr<128, 2, ElemBf16, true>();
+  if (e == cudaSuccess) e = set_fwd_smem_attr<256, 1, ElemBf16, true>();
   return e;
 }
 
 cudaError_t launch_attn_fwd_bf16(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                                  const FwdParams& p, int num_sms, cudaStream_t stream) {
+  const bool vl = p.cu_q != nullptr;
   switch (d) {
     case 64:
-      return launch_fwd<64, 2, ElemBf16>(q, k, v, p, num_sms, stream);
+      return vl ? launch_fwd<64, 2, ElemBf16, true>(q, k, v, p, num_sms, stream)
+                : launch_fwd<64, 2, ElemBf16>(q, k, v, p, num_sms, stream);
     case 128:
-      return launch_fwd<128, 2, ElemBf16>(q, k, v, p, num_sms, stream);
+      return vl ? launch_fwd<128, 2, ElemBf16, true>(q, k, v, p, num_sms, stream)
+                : launch_fwd<128, 2, ElemBf16>(q, k, v, p, num_sms, stream);
     case 256:
-      return launch_fwd<256, 1, ElemBf16>(q, k, v, p, num_sms, stream);
+      return vl ? launch_fwd<256, 1, ElemBf16, true>(q, k, v, p, num_sms, stream)
+                : launch_fwd<256, 1, ElemBf16>(q, k, v, p, num_sms, stream);
     default:
       return cudaErrorInvalidValue;
   }

@@ -6,6 +6,10 @@
 
 namespace ea {
 
+// Device status word bits (OR-ed into the library's per-device status word).
+constexpr int kDevStatusTimeout = 1;
+constexpr int kDevStatusBadSeqlens = 2;  // packed-sequence offsets that break their bounds
+
 // Parameters of the attention forward kernels (bf16 and E4M3).
 struct FwdParams {
   void* o;          // [BH, N, d] bf16 or f32
@@ -29,6 +33,14 @@ struct FwdParams {
   float scale_log2; // softmax scale * log2(e)
   int causal;
   int o_fp32;
+  // Packed variable-length batches (bf16 only): sequence b holds rows [cu_q[b], cu_q[b+1]) of
+  // Q and O and rows [cu_k[b], cu_k[b+1]) of K and V (device arrays of B + 1 entries); N is
+  // then the longest query length the launch covers, BH = B * H, and LSE is [H, total_q].
+  // cu_q == nullptr for fixed-length batches.
+  const int* cu_q;
+  const int* cu_k;
+  int total_q;
+  int total_k;
 };
 
 // Q tiles of 128 rows handled together by one unit of the bf16 kernel for head dim d.

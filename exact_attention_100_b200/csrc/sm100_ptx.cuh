@@ -7,12 +7,10 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "attn_kernels.h"
+
 namespace ea {
 
-// ---------------------------------------------------------------------------------------------
-// Device status word bits (OR-ed into the library's per-device status word).
-// ---------------------------------------------------------------------------------------------
-constexpr int kDevStatusTimeout = 1;
 
 // Bound on any single mbarrier wait, in nanoseconds of %globaltimer.  Every wait in these
 // kernels is on work of the same CTA that takes microseconds; a wait this long means the

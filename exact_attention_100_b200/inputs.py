@@ -16,6 +16,10 @@ Recipe (the same for every workload):
   V ``[B, H, Nk, d]``, in that order, from the same generator.
 * The upstream gradient dO of the backward workloads is ``default_rng(seed).standard_normal``
   float32 of shape ``[B, H, N, d]`` with seed 7 unless stated, rounded to bf16.
+* Packed variable-length workloads: sequence lengths are ``default_rng(seed).integers(lo,
+  hi + 1, B)`` (queries; keys the same unless given), the offsets their running sums from 0,
+  and Q ``[total_q, H, d]``, K, V ``[total_k, H, d]`` are drawn iid N(0, 1) in that order from
+  ``default_rng(seed + 1)``, rounded to bf16.
 """
 
 from __future__ import annotations
@@ -74,3 +78,21 @@ def normal_qkv_lengths(B: int, H: int, Nq: int, Nk: int, d: int, seed: int = 0):
     k = rng.standard_normal((B, H, Nk, d), dtype=np.float32)
     v = rng.standard_normal((B, H, Nk, d), dtype=np.float32)
     return round_to_bf16(q), round_to_bf16(k), round_to_bf16(v)
+
+
+def uniform_lengths(B: int, lo: int, hi: int, seed: int = 0) -> np.ndarray:
+    """B sequence lengths drawn uniformly from [lo, hi] (int64)."""
+    return np.random.default_rng(seed).integers(lo, hi + 1, B).astype(np.int64)
+
+
+def normal_qkv_packed(lengths_q, lengths_k, H: int, d: int, seed: int = 0):
+    """(q, k, v, cu_q, cu_k) for a packed batch: q [sum(lengths_q), H, d], k, v
+    [sum(lengths_k), H, d] float32 arrays of bf16 values, iid N(0, 1), drawn in the order Q, K,
+    V; cu_q, cu_k the int32 offsets (B + 1 entries, starting at 0)."""
+    cu_q = np.concatenate([[0], np.cumsum(lengths_q)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lengths_k)]).astype(np.int32)
+    rng = np.random.default_rng(seed + 1)
+    q = rng.standard_normal((int(cu_q[-1]), H, d), dtype=np.float32)
+    k = rng.standard_normal((int(cu_k[-1]), H, d), dtype=np.float32)
+    v = rng.standard_normal((int(cu_k[-1]), H, d), dtype=np.float32)
+    return round_to_bf16(q), round_to_bf16(k), round_to_bf16(v), cu_q, cu_k

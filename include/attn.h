@@ -113,6 +113,36 @@ int attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float
                      float scale, int causal, int dtype, int o_dtype, void* stream);
 
 /*
+ * attn_fwd_varlen -- attention over a packed batch of B sequences of different lengths, each an
+ * independent problem ("FlashAttention-2/3" motivates long and variable contexts; the packing
+ * is this library's).
+ *
+ *   q, o        [total_q, H, d] (bf16; o of o_dtype), device: sequence b owns rows
+ *               cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1.
+ *   k, v        [total_k, H, d] bf16, device: sequence b owns rows cu_seqlens_k[b] .. [b+1]-1.
+ *   lse         [H, total_q] float32 or NULL, written for every row of every sequence.
+ *   cu_seqlens_q, cu_seqlens_k   DEVICE int32 arrays of B + 1 non-decreasing offsets with
+ *               cu[B] <= total (cu[0] is normally 0); lengths may be 0.
+ *   max_seqlen_q  >= every query length cu_seqlens_q[b+1] - cu_seqlens_q[b]; the launch is
+ *               sized for it (no device-to-host read of the offsets).
+ *   strides     HOST pointer to 8 int64 values {row stride, head stride} for q, k, v and o, in
+ *               elements, each a positive multiple of 8 below 2^36 (head stride of H = 1
+ *               ignored); the head dimension is contiguous.
+ *   causal      per sequence, bottom-right aligned as in attn_fwd_qk (key j visible to query
+ *               i iff j <= i + Nk_b - Nq_b); rows with no visible key get O = 0, LSE = -inf.
+ * Rows of another sequence that share a 128-row block with this sequence's last keys are read
+ * and weighted by exact zeros, so all of k and v must be finite.  Offsets that break the
+ * rules above are found on the device: that sequence is skipped (its rows are not written)
+ * and the next attn_device_status() returns ATTN_ERR_INVALID_ARG.
+ * Other arguments, arithmetic and host-side errors as for attn_fwd.
+ */
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H,
+                    int total_q, int total_k, int max_seqlen_q, int d,
+                    const long long* strides, float scale, int causal,
+                    int dtype, int o_dtype, void* stream);
+
+/*
  * attn_hadamard_quant -- random-sign Hadamard transform plus per-block E4M3 quantisation.
  *
  *   x       [B, H, N, d] bf16, device (read).
@@ -240,7 +270,8 @@ int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float
  * attn_device_status -- synchronises `stream`, returns the current device's status word and
  * clears it.  ATTN_OK if no kernel of this library reported a problem since the last call;
  * ATTN_ERR_TIMEOUT if a bounded wait inside a kernel ran out (that kernel's outputs are then
- * undefined, the CUDA context stays usable); ATTN_ERR_CUDA if synchronising failed.
+ * undefined, the CUDA context stays usable); otherwise ATTN_ERR_INVALID_ARG if attn_fwd_varlen
+ * found sequence offsets that break their rules; ATTN_ERR_CUDA if synchronising failed.
  */
 int attn_device_status(void* stream);
 

@@ -20,7 +20,8 @@ Sources (the three pages this project restates; cited by page title and section)
 Modules
 -------
 ``oracle.attention``  two-pass attention (the definition), the pages' blockwise m/l
-                      recurrence, and a lazy-rescale blockwise variant in base 2.
+                      recurrence, a lazy-rescale blockwise variant in base 2, and a packed
+                      batch of sequences of different lengths built on the definition.
 ``oracle.fp8``        Sylvester Hadamard matrix, fast Walsh-Hadamard transform in float32,
                       E4M3 (OCP E4M3FN) rounding/encoding, per-block quantisation.
 ``oracle.attention_bwd``  the backward pass (dQ, dK, dV) from the chain rule on whole score
@@ -37,6 +38,7 @@ from .attention import (  # noqa: F401
     attention_ref,
     attention_blockwise_ref,
     attention_blockwise_lazy_ref,
+    attention_varlen_ref,
     visible_mask,
 )
 from .attention_bwd import (  # noqa: F401

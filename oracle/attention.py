@@ -29,7 +29,7 @@ def visible_mask(n_q: int, n_k: int, causal: bool) -> np.ndarray:
 
     The pages do not state how a causal mask aligns when the query and key lengths differ;
     the reading taken is bottom-right alignment, ``j <= i + (n_k - n_q)``, which is the
-    plain ``j <= i`` whenever the lengths are equal (the only case the kernels support).
+    plain ``j <= i`` whenever the lengths are equal.
     """
     if not causal:
         return np.ones((n_q, n_k), dtype=bool)
@@ -194,3 +194,32 @@ def attention_blockwise_lazy_ref(q, k, v, scale: float, causal: bool, block_c: i
             out[b] = np.where((l > 0)[:, None], o_acc / np.where(l > 0, l, 1.0)[:, None], 0.0)
             lse[b] = np.where(l > 0, (m + np.log2(np.where(l > 0, l, 1.0))) * LN2, -np.inf)
     return out.reshape(lead + (n_q, d_v)), lse.reshape(lead + (n_q,))
+
+
+def attention_varlen_ref(q, k, v, cu_q, cu_k, scale: float, causal: bool = False):
+    """A packed batch of independent sequences of different lengths, in float64.
+
+    ``q`` is ``[total_q, H, d]`` and ``k``, ``v`` are ``[total_k, H, d]``; sequence ``b`` owns
+    query rows ``cu_q[b]:cu_q[b+1]`` and key/value rows ``cu_k[b]:cu_k[b+1]``.  Each sequence and
+    head is the problem :func:`attention_ref` defines (its own causal alignment, from its own
+    two lengths); the pages motivate variable context lengths ("FlashAttention-2/3") but fix no
+    packing, so this one is the plain reading: rows of one sequence are contiguous.
+
+    Returns ``(O [total_q, H, d_v], LSE [H, total_q])``.  A sequence with no keys gives its
+    rows ``O = 0``, ``LSE = -inf``; rows that belong to no sequence stay ``0`` / ``-inf``.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    total_q, h, _ = q.shape
+    out = np.zeros((total_q, h, v.shape[2]), dtype=np.float64)
+    lse = np.full((h, total_q), -np.inf, dtype=np.float64)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        if q1 == q0 or k1 == k0:
+            continue  # no rows, or no keys: O = 0, LSE = -inf as initialised
+        o_b, lse_b = attention_ref(q[q0:q1].transpose(1, 0, 2), k[k0:k1].transpose(1, 0, 2),
+                                   v[k0:k1].transpose(1, 0, 2), scale, causal)
+        out[q0:q1] = o_b.transpose(1, 0, 2)
+        lse[:, q0:q1] = lse_b
+    return out, lse

@@ -31,7 +31,8 @@ def test_header_declares_the_boundary():
     assert names == sorted(["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status",
                             "attn_status_string", "attn_num_kernel_launches", "attn_shutdown",
                             "attn_fwd_noalloc", "attn_hadamard_quant_qkv", "attn_bwd",
-                            "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided"])
+                            "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided",
+                            "attn_fwd_varlen"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -165,6 +166,42 @@ def test_fwd_strided_rejects_bad_arguments(L):
         assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
 
 
+def test_fwd_varlen_rejects_bad_arguments(L):
+    f = L.attn_fwd_varlen
+    H, d = 4, 128
+    CU = ctypes.c_void_p(0x30000)  # 4-byte aligned suffices for the offset arrays
+
+    def strides(vals):
+        return ctypes.cast((ctypes.c_longlong * 8)(*vals), ctypes.c_void_p)
+
+    good = [H * d, d] * 4  # {row, head} for q, k, v, o
+    ok = [P, P, P, P2, NULL, CU, CU, 3, H, 1000, 900, 512, d, strides(good), 0.1, 1, 0, 0, NULL]
+    for i in (0, 1, 2, 3, 5, 6, 13):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for i in (5, 6):
+        a = list(ok)
+        a[i] = ctypes.c_void_p(0x30002)
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for idx, val in [(7, 0), (8, 0), (9, 0), (10, -1), (11, 0), (14, 0.0), (15, 2), (17, 4)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+    for pos, val in [(0, 4), (1, 0), (3, -8), (6, 12), (7, 1 << 36)]:
+        bad = list(good)
+        bad[pos] = val
+        a = list(ok)
+        a[13] = strides(bad)
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (pos, val)
+    a = list(ok)
+    a[12] = 96
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+    a = list(ok)
+    a[16] = 2  # E4M3 inputs are not built for packed batches
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+
+
 def test_bwd_workspace_bytes(L):
     assert L.attn_bwd_workspace_bytes(1, 1, 1) == 2 * 128 * 4
     assert L.attn_bwd_workspace_bytes(2, 16, 8192) == 2 * 32 * 8192 * 4
@@ -213,5 +250,6 @@ def test_bwd_qk_rejects_bad_arguments(L):
 def test_python_binding_has_same_names():
     for name in ["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status", "attn_status_string",
                  "attn_num_kernel_launches", "attn_shutdown", "attn_fwd_noalloc", "attn_hadamard_quant_qkv",
-                 "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided"]:
+                 "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided",
+                 "attn_fwd_varlen"]:
         assert callable(getattr(ea, name)), name
