@@ -16,6 +16,8 @@ Recipe (the same for every workload):
   V ``[B, H, Nk, d]``, in that order, from the same generator.
 * The upstream gradient dO of the backward workloads is ``default_rng(seed).standard_normal``
   float32 of shape ``[B, H, N, d]`` with seed 7 unless stated, rounded to bf16.
+* Rotary tables: ``cos``/``sin`` ``[n_pos, d/2]`` of the angles ``n * 10000^(-2i/d)``, computed
+  in float64 and rounded to float32 once (an input, like the signs: the kernels take any table).
 * Packed variable-length workloads: sequence lengths are ``default_rng(seed).integers(lo,
   hi + 1, B)`` (queries; keys the same unless given), the offsets their running sums from 0,
   and Q ``[total_q, H, d]``, K, V ``[total_k, H, d]`` are drawn iid N(0, 1) in that order from
@@ -96,3 +98,12 @@ def normal_qkv_packed(lengths_q, lengths_k, H: int, d: int, seed: int = 0):
     k = rng.standard_normal((int(cu_k[-1]), H, d), dtype=np.float32)
     v = rng.standard_normal((int(cu_k[-1]), H, d), dtype=np.float32)
     return round_to_bf16(q), round_to_bf16(k), round_to_bf16(v), cu_q, cu_k
+
+
+def rope_tables(n_pos: int, d: int, base: float = 10000.0):
+    """float32 ``(cos, sin)`` tables ``[n_pos, d/2]`` for the angles ``n * base^(-2i/d)``,
+    computed in float64 and rounded once."""
+    i = np.arange(d // 2, dtype=np.float64)
+    theta = base ** (-2.0 * i / d)
+    ang = np.arange(n_pos, dtype=np.float64)[:, None] * theta[None, :]
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)

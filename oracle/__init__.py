@@ -24,6 +24,8 @@ Modules
                       batch of sequences of different lengths built on the definition.
 ``oracle.fp8``        Sylvester Hadamard matrix, fast Walsh-Hadamard transform in float32,
                       E4M3 (OCP E4M3FN) rounding/encoding, per-block quantisation.
+``oracle.rope``       rotary position embedding (rotate-half pairing, caller's cos/sin
+                      tables) in float32, ahead of the Hadamard/E4M3 pre-processing.
 ``oracle.attention_bwd``  the backward pass (dQ, dK, dV) from the chain rule on whole score
                       matrices; the pages only state that it exists and recomputes the softmax
                       ("FlashAttention-3", "适用范围和工程限制"; "Flash Attention V3 解析" 2.1).
@@ -58,3 +60,4 @@ from .fp8 import (  # noqa: F401
     hadamard_quant_ref,
     dequant_ref,
 )
+from .rope import rope_ref  # noqa: F401
