@@ -402,6 +402,32 @@ def fp8_section(args, dev, rank):
            "prekernel": {"ms_3_tensors": pre_ms, "achieved_gbs": gbs, "peak_gbs": float(peaks["hbm_gbs"]),
                          "frac": gbs / float(peaks["hbm_gbs"]), "bound": "hbm",
                          "bytes_per_call": pre_bytes, "peak_source": peaks["source"]}}
+
+    # the same launch with the rotary embedding of Q and K fused in front of the transform
+    from exact_attention_100_b200.inputs import rope_tables
+    cos_n, sin_n = rope_tables(N, d)  # [N, d/2]; the kernel takes them frequency-major
+    cos, sin = (torch.from_numpy(np.ascontiguousarray(t.T)).to(dev) for t in (cos_n, sin_n))
+
+    def pre_rope():
+        ea.attn_rope_hadamard_quant_qkv(q, k, v, signs, cos, sin, outs=outs, stream=stream)
+
+    for _ in range(3):
+        pre_rope()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        pre_rope()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    rope_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    rope_bytes = pre_bytes + 2 * N * (d // 2) * 4  # plus the cos and sin tables, read once from HBM
+    rgbs = rope_bytes / (rope_ms * 1e-3) / 1e9
+    out["prekernel_rope"] = {"ms_3_tensors": rope_ms, "achieved_gbs": rgbs, "peak_gbs": float(peaks["hbm_gbs"]),
+                             "frac": rgbs / float(peaks["hbm_gbs"]), "bound": "hbm", "bytes_per_call": rope_bytes,
+                             "vs_unrotated": rope_ms / pre_ms, "peak_source": peaks["source"],
+                             "note": "Q and K rotated (frequency-major tables [64, 8192] float32, L2-resident "
+                                     "after the first read), then H D and E4M3; V quantised as it is"}
     try:
         o = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
         lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
@@ -579,6 +605,22 @@ def run_profile_case(args):
     if args.profile_case == "fwd":
         for _ in range(args.reps):
             ea.attn_fwd(q, k, v, causal=bool(causal))
+    elif args.profile_case == "hq_rope":
+        from exact_attention_100_b200.inputs import rope_tables
+        cos, sin = (torch.from_numpy(np.ascontiguousarray(t.T)).to(dev) for t in rope_tables(N, d))
+        outs = None
+        for _ in range(args.reps):
+            outs = ea.attn_rope_hadamard_quant_qkv(q, k, v, signs, cos, sin, outs=outs)
+    elif args.profile_case == "varlen":
+        # the bench's packed workload (the shape's H and d; lengths from the packed recipe)
+        from exact_attention_100_b200.inputs import normal_qkv_packed
+        w = VARLEN_WORKLOAD
+        lens = varlen_lengths(w["total"], w["lo"], w["hi"], w["seed"])
+        qn, kn, vn, cq, ck = normal_qkv_packed(lens, lens, H, d, seed=w["seed"])
+        pq, pk, pv = (torch.from_numpy(a).to(torch.bfloat16).to(dev) for a in (qn, kn, vn))
+        cu_q, cu_k = torch.from_numpy(cq).to(dev), torch.from_numpy(ck).to(dev)
+        for _ in range(args.reps):
+            ea.attn_fwd_varlen(pq, pk, pv, cu_q, cu_k, max(lens), causal=bool(causal))
     elif args.profile_case == "bwd":
         o, lse = ea.attn_fwd(q, k, v, causal=bool(causal))
         do = torch.randn_like(q)
@@ -609,7 +651,7 @@ def main():
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv", "bwd"], default=None,
+    ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv", "hq_rope", "varlen", "bwd"], default=None,
                     help="run --reps untimed calls of one entry point (for an ncu capture) and exit")
     ap.add_argument("--shape", type=int, nargs=5, default=[2, 16, 8192, 128, 1], metavar=("B", "H", "N", "d", "CAUSAL"))
     ap.add_argument("--reps", type=int, default=3)

@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.attn_hadamard_quant.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
         L.attn_hadamard_quant.restype = i
         L.attn_hadamard_quant_qkv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
+        L.attn_rope_hadamard_quant_qkv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+        L.attn_rope_hadamard_quant_qkv.restype = i
         L.attn_hadamard_quant_qkv.restype = i
         L.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
         L.attn_fwd_fp8.restype = i
@@ -329,6 +331,32 @@ def attn_hadamard_quant_qkv(q, k, v, signs, outs=None, stream=None):
     _check(lib().attn_hadamard_quant_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs), _ptr(ks),
                                          _ptr(vs), _ptr(signs), B, H, N, d, _stream_ptr(stream)),
            "attn_hadamard_quant_qkv")
+    return outs
+
+
+def attn_rope_hadamard_quant_qkv(q, k, v, signs, cos, sin, outs=None, stream=None):
+    """attn_hadamard_quant_qkv with Q and K first rotated by the rotary tables ``cos``, ``sin``
+    (frequency-major [d/2, n_pos] float32 cuda tensors, n_pos >= N; row n of each sequence uses
+    column n).  Returns ``(q8, k8, v8, q_scale, k_scale, v_scale)``."""
+    import torch
+    B, H, N, d = _dims(q)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError("q, k, v must be contiguous bf16 tensors of one shape")
+    for t in (cos, sin):
+        if t.dtype != torch.float32 or not t.is_contiguous() or t.dim() != 2 or t.shape[0] != d // 2:
+            raise ValueError("cos and sin must be contiguous float32 [d/2, n_pos]")
+    if cos.shape != sin.shape:
+        raise ValueError("cos and sin must have one shape")
+    nb = (N + 127) // 128
+    if outs is None:
+        outs = tuple(torch.empty(q.shape, dtype=torch.uint8, device=q.device) for _ in range(3)) + \
+            tuple(torch.empty((B, H, nb), dtype=torch.float32, device=q.device) for _ in range(3))
+    q8, k8, v8, qs, ks, vs = outs
+    _check(lib().attn_rope_hadamard_quant_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs),
+                                              _ptr(ks), _ptr(vs), _ptr(signs), _ptr(cos), _ptr(sin),
+                                              int(cos.shape[1]), B, H, N, d, _stream_ptr(stream)),
+           "attn_rope_hadamard_quant_qkv")
     return outs
 
 

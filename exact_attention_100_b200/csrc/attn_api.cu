@@ -316,16 +316,22 @@ int attn_hadamard_quant(const void* x, void* x8, float* scales, const signed cha
   if (!encode_rows_map(&mx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H)) return ATTN_ERR_CUDA;
   uint8_t* out = static_cast<uint8_t*>(x8);
   const int transform = signs != nullptr ? 1 : 0;
-  if (ea::launch_hadamard_quant(&mx, 1, &out, &scales, &post, &transform, signs, B * H, N, d, st->num_sms, st->status,
+  if (ea::launch_hadamard_quant(&mx, 1, &out, &scales, &post, &transform, signs, B * H, N, d, nullptr, nullptr,
+                                nullptr, 0, st->num_sms, st->status,
                                static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
   return ATTN_OK;
 }
 
-int attn_hadamard_quant_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8,
-                            float* q_scale, float* k_scale, float* v_scale, const signed char* signs, int B, int H,
-                            int N, int d, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// attn_hadamard_quant_qkv and attn_rope_hadamard_quant_qkv (cos/sin NULL: no rotation).
+int hq_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8, float* q_scale, float* k_scale,
+           float* v_scale, const signed char* signs, const float* cos, const float* sin, int n_pos, int B, int H, int N,
+           int d, void* stream) {
   const void* in[3] = {q, k, v};
   void* out[3] = {q8, k8, v8};
   float* sc[3] = {q_scale, k_scale, v_scale};
@@ -346,11 +352,30 @@ int attn_hadamard_quant_qkv(const void* q, const void* k, const void* v, void* q
   uint8_t* o8[3] = {static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8), static_cast<uint8_t*>(v8)};
   const float post[3] = {rsd, rsd, 1.0f};
   const int transform[3] = {1, 1, 0};
-  if (ea::launch_hadamard_quant(maps, 3, o8, sc, post, transform, signs, B * H, N, d, st->num_sms, st->status,
-                               static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  const int rope[3] = {1, 1, 0};  // Q and K rotated, V not
+  if (ea::launch_hadamard_quant(maps, 3, o8, sc, post, transform, signs, B * H, N, d, cos ? rope : nullptr, cos, sin,
+                                n_pos, st->num_sms, st->status, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
   return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_hadamard_quant_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8,
+                            float* q_scale, float* k_scale, float* v_scale, const signed char* signs, int B, int H,
+                            int N, int d, void* stream) {
+  return hq_qkv(q, k, v, q8, k8, v8, q_scale, k_scale, v_scale, signs, nullptr, nullptr, 0, B, H, N, d, stream);
+}
+
+int attn_rope_hadamard_quant_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8,
+                                 float* q_scale, float* k_scale, float* v_scale, const signed char* signs,
+                                 const float* cos, const float* sin, int n_pos, int B, int H, int N, int d,
+                                 void* stream) {
+  if (!cos || !sin || !aligned16(cos) || !aligned16(sin) || n_pos < N) return ATTN_ERR_INVALID_ARG;
+  return hq_qkv(q, k, v, q8, k8, v8, q_scale, k_scale, v_scale, signs, cos, sin, n_pos, B, H, N, d, stream);
 }
 
 int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,

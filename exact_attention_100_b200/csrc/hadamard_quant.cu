@@ -9,13 +9,22 @@
 // brought into shared memory by TMA (128-byte swizzle, rows past the sequence end read as
 // zero); two blocks are in flight per CTA, the next load being issued as soon as every thread
 // has copied the current block into registers.  One thread holds a whole row (d = 64, 128) or
-// a quarter of it (d = 256, 64 elements each, four adjacent lanes): the unnormalised transform
-// y = H_d (D x) runs in float32 registers with butterfly stages of stride 1, 2, ..., 32/64
-// inside a thread and, for d = 256, 64 and 128 between the lanes of a row (shuffles) -- the
+// 64 elements of it (d = 256, and d = 128 with the rotary embedding; adjacent lanes): the
+// unnormalised transform y = H_d (D x) runs in float32 registers with butterfly stages of
+// stride 1, 2, ..., inside a thread and the remaining strides between the lanes of a row -- the
 // textbook stage order, so every element sees the same float32 additions in the same order
 // as a plain sequential transform.  The block's largest |y| sets s_u = max(amax / 448, 2^-126);
 // codes are E4M3(y * (1/s_u)) (round to nearest even, saturating); the stored dequantisation
 // scale is s_u * post_scale (post_scale = 1/sqrt(d) with the transform, 1 without).
+//
+// With ROPE, the tensors marked for it are first given the rotary position embedding the same
+// page names as a bandwidth-bound step to fuse with the transform: coordinates i and i + d/2 of
+// row n are rotated by the angle whose cosine and sine the caller's tables hold at [i, n],
+// in float32 with each product and the sum rounded (no fused multiply-add); then D (an exact
+// sign flip) and the butterflies run on the rotated float32 row.  The tables are frequency-major
+// so that the 32 rows of a warp read one contiguous 128-byte line per frequency (row-major
+// tables cost each warp load 32 lines and made the kernel L1-bound).  For d = 256 the partner
+// coordinate sits two lanes away.
 
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -66,14 +75,16 @@ __device__ __forceinline__ void thread_wait(uint64_t* bar, uint32_t parity, vola
   }
 }
 
-template <int D>
+template <int D, bool ROPE = false>
 struct HqCfg {
-  static constexpr int kElems = D == 256 ? 64 : D;  // elements of a row held by one thread
+  // elements of a row held by one thread: at most 64 with the rotary embedding, whose table
+  // loads need registers to be in flight (a whole d = 128 row per thread left too few)
+  static constexpr int kElems = (D == 256 || ROPE) ? 64 : D;
   static constexpr int kThreadsPerRow = D / kElems;
   static constexpr int kThreads = 128 * kThreadsPerRow;
   static constexpr int kBoxes = D / 64;             // 128-byte TMA boxes per row
   static constexpr int kBufBytes = 128 * D * 2;
-  static constexpr int kCtasPerSm = D == 256 ? 1 : (D == 128 ? 3 : 5);
+  static constexpr int kCtasPerSm = D == 256 ? 1 : (D == 128 ? (ROPE ? 2 : 3) : 5);
 };
 
 // Up to three tensors of one shape in one launch (Q and K with the transform, V without).
@@ -82,15 +93,19 @@ struct HqJob {
   float* scales[3];
   float post[3];
   int transform[3];
+  int rope[3];        // ROPE kernels: rotate this tensor's rows first
+  const float* cos;   // [d/2, n_pos] float32 rotary tables, frequency-major (ROPE kernels)
+  const float* sin;
+  int n_pos;
   int blocks_per_tensor;
 };
 
-template <int D>
-__global__ void __launch_bounds__(HqCfg<D>::kThreads, HqCfg<D>::kCtasPerSm)
+template <int D, bool ROPE>
+__global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCtasPerSm)
     hadamard_quant_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
                           const __grid_constant__ CUtensorMap tm2, const HqJob job,
                           const signed char* __restrict__ signs, int N, int n_blocks, int total_blocks, int* status) {
-  using C = HqCfg<D>;
+  using C = HqCfg<D, ROPE>;
   constexpr int kE = C::kElems;
   constexpr int kWarps = C::kThreads / 32;
   extern __shared__ uint8_t smem_raw[];
@@ -160,7 +175,23 @@ __global__ void __launch_bounds__(HqCfg<D>::kThreads, HqCfg<D>::kCtasPerSm)
     // 16-byte chunk ((e0 % 64) / 8) ^ (row % 8) of the row (128-byte swizzle).  With the
     // transform, D x is a flip of bf16 sign bits, and the stride-1 butterflies of H run here.
     float v[kE];
-    if (transform) {
+    // x = the raw bf16 row part, as float32
+    auto unpack_raw = [&]() {
+#pragma unroll
+      for (int c = 0; c < kE / 8; ++c) {
+        const int e0 = part * kE + c * 8;
+        const uint4 w = *reinterpret_cast<const uint4*>(sb + (e0 >> 6) * 16384 + row * 128 +
+                                                        ((((e0 & 63) >> 3) ^ (row & 7)) << 4));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          v[c * 8 + 2 * k] = __uint_as_float(ws[k] << 16);
+          v[c * 8 + 2 * k + 1] = __uint_as_float(ws[k] & 0xFFFF0000u);
+        }
+      }
+    };
+    // D x as a flip of bf16 sign bits, fused with the stride-1 butterflies of H
+    auto unpack_signed_stage1 = [&]() {
 #pragma unroll
       for (int c = 0; c < kE / 8; ++c) {
         const int e0 = part * kE + c * 8;
@@ -176,6 +207,9 @@ __global__ void __launch_bounds__(HqCfg<D>::kThreads, HqCfg<D>::kCtasPerSm)
           v[c * 8 + 2 * k + 1] = lo - hi;
         }
       }
+    };
+    // the butterflies of stride 2 .. D/2
+    auto later_stages = [&]() {
       // strides 2 .. kE/2 inside the thread, on register pairs (e, e+1): one packed add and one
       // packed sub make two butterflies, each lane rounding like a scalar operation
 #pragma unroll
@@ -205,18 +239,73 @@ __global__ void __launch_bounds__(HqCfg<D>::kThreads, HqCfg<D>::kCtasPerSm)
           fma2_rn(v[e], v[e + 1], sgn, o0, o1);
         }
       }
-    } else {
+    };
+    // rotary embedding of the float32 row (pairs i, i + D/2), then, with the transform, the sign
+    // flips of D and the stride-1 butterflies
+    auto rotate_row = [&]() {
+      // rows past the sequence end hold zeros (TMA fill): any table row leaves them zero
+      const int pos = min(blk * 128 + row, N - 1);
+      const size_t np = static_cast<size_t>(job.n_pos);
+      if constexpr (C::kThreadsPerRow == 1) {
+        const float* cr = job.cos + pos;
+        const float* sr = job.sin + pos;
 #pragma unroll
-      for (int c = 0; c < kE / 8; ++c) {
-        const int e0 = part * kE + c * 8;
-        const uint4 w = *reinterpret_cast<const uint4*>(sb + (e0 >> 6) * 16384 + row * 128 +
-                                                        ((((e0 & 63) >> 3) ^ (row & 7)) << 4));
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          v[c * 8 + 2 * k] = __uint_as_float(ws[k] << 16);
-          v[c * 8 + 2 * k + 1] = __uint_as_float(ws[k] & 0xFFFF0000u);
+        for (int i = 0; i < D / 2; ++i) {
+          const float c = __ldg(cr + i * np), s = __ldg(sr + i * np);
+          const float a = v[i], b = v[i + D / 2];
+          v[i] = __fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s));
+          v[i + D / 2] = __fadd_rn(__fmul_rn(b, c), __fmul_rn(a, s));
         }
+      } else {
+        // the lower half of the parts holds coordinates 0 .. D/2-1, the upper half their
+        // partners D/2 .. D-1, kThreadsPerRow/2 lanes away
+        constexpr int kHalf = C::kThreadsPerRow / 2;
+        const bool upper = part >= kHalf;
+        const int i0 = (part % kHalf) * kE;
+        const float* cr = job.cos + i0 * np + pos;
+        const float* sr = job.sin + i0 * np + pos;
+#pragma unroll
+        for (int e = 0; e < kE; ++e) {
+          const float c = __ldg(cr + e * np), s = __ldg(sr + e * np);
+          const float own = v[e];
+          const float other = __shfl_xor_sync(0xffffffffu, own, kHalf);
+          v[e] = upper ? __fadd_rn(__fmul_rn(own, c), __fmul_rn(other, s))
+                       : __fsub_rn(__fmul_rn(own, c), __fmul_rn(other, s));
+        }
+      }
+    };
+    auto signed_stage1 = [&]() {
+#pragma unroll
+      for (int e = 0; e < kE; e += 2) {
+        const uint32_t mk = smask[(part * kE + e) / 2];
+        const float a = __uint_as_float(__float_as_uint(v[e]) ^ (mk << 16));
+        const float b = __uint_as_float(__float_as_uint(v[e + 1]) ^ (mk & 0x80000000u));
+        v[e] = a + b;
+        v[e + 1] = a - b;
+      }
+    };
+
+    if constexpr (ROPE) {
+      const bool rotate = (t == 0 ? job.rope[0] : (t == 1 ? job.rope[1] : job.rope[2])) != 0;
+      if (rotate) {
+        unpack_raw();
+        rotate_row();
+        if (transform) {
+          signed_stage1();
+          later_stages();
+        }
+      } else if (transform) {
+        unpack_signed_stage1();
+        later_stages();
+      } else {
+        unpack_raw();
+      }
+    } else {
+      if (transform) {
+        unpack_signed_stage1();
+        later_stages();
+      } else {
+        unpack_raw();
       }
     }
 
@@ -283,10 +372,10 @@ __global__ void __launch_bounds__(HqCfg<D>::kThreads, HqCfg<D>::kCtasPerSm)
   }
 }
 
-template <int D>
+template <int D, bool ROPE>
 static cudaError_t launch_hq(const CUtensorMap* tm, int ntensors, const HqJob& job0, const signed char* signs, int BH,
                              int N, int num_sms, int* status, cudaStream_t stream) {
-  using C = HqCfg<D>;
+  using C = HqCfg<D, ROPE>;
   const int n_blocks = (N + 127) / 128;
   const long long per = static_cast<long long>(BH) * n_blocks;
   const long long total = per * ntensors;
@@ -295,7 +384,7 @@ static cudaError_t launch_hq(const CUtensorMap* tm, int ntensors, const HqJob& j
   job.blocks_per_tensor = static_cast<int>(per);
   const long long cap = static_cast<long long>(num_sms) * C::kCtasPerSm;
   const int grid = static_cast<int>(total < cap ? total : cap);
-  hadamard_quant_kernel<D><<<grid, C::kThreads, 2 * C::kBufBytes + 1024, stream>>>(
+  hadamard_quant_kernel<D, ROPE><<<grid, C::kThreads, 2 * C::kBufBytes + 1024, stream>>>(
       tm[0], tm[ntensors > 1 ? 1 : 0], tm[ntensors > 2 ? 2 : 0], job, signs, N, n_blocks, static_cast<int>(total),
       status);
   return cudaGetLastError();
@@ -303,8 +392,12 @@ static cudaError_t launch_hq(const CUtensorMap* tm, int ntensors, const HqJob& j
 
 template <int D>
 static cudaError_t set_hq_attr() {
-  return cudaFuncSetAttribute(hadamard_quant_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              2 * HqCfg<D>::kBufBytes + 1024);
+  cudaError_t e = cudaFuncSetAttribute(hadamard_quant_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       2 * HqCfg<D>::kBufBytes + 1024);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(hadamard_quant_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             2 * HqCfg<D, true>::kBufBytes + 1024);
+  return e;
 }
 
 cudaError_t setup_hadamard_quant_kernels() {
@@ -316,8 +409,11 @@ cudaError_t setup_hadamard_quant_kernels() {
 
 cudaError_t launch_hadamard_quant(const CUtensorMap* tm, int ntensors, uint8_t* const* x8, float* const* scales,
                                   const float* post, const int* transform, const signed char* signs, int BH, int N,
-                                  int d, int num_sms, int* status, cudaStream_t stream) {
+                                  int d, const int* rope, const float* cos, const float* sin, int n_pos, int num_sms,
+                                  int* status, cudaStream_t stream) {
   if (ntensors < 1 || ntensors > 3) return cudaErrorInvalidValue;
+  const bool with_rope = rope != nullptr;
+  if (with_rope && (cos == nullptr || sin == nullptr)) return cudaErrorInvalidValue;
   HqJob job{};
   for (int t = 0; t < 3; ++t) {
     const int s = t < ntensors ? t : 0;
@@ -325,14 +421,21 @@ cudaError_t launch_hadamard_quant(const CUtensorMap* tm, int ntensors, uint8_t* 
     job.scales[t] = scales[s];
     job.post[t] = post[s];
     job.transform[t] = transform[s];
+    job.rope[t] = with_rope ? rope[s] : 0;
   }
+  job.cos = cos;
+  job.sin = sin;
+  job.n_pos = n_pos;
   switch (d) {
     case 64:
-      return launch_hq<64>(tm, ntensors, job, signs, BH, N, num_sms, status, stream);
+      return with_rope ? launch_hq<64, true>(tm, ntensors, job, signs, BH, N, num_sms, status, stream)
+                       : launch_hq<64, false>(tm, ntensors, job, signs, BH, N, num_sms, status, stream);
     case 128:
-      return launch_hq<128>(tm, ntensors, job, signs, BH, N, num_sms, status, stream);
+      return with_rope ? launch_hq<128, true>(tm, ntensors, job, signs, BH, N, num_sms, status, stream)
+                       : launch_hq<128, false>(tm, ntensors, job, signs, BH, N, num_sms, status, stream);
     case 256:
-      return launch_hq<256>(tm, ntensors, job, signs, BH, N, num_sms, status, stream);
+      return with_rope ? launch_hq<256, true>(tm, ntensors, job, signs, BH, N, num_sms, status, stream)
+                       : launch_hq<256, false>(tm, ntensors, job, signs, BH, N, num_sms, status, stream);
     default:
       return cudaErrorInvalidValue;
   }

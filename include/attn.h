@@ -180,6 +180,27 @@ int attn_hadamard_quant_qkv(const void* q, const void* k, const void* v, void* q
                             int B, int H, int N, int d, void* stream);
 
 /*
+ * attn_rope_hadamard_quant_qkv -- attn_hadamard_quant_qkv with the rotary position embedding of
+ * Q and K fused in front of the transform ("FlashAttention-3", section "为什么 Hadamard 适合放到
+ * 内核里": the transform fuses with RoPE, another bandwidth-bound step; the pages do not define
+ * RoPE, the rotate-half form below is this library's reading).
+ *
+ *   cos, sin    [d/2, n_pos] float32, device, 16-byte aligned (read), frequency-major (each
+ *               frequency's positions contiguous): row n of every sequence rotates
+ *               coordinates i and i + d/2 by the angle these tables hold at [i, n]:
+ *                 y_i       = x_i       * cos[i,n] - x_{i+d/2} * sin[i,n]
+ *                 y_{i+d/2} = x_{i+d/2} * cos[i,n] + x_i       * sin[i,n]
+ *               in float32, each product and the sum rounded (no fused multiply-add).
+ *   n_pos       positions in the tables (their row length), >= N.
+ * Q and K are rotated, then transformed (H D) and quantised; V is quantised as it is.  Other
+ * arguments, outputs and errors as for attn_hadamard_quant_qkv.
+ */
+int attn_rope_hadamard_quant_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8,
+                                 float* q_scale, float* k_scale, float* v_scale, const signed char* signs,
+                                 const float* cos, const float* sin, int n_pos,
+                                 int B, int H, int N, int d, void* stream);
+
+/*
  * attn_fwd_fp8 -- exact-attention forward on per-block E4M3 inputs (approximate: the inputs
  * and P carry E4M3 rounding).
  *

@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
                             "attn_status_string", "attn_num_kernel_launches", "attn_shutdown",
                             "attn_fwd_noalloc", "attn_hadamard_quant_qkv", "attn_bwd",
                             "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided",
-                            "attn_fwd_varlen"])
+                            "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -202,6 +202,26 @@ def test_fwd_varlen_rejects_bad_arguments(L):
     assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
 
 
+def test_rope_hadamard_quant_qkv_rejects_bad_arguments(L):
+    f = L.attn_rope_hadamard_quant_qkv
+    ok = [P, P, P, P2, P2, P2, P2, P2, P2, P, P, P, 256, 1, 2, 256, 128, NULL]
+    for i in range(12):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for i in (10, 11):
+        a = list(ok)
+        a[i] = MIS
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for idx, val in [(12, 255), (13, 0), (14, 0), (15, 0)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+    a = list(ok)
+    a[16] = 96
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+
+
 def test_bwd_workspace_bytes(L):
     assert L.attn_bwd_workspace_bytes(1, 1, 1) == 2 * 128 * 4
     assert L.attn_bwd_workspace_bytes(2, 16, 8192) == 2 * 32 * 8192 * 4
@@ -251,5 +271,5 @@ def test_python_binding_has_same_names():
     for name in ["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status", "attn_status_string",
                  "attn_num_kernel_launches", "attn_shutdown", "attn_fwd_noalloc", "attn_hadamard_quant_qkv",
                  "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided",
-                 "attn_fwd_varlen"]:
+                 "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv"]:
         assert callable(getattr(ea, name)), name
