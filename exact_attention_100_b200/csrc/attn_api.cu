@@ -147,6 +147,7 @@ void fill_params(ea::FwdParams& p, void* o, float* lse, int* status, int B, int 
   p.q_scale = p.k_scale = p.v_scale = nullptr;
   p.cu_q = p.cu_k = nullptr;
   p.total_q = p.total_k = 0;
+  p.vl_sched = 0;
   p.N = N;
   p.BH = B * H;
   p.H = H;
@@ -295,6 +296,8 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   p.cu_k = cu_seqlens_k;
   p.total_q = total_q;
   p.total_k = total_k;
+  // the in-kernel schedule's shared-memory tables hold up to 1024 sequences and 1023 pairs
+  p.vl_sched = (B <= 1024 && p.n_pairs <= 1023) ? 1 : 0;
   if (ea::launch_attn_fwd_bf16(d, mq, mk, mv, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);

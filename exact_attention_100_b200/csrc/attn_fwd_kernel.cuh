@@ -68,6 +68,9 @@ struct ElemE4m3 {
   static constexpr int kPCols = 32;
 };
 
+// Schedule of a packed batch in shared memory: at most this many sequences and tile pairs.
+constexpr int kVlSchedSeqs = 1024, kVlSchedRounds = 1023;
+
 template <int D, int NQ, class E>
 struct FwdCfg {
   static constexpr int kBoxBytes = 128 * 128;                 // one TMA box: 128 rows x 128 bytes
@@ -95,7 +98,10 @@ struct FwdCfg {
   static constexpr int kFlagOff = kRowLOff + NQ * 2 * 128 * 4;  // [NQ][2] int, one byte per warp
   static constexpr int kEventOff = kFlagOff + 16;               // [kEvents][4] int
   static constexpr int kMiscOff = kEventOff + kEvents * 16;
-  static constexpr int kSmemBytes = kMiscOff + 16;
+  // packed batches: sorted sequence keys [kSchedSeqs] and the unit prefix [kSchedRounds + 1]
+  static constexpr int kSchedSeqs = kVlSchedSeqs, kSchedRounds = kVlSchedRounds;
+  static constexpr int kSchedOff = kMiscOff + 16;
+  static constexpr int kSmemBytes = kSchedOff + (kSchedSeqs + kSchedRounds + 1) * 4;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;        // room to align the base to 1024 bytes
   static_assert(kSlots >= 2, "K/V ring");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
@@ -164,13 +170,33 @@ struct Unit {
   Seq s;
 };
 
+// Unit u of the launch.  Fixed-length batches (and packed ones without the schedule): round
+// r = u / BH, (batch, head) = u % BH, tile pair n_pairs - 1 - r when causal (longest units
+// first) or r.  Packed batches with the schedule (`sched` = the sorted sequence keys, then the
+// unit prefix C[0..n_pairs]): round r holds, for tile pair n_pairs - 1 - r, every sequence that
+// has that pair (a prefix of the sorted keys) times every head, so no unit is empty.
 template <int NQ, bool VL>
-__device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p) {
+__device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p, const int* sched) {
   Unit U;
-  const int r = u / p.BH;
-  U.bh = u - r * p.BH;
+  int pair;
+  if (VL && sched != nullptr) {
+    const int* pre = sched + kVlSchedSeqs;
+    int lo = 0, hi = p.n_pairs;  // pre[lo] <= u < pre[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pre[mid] <= u) lo = mid;
+      else hi = mid;
+    }
+    const int idx = u - pre[lo];
+    const int i = idx / p.H;
+    U.bh = (sched[i] & 0xFFFF) * p.H + (idx - i * p.H);
+    pair = p.n_pairs - 1 - lo;
+  } else {
+    const int r = u / p.BH;
+    U.bh = u - r * p.BH;
+    pair = p.causal ? (p.n_pairs - 1 - r) : r;  // causal: longest units first
+  }
   U.s = seq_of<VL>(U.bh, p);
-  const int pair = p.causal ? (p.n_pairs - 1 - r) : r;  // causal: longest units first
   U.tile0 = pair * NQ;
   U.present = U.tile0 * 128 < U.s.N;
   U.n_max = 0;
@@ -366,10 +392,84 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
+  const int* sched = nullptr;
+  int num_units = p.num_units;
+  if constexpr (VL) {
+    if (p.vl_sched) {
+      // every CTA builds the same schedule: sequence keys (n_pairs - pairs) << 16 | b sorted
+      // ascending (bitonic sort; unique keys, so the order is the same in every CTA), then the
+      // units per round, prefix-summed
+      int* key = reinterpret_cast<int*>(smem + C::kSchedOff);
+      int* pre = key + C::kSchedSeqs;
+      const int B = p.BH / p.H;
+      int Bp = 1;
+      while (Bp < B) Bp <<= 1;
+      for (int i = threadIdx.x; i < Bp; i += C::kThreads) {
+        int k = 0x7FFFFFFF;  // padding sorts last
+        if (i < B) {
+          const Seq s = seq_of<true>(i * p.H, p);
+          if (s.bad && blockIdx.x == 0) atomicOr(p.status, kDevStatusBadSeqlens);
+          const int pairs = (s.N + 128 * NQ - 1) / (128 * NQ);
+          k = ((p.n_pairs - pairs) << 16) | i;
+        }
+        key[i] = k;
+      }
+      __syncthreads();
+      for (int kk = 2; kk <= Bp; kk <<= 1) {
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+          for (int i = threadIdx.x; i < Bp; i += C::kThreads) {
+            const int ixj = i ^ j;
+            if (ixj > i) {
+              const int a = key[i], b = key[ixj];
+              if ((a > b) == ((i & kk) == 0)) {
+                key[i] = b;
+                key[ixj] = a;
+              }
+            }
+          }
+          __syncthreads();
+        }
+      }
+      // round r has every sequence whose key >> 16 is <= r, i.e. with at least n_pairs - r pairs
+      for (int r = threadIdx.x; r < p.n_pairs; r += C::kThreads) {
+        int lo = 0, hi = B;  // first index whose key >> 16 exceeds r
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if ((key[mid] >> 16) <= r) lo = mid + 1;
+          else hi = mid;
+        }
+        pre[r + 1] = lo * p.H;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // inclusive scan of pre[1..n_pairs] by one warp: each lane a contiguous chunk
+        const int per = (p.n_pairs + 31) / 32;
+        const int r0 = 1 + lane * per;
+        int sum = 0;
+        for (int r = r0; r < r0 + per && r <= p.n_pairs; ++r) sum += pre[r];
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        int run = incl - sum;
+        for (int r = r0; r < r0 + per && r <= p.n_pairs; ++r) {
+          run += pre[r];
+          pre[r] = run;
+        }
+        if (lane == 0) pre[0] = 0;
+      }
+      sched = key;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if constexpr (VL) {
+    if (sched != nullptr) num_units = sched[C::kSchedSeqs + p.n_pairs];
+  }
   const AbortState ab{abort_flag, p.status};
   const int nb = p.n_blocks;
 
@@ -385,8 +485,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int u = unit_index(k);
-      if (u >= p.num_units) break;
-      const Unit U = decode_unit<NQ, VL>(u, p);
+      if (u >= num_units) break;
+      const Unit U = decode_unit<NQ, VL>(u, p, sched);
       const Seq& S = U.s;
       const int n = U.n[q];
       const int tile_row0 = (U.tile0 + q) * 128;
@@ -684,8 +784,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int u = unit_index(k);
-        if (u >= p.num_units) break;
-        const Unit U = decode_unit<NQ, VL>(u, p);
+        if (u >= num_units) break;
+        const Unit U = decode_unit<NQ, VL>(u, p, sched);
         if constexpr (VL) {
           if (!U.present) continue;  // past its sequence's end: the producer skips it too
         }
@@ -767,8 +867,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int u = unit_index(k);
-        if (u >= p.num_units) break;
-        const Unit U = decode_unit<NQ, VL>(u, p);
+        if (u >= num_units) break;
+        const Unit U = decode_unit<NQ, VL>(u, p, sched);
         const Seq& S = U.s;
         if constexpr (VL) {
           if (S.bad && U.tile0 == 0) atomicOr(p.status, kDevStatusBadSeqlens);

@@ -41,6 +41,9 @@ struct FwdParams {
   const int* cu_k;
   int total_q;
   int total_k;
+  // packed batches with B <= 1024 and n_pairs <= 1023: every CTA sorts the sequences by their
+  // number of tile pairs and deals out only the units that exist, longest first
+  int vl_sched;
 };
 
 // Q tiles of 128 rows handled together by one unit of the bf16 kernel for head dim d.

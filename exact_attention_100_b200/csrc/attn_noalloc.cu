@@ -138,6 +138,7 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
   p.q_scale = p.k_scale = p.v_scale = nullptr;
   p.cu_q = p.cu_k = nullptr;
   p.total_q = p.total_k = 0;
+  p.vl_sched = 0;
   p.N = N;
   p.BH = B * H;
   p.H = H;

@@ -123,3 +123,17 @@ def test_bad_offsets_are_reported_and_skipped():
     ea.attn_fwd_varlen(tq, tk, tv, tcq, tck, 250, o=o, causal=False)
     assert ea.attn_device_status() == ea.ATTN_ERR_INVALID_ARG
     assert torch.isnan(o[:300]).all() and not torch.isnan(o[300:]).any()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_more_sequences_than_the_schedule_holds(causal):
+    """1100 short sequences: more than the in-kernel schedule's 1024, so the launch deals out
+    units in the plain round order (empty ones skipped) -- same results."""
+    lq = [int(x) for x in uniform_lengths(1100, 1, 24, seed=9)]
+    _run(lq, lq, 1, 64, causal, seed=10)
+
+
+def test_schedule_covers_sequences_of_one_length_and_empty_ones():
+    """Sorting by tile pairs with many ties and zero-length sequences in between."""
+    lq = [256, 0, 256, 512, 0, 1, 256, 257, 0, 512]
+    _run(lq, lq, 2, 128, True, seed=11)
