@@ -53,6 +53,10 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_strided.restype = i
         L.attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, f, i, i, i, vp]
         L.attn_fwd_varlen.restype = i
+        L.attn_bwd_strided.argtypes = [vp] * 10 + [i, i, i, i, i, vp, f, i, i, vp]
+        L.attn_bwd_strided.restype = i
+        L.attn_bwd_varlen.argtypes = [vp] * 12 + [i, i, i, i, i, i, i, vp, f, i, i, vp]
+        L.attn_bwd_varlen.restype = i
         L.attn_hadamard_quant.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
         L.attn_hadamard_quant.restype = i
         L.attn_hadamard_quant_qkv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
@@ -283,6 +287,83 @@ def attn_bwd_qk(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None
     _check(lib().attn_bwd_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
                              _ptr(workspace), B, H, Nq, Nk, d, s, int(bool(causal)), gcode, _stream_ptr(stream)),
            "attn_bwd_qk")
+    return dq, dk, dv
+
+
+def attn_bwd_strided(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None, scale=None, causal=False,
+                     g_dtype=None, stream=None):
+    """attn_bwd_qk on logical [B, H, N, d] bf16 views with any strides whose last one is 1 (the
+    backward of :func:`attn_fwd_strided`); ``lse`` [B, H, Nq] contiguous.  Gradients default to
+    tensors with their input's memory order.  Returns ``(dq, dk, dv)``."""
+    import torch
+    B, H, Nq, d = _dims(q)
+    Nk = int(k.shape[2])
+    if k.shape != v.shape or tuple(k.shape) != (B, H, Nk, d) or o.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("expected q, o, dout [B, H, Nq, d] and k, v [B, H, Nk, d]")
+    for t in (q, k, v, o, dout):
+        if t.dtype != torch.bfloat16 or t.stride(-1) != 1:
+            raise ValueError("q, k, v, o, dout must be bf16 with a contiguous last dimension")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, H, Nq):
+        raise ValueError("lse must be contiguous float32 [B, H, Nq]")
+    gd = g_dtype or (dq.dtype if dq is not None else torch.bfloat16)
+    dq = dq if dq is not None else torch.empty_like(q, dtype=gd)
+    dk = dk if dk is not None else torch.empty_like(k, dtype=gd)
+    dv = dv if dv is not None else torch.empty_like(v, dtype=gd)
+    for g, ref in ((dq, q), (dk, k), (dv, k)):
+        if g.shape != ref.shape or g.stride(-1) != 1:
+            raise ValueError("gradients must have their input's shape and a contiguous last dimension")
+    if workspace is None:
+        workspace = torch.empty(attn_bwd_workspace_bytes(B, H, Nq) // 4, dtype=torch.float32, device=q.device)
+    strides = (ctypes.c_longlong * 24)(*[int(x) for t in (q, k, v, o, dout, dq, dk, dv) for x in t.stride()[:3]])
+    gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_bwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                  _ptr(dv), _ptr(workspace), B, H, Nq, Nk, d, ctypes.cast(strides, ctypes.c_void_p),
+                                  s, int(bool(causal)), gcode, _stream_ptr(stream)), "attn_bwd_strided")
+    return dq, dk, dv
+
+
+def attn_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, dq=None, dk=None,
+                    dv=None, workspace=None, scale=None, causal=False, g_dtype=None, stream=None):
+    """The backward of :func:`attn_fwd_varlen`: ``q``, ``o``, ``dout`` [total_q, H, d], ``k``, ``v``
+    [total_k, H, d] (bf16, row and head strides free, last dimension contiguous), ``lse``
+    [H, total_q].  Returns ``(dq, dk, dv)``."""
+    import torch
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape or o.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("expected q, o, dout [total_q, H, d] and k, v [total_k, H, d]")
+    total_q, H, d = (int(x) for x in q.shape)
+    total_k = int(k.shape[0])
+    if (int(k.shape[1]), int(k.shape[2])) != (H, d):
+        raise ValueError("k and v must have q's H and d")
+    for t in (q, k, v, o, dout):
+        if t.dtype != torch.bfloat16 or t.stride(-1) != 1:
+            raise ValueError("q, k, v, o, dout must be bf16 with a contiguous last dimension")
+    for c in (cu_seqlens_q, cu_seqlens_k):
+        if c.dtype != torch.int32 or c.dim() != 1 or not c.is_contiguous() or not c.is_cuda:
+            raise ValueError("cu_seqlens must be contiguous int32 cuda tensors")
+    if cu_seqlens_k.shape != cu_seqlens_q.shape:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B + 1 entries")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (H, total_q):
+        raise ValueError("lse must be contiguous float32 [H, total_q]")
+    B = int(cu_seqlens_q.shape[0]) - 1
+    gd = g_dtype or (dq.dtype if dq is not None else torch.bfloat16)
+    dq = dq if dq is not None else torch.empty_like(q, dtype=gd)
+    dk = dk if dk is not None else torch.empty_like(k, dtype=gd)
+    dv = dv if dv is not None else torch.empty_like(v, dtype=gd)
+    for g, ref in ((dq, q), (dk, k), (dv, k)):
+        if g.shape != ref.shape or g.stride(-1) != 1:
+            raise ValueError("gradients must have their input's shape and a contiguous last dimension")
+    mq = min(int(max_seqlen_q), total_q)
+    if workspace is None:
+        workspace = torch.empty(attn_bwd_workspace_bytes(B, H, mq) // 4, dtype=torch.float32, device=q.device)
+    strides = (ctypes.c_longlong * 16)(*[int(x) for t in (q, k, v, o, dout, dq, dk, dv) for x in t.stride()[:2]])
+    gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                 _ptr(dv), _ptr(workspace), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, H, total_q,
+                                 total_k, int(max_seqlen_q), int(max_seqlen_k), d,
+                                 ctypes.cast(strides, ctypes.c_void_p), s, int(bool(causal)), gcode,
+                                 _stream_ptr(stream)), "attn_bwd_varlen")
     return dq, dk, dv
 
 

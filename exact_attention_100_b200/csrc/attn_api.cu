@@ -424,9 +424,18 @@ unsigned long long attn_bwd_workspace_bytes(int B, int H, int N) {
 
 namespace {
 
+// Packed-batch description for the backward (nullptr: fixed-length batch).
+struct Packed {
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
+};
+
+// attn_bwd, attn_bwd_qk, attn_bwd_strided and attn_bwd_varlen.  st8: element strides of q, k, v,
+// o, dout, dq, dk, dv.  Fixed-length batches: Nq, Nk are the lengths; packed ones: the longest.
 int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-             void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
-             int causal, int g_dtype, void* stream) {
+             void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk, int d, const Strides* st8,
+             const Packed* pk, float scale, int causal, int g_dtype, void* stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
@@ -444,17 +453,20 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const v
   DeviceState* st = nullptr;
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
+  const int rows_q = pk ? pk->total_q : Nq, rows_k = pk ? pk->total_k : Nk, nbat = pk ? 1 : B;
+  const Strides &sq = st8[0], &sk = st8[1], &sv = st8[2], &so = st8[3], &sdo = st8[4];
   CUtensorMap mq, mk, mv, mdo;
-  if (!encode_rows_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nq, B * H) ||
-      !encode_rows_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nk, B * H) ||
-      !encode_rows_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nk, B * H) ||
-      !encode_rows_map(&mdo, dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nq, B * H))
+  if (!encode_fwd_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, rows_q, H, nbat, sq.sn, sq.sh, sq.sb) ||
+      !encode_fwd_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, rows_k, H, nbat, sk.sn, sk.sh, sk.sb) ||
+      !encode_fwd_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, rows_k, H, nbat, sv.sn, sv.sh, sv.sb) ||
+      !encode_fwd_map(&mdo, dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, rows_q, H, nbat, sdo.sn, sdo.sh, sdo.sb))
     return ATTN_ERR_CUDA;
   ea::BwdParams p;
   p.lse = lse;
   p.o = o;
   p.dout = dout;
   p.BH = B * H;
+  p.H = H;
   p.N = Nq;
   p.n_blocks = static_cast<int>(n_blocks);
   p.n_pad = static_cast<int>(n_blocks * 128);
@@ -471,6 +483,15 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const v
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.causal = causal;
   p.g_fp32 = g_dtype == ATTN_FP32 ? 1 : 0;
+  p.o_sb = so.sb, p.o_sh = so.sh, p.o_sn = so.sn;
+  p.do_sb = sdo.sb, p.do_sh = sdo.sh, p.do_sn = sdo.sn;
+  p.dq_sb = st8[5].sb, p.dq_sh = st8[5].sh, p.dq_sn = st8[5].sn;
+  p.dk_sb = st8[6].sb, p.dk_sh = st8[6].sh, p.dk_sn = st8[6].sn;
+  p.dv_sb = st8[7].sb, p.dv_sh = st8[7].sh, p.dv_sn = st8[7].sn;
+  p.cu_q = pk ? pk->cu_q : nullptr;
+  p.cu_k = pk ? pk->cu_k : nullptr;
+  p.total_q = pk ? pk->total_q : 0;
+  p.total_k = pk ? pk->total_k : 0;
   if (ea::launch_attn_bwd(d, mq, mk, mv, mdo, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(3);
@@ -484,13 +505,56 @@ extern "C" {
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
              void* dq, void* dk, void* dv, void* workspace, int B, int H, int N, int d, float scale, int causal,
              int g_dtype, void* stream) {
-  return bwd_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, N, N, d, scale, causal, g_dtype, stream);
+  const Strides s = contiguous_strides(H, N, d);
+  const Strides st8[8] = {s, s, s, s, s, s, s, s};
+  return bwd_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, N, N, d, st8, nullptr, scale, causal, g_dtype,
+                  stream);
 }
 
 int attn_bwd_qk(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                 void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
                 int causal, int g_dtype, void* stream) {
-  return bwd_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale, causal, g_dtype, stream);
+  const Strides a = contiguous_strides(H, Nq, d), c = contiguous_strides(H, Nk, d);
+  const Strides st8[8] = {a, c, c, a, a, a, c, c};
+  return bwd_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Nq, Nk, d, st8, nullptr, scale, causal, g_dtype,
+                  stream);
+}
+
+int attn_bwd_strided(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                     void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk, int d,
+                     const long long* strides, float scale, int causal, int g_dtype, void* stream) {
+  if (strides == nullptr || B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0) return ATTN_ERR_INVALID_ARG;
+  Strides st8[8];
+  for (int t = 0; t < 8; ++t) {
+    const bool key_side = t == 1 || t == 2 || t == 6 || t == 7;  // k, v, dk, dv
+    if (!canonical_strides(strides + 3 * t, B, H, key_side ? Nk : Nq, &st8[t])) return ATTN_ERR_INVALID_ARG;
+  }
+  return bwd_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Nq, Nk, d, st8, nullptr, scale, causal, g_dtype,
+                  stream);
+}
+
+int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                    void* dq, void* dk, void* dv, void* workspace, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                    int B, int H, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                    const long long* strides, float scale, int causal, int g_dtype, void* stream) {
+  if (!cu_seqlens_q || !cu_seqlens_k || !strides || B <= 0 || H <= 0) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
+    return ATTN_ERR_INVALID_ARG;
+  constexpr int kMaxRows = 0x7FFFFFFF - (1 << 20);
+  if (total_q <= 0 || total_k <= 0 || total_q > kMaxRows || total_k > kMaxRows || max_seqlen_q <= 0 ||
+      max_seqlen_k <= 0 || max_seqlen_q > kMaxRows || max_seqlen_k > kMaxRows)
+    return ATTN_ERR_INVALID_ARG;
+  if (max_seqlen_q > total_q) max_seqlen_q = total_q;  // no sequence is longer than its tensor
+  if (max_seqlen_k > total_k) max_seqlen_k = total_k;
+  Strides st8[8];
+  for (int t = 0; t < 8; ++t) {
+    const bool key_side = t == 1 || t == 2 || t == 6 || t == 7;
+    const long long s3[3] = {8, strides[2 * t + 1], strides[2 * t]};  // {batch (unused), head, row}
+    if (!canonical_strides(s3, 1, H, key_side ? total_k : total_q, &st8[t])) return ATTN_ERR_INVALID_ARG;
+  }
+  const Packed pk{cu_seqlens_q, cu_seqlens_k, total_q, total_k};
+  return bwd_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, max_seqlen_q, max_seqlen_k, d, st8, &pk, scale,
+                  causal, g_dtype, stream);
 }
 
 int attn_device_status(void* stream) {

@@ -54,10 +54,58 @@ __device__ __forceinline__ void exp2_pair(float& p0, float& p1, float x0, float 
   p1 = ex2_approx(x1);
 }
 
+// The sequence of one (batch entry, head) pair: fixed-length batches take every field from the
+// parameters, packed batches (VL) read the row ranges from the offset arrays.
+struct BSeq {
+  int h, bc;        // head; batch coordinate of the tensors (0 for packed batches)
+  int N, Nk;        // query and key lengths
+  int nb, nbk;      // 128-row query and key blocks
+  int off;          // Nk - N: key j is visible to query i iff j <= i + off (causal)
+  int q0, k0;       // first query and key row (0 unless packed)
+  long long lse0;   // LSE index of the sequence's row 0 for this head
+  bool bad;         // packed offsets out of order, outside the tensors or too long
+};
+
+template <bool VL>
+__device__ __forceinline__ BSeq bseq_of(int bh, const BwdParams& p) {
+  BSeq s;
+  const int b = bh / p.H;
+  s.h = bh - b * p.H;
+  s.bad = false;
+  if constexpr (!VL) {
+    s.bc = b;
+    s.N = p.N;
+    s.Nk = p.Nk;
+    s.nb = p.n_blocks;
+    s.nbk = p.nbk;
+    s.off = p.off;
+    s.q0 = s.k0 = 0;
+    s.lse0 = static_cast<long long>(bh) * p.N;
+  } else {
+    int q0 = __ldg(p.cu_q + b), q1 = __ldg(p.cu_q + b + 1);
+    int k0 = __ldg(p.cu_k + b), k1 = __ldg(p.cu_k + b + 1);
+    if (!(0 <= q0 && q0 <= q1 && q1 <= p.total_q && q1 - q0 <= p.N && 0 <= k0 && k0 <= k1 && k1 <= p.total_k &&
+          k1 - k0 <= p.Nk)) {
+      s.bad = true;
+      q0 = q1 = k0 = k1 = 0;
+    }
+    s.bc = 0;
+    s.N = q1 - q0;
+    s.Nk = k1 - k0;
+    s.nb = (s.N + 127) / 128;
+    s.nbk = (s.Nk + 127) / 128;
+    s.off = s.Nk - s.N;
+    s.q0 = q0;
+    s.k0 = k0;
+    s.lse0 = static_cast<long long>(s.h) * p.total_q + q0;
+  }
+  return s;
+}
+
 // ------------------------------------------------------------------------------ preparation
 // One row per group of d/16 lanes: D = sum_c dO * O (f32), lse2 = LSE * log2 e; rows past N get
 // D = 0 and lse2 = +inf, so that their P (= 2^(s - lse2)) is exactly zero in the main kernels.
-template <int D>
+template <int D, bool VL>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
   constexpr int kLanes = D / 16;
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -67,12 +115,18 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
   const bool in_range = row < total;
   const int bh = in_range ? static_cast<int>(row / p.n_pad) : 0;
   const int r = in_range ? static_cast<int>(row % p.n_pad) : 0;
-  const bool valid = in_range && r < p.N;
+  const BSeq S = bseq_of<VL>(bh, p);
+  if constexpr (VL) {
+    if (S.bad && in_range && r == 0 && part == 0) atomicOr(p.status, kDevStatusBadSeqlens);
+  }
+  const bool valid = in_range && r < S.N;
   float acc = 0.f;
   if (valid) {
-    const size_t off = (static_cast<size_t>(bh) * p.N + r) * D + part * 16;
-    const uint4* po = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.o) + off);
-    const uint4* pd = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dout) + off);
+    const long long row_q = S.q0 + r;
+    const long long oo = S.bc * p.o_sb + S.h * p.o_sh + row_q * p.o_sn + part * 16;
+    const long long od = S.bc * p.do_sb + S.h * p.do_sh + row_q * p.do_sn + part * 16;
+    const uint4* po = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.o) + oo);
+    const uint4* pd = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dout) + od);
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const uint4 a = __ldg(po + c), b = __ldg(pd + c);
@@ -88,7 +142,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
   for (int o = kLanes / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if (in_range && part == 0) {
     p.delta[row] = valid ? acc : 0.f;
-    p.lse2[row] = valid ? p.lse[static_cast<size_t>(bh) * p.N + r] * kLog2e : INFINITY;
+    p.lse2[row] = valid ? p.lse[S.lse0 + r] * kLog2e : INFINITY;
   }
 }
 
@@ -106,13 +160,14 @@ struct BwdCfg {
   static constexpr uint32_t kIdD = make_idesc(128, D, 1, true);     // accumulations, B MN-major
 };
 
-// Loads a 128-row tile at rows [row0, row0 + 128) of head bh: one 128-row x 128-byte TMA box
-// per column box (the maps the forward uses).
+// Loads a 128-row tile at rows [row0, row0 + 128) of head h, batch coordinate bc: one 128-row x
+// 128-byte TMA box per column box (4-D maps (d, rows, heads, batch), as the forward's).
 template <int D>
-__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row0, int bh) {
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row0, int h,
+                                          int bc) {
   using C = BwdCfg<D>;
 #pragma unroll
-  for (int b = 0; b < C::kBoxes; ++b) tma_load_3d(dst + b * C::kBoxBytes, map, bar, b * 64, row0, bh);
+  for (int b = 0; b < C::kBoxes; ++b) tma_load_4d(dst + b * C::kBoxBytes, map, bar, b * 64, row0, h, bc);
 }
 
 // X[tmem, 128 x 128] = A B^T with A and B 128 x D tiles in shared memory, both K-major.
@@ -180,14 +235,20 @@ __device__ __forceinline__ int unit_of(int k) {
 
 // dK/dV unit u: key block kb of head bh and the first query block i0 that sees any of its keys
 // (causal, bottom-right: query r sees key c iff c <= r + off); i0 >= n_blocks: no query does.
+// `present`: the block lies inside its sequence (always, unless packed).
 struct KvUnit {
   int bh, kb, i0;
+  bool present;
+  BSeq S;
 };
+template <bool VL>
 __device__ __forceinline__ KvUnit kv_unit(int u, const BwdParams& p) {
   KvUnit U;
   U.bh = u % p.BH;
   U.kb = u / p.BH;
-  const int first_q = U.kb * 128 - p.off;  // the smallest query that sees the block's first key
+  U.S = bseq_of<VL>(U.bh, p);
+  U.present = U.kb < U.S.nbk;
+  const int first_q = U.kb * 128 - U.S.off;  // the smallest query that sees the block's first key
   U.i0 = (!p.causal || first_q <= 0) ? 0 : first_q / 128;
   return U;
 }
@@ -196,16 +257,21 @@ __device__ __forceinline__ KvUnit kv_unit(int u, const BwdParams& p) {
 // blocks (0: its rows see no key).
 struct QUnit {
   int bh, qb, n;
+  bool present;
+  BSeq S;
 };
+template <bool VL>
 __device__ __forceinline__ QUnit q_unit(int u, const BwdParams& p) {
   QUnit U;
   U.bh = u % p.BH;
   U.qb = p.causal ? p.n_blocks - 1 - u / p.BH : u / p.BH;
+  U.S = bseq_of<VL>(U.bh, p);
+  U.present = U.qb < U.S.nb;
   if (!p.causal) {
-    U.n = p.nbk;
+    U.n = U.S.nbk;
   } else {
-    const int last = min(U.qb * 128 + 127, p.N - 1) + p.off;
-    U.n = last < 0 ? 0 : min(last / 128 + 1, p.nbk);
+    const int last = min(U.qb * 128 + 127, U.S.N - 1) + U.S.off;
+    U.n = last < 0 ? 0 : min(last / 128 + 1, U.S.nbk);
   }
   return U;
 }
@@ -256,7 +322,7 @@ struct DkdvCfg : BwdCfg<D> {
   static_assert(256 + 2 * D <= 512, "TMEM budget");
 };
 
-template <int D>
+template <int D, bool VL>
 __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -313,7 +379,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const AbortState ab{abort_flag, p.status};
-  const int nb = p.n_blocks;
   const int num_units = p.BH * p.nbk;
 
   if (warp < C::kComputeWarps) {
@@ -326,15 +391,21 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     for (int k = 0; ok; ++k) {
       const int u = unit_of(k);
       if (u >= num_units) break;
-      const KvUnit U = kv_unit(u, p);
-      const int bh = U.bh, kb = U.kb, i0 = U.i0;
+      const KvUnit U = kv_unit<VL>(u, p);
+      if constexpr (VL) {
+        if (!U.present) continue;  // past its sequence's keys: every role skips it
+      }
+      const BSeq& S = U.S;
+      const int kb = U.kb, i0 = U.i0, nb = S.nb;
       const int key_g = kb * 128 + row;
+      const long long key_row = S.k0 + key_g;
+      const size_t off_v = static_cast<size_t>(S.bc * p.dv_sb + S.h * p.dv_sh + key_row * p.dv_sn) + h * (D / 2);
+      const size_t off_k = static_cast<size_t>(S.bc * p.dk_sb + S.h * p.dk_sh + key_row * p.dk_sn) + h * (D / 2);
       if (i0 >= nb) {
         // no query sees these keys (causal, more keys than queries): dK = dV = 0
-        if (key_g < p.Nk) {
-          const size_t off = (static_cast<size_t>(bh) * p.Nk + key_g) * D + h * (D / 2);
-          zero_row<D / 2>(p.dv, off, p.g_fp32 != 0);
-          zero_row<D / 2>(p.dk, off, p.g_fp32 != 0);
+        if (key_g < S.Nk) {
+          zero_row<D / 2>(p.dv, off_v, p.g_fp32 != 0);
+          zero_row<D / 2>(p.dk, off_k, p.g_fp32 != 0);
         }
         continue;
       }
@@ -347,7 +418,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                                                            2 * C::kTileBytes);
         const float* dlt = lse2 + 128;
         // some query of block i misses some key of block kb (bottom-right causal mask)
-        const bool diag = p.causal && kb * 128 + 127 > i * 128 + p.off;
+        const bool diag = p.causal && kb * 128 + 127 > i * 128 + S.off;
         // pass 1, from S^T alone: P^T, kept in registers and stored as bf16 over this half's first
         // 32 S^T columns [64h, 64h + 32) (already read by this thread)
         ok = warp_all(wait_bar(st_s, qc & 1u, ab));
@@ -369,8 +440,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
             f2_fma(x0, x1, __uint_as_float(sv[2 * t]), __uint_as_float(sv[2 * t + 1]), p.scale_log2, p.scale_log2,
                    -lse2[qq], -lse2[qq + 1]);
             exp2_pair(p0, p1, x0, x1);
-            if (diag && i * 128 + qq + p.off < key_g) p0 = 0.f;  // key after the query's diagonal
-            if (diag && i * 128 + qq + 1 + p.off < key_g) p1 = 0.f;
+            if (diag && i * 128 + qq + S.off < key_g) p0 = 0.f;  // key after the query's diagonal
+            if (diag && i * 128 + qq + 1 + S.off < key_g) p1 = 0.f;
             pr[ql] = p0;
             pr[ql + 1] = p1;
           }
@@ -413,10 +484,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       ok = warp_all(wait_bar(dkv_done, uit & 1u, ab));
       if (!ok) break;
       tc_fence_after();
-      const bool valid = key_g < p.Nk;
-      const size_t off = (static_cast<size_t>(bh) * p.Nk + key_g) * D + h * (D / 2);  // this half's columns
-      store_row<D / 2>(lane_base + 256 + h * (D / 2), p.dv, off, 1.f, p.g_fp32 != 0, valid);
-      store_row<D / 2>(lane_base + 256 + D + h * (D / 2), p.dk, off, p.scale, p.g_fp32 != 0, valid);
+      const bool valid = key_g < S.Nk;
+      store_row<D / 2>(lane_base + 256 + h * (D / 2), p.dv, off_v, 1.f, p.g_fp32 != 0, valid);
+      store_row<D / 2>(lane_base + 256 + D + h * (D / 2), p.dk, off_k, p.scale, p.g_fp32 != 0, valid);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) bar_arrive(dkv_free);
@@ -432,8 +502,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int u = unit_of(k);
         if (u >= num_units) break;
-        const KvUnit U = kv_unit(u, p);
-        const int i0 = U.i0;
+        const KvUnit U = kv_unit<VL>(u, p);
+        if constexpr (VL) {
+          if (!U.present) continue;
+        }
+        const int i0 = U.i0, nb = U.S.nb;
         if (i0 >= nb) continue;  // no query sees the block: nothing loaded, nothing to compute
         if (!(ok = wait_bar(kv_full, uc & 1u, ab))) break;
         auto q_at = [&](uint32_t c) { return smem_addr(smem + C::kStageOff + (c % C::kStages) * C::kStageBytes); };
@@ -486,21 +559,25 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int u = unit_of(k);
         if (u >= num_units) break;
-        const KvUnit U = kv_unit(u, p);
-        const int bh = U.bh, kb = U.kb, i0 = U.i0;
+        const KvUnit U = kv_unit<VL>(u, p);
+        if constexpr (VL) {
+          if (!U.present) continue;
+        }
+        const BSeq& S = U.S;
+        const int bh = U.bh, kb = U.kb, i0 = U.i0, nb = S.nb;
         if (i0 >= nb) continue;
         if (uc > 0 && !(ok = wait_bar(kv_empty, (uc - 1u) & 1u, ab))) break;
         bar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
-        load_tile<D>(smem + C::kKOff, &tmK, kv_full, kb * 128, bh);
-        load_tile<D>(smem + C::kVOff, &tmV, kv_full, kb * 128, bh);
+        load_tile<D>(smem + C::kKOff, &tmK, kv_full, S.k0 + kb * 128, S.h, S.bc);
+        load_tile<D>(smem + C::kVOff, &tmV, kv_full, S.k0 + kb * 128, S.h, S.bc);
         ++uc;
         for (int i = i0; i < nb && ok; ++i, ++qc) {
           const uint32_t st = qc % C::kStages;
           if (!(ok = wait_bar(&st_empty[st], ((qc / C::kStages) & 1u) ^ 1u, ab))) break;
           uint8_t* base = smem + C::kStageOff + st * C::kStageBytes;
           bar_arrive_expect_tx(&st_full[st], 2 * C::kTileBytes + 1024);
-          load_tile<D>(base, &tmQ, &st_full[st], i * 128, bh);
-          load_tile<D>(base + C::kTileBytes, &tmdO, &st_full[st], i * 128, bh);
+          load_tile<D>(base, &tmQ, &st_full[st], S.q0 + i * 128, S.h, S.bc);
+          load_tile<D>(base + C::kTileBytes, &tmdO, &st_full[st], S.q0 + i * 128, S.h, S.bc);
           const size_t w = static_cast<size_t>(bh) * p.n_pad + static_cast<size_t>(i) * 128;
           bulk_load_g2s(base + 2 * C::kTileBytes, p.lse2 + w, 512, &st_full[st]);
           bulk_load_g2s(base + 2 * C::kTileBytes + 512, p.delta + w, 512, &st_full[st]);
@@ -548,7 +625,7 @@ struct DqCfg : BwdCfg<D> {
   static_assert(256 + D <= 384, "TMEM budget");
 };
 
-template <int D>
+template <int D, bool VL>
 __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -624,12 +701,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     for (int k = 0; ok; ++k) {
       const int u = unit_of(k);
       if (u >= num_units) break;
-      const QUnit U = q_unit(u, p);
+      const QUnit U = q_unit<VL>(u, p);
+      if constexpr (VL) {
+        if (!U.present) continue;  // past its sequence's queries: every role skips it
+      }
+      const BSeq& S = U.S;
       const int bh = U.bh, qb = U.qb, n = U.n;
       const int q_g = qb * 128 + row;
+      const size_t off_q = static_cast<size_t>(S.bc * p.dq_sb + S.h * p.dq_sh + (S.q0 + static_cast<long long>(q_g)) *
+                                               p.dq_sn) + h * (D / 2);
       if (n == 0) {
-        // these queries see no key (causal, more queries than keys): dQ = 0
-        if (q_g < p.N) zero_row<D / 2>(p.dq, (static_cast<size_t>(bh) * p.N + q_g) * D + h * (D / 2), p.g_fp32 != 0);
+        // these queries see no key (causal, more queries than keys, or no keys): dQ = 0
+        if (q_g < S.N) zero_row<D / 2>(p.dq, off_q, p.g_fp32 != 0);
         continue;
       }
       const size_t w = static_cast<size_t>(bh) * p.n_pad + q_g;
@@ -637,8 +720,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       const float dlt = p.delta[w];
       for (int j = 0; j < n && ok; ++j, ++sc) {
         const uint32_t t_ds = lane_base + 384 + (sc & 1u) * 64;
-        const bool mask = (j * 128 + 128 > p.Nk) || (p.causal && j * 128 + 127 > qb * 128 + p.off);
-        const int lim = min(p.Nk, p.causal ? q_g + p.off + 1 : p.Nk) - j * 128;  // visible keys of this block
+        const bool mask = (j * 128 + 128 > S.Nk) || (p.causal && j * 128 + 127 > qb * 128 + S.off);
+        const int lim = min(S.Nk, p.causal ? q_g + S.off + 1 : S.Nk) - j * 128;  // visible keys of this block
         // pass 1, from S alone: P in registers; then S's columns may take the next block
         ok = warp_all(wait_bar(s_full, sc & 1u, ab));
         if (!ok) break;
@@ -695,8 +778,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       ok = warp_all(wait_bar(dq_done, uit & 1u, ab));
       if (!ok) break;
       tc_fence_after();
-      store_row<D / 2>(lane_base + 256 + h * (D / 2), p.dq, (static_cast<size_t>(bh) * p.N + q_g) * D + h * (D / 2),
-                       p.scale, p.g_fp32 != 0, q_g < p.N);
+      store_row<D / 2>(lane_base + 256 + h * (D / 2), p.dq, off_q, p.scale, p.g_fp32 != 0, q_g < S.N);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) bar_arrive(dq_free);
@@ -718,7 +800,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int u = unit_of(k);
         if (u >= num_units) break;
-        const int n = q_unit(u, p).n;
+        const QUnit U = q_unit<VL>(u, p);
+        if constexpr (VL) {
+          if (!U.present) continue;
+        }
+        const int n = U.n;
         const uint32_t kb0 = kit, vb0 = vit;  // K_j = kb0 + j, V_j = vb0 + j
         kit += n;
         vit += n;
@@ -787,23 +873,27 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int u = unit_of(k);
         if (u >= num_units) break;
-        const QUnit U = q_unit(u, p);
-        const int bh = U.bh, qb = U.qb, n = U.n;
+        const QUnit U = q_unit<VL>(u, p);
+        if constexpr (VL) {
+          if (!U.present) continue;
+        }
+        const BSeq& S = U.S;
+        const int qb = U.qb, n = U.n;
         if (qit > 0 && !(ok = wait_bar(qdo_empty, (qit - 1u) & 1u, ab))) break;
         bar_arrive_expect_tx(qdo_full, 2 * C::kTileBytes);
-        load_tile<D>(smem + C::kQOff, &tmQ, qdo_full, qb * 128, bh);
-        load_tile<D>(smem + C::kDoOff, &tmdO, qdo_full, qb * 128, bh);
+        load_tile<D>(smem + C::kQOff, &tmQ, qdo_full, S.q0 + qb * 128, S.h, S.bc);
+        load_tile<D>(smem + C::kDoOff, &tmdO, qdo_full, S.q0 + qb * 128, S.h, S.bc);
         ++qit;
         for (int j = 0; j < n && ok; ++j) {
           const uint32_t ks = kit % C::kKSlots;
           if (!(ok = wait_bar(&kempty[ks], ((kit / C::kKSlots) & 1u) ^ 1u, ab))) break;
           bar_arrive_expect_tx(&kfull[ks], C::kTileBytes);
-          load_tile<D>(smem + C::kKOff + ks * C::kTileBytes, &tmK, &kfull[ks], j * 128, bh);
+          load_tile<D>(smem + C::kKOff + ks * C::kTileBytes, &tmK, &kfull[ks], S.k0 + j * 128, S.h, S.bc);
           ++kit;
           const uint32_t vs = vit % C::kVSlots;
           if (!(ok = wait_bar(&vempty[vs], ((vit / C::kVSlots) & 1u) ^ 1u, ab))) break;
           bar_arrive_expect_tx(&vfull[vs], C::kTileBytes);
-          load_tile<D>(smem + C::kVOff + vs * C::kTileBytes, &tmV, &vfull[vs], j * 128, bh);
+          load_tile<D>(smem + C::kVOff + vs * C::kTileBytes, &tmV, &vfull[vs], S.k0 + j * 128, S.h, S.bc);
           ++vit;
         }
       }
@@ -825,51 +915,57 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool VL>
 cudaError_t setup_d() {
-  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, VL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        DkdvCfg<D>::kSmemAlloc);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DqCfg<D>::kSmemAlloc);
+    e = cudaFuncSetAttribute(bwd_dq_kernel<D, VL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DqCfg<D>::kSmemAlloc);
   return e;
 }
 
-template <int D>
+template <int D, bool VL>
 cudaError_t launch_d(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& dout,
                      const BwdParams& p, int num_sms, cudaStream_t stream) {
   const long long rows = static_cast<long long>(p.BH) * p.n_pad;
   const long long threads = rows * (D / 16);
   const long long blocks = (threads + 255) / 256;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  bwd_prep_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  bwd_prep_kernel<D, VL><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int kv_units = p.BH * p.nbk;
   const int kv_grid = kv_units < num_sms ? kv_units : num_sms;
-  bwd_dkdv_kernel<D><<<kv_grid, BwdCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(q, k, v, dout, p);
+  bwd_dkdv_kernel<D, VL><<<kv_grid, BwdCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(q, k, v, dout, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int q_units = p.BH * p.n_blocks;
   const int q_grid = q_units < num_sms ? q_units : num_sms;
-  bwd_dq_kernel<D><<<q_grid, BwdCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(q, k, v, dout, p);
+  bwd_dq_kernel<D, VL><<<q_grid, BwdCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(q, k, v, dout, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t setup_bwd_kernels() {
-  cudaError_t e = setup_d<64>();
-  if (e == cudaSuccess) e = setup_d<128>();
+  cudaError_t e = setup_d<64, false>();
+  if (e == cudaSuccess) e = setup_d<128, false>();
+  if (e == cudaSuccess) e = setup_d<64, true>();
+  if (e == cudaSuccess) e = setup_d<128, true>();
   return e;
 }
 
 cudaError_t launch_attn_bwd(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                             const CUtensorMap& dout, const BwdParams& p, int num_sms, cudaStream_t stream) {
+  const bool vl = p.cu_q != nullptr;
   switch (d) {
     case 64:
-      return launch_d<64>(q, k, v, dout, p, num_sms, stream);
+      return vl ? launch_d<64, true>(q, k, v, dout, p, num_sms, stream)
+                : launch_d<64, false>(q, k, v, dout, p, num_sms, stream);
     case 128:
-      return launch_d<128>(q, k, v, dout, p, num_sms, stream);
+      return vl ? launch_d<128, true>(q, k, v, dout, p, num_sms, stream)
+                : launch_d<128, false>(q, k, v, dout, p, num_sms, stream);
     default:
       return cudaErrorInvalidValue;
   }

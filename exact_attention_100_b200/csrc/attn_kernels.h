@@ -82,10 +82,24 @@ struct BwdParams {
   float scale_log2;       // scale * log2 e
   int causal;
   int g_fp32;             // gradients stored as f32 (else bf16)
+  int H;                  // heads (bh = b * H + h)
+  // element strides (batch, head, row) of O and dO (read by the preparation kernel) and of the
+  // gradients (d contiguous); Q, K, V and dO reach the main kernels through 4-D tensor maps
+  long long o_sb, o_sh, o_sn, do_sb, do_sh, do_sn;
+  long long dq_sb, dq_sh, dq_sn, dk_sb, dk_sh, dk_sn, dv_sb, dv_sh, dv_sn;
+  // packed batches (cu_q == nullptr: fixed lengths): sequence b owns query rows
+  // [cu_q[b], cu_q[b+1]) and key rows [cu_k[b], cu_k[b+1]); N and Nk are then the longest
+  // lengths the launch covers, LSE is [H, total_q], and the workspace keeps n_pad rows per
+  // (sequence, head)
+  const int* cu_q;
+  const int* cu_k;
+  int total_q;
+  int total_k;
 };
 
 cudaError_t setup_bwd_kernels();
-// D and LSE*log2e into the workspace, then dK/dV and dQ; q/k/v/dout maps as for the forward.
+// D and LSE*log2e into the workspace, then dK/dV and dQ; q/k/v/dout are 4-D maps as for the
+// forward (p.cu_q selects the packed-batch kernels).
 cudaError_t launch_attn_bwd(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                             const CUtensorMap& dout, const BwdParams& p, int num_sms, cudaStream_t stream);
 

@@ -264,6 +264,47 @@ int attn_bwd_qk(const void* q, const void* k, const void* v, const void* o, cons
                 void* stream);
 
 /*
+ * attn_bwd_strided -- attn_bwd_qk on tensors laid out with arbitrary strides (the backward of
+ * attn_fwd_strided).
+ *
+ *   q, k, v, o, dout, dq, dk, dv   logical [B, H, N, d] tensors (N = Nq for q, o, dout, dq;
+ *               Nk for k, v, dk, dv); element (b, h, n, c) at base + b*sb + h*sh + n*sn + c.
+ *   strides     HOST pointer to 24 int64 values: {sb, sh, sn} for q, k, v, o, dout, dq, dk, dv in
+ *               that order, in elements, with the rules of attn_fwd_strided.  The gradients
+ *               must not overlap the inputs or one another.
+ *   lse         [B, H, Nq] float32, contiguous (as attn_fwd_strided writes it).
+ * Other arguments, arithmetic and errors as for attn_bwd_qk, which is attn_bwd_strided with
+ * contiguous strides.
+ */
+int attn_bwd_strided(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                     int B, int H, int Nq, int Nk, int d, const long long* strides,
+                     float scale, int causal, int g_dtype, void* stream);
+
+/*
+ * attn_bwd_varlen -- the backward of attn_fwd_varlen: a packed batch of B sequences.
+ *
+ *   q, o, dout, dq   [total_q, H, d]; k, v, dk, dv [total_k, H, d] (bf16 inputs; gradients of
+ *               g_dtype), device; sequence b owns query rows cu_seqlens_q[b] .. [b+1]-1 and key
+ *               rows cu_seqlens_k[b] .. [b+1]-1.
+ *   lse         [H, total_q] float32 from attn_fwd_varlen.
+ *   cu_seqlens_q, cu_seqlens_k   DEVICE int32 arrays of B + 1 offsets, as for attn_fwd_varlen.
+ *   max_seqlen_q, max_seqlen_k   >= every query / key length; the launches are sized for them.
+ *   strides     HOST pointer to 16 int64 values: {row stride, head stride} for q, k, v, o, dout,
+ *               dq, dk, dv in that order, in elements, with the rules of attn_fwd_varlen.
+ *   workspace   attn_bwd_workspace_bytes(B, H, max_seqlen_q) bytes, device.
+ * Per sequence the arithmetic, the zero gradients of unseen keys and key-less queries, and the
+ * finiteness requirement on rows read past a sequence's end are those of attn_bwd_qk and
+ * attn_fwd_varlen; a sequence whose offsets break the rules is skipped and reported by
+ * attn_device_status() as ATTN_ERR_INVALID_ARG.
+ */
+int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                    const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                    const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H,
+                    int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                    const long long* strides, float scale, int causal, int g_dtype, void* stream);
+
+/*
  * attn_fwd_noalloc -- attn_fwd for callers that cannot allocate device memory.  The pages have
  * no counterpart; it exists for this library's users.
  *

@@ -46,6 +46,7 @@ from .attention import (  # noqa: F401
 from .attention_bwd import (  # noqa: F401
     attention_bwd_ref,
     attention_bwd_terms,
+    attention_varlen_bwd_ref,
     softmax_bwd_delta,
     softmax_probs,
 )

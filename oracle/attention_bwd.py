@@ -83,3 +83,26 @@ def attention_bwd_terms(q, k, v, do, scale: float, causal: bool = False):
     tq = scale * np.einsum("bij,bjc->bic", np.abs(ds), np.abs(k3))
     tk = scale * np.einsum("bij,bic->bjc", np.abs(ds), np.abs(q3))
     return tq.reshape(q.shape), tk.reshape(k.shape), tv.reshape(v.shape)
+
+
+def attention_varlen_bwd_ref(q, k, v, do, cu_q, cu_k, scale: float, causal: bool = False):
+    """(dQ, dK, dV) of the packed batch ``attention_varlen_ref`` defines, float64.
+
+    ``q``, ``do`` are ``[total_q, H, d]``, ``k``, ``v`` ``[total_k, H, d]``; sequence ``b`` owns
+    query rows ``cu_q[b]:cu_q[b+1]`` and key rows ``cu_k[b]:cu_k[b+1]``.  Each sequence is its
+    own problem, so its gradients are :func:`attention_bwd_ref` of its own rows; a sequence with
+    no keys (or no queries) has zero gradients, and rows outside every sequence stay zero.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        if q1 == q0 or k1 == k0:
+            continue
+        t = lambda x: x.transpose(1, 0, 2)  # [rows, H, d] <-> [H, rows, d]
+        g = attention_bwd_ref(t(q[q0:q1]), t(k[k0:k1]), t(v[k0:k1]), t(do[q0:q1]), scale, causal)
+        dq[q0:q1], dk[k0:k1], dv[k0:k1] = (t(x) for x in g)
+    return dq, dk, dv

@@ -32,7 +32,8 @@ def test_header_declares_the_boundary():
                             "attn_status_string", "attn_num_kernel_launches", "attn_shutdown",
                             "attn_fwd_noalloc", "attn_hadamard_quant_qkv", "attn_bwd",
                             "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided",
-                            "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv"])
+                            "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv", "attn_bwd_strided",
+                            "attn_bwd_varlen"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -222,6 +223,62 @@ def test_rope_hadamard_quant_qkv_rejects_bad_arguments(L):
     assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
 
 
+def _strides(vals):
+    return ctypes.cast((ctypes.c_longlong * len(vals))(*vals), ctypes.c_void_p)
+
+
+def test_bwd_strided_rejects_bad_arguments(L):
+    f = L.attn_bwd_strided
+    B, H, Nq, Nk, d = 2, 4, 128, 300, 128
+    q_s, k_s = [Nq * H * d, d, H * d], [Nk * H * d, d, H * d]
+    good = q_s + k_s + k_s + q_s + q_s + q_s + k_s + k_s  # q k v o dout dq dk dv
+    ok = [P, P, P, P, P, P, P2, P2, P2, P2, B, H, Nq, Nk, d, _strides(good), 0.1, 1, 0, NULL]
+    a = list(ok)
+    a[15] = NULL
+    assert f(*a) == ea.ATTN_ERR_INVALID_ARG
+    for i in range(10):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for pos, val in [(2, 4), (5, 0), (14, -8), (23, 1 << 36), (20, 12)]:
+        bad = list(good)
+        bad[pos] = val
+        a = list(ok)
+        a[15] = _strides(bad)
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (pos, val)
+    a = list(ok)
+    a[14] = 256
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+
+
+def test_bwd_varlen_rejects_bad_arguments(L):
+    f = L.attn_bwd_varlen
+    H, d = 4, 64
+    CU = ctypes.c_void_p(0x30000)
+    good = [H * d, d] * 8
+    ok = [P, P, P, P, P, P, P2, P2, P2, P2, CU, CU, 3, H, 1000, 900, 512, 600, d, _strides(good), 0.1, 1, 0, NULL]
+    for i in (0, 4, 5, 9, 10, 11, 19):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for i in (10, 11):
+        a = list(ok)
+        a[i] = ctypes.c_void_p(0x30002)
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for idx, val in [(12, 0), (13, 0), (14, 0), (15, -1), (16, 0), (17, 0), (20, 0.0), (21, 2), (22, 5)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+    bad = list(good)
+    bad[0] = 12
+    a = list(ok)
+    a[19] = _strides(bad)
+    assert f(*a) == ea.ATTN_ERR_INVALID_ARG
+    a = list(ok)
+    a[18] = 256
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+
+
 def test_bwd_workspace_bytes(L):
     assert L.attn_bwd_workspace_bytes(1, 1, 1) == 2 * 128 * 4
     assert L.attn_bwd_workspace_bytes(2, 16, 8192) == 2 * 32 * 8192 * 4
@@ -271,5 +328,5 @@ def test_python_binding_has_same_names():
     for name in ["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status", "attn_status_string",
                  "attn_num_kernel_launches", "attn_shutdown", "attn_fwd_noalloc", "attn_hadamard_quant_qkv",
                  "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided",
-                 "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv"]:
+                 "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv", "attn_bwd_strided", "attn_bwd_varlen"]:
         assert callable(getattr(ea, name)), name

@@ -141,3 +141,42 @@ def _mutant(kind):
 @pytest.mark.parametrize("kind", ["query_offsets_for_keys", "one_row_short", "top_left_causal", "lse_wrong_head"])
 def test_planted_packing_mistake_is_caught(kind):
     assert _pins(_mutant(kind)) != []
+
+
+# ---- the packed backward ---------------------------------------------------------------
+
+def test_varlen_backward_matches_finite_differences():
+    """Central differences of the packed forward oracle (an independent route to the gradient)
+    on a tiny batch with an empty key sequence and more queries than keys."""
+    from oracle import attention_varlen_bwd_ref
+    lengths = [(3, 4), (2, 0), (4, 2)]
+    q, k, v, cu_q, cu_k = _packed(lengths, 2, 3, seed=21)
+    do = np.random.default_rng(22).standard_normal(q.shape)
+    for causal in (False, True):
+        dq, dk, dv = attention_varlen_bwd_ref(q, k, v, do, cu_q, cu_k, 0.6, causal)
+        loss = lambda q_, k_, v_: float((attention_varlen_ref(q_, k_, v_, cu_q, cu_k, 0.6, causal)[0] * do).sum())
+        eps = 1e-6
+        for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+            num = np.zeros_like(x)
+            for idx in np.ndindex(*x.shape):
+                xp, xm = x.copy(), x.copy()
+                xp[idx] += eps
+                xm[idx] -= eps
+                args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+                args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+                num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert np.allclose(g, num, atol=1e-6, rtol=1e-5), (name, causal)
+
+
+def test_varlen_backward_equal_lengths_is_the_batched_oracle():
+    from oracle import attention_bwd_ref, attention_varlen_bwd_ref
+    B, H, N, d = 3, 2, 6, 4
+    rng = np.random.default_rng(23)
+    qb, kb, vb, dob = (rng.standard_normal((B, H, N, d)) for _ in range(4))
+    pack = lambda x: x.transpose(0, 2, 1, 3).reshape(B * N, H, d)
+    cu = np.arange(B + 1) * N
+    for causal in (False, True):
+        got = attention_varlen_bwd_ref(pack(qb), pack(kb), pack(vb), pack(dob), cu, cu, 0.5, causal)
+        ref = attention_bwd_ref(qb, kb, vb, dob, 0.5, causal)
+        for a, r in zip(got, ref):
+            assert np.allclose(a, pack(r), atol=1e-12, rtol=0)
