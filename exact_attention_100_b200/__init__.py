@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
         L.attn_hadamard_quant_qkv.restype = i
         L.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
         L.attn_fwd_fp8.restype = i
+        L.attn_fwd_fp8_qk.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+        L.attn_fwd_fp8_qk.restype = i
         L.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
         L.attn_fwd_noalloc.restype = i
         L.attn_bwd_workspace_bytes.argtypes = [i, i, i]
@@ -455,6 +457,27 @@ def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o=None, lse=None, scale=
     _check(lib().attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
                               _ptr(o), _ptr(lse), B, H, N, d, s, int(bool(causal)), od, _stream_ptr(stream)),
            "attn_fwd_fp8")
+    return o, lse
+
+
+def attn_fwd_fp8_qk(q8, k8, v8, q_scale, k_scale, v_scale, o=None, lse=None, scale=None, causal=False,
+                    o_dtype=None, stream=None):
+    """attn_fwd_fp8 with keys/values [B, H, Nk, d] of another length than the queries
+    [B, H, Nq, d] (bottom-right causal alignment, as attn_fwd_qk)."""
+    import torch
+    B, H, Nq, d = _dims(q8)
+    Nk = int(k8.shape[2])
+    if tuple(k8.shape) != (B, H, Nk, d) or v8.shape != k8.shape:
+        raise ValueError("k8 and v8 must be [B, H, Nk, d] with q8's B, H, d")
+    if o is None:
+        o = torch.empty((B, H, Nq, d), dtype=o_dtype or torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q8.device)
+    od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_fwd_fp8_qk(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
+                                 _ptr(o), _ptr(lse), B, H, Nq, Nk, d, s, int(bool(causal)), od, _stream_ptr(stream)),
+           "attn_fwd_fp8_qk")
     return o, lse
 
 

@@ -381,27 +381,33 @@ int attn_rope_hadamard_quant_qkv(const void* q, const void* k, const void* v, vo
   return hq_qkv(q, k, v, q8, k8, v8, q_scale, k_scale, v_scale, signs, cos, sin, n_pos, B, H, N, d, stream);
 }
 
-int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
-                 const float* v_scale, void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
-                 int o_dtype, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// attn_fwd_fp8 and attn_fwd_fp8_qk: E4M3 Q [B, H, Nq, d], K and V [B, H, Nk, d], contiguous.
+int fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
+            const float* v_scale, void* o, float* lse, int B, int H, int Nq, int Nk, int d, float scale, int causal,
+            int o_dtype, void* stream) {
   if (!q8 || !k8 || !v8 || !q_scale || !k_scale || !v_scale || !o) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || (lse && !aligned16(lse)) ||
       !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(v_scale))
     return ATTN_ERR_INVALID_ARG;
-  int rc = check_common(B, H, N, scale, causal, o_dtype);
+  int rc = check_common(B, H, Nq, scale, causal, o_dtype);
   if (rc != ATTN_OK) return rc;
+  if (Nk <= 0 || !units_fit(B, H, Nq)) return ATTN_ERR_INVALID_ARG;
   if (d != 128) return ATTN_ERR_UNSUPPORTED;
   DeviceState* st = nullptr;
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
-  const Strides s = contiguous_strides(H, N, d);
+  const Strides s = contiguous_strides(H, Nq, d), sk = contiguous_strides(H, Nk, d);
   CUtensorMap mq, mk, mv;
-  if (!encode_fwd_map(&mq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, H, B, s.sn, s.sh, s.sb) ||
-      !encode_fwd_map(&mk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, H, B, s.sn, s.sh, s.sb) ||
-      !encode_fwd_map(&mv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, H, B, s.sn, s.sh, s.sb))
+  if (!encode_fwd_map(&mq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Nq, H, B, s.sn, s.sh, s.sb) ||
+      !encode_fwd_map(&mk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Nk, H, B, sk.sn, sk.sh, sk.sb) ||
+      !encode_fwd_map(&mv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Nk, H, B, sk.sn, sk.sh, sk.sb))
     return ATTN_ERR_CUDA;
   ea::FwdParams p;
-  fill_params(p, o, lse, st->status, B, H, N, N, 2, scale, causal, o_dtype);
+  fill_params(p, o, lse, st->status, B, H, Nq, Nk, 2, scale, causal, o_dtype);
   p.o_sb = s.sb;
   p.o_sh = s.sh;
   p.o_sn = s.sn;
@@ -412,6 +418,22 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
   return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
+                 const float* v_scale, void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
+                 int o_dtype, void* stream) {
+  return fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, N, d, scale, causal, o_dtype, stream);
+}
+
+int attn_fwd_fp8_qk(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
+                    const float* v_scale, void* o, float* lse, int B, int H, int Nq, int Nk, int d, float scale,
+                    int causal, int o_dtype, void* stream) {
+  return fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, Nq, Nk, d, scale, causal, o_dtype, stream);
 }
 
 unsigned long long attn_bwd_workspace_bytes(int B, int H, int N) {

@@ -221,6 +221,19 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
                  int o_dtype, void* stream);
 
 /*
+ * attn_fwd_fp8_qk -- attn_fwd_fp8 with a key/value length Nk that may differ from the query
+ * length Nq: q8 [B, H, Nq, d] with q_scale [B, H, ceil(Nq/128)], k8 and v8 [B, H, Nk, d] with
+ * k_scale, v_scale [B, H, ceil(Nk/128)] (from attn_hadamard_quant on each tensor).  Causal
+ * masking bottom-right aligned and rows with no visible key as in attn_fwd_qk; other
+ * arguments, arithmetic and errors as for attn_fwd_fp8, which is attn_fwd_fp8_qk with
+ * Nq = Nk = N.
+ */
+int attn_fwd_fp8_qk(const void* q8, const void* k8, const void* v8,
+                    const float* q_scale, const float* k_scale, const float* v_scale,
+                    void* o, float* lse, int B, int H, int Nq, int Nk, int d, float scale,
+                    int causal, int o_dtype, void* stream);
+
+/*
  * attn_bwd_workspace_bytes -- size of the float32 workspace attn_bwd needs:
  * 2 * B * H * ceil(N / 128) * 128 * 4 bytes (per row, padded to whole 128-row blocks: the
  * rowsum D of dO * O and LSE * log2 e).  Returns 0 if a size is not positive.

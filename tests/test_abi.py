@@ -33,7 +33,7 @@ def test_header_declares_the_boundary():
                             "attn_fwd_noalloc", "attn_hadamard_quant_qkv", "attn_bwd",
                             "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided",
                             "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv", "attn_bwd_strided",
-                            "attn_bwd_varlen"])
+                            "attn_bwd_varlen", "attn_fwd_fp8_qk"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -279,6 +279,22 @@ def test_bwd_varlen_rejects_bad_arguments(L):
     assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
 
 
+def test_fwd_fp8_qk_rejects_bad_arguments(L):
+    f = L.attn_fwd_fp8_qk
+    ok = [P, P, P, P, P, P, P2, NULL, 1, 2, 128, 300, 128, 0.1, 1, 0, NULL]
+    for i in range(7):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for idx, val in [(8, 0), (10, 0), (11, 0), (11, -2), (13, 0.0), (14, 2), (15, 7)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+    a = list(ok)
+    a[12] = 64
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+
+
 def test_bwd_workspace_bytes(L):
     assert L.attn_bwd_workspace_bytes(1, 1, 1) == 2 * 128 * 4
     assert L.attn_bwd_workspace_bytes(2, 16, 8192) == 2 * 32 * 8192 * 4
@@ -328,5 +344,6 @@ def test_python_binding_has_same_names():
     for name in ["attn_fwd", "attn_hadamard_quant", "attn_fwd_fp8", "attn_device_status", "attn_status_string",
                  "attn_num_kernel_launches", "attn_shutdown", "attn_fwd_noalloc", "attn_hadamard_quant_qkv",
                  "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided",
-                 "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv", "attn_bwd_strided", "attn_bwd_varlen"]:
+                 "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv", "attn_bwd_strided", "attn_bwd_varlen",
+                 "attn_fwd_fp8_qk"]:
         assert callable(getattr(ea, name)), name

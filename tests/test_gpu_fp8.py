@@ -85,3 +85,41 @@ def test_fp8_workload_rmse_with_and_without_hadamard():
         rmse[use] = float(np.sqrt(np.mean(np.square(err))))
     assert rmse[True] <= 3e-2 and rmse[False] <= 3e-2, rmse
     assert rmse[True] < rmse[False], rmse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("nq,nk", [(128, 300), (300, 128), (1, 513), (513, 1), (640, 130)])
+def test_fp8_qk_against_oracle_on_dequantised_inputs(nq, nk, causal):
+    """attn_fwd_fp8_qk: key length different from the query length (bottom-right causal); the
+    same bars as the equal-length case on rows that see a key, O = 0 and LSE = -inf on rows
+    that see none."""
+    from exact_attention_100_b200.inputs import normal_qkv_lengths
+    d = 128
+    q, k, v = normal_qkv_lengths(1, 2, nq, nk, d, seed=nq + nk)
+    q8, qs, k8, ks, v8, vs = _quantise(q, k, v, hadamard_signs(d))
+    o, lse = ea.attn_fwd_fp8_qk(q8, k8, v8, qs, ks, vs, causal=causal, o_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+    qd = dequant_ref(q8.cpu().numpy(), qs.cpu().numpy())
+    kd = dequant_ref(k8.cpu().numpy(), ks.cpu().numpy())
+    vd = dequant_ref(v8.cpu().numpy(), vs.cpu().numpy())
+    o_ref, lse_ref = attention_ref(qd, kd, vd, 1 / math.sqrt(d), causal)
+    og = o.cpu().numpy().astype(np.float64)
+    lg = lse.cpu().numpy().astype(np.float64)
+    empty = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lg), empty) and np.all(og[empty] == 0.0)
+    err = (og - o_ref)[~empty]
+    if err.size:
+        assert float(np.sqrt(np.mean(err ** 2))) <= 1e-2
+        assert np.abs(err).max() <= (2.0 ** -4 + 1e-2) * np.abs(vd).max()
+        assert (np.abs(lg[~empty] - lse_ref[~empty]) / np.abs(lse_ref[~empty])).max() <= 1e-3
+
+
+def test_fp8_qk_equal_lengths_is_attn_fwd_fp8():
+    d = 128
+    q, k, v = normal_qkv(1, 2, 333, d, seed=4)
+    q8, qs, k8, ks, v8, vs = _quantise(q, k, v, hadamard_signs(d))
+    a = ea.attn_fwd_fp8(q8, k8, v8, qs, ks, vs, causal=True)
+    b = ea.attn_fwd_fp8_qk(q8, k8, v8, qs, ks, vs, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
