@@ -41,6 +41,7 @@ from .attention import (  # noqa: F401
     attention_blockwise_ref,
     attention_blockwise_lazy_ref,
     attention_varlen_ref,
+    merge_partials_ref,
     visible_mask,
 )
 from .attention_bwd import (  # noqa: F401

@@ -223,3 +223,29 @@ def attention_varlen_ref(q, k, v, cu_q, cu_k, scale: float, causal: bool = False
         out[q0:q1] = o_b.transpose(1, 0, 2)
         lse[:, q0:q1] = lse_b
     return out, lse
+
+
+def merge_partials_ref(o_a, lse_a, o_b, lse_b):
+    """Combine two attention results of the same queries over disjoint key sets, float64.
+
+    With ``l = exp(LSE)`` the softmax denominator of each part, the result over the union of the
+    keys is ``O = (l_a O_a + l_b O_b) / (l_a + l_b)`` and ``LSE = log(l_a + l_b)``: the running
+    rescale of the pages' tiled recurrence ("FlashAttention-2/3", "技术原理") applied to two
+    finished parts, and the merge a sequence-sharded (ring) attention needs (the same page names
+    long-context parallel systems).  A part with ``LSE = -inf`` (no visible key) contributes
+    nothing; if both are ``-inf`` the result is ``O = 0``, ``LSE = -inf``.
+    Shapes: O ``[..., N, d]``, LSE ``[..., N]``.
+    """
+    o_a, o_b = np.asarray(o_a, dtype=np.float64), np.asarray(o_b, dtype=np.float64)
+    lse_a, lse_b = np.asarray(lse_a, dtype=np.float64), np.asarray(lse_b, dtype=np.float64)
+    m = np.maximum(lse_a, lse_b)
+    has = np.isfinite(m)
+    m0 = np.where(has, m, 0.0)
+    wa = np.where(np.isfinite(lse_a), np.exp(lse_a - m0), 0.0)
+    wb = np.where(np.isfinite(lse_b), np.exp(lse_b - m0), 0.0)
+    tot = wa + wb
+    with np.errstate(divide="ignore", invalid="ignore"):
+        o = np.where(has[..., None], (wa[..., None] * o_a + wb[..., None] * o_b) / np.where(has, tot, 1.0)[..., None],
+                     0.0)
+        lse = np.where(has, m0 + np.log(np.where(has, tot, 1.0)), -np.inf)
+    return o, lse
