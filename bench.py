@@ -352,6 +352,7 @@ def run_ours(args):
     fp8 = fp8_section(args, dev, rank) if not args.no_fp8 else None
     bwd = bwd_section(args, dev, rank) if not args.no_bwd else None
     varlen = varlen_section(args, dev, rank) if not args.no_varlen else None
+    ring = ring_section(args, dev, rank) if not args.no_ring else None
     barrier()
     if rank == 0:
         peaks = load_peaks()
@@ -399,6 +400,8 @@ def run_ours(args):
             line["bwd"] = bwd
         if varlen is not None:
             line["varlen"] = varlen
+        if ring is not None:
+            line["ring_merge"] = ring
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -495,6 +498,39 @@ def fp8_section(args, dev, rank):
     except Exception as e:  # the E4M3 forward reports unsupported until it is built
         out["forward"] = {"unavailable": str(e)}
     return out
+
+
+def ring_section(args, dev, rank):
+    """Times the partial-result merge of the ring attention (attn_merge_partials) on the
+    headline's rows: float32 accumulator [2, 16, 8192, 128], bf16 part; HBM-bound."""
+    import torch
+    import exact_attention_100_b200 as ea
+    B, H, N, d = 2, 16, 8192, 128
+    g = torch.Generator(device=dev).manual_seed(17 + rank)
+    acc_o = torch.randn(B, H, N, d, device=dev, generator=g)
+    acc_l = torch.randn(B, H, N, device=dev, generator=g)
+    part_o = torch.randn(B, H, N, d, device=dev, generator=g).to(torch.bfloat16)
+    part_l = torch.randn(B, H, N, device=dev, generator=g)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for _ in range(3):
+        ea.attn_merge_partials(acc_o, acc_l, part_o, part_l, stream=stream)
+    steps = max(3, min(args.steps, 50))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        ea.attn_merge_partials(acc_o, acc_l, part_o, part_l, stream=stream)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    rows = B * H * N
+    nbytes = rows * d * (4 + 2 + 4) + rows * 4 * 3  # acc read + part read + acc written; three LSE rows
+    peaks = load_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": "merge of a bf16 partial (O, LSE) into a float32 accumulator, rows [2, 16, 8192], d=128",
+            "ms": ms, "achieved_gbs": gbs, "peak_gbs": float(peaks["hbm_gbs"]), "frac": gbs / float(peaks["hbm_gbs"]),
+            "bound": "hbm", "bytes_per_call": nbytes, "peak_source": peaks["source"]}
 
 
 VARLEN_WORKLOAD = dict(total=16384, lo=512, hi=4096, H=16, d=128, causal=True, seed=11)
@@ -692,6 +728,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
+    ap.add_argument("--no-ring", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv", "hq_rope", "varlen", "bwd"], default=None,
                     help="run --reps untimed calls of one entry point (for an ncu capture) and exit")

@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_fp8.restype = i
         L.attn_fwd_fp8_qk.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
         L.attn_fwd_fp8_qk.restype = i
+        L.attn_merge_partials.argtypes = [vp, vp, vp, vp, ctypes.c_longlong, i, i, vp]
+        L.attn_merge_partials.restype = i
         L.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
         L.attn_fwd_noalloc.restype = i
         L.attn_bwd_workspace_bytes.argtypes = [i, i, i]
@@ -479,6 +481,27 @@ def attn_fwd_fp8_qk(q8, k8, v8, q_scale, k_scale, v_scale, o=None, lse=None, sca
                                  _ptr(o), _ptr(lse), B, H, Nq, Nk, d, s, int(bool(causal)), od, _stream_ptr(stream)),
            "attn_fwd_fp8_qk")
     return o, lse
+
+
+def attn_merge_partials(o_acc, lse_acc, o_part, lse_part, stream=None):
+    """In place: (o_acc float32 [..., N, d], lse_acc float32 [..., N]) <- the attention result over
+    the union of their keys and those of (o_part [..., N, d] bf16 or float32, lse_part)."""
+    import torch
+    if o_acc.dtype != torch.float32 or lse_acc.dtype != torch.float32 or lse_part.dtype != torch.float32:
+        raise ValueError("o_acc, lse_acc and lse_part must be float32")
+    if o_part.dtype not in (torch.bfloat16, torch.float32) or o_part.shape != o_acc.shape:
+        raise ValueError("o_part must be bf16 or float32 with o_acc's shape")
+    if lse_acc.shape != o_acc.shape[:-1] or lse_part.shape != lse_acc.shape:
+        raise ValueError("lse_acc and lse_part must be o_acc's shape without its last dimension")
+    for t in (o_acc, lse_acc, o_part, lse_part):
+        if not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+    d = int(o_acc.shape[-1])
+    rows = int(lse_acc.numel())
+    pd = ATTN_FP32 if o_part.dtype == torch.float32 else ATTN_BF16
+    _check(lib().attn_merge_partials(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part), rows, d, pd,
+                                     _stream_ptr(stream)), "attn_merge_partials")
+    return o_acc, lse_acc
 
 
 def attn_device_status(stream=None) -> int:

@@ -9,6 +9,7 @@
 
 #include "../../include/attn.h"
 #include "attn_kernels.h"
+#include "attn_merge.h"
 
 namespace ea {
 cudaError_t setup_fwd_bf16_kernels();
@@ -187,6 +188,21 @@ const char* attn_status_string(int status) {
 }
 
 unsigned long long attn_num_kernel_launches(void) { return g_launches.load(); }
+
+int attn_merge_partials(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, long long rows,
+                        int d, int part_dtype, void* stream) {
+  if (!o_acc || !lse_acc || !o_part || !lse_part) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o_acc) || !aligned16(o_part) || (reinterpret_cast<uintptr_t>(lse_acc) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(lse_part) & 3u) != 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (rows <= 0 || rows > (1ll << 40) || d < 4 || d > 1024 || (d & 3) != 0) return ATTN_ERR_INVALID_ARG;
+  if (part_dtype != ATTN_BF16 && part_dtype != ATTN_FP32) return ATTN_ERR_INVALID_ARG;
+  if (ea::launch_merge_partials(o_acc, lse_acc, o_part, lse_part, rows, d, part_dtype == ATTN_FP32 ? 1 : 0,
+                                static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return ATTN_OK;
+}
 
 }  // extern "C"
 

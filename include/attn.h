@@ -350,6 +350,25 @@ int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float
  */
 int attn_device_status(void* stream);
 
+/*
+ * attn_merge_partials -- merge of two attention results of the same queries over disjoint key
+ * sets, in place: (o_acc, lse_acc) <- the result over the union of their keys.  With
+ * l = exp(LSE) the softmax denominator of a part, O = (l_a O_a + l_b O_b) / (l_a + l_b) and
+ * LSE = log(l_a + l_b) ("FlashAttention-2/3", section "技术原理": the running rescale applied to
+ * two finished parts); the step a sequence-sharded (ring) attention takes after each hop.
+ *
+ *   o_acc       [rows, d] float32, device, read and written (start from zeros).
+ *   lse_acc     [rows] float32, device, read and written (start from -inf: no key yet).
+ *   o_part      [rows, d] of part_dtype (ATTN_BF16 or ATTN_FP32), device: O of the new part.
+ *   lse_part    [rows] float32, device: its natural-log LSE (-inf: the row sees no key there).
+ *   rows        1 .. 2^40; any [B, H, N] of contiguous rows.   d  4 .. 1024, a multiple of 4.
+ * Arithmetic: float32, weights exp(LSE - max) so neither exponential overflows.  A row whose
+ * two LSEs are -inf keeps O = 0, LSE = -inf.  o_acc and o_part 16-byte aligned; the LSE arrays
+ * 4-byte aligned.  Returns ATTN_OK once the kernel is enqueued.
+ */
+int attn_merge_partials(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                        long long rows, int d, int part_dtype, void* stream);
+
 /* attn_status_string -- static, human-readable name of a status code (never NULL). */
 const char* attn_status_string(int status);
 

@@ -33,7 +33,7 @@ def test_header_declares_the_boundary():
                             "attn_fwd_noalloc", "attn_hadamard_quant_qkv", "attn_bwd",
                             "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided",
                             "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv", "attn_bwd_strided",
-                            "attn_bwd_varlen", "attn_fwd_fp8_qk"])
+                            "attn_bwd_varlen", "attn_fwd_fp8_qk", "attn_merge_partials"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -295,6 +295,26 @@ def test_fwd_fp8_qk_rejects_bad_arguments(L):
     assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
 
 
+def test_merge_partials_rejects_bad_arguments(L):
+    f = L.attn_merge_partials
+    ok = [P, P, P2, P2, 1000, 128, 0, NULL]
+    for i in range(4):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for i in (0, 2):
+        a = list(ok)
+        a[i] = MIS
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    a = list(ok)
+    a[1] = ctypes.c_void_p(0x10002)  # LSE arrays need 4-byte alignment
+    assert f(*a) == ea.ATTN_ERR_INVALID_ARG
+    for idx, val in [(4, 0), (4, -1), (4, (1 << 40) + 1), (5, 0), (5, 6), (5, 2048), (6, 2)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+
+
 def test_bwd_workspace_bytes(L):
     assert L.attn_bwd_workspace_bytes(1, 1, 1) == 2 * 128 * 4
     assert L.attn_bwd_workspace_bytes(2, 16, 8192) == 2 * 32 * 8192 * 4
@@ -345,5 +365,5 @@ def test_python_binding_has_same_names():
                  "attn_num_kernel_launches", "attn_shutdown", "attn_fwd_noalloc", "attn_hadamard_quant_qkv",
                  "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided",
                  "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv", "attn_bwd_strided", "attn_bwd_varlen",
-                 "attn_fwd_fp8_qk"]:
+                 "attn_fwd_fp8_qk", "attn_merge_partials"]:
         assert callable(getattr(ea, name)), name
