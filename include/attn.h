@@ -17,8 +17,9 @@
  *   - Pointers to tensors are DEVICE pointers (cudaMalloc'd or equivalent) on the current CUDA
  *     device, unless an argument says otherwise.  The caller owns every tensor.
  *   - Tensors are contiguous [B, H, N, d] (row-major, d fastest); LSE is contiguous [B, H, N]
- *     float32; per-block scales are contiguous [B, H, ceil(N/128)] float32.
- *   - Every tensor pointer must be 16-byte aligned.
+ *     float32; per-block scales are contiguous [B, H, ceil(N/128)] float32 -- except where an
+ *     entry point states its own layout (the *_strided, *_varlen and merge entry points).
+ *   - Every tensor pointer must be 16-byte aligned unless the entry point states otherwise.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Work is
  *     enqueued asynchronously; the call returns once it is enqueued.
  *   - Arguments are checked before any CUDA call; a bad argument returns an error status and
