@@ -683,6 +683,13 @@ def run_profile_case(args):
     if args.profile_case == "fwd":
         for _ in range(args.reps):
             ea.attn_fwd(q, k, v, causal=bool(causal))
+    elif args.profile_case == "merge":
+        acc_o = torch.randn(B, H, N, d, device=dev)
+        acc_l = torch.randn(B, H, N, device=dev)
+        part_o = torch.randn(B, H, N, d, device=dev).to(torch.bfloat16)
+        part_l = torch.randn(B, H, N, device=dev)
+        for _ in range(args.reps):
+            ea.attn_merge_partials(acc_o, acc_l, part_o, part_l)
     elif args.profile_case == "hq_rope":
         from exact_attention_100_b200.inputs import rope_tables
         cos, sin = (torch.from_numpy(np.ascontiguousarray(t.T)).to(dev) for t in rope_tables(N, d))
@@ -730,7 +737,7 @@ def main():
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-ring", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv", "hq_rope", "varlen", "bwd"], default=None,
+    ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv", "hq_rope", "varlen", "bwd", "merge"], default=None,
                     help="run --reps untimed calls of one entry point (for an ncu capture) and exit")
     ap.add_argument("--shape", type=int, nargs=5, default=[2, 16, 8192, 128, 1], metavar=("B", "H", "N", "d", "CAUSAL"))
     ap.add_argument("--reps", type=int, default=3)
