@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_fp8_qk.restype = i
         L.attn_merge_partials.argtypes = [vp, vp, vp, vp, ctypes.c_longlong, i, i, vp]
         L.attn_merge_partials.restype = i
+        L.attn_selftest_wait_timeout.argtypes = [vp]
+        L.attn_selftest_wait_timeout.restype = i
         L.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
         L.attn_fwd_noalloc.restype = i
         L.attn_bwd_workspace_bytes.argtypes = [i, i, i]
@@ -502,6 +504,12 @@ def attn_merge_partials(o_acc, lse_acc, o_part, lse_part, stream=None):
     _check(lib().attn_merge_partials(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part), rows, d, pd,
                                      _stream_ptr(stream)), "attn_merge_partials")
     return o_acc, lse_acc
+
+
+def attn_selftest_wait_timeout(stream=None) -> None:
+    """Launches the bounded-wait diagnostic: a wait that nothing satisfies gives up after its limit;
+    the next :func:`attn_device_status` returns ATTN_ERR_TIMEOUT."""
+    _check(lib().attn_selftest_wait_timeout(_stream_ptr(stream)), "attn_selftest_wait_timeout")
 
 
 def attn_device_status(stream=None) -> int:

@@ -10,6 +10,7 @@
 #include "../../include/attn.h"
 #include "attn_kernels.h"
 #include "attn_merge.h"
+#include "attn_selftest.h"
 
 namespace ea {
 cudaError_t setup_fwd_bf16_kernels();
@@ -188,6 +189,15 @@ const char* attn_status_string(int status) {
 }
 
 unsigned long long attn_num_kernel_launches(void) { return g_launches.load(); }
+
+int attn_selftest_wait_timeout(void* stream) {
+  DeviceState* st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  if (ea::launch_wait_selftest(st->status, static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return ATTN_OK;
+}
 
 int attn_merge_partials(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, long long rows,
                         int d, int part_dtype, void* stream) {

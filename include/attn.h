@@ -370,6 +370,15 @@ int attn_device_status(void* stream);
 int attn_merge_partials(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
                         long long rows, int d, int part_dtype, void* stream);
 
+/*
+ * attn_selftest_wait_timeout -- diagnostic of the failure detection every kernel relies on: one
+ * thread waits on an mbarrier that nothing arrives at, with the bounded wait the kernels use.
+ * After the bound (2 s) the wait gives up and records a timeout; the kernel returns.  The next
+ * attn_device_status(stream) returns ATTN_ERR_TIMEOUT, and the CUDA context stays usable.
+ * Returns ATTN_OK once the kernel is enqueued.
+ */
+int attn_selftest_wait_timeout(void* stream);
+
 /* attn_status_string -- static, human-readable name of a status code (never NULL). */
 const char* attn_status_string(int status);
 
