@@ -8,6 +8,20 @@ fallback: if the library is missing or a call fails, an exception is raised.
     o, lse = ea.attn_fwd(q, k, v, causal=True)           # q, k, v: [B, H, N, d] bf16 on cuda
     q8, qs = ea.attn_hadamard_quant(q, signs)             # E4M3 codes + per-block scales
     dq, dk, dv = ea.attn_bwd(q, k, v, o, lse, do, causal=True)  # backward (bf16 O from attn_fwd)
+
+Entry points, by family:
+
+* forward: ``attn_fwd``, ``attn_fwd_qk`` (key length != query length), ``attn_fwd_strided``
+  (any strides, e.g. sequence-major or fused QKV), ``attn_fwd_varlen`` (packed batches),
+  ``attn_fwd_noalloc`` (no device allocation);
+* FP8: ``attn_hadamard_quant``, ``attn_hadamard_quant_qkv``, ``attn_rope_hadamard_quant_qkv``
+  (rotary embedding fused), ``attn_fwd_fp8``, ``attn_fwd_fp8_qk``;
+* backward: ``attn_bwd``, ``attn_bwd_qk``, ``attn_bwd_strided``, ``attn_bwd_varlen``,
+  ``attn_bwd_workspace_bytes``;
+* sequence parallelism: ``attn_merge_partials`` and the ring driver in
+  :mod:`exact_attention_100_b200.ring`;
+* status: ``attn_device_status``, ``attn_status_string``, ``attn_num_kernel_launches``,
+  ``attn_selftest_wait_timeout``, ``attn_shutdown``.
 """
 
 from __future__ import annotations
