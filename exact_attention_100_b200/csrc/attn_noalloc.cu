@@ -113,6 +113,9 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
   if (!is_aligned16(q) || !is_aligned16(k) || !is_aligned16(v) || !is_aligned16(o) || (lse && !is_aligned16(lse)))
     return ATTN_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || N <= 0 || static_cast<long long>(B) * H > 0x7FFFFFFFLL) return ATTN_ERR_INVALID_ARG;
+  // the persistent kernel indexes its work units with int: B * H * ceil(N / 128) must fit
+  if (static_cast<long long>(B) * H * ((static_cast<long long>(N) + 127) / 128) >= 0x7FFFFFFFLL)
+    return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
   if (o_dtype != ATTN_BF16 && o_dtype != ATTN_FP32) return ATTN_ERR_INVALID_ARG;

@@ -316,6 +316,14 @@ def test_merge_partials_rejects_bad_arguments(L):
         assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
 
 
+def test_work_unit_count_overflow_is_refused(L):
+    """B * H * ceil(N / 128) units must fit an int: refused on the host, before any CUDA call."""
+    for f in (L.attn_fwd, L.attn_fwd_noalloc):
+        assert f(P, P, P, P2, NULL, 65536, 1024, 1 << 30, 128, 0.1, 0, 0, 0, NULL) == ea.ATTN_ERR_INVALID_ARG
+    assert L.attn_fwd_qk(P, P, P, P2, NULL, 65536, 1024, 1 << 30, 128, 128, 0.1, 0, 0, 0, NULL) == \
+        ea.ATTN_ERR_INVALID_ARG
+
+
 def test_bwd_workspace_bytes(L):
     assert L.attn_bwd_workspace_bytes(1, 1, 1) == 2 * 128 * 4
     assert L.attn_bwd_workspace_bytes(2, 16, 8192) == 2 * 32 * 8192 * 4
