@@ -217,6 +217,25 @@ def run_reference(args):
     }), flush=True)
 
 
+# ------------------------------------------------------------------------- rank aggregation
+def max_over_ranks(x, world, device):
+    """The largest ``x`` over the ranks of the default process group (the slowest rank's time);
+    ``x`` itself with one rank.  ``device`` is where the reduction's tensor lives (the rank's GPU
+    under NCCL, the CPU under gloo)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world, flops_per_rank, ms_max):
+    """Throughput of the whole job: every rank's work divided by the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------------- GPU arm
 def run_ours(args):
     import torch
@@ -237,12 +256,8 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def slowest(x):
+        return max_over_ranks(x, world, dev)
 
     w = WORKLOAD
     B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
@@ -292,8 +307,8 @@ def run_ours(args):
     ms = float(np.mean([s.elapsed_time(e) for s, e in zip(starts, ends)]))
     clocks = sampler.stop(t_begin, t_end) if sampler else None
     assert ea.attn_device_status() == ea.ATTN_OK
-    ms_max = max_over_ranks(ms)
-    value = world * flops / (ms_max * 1e-3) / 1e12
+    ms_max = slowest(ms)
+    value = whole_job_tflops(world, flops, ms_max)
 
     # e2e: pinned host inputs -> device -> attn_fwd -> O and LSE back to pinned host memory, every
     # step.  Two buffer slots and three streams: the host-to-device copy of step i+1 and the
@@ -344,7 +359,7 @@ def run_ours(args):
     stream.wait_event(slots[e2e_steps % 2]["ev_out"])
     ev1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps)
+    e2e_ms = slowest(ev0.elapsed_time(ev1) / e2e_steps)
     pin_o, pin_l = slots[0]["pin_o"], slots[0]["pin_l"]
     h2d = sum(t.numel() * t.element_size() for t in pin_in)
     d2h = pin_o.numel() * pin_o.element_size() + pin_l.numel() * pin_l.element_size()
@@ -386,7 +401,7 @@ def run_ours(args):
                          "frac_of_measured_sustained": achieved / sustained if sustained else None,
                          "frac_of_datasheet_2250": achieved / 2250.0},
             "cpu_baseline": cpu,
-            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": whole_job_tflops(world, flops, e2e_ms), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "path": "pinned host -> H2D copies -> attn_fwd (C ABI) -> D2H O, LSE",
                     "overlap": "two buffer slots, three streams: H2D of step i+1 and D2H of step i-1 overlap the "
