@@ -20,15 +20,17 @@ Sources (the three pages this project restates; cited by page title and section)
 Modules
 -------
 ``oracle.attention``  two-pass attention (the definition), the pages' blockwise m/l
-                      recurrence, a lazy-rescale blockwise variant in base 2, and a packed
-                      batch of sequences of different lengths built on the definition.
+                      recurrence, a lazy-rescale blockwise variant in base 2, a packed
+                      batch of sequences of different lengths built on the definition, and
+                      the merge of two partial results over disjoint key sets.
 ``oracle.fp8``        Sylvester Hadamard matrix, fast Walsh-Hadamard transform in float32,
                       E4M3 (OCP E4M3FN) rounding/encoding, per-block quantisation.
 ``oracle.rope``       rotary position embedding (rotate-half pairing, caller's cos/sin
                       tables) in float32, ahead of the Hadamard/E4M3 pre-processing.
 ``oracle.attention_bwd``  the backward pass (dQ, dK, dV) from the chain rule on whole score
-                      matrices; the pages only state that it exists and recomputes the softmax
-                      ("FlashAttention-3", "适用范围和工程限制"; "Flash Attention V3 解析" 2.1).
+                      matrices, also per sequence of a packed batch; the pages only state that
+                      it exists and recomputes the softmax ("FlashAttention-3", "适用范围和工程限制";
+                      "Flash Attention V3 解析" 2.1).
 
 Every function is pinned by ``tests/test_oracle_*.py`` against closed forms, invariants,
 library routines (torch SDPA in float64, scipy's Hadamard, ml_dtypes/torch float8), central
