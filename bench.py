@@ -195,7 +195,6 @@ def run_reference(args):
     flops = sum(4.0 * w["d"] * (i + 1) for i in rows)  # causal: row i sees keys 0..i
 
     def step():
-        i0 = w["N"] - R
         for i in rows:  # the oracle on keys 0..i for each causal row
             attention_ref(q[0, 0, i:i + 1], k[0, 0, :i + 1], v[0, 0, :i + 1], scale, False)
 
