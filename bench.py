@@ -684,6 +684,95 @@ def run_sweep(args):
                       flush=True)
 
 
+def run_rows(args):
+    """Timings of the entry points the headline line does not cover, one JSON line: the strided
+    forward and backward on the headline in sequence-major memory (against the contiguous entry
+    points in the same run), the packed backward on the packed workload, the E4M3 forward with
+    two lengths, and the d=64 backward.  20 steps each after 3 warm-ups, L2 flushed between."""
+    import torch
+    import exact_attention_100_b200 as ea
+    from exact_attention_100_b200.inputs import hadamard_signs, normal_qkv_lengths, normal_qkv_packed
+    dev = torch.device("cuda", 0)
+    torch.manual_seed(0)
+    flush = torch.empty(256 * 1024 * 1024 // 4, device=dev)
+    steps = max(3, min(args.steps, 50))
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(float(i))
+            evs[i][0].record()
+            fn()
+            evs[i][1].record()
+        torch.cuda.synchronize()
+        if ea.attn_device_status() != ea.ATTN_OK:
+            raise SystemExit("device status set")
+        return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+    peak = float(load_peaks()["bf16_tflops"])
+    out = {}
+    B, H, N, d = 2, 16, 8192, 128
+    q, k, v = (torch.randn(B, N, H, d, device=dev).to(torch.bfloat16).transpose(1, 2) for _ in range(3))
+    qc, kc, vc = (x.contiguous() for x in (q, k, v))
+    fl = attn_flops(B, H, N, d, True)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, N, device=dev)
+    ms_s = timed(lambda: ea.attn_fwd_strided(q, k, v, o=o, lse=lse, causal=True))
+    ms_c = timed(lambda: ea.attn_fwd(qc, kc, vc, causal=True))
+    out["fwd_strided_seq_major"] = {"ms": ms_s, "tflops": fl / ms_s / 1e9, "frac": fl / ms_s / 1e9 / peak,
+                                    "contiguous_ms": ms_c, "contiguous_tflops": fl / ms_c / 1e9}
+    do = torch.randn_like(qc)
+    dos = do.transpose(1, 2).contiguous().transpose(1, 2)
+    oc, lc = ea.attn_fwd(qc, kc, vc, causal=True)
+    os_ = oc.transpose(1, 2).contiguous().transpose(1, 2)
+    ws = torch.empty(ea.attn_bwd_workspace_bytes(B, H, N) // 4, device=dev)
+    g = [torch.empty_like(q) for _ in range(3)]
+    gc = [torch.empty_like(qc) for _ in range(3)]
+    ms_bs = timed(lambda: ea.attn_bwd_strided(q, k, v, os_, lc, dos, dq=g[0], dk=g[1], dv=g[2], workspace=ws,
+                                              causal=True))
+    ms_bc = timed(lambda: ea.attn_bwd(qc, kc, vc, oc, lc, do, dq=gc[0], dk=gc[1], dv=gc[2], workspace=ws, causal=True))
+    out["bwd_strided_seq_major"] = {"ms": ms_bs, "tflops": 2.5 * fl / ms_bs / 1e9, "frac": 2.5 * fl / ms_bs / 1e9 / peak,
+                                    "contiguous_ms": ms_bc, "contiguous_tflops": 2.5 * fl / ms_bc / 1e9}
+    w = VARLEN_WORKLOAD
+    lens = varlen_lengths(w["total"], w["lo"], w["hi"], w["seed"])
+    qn, kn, vn, cq, ck = normal_qkv_packed(lens, lens, w["H"], w["d"], seed=w["seed"])
+    pq, pk, pv = (torch.from_numpy(a).to(torch.bfloat16).to(dev) for a in (qn, kn, vn))
+    tcq, tck = torch.from_numpy(cq).to(dev), torch.from_numpy(ck).to(dev)
+    po, pl = ea.attn_fwd_varlen(pq, pk, pv, tcq, tck, max(lens), causal=True)
+    pdo = torch.randn_like(pq)
+    pws = torch.empty(ea.attn_bwd_workspace_bytes(len(lens), w["H"], max(lens)) // 4, device=dev)
+    pg = [torch.empty_like(pq) for _ in range(3)]
+    vfl = sum(attn_flops(1, w["H"], n, w["d"], True) for n in lens)
+    ms_pv = timed(lambda: ea.attn_bwd_varlen(pq, pk, pv, po, pl, pdo, tcq, tck, max(lens), max(lens), dq=pg[0], dk=pg[1],
+                                             dv=pg[2], workspace=pws, causal=True))
+    out["bwd_varlen"] = {"ms": ms_pv, "tflops": 2.5 * vfl / ms_pv / 1e9, "frac": 2.5 * vfl / ms_pv / 1e9 / peak,
+                         "lengths": lens}
+    qn, kn, vn = normal_qkv_lengths(2, 16, 4096, 8192, 128, seed=3)
+    tq, tk, tv = (torch.from_numpy(a).to(torch.bfloat16).to(dev) for a in (qn, kn, vn))
+    sg = torch.from_numpy(hadamard_signs(128)).to(dev)
+    q8, qs = ea.attn_hadamard_quant(tq, sg)
+    k8, ks = ea.attn_hadamard_quant(tk, sg)
+    v8, vs = ea.attn_hadamard_quant(tv, None)
+    o8 = torch.empty(2, 16, 4096, 128, dtype=torch.bfloat16, device=dev)
+    l8 = torch.empty(2, 16, 4096, device=dev)
+    ms8 = timed(lambda: ea.attn_fwd_fp8_qk(q8, k8, v8, qs, ks, vs, o=o8, lse=l8, causal=False))
+    fl8 = 4.0 * 2 * 16 * 4096 * 8192 * 128
+    out["fp8_qk"] = {"ms": ms8, "tflops": fl8 / ms8 / 1e9, "frac": fl8 / ms8 / 1e9 / (2 * peak),
+                     "workload": "B=2 H=16 Nq=4096 Nk=8192 d=128 non-causal, peak 2 x bf16"}
+    q6, k6, v6 = (torch.randn(2, 32, 8192, 64, device=dev).to(torch.bfloat16) for _ in range(3))
+    o6, l6 = ea.attn_fwd(q6, k6, v6, causal=True)
+    do6 = torch.randn_like(q6)
+    ws6 = torch.empty(ea.attn_bwd_workspace_bytes(2, 32, 8192) // 4, device=dev)
+    g6 = [torch.empty_like(q6) for _ in range(3)]
+    ms6 = timed(lambda: ea.attn_bwd(q6, k6, v6, o6, l6, do6, dq=g6[0], dk=g6[1], dv=g6[2], workspace=ws6, causal=True))
+    fl6 = 2.5 * attn_flops(2, 32, 8192, 64, True)
+    out["bwd_d64"] = {"ms": ms6, "tflops": fl6 / ms6 / 1e9, "frac": fl6 / ms6 / 1e9 / peak,
+                      "workload": "B=2 H=32 N=8192 d=64 causal"}
+    print(json.dumps({"rows": out, "peak_tflops": peak, "steps": steps}), flush=True)
+
+
 def run_profile_case(args):
     """A few untimed calls of one entry point on a small case, for an ncu capture (no JSON line)."""
     import torch
@@ -745,6 +834,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--rows", action="store_true",
+                    help="time the entry points the headline line does not cover and exit")
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
@@ -765,6 +856,8 @@ def main():
         run_reference(args)
     elif args.sweep:
         run_sweep(args)
+    elif args.rows:
+        run_rows(args)
     else:
         run_ours(args)
 
