@@ -1,9 +1,11 @@
 #!/usr/bin/env python
 """Benchmark of the exact attention forward on B200: one JSON line on rank 0.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--sweep]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--sweep] [--rows]
 
-Defaults: 5 warm-up steps, then 20 timed steps.
+Defaults: 5 warm-up steps, then 20 timed steps.  ``--sweep`` times the head-dim x length grid,
+``--rows`` the strided, packed, FP8-with-two-lengths and d=64 entry points; ``--profile-case``
+runs a few untimed calls of one entry point for an ncu capture.
 
 A step is one call of the bf16 forward (``attn_fwd``) on the headline workload, bf16 B=2 H=16
 N=8192 d=128 causal, inputs iid N(0,1) (seed 0 + rank), already resident in device memory.
