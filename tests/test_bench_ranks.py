@@ -49,3 +49,15 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(0.7, 1, "cpu") == 0.7
     assert abs(bench.whole_job_tflops(1, 5.498e11, 0.55) - 999.6363636) < 1e-6
+
+
+def test_workload_helpers():
+    """The FLOP count the lines divide by, and the packed workload's lengths."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.attn_flops(2, 16, 8192, 128, True) == 5.497558138880e11  # 4 B H N^2 d / 2
+    assert bench.attn_flops(1, 1, 4, 2, False) == 4 * 16 * 2
+    w = bench.VARLEN_WORKLOAD
+    lens = bench.varlen_lengths(w["total"], w["lo"], w["hi"], w["seed"])
+    assert sum(lens) == w["total"] and all(0 < n <= w["hi"] for n in lens)
+    assert lens == bench.varlen_lengths(w["total"], w["lo"], w["hi"], w["seed"])  # seeded
