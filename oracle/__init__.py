@@ -28,7 +28,8 @@ Modules
 ``oracle.rope``       rotary position embedding (rotate-half pairing, caller's cos/sin
                       tables) in float32, ahead of the Hadamard/E4M3 pre-processing.
 ``oracle.attention_bwd``  the backward pass (dQ, dK, dV) from the chain rule on whole score
-                      matrices, also per sequence of a packed batch; the pages only state that
+                      matrices, the same evaluated a block of query rows at a time (for long
+                      sequences), also per sequence of a packed batch; the pages only state that
                       it exists and recomputes the softmax ("FlashAttention-3", "适用范围和工程限制";
                       "Flash Attention V3 解析" 2.1).
 
@@ -48,7 +49,7 @@ from .attention import (  # noqa: F401
 )
 from .attention_bwd import (  # noqa: F401
     attention_bwd_ref,
-    attention_bwd_terms,
+    attention_bwd_chunked_ref,
     attention_varlen_bwd_ref,
     softmax_bwd_delta,
     softmax_probs,

@@ -68,21 +68,42 @@ def attention_bwd_ref(q, k, v, do, scale: float, causal: bool = False):
     return dq.reshape(q.shape), dk.reshape(k.shape), dv.reshape(v.shape)
 
 
-def attention_bwd_terms(q, k, v, do, scale: float, causal: bool = False):
-    """Elementwise magnitudes that bound the rounding error of a kernel that rounds P and dS
-    to bf16 before the three products (used by the GPU tests to state their tolerance):
-    ``|P|^T |dO|`` for dV, ``scale |dS| |K|`` for dQ and ``scale |dS|^T |Q|`` for dK."""
-    q3, lead = _as_3d(np.asarray(q, dtype=np.float64))
+def attention_bwd_chunked_ref(q, k, v, do, scale: float, causal: bool = False, row_chunk: int = 1024):
+    """(dQ, dK, dV) of :func:`attention_bwd_ref`, evaluated ``row_chunk`` query rows at a time.
+
+    The same chain rule on the same definition, for problems whose full score matrix does not
+    fit in memory (N = 8192 and beyond).  For every block of query rows ``c`` it forms
+    ``P_c`` (softmax over the visible keys of those rows), ``dP_c = dO_c V^T`` and
+    ``dS_c = P_c * (dP_c - rowsum(P_c * dP_c))``; ``dQ_c = scale dS_c K`` is complete within the
+    block, while ``dV = sum_c P_c^T dO_c`` and ``dK = scale sum_c dS_c^T Q_c`` are summed over the
+    blocks.  Only the order of the float64 sums differs from the whole-matrix form.  Inputs are
+    ``[..., N, d]`` (``k``, ``v`` may have another length than ``q``; causal masking is
+    bottom-right aligned as in :func:`oracle.attention.visible_mask`).
+    """
+    q3, _ = _as_3d(np.asarray(q, dtype=np.float64))
     k3, _ = _as_3d(np.asarray(k, dtype=np.float64))
     v3, _ = _as_3d(np.asarray(v, dtype=np.float64))
     do3, _ = _as_3d(np.asarray(do, dtype=np.float64))
-    p = softmax_probs(q3, k3, scale, causal)
-    dp = np.einsum("bic,bjc->bij", do3, v3)
-    ds = p * (dp - (p * dp).sum(axis=-1, keepdims=True))
-    tv = np.einsum("bij,bic->bjc", np.abs(p), np.abs(do3))
-    tq = scale * np.einsum("bij,bjc->bic", np.abs(ds), np.abs(k3))
-    tk = scale * np.einsum("bij,bic->bjc", np.abs(ds), np.abs(q3))
-    return tq.reshape(q.shape), tk.reshape(k.shape), tv.reshape(v.shape)
+    g, n_q, _ = q3.shape
+    n_k = k3.shape[1]
+    dq, dk, dv = np.zeros_like(q3), np.zeros_like(k3), np.zeros_like(v3)
+    for b in range(g):
+        for r0 in range(0, n_q, row_chunk):
+            r1 = min(n_q, r0 + row_chunk)
+            s = scale * (q3[b, r0:r1] @ k3[b].T)
+            vis = visible_mask(n_q, n_k, causal)[r0:r1]
+            s = np.where(vis, s, -np.inf)
+            m = s.max(axis=1, keepdims=True)
+            m = np.where(np.isfinite(m), m, 0.0)
+            e = np.where(vis, np.exp(s - m), 0.0)
+            den = e.sum(axis=1, keepdims=True)
+            p = np.divide(e, den, out=np.zeros_like(e), where=den > 0)
+            dv[b] += p.T @ do3[b, r0:r1]
+            dp = do3[b, r0:r1] @ v3[b].T
+            ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+            dq[b, r0:r1] = scale * (ds @ k3[b])
+            dk[b] += scale * (ds.T @ q3[b, r0:r1])
+    return dq.reshape(np.shape(q)), dk.reshape(np.shape(k)), dv.reshape(np.shape(v))
 
 
 def attention_varlen_bwd_ref(q, k, v, do, cu_q, cu_k, scale: float, causal: bool = False):

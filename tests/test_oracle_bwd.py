@@ -169,3 +169,46 @@ def test_pins_accept_the_oracle():
                                       "ds_not_transposed", "strict_causal"])
 def test_planted_mistake_fails_a_pin(mutation):
     assert not _pins_pass(_mutant_bwd(mutation))
+
+
+# ---- the row-chunked backward (used at sizes whose score matrix does not fit in memory) -------
+
+from oracle import attention_bwd_chunked_ref  # noqa: E402
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("nq,nk,chunk", [(37, 37, 1), (37, 37, 5), (40, 23, 7), (23, 40, 16), (64, 64, 64),
+                                         (50, 50, 1024)])
+def test_chunked_backward_equals_whole_matrix(nq, nk, chunk, causal):
+    """Query-row blocks of any size (dividing N or not, longer than N) give the whole-matrix
+    gradients: dQ rows are local to their block, dK and dV are sums over the blocks."""
+    rng = np.random.default_rng(nq * 100 + nk + chunk)
+    q, k, v = (rng.standard_normal((2, n, 16)) for n in (nq, nk, nk))
+    do = rng.standard_normal((2, nq, 16))
+    a = attention_bwd_ref(q, k, v, do, 0.3, causal)
+    b = attention_bwd_chunked_ref(q, k, v, do, 0.3, causal, row_chunk=chunk)
+    for x, y in zip(a, b):
+        assert x.shape == y.shape
+        assert np.abs(x - y).max() <= 1e-12 * max(1.0, np.abs(x).max())
+
+
+def test_chunked_backward_matches_finite_differences():
+    """Independently of the whole-matrix form: central differences of the forward oracle."""
+    q, k, v = (_rand((1, 9, 4), s) for s in (31, 32, 33))
+    do = _rand((1, 9, 4), 34)
+    got = attention_bwd_chunked_ref(q, k, v, do, 0.7, True, row_chunk=4)
+    for g, r in zip(got, _fd_grads(q, k, v, do, 0.7, True)):
+        assert np.abs(g - r).max() <= 1e-6
+
+
+def test_chunked_backward_planted_mistake_fails():
+    """dV taken from the last block only (assigned, not summed) must fail the equality pin."""
+    rng = np.random.default_rng(5)
+    q, k, v = (rng.standard_normal((1, 30, 8)) for _ in range(3))
+    do = rng.standard_normal((1, 30, 8))
+    ref = attention_bwd_ref(q, k, v, do, 0.5, False)[2]
+    wrong = np.zeros_like(v)
+    for r0 in range(0, 30, 7):
+        p = softmax_probs(q[:, r0:r0 + 7], k, 0.5, False)
+        wrong[0] = p[0].T @ do[0, r0:r0 + 7]
+    assert np.abs(wrong - ref).max() > 1e-3
