@@ -25,7 +25,7 @@ import torch
 
 import exact_attention_100_b200 as ea
 from exact_attention_100_b200.inputs import normal_dout
-from oracle import attention_bwd_ref, softmax_probs
+from oracle import attention_bwd_chunked_ref, attention_bwd_ref, attention_ref, visible_mask
 
 from gpu_util import device_qkv
 
@@ -34,21 +34,46 @@ pytestmark = pytest.mark.gpu
 U = 2.0 ** -9
 
 
-def _bounds(q, k, v, do, o_ref, scale, causal):
-    p = softmax_probs(q, k, scale, causal)
-    dp = np.einsum("bhic,bhjc->bhij", do, v)
-    ds = p * (dp - (p * dp).sum(-1, keepdims=True))
-    ap, ads = np.abs(p), np.abs(ds)
-    n, d = q.shape[-2], q.shape[-1]
-    pv = np.einsum("bhij,bhjc->bhic", ap, np.abs(v))
-    d_err = np.einsum("bhic,bhic->bhi", np.abs(do), U * np.abs(o_ref) + 2 * U * pv)
-    dp_err = d * 2.0 ** -23 * np.einsum("bhic,bhjc->bhij", np.abs(do), np.abs(v))
-    ds_err = (U + 1e-4) * ads + ap * (d_err[..., None] + dp_err)
+def _probs_rows(q, k, scale, causal, r0, r1):
+    """P for query rows r0..r1-1 of one head (float64, bottom-right causal alignment)."""
+    s = scale * (q[r0:r1] @ k.T)
+    vis = visible_mask(q.shape[0], k.shape[0], causal)[r0:r1]
+    s = np.where(vis, s, -np.inf)
+    m = s.max(axis=1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    e = np.where(vis, np.exp(s - m), 0.0)
+    den = e.sum(axis=1, keepdims=True)
+    return np.divide(e, den, out=np.zeros_like(e), where=den > 0)
+
+
+def _bounds(q, k, v, do, o_ref, scale, causal, row_chunk=1024):
+    """The elementwise bounds of the module docstring for dQ, dK, dV (shapes of q, k, v).
+
+    Evaluated a block of query rows at a time, so that the bench's N = 8192 fits in memory:
+    every term of dQ's bound is local to its rows, and dK's and dV's are sums over the rows."""
+    shp = [np.shape(x) for x in (q, k, v)]
+    q3, k3, v3, do3, o3 = (np.asarray(x, dtype=np.float64).reshape((-1,) + np.shape(x)[-2:])
+                           for x in (q, k, v, do, o_ref))
+    n, d = q3.shape[1], q3.shape[2]
     acc = n * 2.0 ** -23
-    bv = np.einsum("bhij,bhic->bhjc", (U + 1e-4 + acc) * ap, np.abs(do))
-    bq = scale * (np.einsum("bhij,bhjc->bhic", ds_err + acc * ads, np.abs(k)))
-    bk = scale * (np.einsum("bhij,bhic->bhjc", ds_err + acc * ads, np.abs(q)))
-    return bq, bk, bv
+    bq, bk, bv = np.zeros_like(q3), np.zeros_like(k3), np.zeros_like(v3)
+    for b in range(q3.shape[0]):
+        aq, ak, av, ado = np.abs(q3[b]), np.abs(k3[b]), np.abs(v3[b]), np.abs(do3[b])
+        for r0 in range(0, n, row_chunk):
+            r1 = min(n, r0 + row_chunk)
+            p = _probs_rows(q3[b], k3[b], scale, causal, r0, r1)
+            dp = do3[b, r0:r1] @ v3[b].T
+            ds = p * (dp - (p * dp).sum(-1, keepdims=True))
+            ap, ads = np.abs(p), np.abs(ds)
+            pv = ap @ av
+            d_err = (ado[r0:r1] * (U * np.abs(o3[b, r0:r1]) + 2 * U * pv)).sum(-1)
+            dp_err = d * 2.0 ** -23 * (ado[r0:r1] @ av.T)
+            ds_err = (U + 1e-4) * ads + ap * (d_err[:, None] + dp_err)
+            bv[b] += ((U + 1e-4 + acc) * ap).T @ ado[r0:r1]
+            t = ds_err + acc * ads
+            bq[b, r0:r1] = scale * (t @ ak)
+            bk[b] += scale * (t.T @ aq[r0:r1])
+    return bq.reshape(shp[0]), bk.reshape(shp[1]), bv.reshape(shp[2])
 
 
 def _run(B, H, N, d, causal, g_dtype=torch.float32, seed=0):
@@ -66,7 +91,6 @@ def _run(B, H, N, d, causal, g_dtype=torch.float32, seed=0):
 def _check(inputs, grads, causal, bf16_out=False):
     q, k, v, do, scale = inputs
     refs = attention_bwd_ref(q, k, v, do, scale, causal)
-    from oracle import attention_ref
     o_ref, _ = attention_ref(q, k, v, scale, causal)
     bounds = _bounds(q, k, v, do, o_ref, scale, causal)
     for name, g, r, b in zip(("dq", "dk", "dv"), grads, refs, bounds):
@@ -166,3 +190,40 @@ def test_bwd_qk_equal_lengths_is_attn_bwd(causal):
     torch.cuda.synchronize()
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+def test_bwd_bench_workload_whole_heads():
+    """The workload and call the bench times: B=2 H=16 N=8192 d=128 causal, bf16 O and bf16
+    gradients, dO from the recipe (seed 7).  Two whole heads, (0, 0) and (1, 15), against the
+    float64 oracle element by element under the bound above (the oracle and the bound taken
+    1024 query rows at a time), and a second call bit-identical to the first."""
+    B, H, N, d = 2, 16, 8192, 128
+    (q, k, v), (tq, tk, tv) = device_qkv(B, H, N, d, seed=0)
+    do = normal_dout(B, H, N, d, seed=7)
+    tdo = torch.from_numpy(do).to(torch.bfloat16).cuda()
+    scale = 1.0 / math.sqrt(d)
+    o, lse = ea.attn_fwd(tq, tk, tv, causal=True)
+    ws = torch.empty(ea.attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device="cuda")
+    g1 = [torch.empty_like(tq) for _ in range(3)]
+    g2 = [torch.empty_like(tq) for _ in range(3)]
+    ea.attn_bwd(tq, tk, tv, o, lse, tdo, *g1, ws, causal=True)
+    ea.attn_bwd(tq, tk, tv, o, lse, tdo, *g2, ws, causal=True)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
+    for (b, h) in [(0, 0), (1, 15)]:
+        sel = lambda x: x[b:b + 1, h:h + 1]
+        inputs = (sel(q), sel(k), sel(v), sel(do), scale)
+        refs = attention_bwd_chunked_ref(*inputs[:4], scale, True)
+        o_ref, _ = attention_ref(*inputs[:3], scale, True)
+        bounds = _bounds(*inputs[:4], o_ref, scale, True)
+        grads = [g[b:b + 1, h:h + 1].float().cpu().numpy() for g in g1]
+        for name, g, r, bd in zip(("dq", "dk", "dv"), grads, refs, bounds):
+            g = g.astype(np.float64)
+            assert np.isfinite(g).all(), name
+            tol = 2.0 * bd + 1e-6 * np.abs(r).max() + U * np.abs(r)
+            err = np.abs(g - r)
+            assert np.all(err[tol == 0] == 0), name
+            worst = float(np.divide(err, tol, out=np.zeros_like(err), where=tol > 0).max())
+            assert worst <= 1.0, ((b, h), name, worst, float(err.max()))

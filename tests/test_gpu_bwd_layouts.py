@@ -11,7 +11,7 @@ import torch
 
 import exact_attention_100_b200 as ea
 from exact_attention_100_b200.inputs import normal_dout, normal_qkv_lengths, normal_qkv_packed
-from oracle import attention_ref, attention_bwd_ref, attention_varlen_bwd_ref
+from oracle import attention_ref, attention_bwd_chunked_ref, attention_bwd_ref, attention_varlen_bwd_ref
 
 from test_gpu_bwd import _bounds
 
@@ -147,6 +147,26 @@ def test_packed_is_per_sequence_attn_bwd_qk(lk, layout, causal):
         assert np.array_equal(grads[0][q0:q1], back(ref[0]))
         assert np.array_equal(grads[1][k0:k1], back(ref[1]))
         assert np.array_equal(grads[2][k0:k1], back(ref[2]))
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_packed_bench_batch_two_heads(causal):
+    """The bench's packed workload (8 sequences of 391..3369 tokens, 16384 in all, H=16 d=128,
+    seed 11): every sequence of heads 0 and 15 against the float64 oracle under the derived
+    bound (oracle and bound taken 1024 query rows at a time)."""
+    from bench import VARLEN_WORKLOAD, varlen_lengths
+    w = VARLEN_WORKLOAD
+    lens = varlen_lengths(w["total"], w["lo"], w["hi"], w["seed"])
+    assert sum(lens) == w["total"] and len(lens) == 8
+    (q, k, v, do, cq, ck, scale), _, grads = _packed_run(lens, lens, w["H"], w["d"], causal, seed=w["seed"])
+    for h in (0, w["H"] - 1):
+        for b in range(len(lens)):
+            q0, q1 = int(cq[b]), int(cq[b + 1])
+            t = lambda x: x[q0:q1, h][None, None]  # [1, 1, rows, d]
+            qs, ks, vs, dos = t(q), t(k), t(v), t(do)
+            refs = attention_bwd_chunked_ref(qs, ks, vs, dos, scale, causal)
+            o_ref, _ = attention_ref(qs, ks, vs, scale, causal)
+            _check_grads([t(g) for g in grads], refs, _bounds(qs, ks, vs, dos, o_ref, scale, causal))
 
 
 def test_packed_bad_offsets_are_reported():

@@ -137,3 +137,14 @@ def test_schedule_covers_sequences_of_one_length_and_empty_ones():
     """Sorting by tile pairs with many ties and zero-length sequences in between."""
     lq = [256, 0, 256, 512, 0, 1, 256, 257, 0, 512]
     _run(lq, lq, 2, 128, True, seed=11)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_bench_packed_batch_all_heads(causal):
+    """The packed batch the bench times: 8 sequences of 391..3369 tokens (16384 in all), H=16
+    d=128, seed 11, bf16 O; every row of every head against the float64 oracle."""
+    from bench import VARLEN_WORKLOAD, varlen_lengths
+    w = VARLEN_WORKLOAD
+    lens = varlen_lengths(w["total"], w["lo"], w["hi"], w["seed"])
+    assert sum(lens) == w["total"] and len(lens) == 8
+    _run(lens, lens, w["H"], w["d"], causal, seed=w["seed"], o_dtype=torch.bfloat16)
