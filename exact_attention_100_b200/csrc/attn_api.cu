@@ -104,6 +104,24 @@ bool encode_fwd_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, 
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D tiled map over O for the forward's TMA stores: dims (d, rows, heads, batch), the caller's
+// element strides, box = 64 bytes x 128 rows x 1 x 1 (32 bf16 or 16 f32 columns), 64-byte swizzle;
+// rows past the last one are not written.
+bool encode_o_map(CUtensorMap* map, void* base, int o_dtype, int d, int N, int H, int B, long long sn, long long sh,
+                  long long sb) {
+  const bool f32 = o_dtype == ATTN_FP32;
+  const int eb = f32 ? 4 : 2;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(sn) * eb, static_cast<cuuint64_t>(sh) * eb,
+                                 static_cast<cuuint64_t>(sb) * eb};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(64 / eb), 128u, 1u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return g_encode(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Element strides (batch, head, row) of one [B, H, N, d] tensor; the forward's maps and its O
 // stores take any strides that are positive multiples of 8 elements below 2^36.  A stride of a
 // dimension of extent 1 is never used to address anything and is replaced by 8.
@@ -235,17 +253,18 @@ int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, i
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
   const Strides &sq = st4[0], &sk = st4[1], &sv = st4[2], &so = st4[3];
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!encode_fwd_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nq, H, B, sq.sn, sq.sh, sq.sb) ||
       !encode_fwd_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nk, H, B, sk.sn, sk.sh, sk.sb) ||
-      !encode_fwd_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nk, H, B, sv.sn, sv.sh, sv.sb))
+      !encode_fwd_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, Nk, H, B, sv.sn, sv.sh, sv.sb) ||
+      !encode_o_map(&mo, o, o_dtype, d, Nq, H, B, so.sn, so.sh, so.sb))
     return ATTN_ERR_CUDA;
   ea::FwdParams p;
   fill_params(p, o, lse, st->status, B, H, Nq, Nk, ea::fwd_units_per_tile_pair(d), scale, causal, o_dtype);
   p.o_sb = so.sb;
   p.o_sh = so.sh;
   p.o_sn = so.sn;
-  if (ea::launch_attn_fwd_bf16(d, mq, mk, mv, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (ea::launch_attn_fwd_bf16(d, mq, mk, mv, mo, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
   return ATTN_OK;
@@ -306,10 +325,11 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
   const Strides &sq = st4[0], &sk = st4[1], &sv = st4[2], &so = st4[3];
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!encode_fwd_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, total_q, H, 1, sq.sn, sq.sh, sq.sb) ||
       !encode_fwd_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, total_k, H, 1, sk.sn, sk.sh, sk.sb) ||
-      !encode_fwd_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, total_k, H, 1, sv.sn, sv.sh, sv.sb))
+      !encode_fwd_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, total_k, H, 1, sv.sn, sv.sh, sv.sb) ||
+      !encode_o_map(&mo, o, o_dtype, d, total_q, H, 1, so.sn, so.sh, so.sb))
     return ATTN_ERR_CUDA;
   ea::FwdParams p;
   // sized for B sequences of max_seqlen_q queries each; shorter ones skip the surplus units
@@ -324,7 +344,7 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   p.total_k = total_k;
   // the in-kernel schedule's shared-memory tables hold up to 1024 sequences and 1023 pairs
   p.vl_sched = (B <= 1024 && p.n_pairs <= 1023) ? 1 : 0;
-  if (ea::launch_attn_fwd_bf16(d, mq, mk, mv, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (ea::launch_attn_fwd_bf16(d, mq, mk, mv, mo, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
   return ATTN_OK;
@@ -427,10 +447,11 @@ int fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
   const Strides s = contiguous_strides(H, Nq, d), sk = contiguous_strides(H, Nk, d);
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!encode_fwd_map(&mq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Nq, H, B, s.sn, s.sh, s.sb) ||
       !encode_fwd_map(&mk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Nk, H, B, sk.sn, sk.sh, sk.sb) ||
-      !encode_fwd_map(&mv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Nk, H, B, sk.sn, sk.sh, sk.sb))
+      !encode_fwd_map(&mv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Nk, H, B, sk.sn, sk.sh, sk.sb) ||
+      !encode_o_map(&mo, o, o_dtype, d, Nq, H, B, s.sn, s.sh, s.sb))
     return ATTN_ERR_CUDA;
   ea::FwdParams p;
   fill_params(p, o, lse, st->status, B, H, Nq, Nk, 2, scale, causal, o_dtype);
@@ -440,7 +461,7 @@ int fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.v_scale = v_scale;
-  if (ea::launch_attn_fwd_fp8(d, mq, mk, mv, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (ea::launch_attn_fwd_fp8(d, mq, mk, mv, mo, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
   return ATTN_OK;

@@ -11,10 +11,14 @@
 // Roles (warp specialisation, "FlashAttention-3", section "异步搬运与异步计算"):
 //   warps 0..4*NQ-1   softmax warpgroup q = warp/4: one thread per S row (= TMEM lane)
 //   next 4 warps      correction warpgroup: serves events from the MMA thread -- a lazy O
-//                     rescale before a P.V, or the epilogue of a finished Q tile
+//                     rescale before a P.V, or the epilogue of a finished Q tile (O / l into
+//                     shared-memory stage buffers, LSE)
 //   next warp         MMA issuer (one thread issues every tcgen05.mma)
 //   next warp         TMA producer (one thread; Q tiles and a ring of K/V slots)
-//   remaining warps   idle (the CTA is a whole number of warpgroups)
+//   next warp         store warp (one thread): TMA stores of the staged O slices and bulk
+//                     copies of the LSE rows ("Flash Attention V3 解析", section 3.2.1: the
+//                     asynchronous copy engine moves tiles both ways)
+//   remaining warp    idle (the CTA is a whole number of warpgroups)
 //
 // Overlap ("FlashAttention-3", sections "Ping-pong 调度" and "同一个 warpgroup 内部也能再叠一层";
 // "Flash Attention V3 解析", section 3.2.3):
@@ -84,26 +88,34 @@ struct FwdCfg {
   static constexpr int kCorrWarp0 = 4 * NQ;
   static constexpr int kMmaWarp = 4 * NQ + 4;
   static constexpr int kLoadWarp = 4 * NQ + 5;
+  static constexpr int kEpiWarp = 4 * NQ + 6;                 // issues the TMA stores of O and LSE
   static constexpr int kThreads = (4 * NQ + 8) * 32;
   static constexpr int kEvents = 4;                           // correction event ring
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = NQ * kTileBytes;
-  static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
+  // O leaves through two stage buffers of 128 rows x 64 bytes (32 bf16 or 16 f32 columns, the
+  // O map's box, 64-byte swizzle) and the LSE of a tile through [2][128] f32
+  static constexpr int kStageBytes = 128 * 64;
+  static constexpr int kStageOff = kRingOff + kSlots * kTileBytes;
+  static constexpr int kLseStageOff = kStageOff + 2 * kStageBytes;
+  static constexpr int kBarOff = kLseStageOff + 2 * 128 * 4;
   // full[kSlots], empty[kSlots], q_full, q_empty, s_full[kSBufs], p_full[kSBufs], o_corr[NQ],
-  // o_done[NQ], o_free[NQ], ev_full[kEvents], ev_empty[kEvents], drain
-  static constexpr int kNumBars = 2 * kSlots + 2 + 2 * kSBufs + 3 * NQ + 2 * kEvents + 1;
+  // o_done[NQ], o_free[NQ], ev_full[kEvents], ev_empty[kEvents], drain, st_full[2], st_empty[2]
+  static constexpr int kNumBars = 2 * kSlots + 2 + 2 * kSBufs + 3 * NQ + 2 * kEvents + 1 + 4;
   static constexpr int kAlphaOff = kBarOff + ((kNumBars * 8 + 15) / 16) * 16;
   static constexpr int kRowMOff = kAlphaOff + NQ * 2 * 128 * 4;
   static constexpr int kRowLOff = kRowMOff + NQ * 2 * 128 * 4;
   static constexpr int kFlagOff = kRowLOff + NQ * 2 * 128 * 4;  // [NQ][2] int, one byte per warp
   static constexpr int kEventOff = kFlagOff + 16;               // [kEvents][4] int
-  static constexpr int kMiscOff = kEventOff + kEvents * 16;
+  static constexpr int kStageInfoOff = kEventOff + kEvents * 16;  // [2][8] int: what a stage holds
+  static constexpr int kMiscOff = kStageInfoOff + 2 * 8 * 4;
   // packed batches: sorted sequence keys [kSchedSeqs] and the unit prefix [kSchedRounds + 1]
   static constexpr int kSchedSeqs = kVlSchedSeqs, kSchedRounds = kVlSchedRounds;
   static constexpr int kSchedOff = kMiscOff + 16;
   static constexpr int kSmemBytes = kSchedOff + (kSchedSeqs + kSchedRounds + 1) * 4;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;        // room to align the base to 1024 bytes
   static_assert(kSlots >= 2, "K/V ring");
+  static_assert(kStageOff % 1024 == 0, "stage buffers: 64-byte swizzle atoms");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
   static_assert(kSBufs * 128 <= kOCol && kOCol + NQ * D <= kTmemCols, "TMEM budget");
   // register split (setmaxnreg) for NQ = 2: 2 softmax warpgroups, 1 correction, 1 MMA/TMA
@@ -328,7 +340,8 @@ __device__ __forceinline__ float softmax_block(uint32_t (&r)[128], uint32_t* pk,
 template <int D, int NQ, class E, bool VL>
 __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                    const FwdParams p) {
   using C = FwdCfg<D, NQ, E>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
@@ -349,6 +362,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
   uint64_t* ev_full = o_free + NQ;         // [kEvents] event posted (MMA thread)
   uint64_t* ev_empty = ev_full + C::kEvents;  // [kEvents] event taken (correction warps)
   uint64_t* drain = ev_empty + C::kEvents;
+  uint64_t* st_full = drain + 1;           // [2] stage buffer written (128 correction threads)
+  uint64_t* st_empty = st_full + 2;        // [2] stage buffer read by its store (store warp)
+  uint8_t* stage = smem + C::kStageOff;                                   // [2][128 rows][64 B]
+  float* lse_stage = reinterpret_cast<float*>(smem + C::kLseStageOff);    // [2][128]
+  volatile int* stage_info = reinterpret_cast<volatile int*>(smem + C::kStageInfoOff);  // [2][8]
   float* alpha_s = reinterpret_cast<float*>(smem + C::kAlphaOff);  // [NQ][2][128]
   // [NQ][2][128], slot = parity of the tile's unit count: a tile with a single K/V block writes
   // the next unit's values before the previous epilogue has necessarily read its own
@@ -380,6 +398,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       bar_init(&ev_empty[e], 4);
     }
     bar_init(drain, 1);
+    for (int b = 0; b < 2; ++b) {
+      bar_init(&st_full[b], 128);
+      bar_init(&st_empty[b], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -388,6 +410,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
     prefetch_tensor_map(&tmK);
     prefetch_tensor_map(&tmV);
   }
+  if (warp == C::kEpiWarp && lane == 0) prefetch_tensor_map(&tmO);
   if (warp == 0) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
@@ -612,7 +635,29 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     uint32_t eit = 0;
+    uint32_t stc = 0;  // stage buffers filled so far (buffer stc & 1)
     bool ok = true;
+    // waits until stage buffer stc & 1 is free again (its previous store has read it)
+    auto stage_acquire = [&]() {
+      return warp_all(wait_bar(&st_empty[stc & 1u], ((stc >> 1) & 1u) ^ 1u, ab));
+    };
+    // hands the stage buffer to the store warp: info = {kind, x, row, head, batch, lse, lse lo, hi}
+    auto stage_release = [&](int x, int y, int h, int bc, bool lse, long long lse_idx) {
+      volatile int* info = stage_info + (stc & 1u) * 8;
+      if (row == 0) {
+        info[0] = 1;
+        info[1] = x;
+        info[2] = y;
+        info[3] = h;
+        info[4] = bc;
+        info[5] = lse ? 1 : 0;
+        info[6] = static_cast<int>(lse_idx & 0xFFFFFFFFll);
+        info[7] = static_cast<int>(lse_idx >> 32);
+      }
+      fence_proxy_async_smem();
+      bar_arrive(&st_full[stc & 1u]);
+      ++stc;
+    };
     while (ok) {
       const uint32_t es = eit % C::kEvents;
       ok = warp_all(wait_bar(&ev_full[es], (eit / C::kEvents) & 1u, ab));
@@ -627,7 +672,14 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       const int kind = kq & 0xff;
       const int q = (kq >> 8) & 0xff;
       const int uslot = kq >> 16;
-      if (kind == kEvEnd) break;
+      if (kind == kEvEnd) {
+        // tells the store warp to finish
+        if ((ok = stage_acquire())) {
+          if (row == 0) stage_info[(stc & 1u) * 8] = 0;
+          bar_arrive(&st_full[stc & 1u]);
+        }
+        break;
+      }
       const uint32_t tO = tmem + lane_off + C::kOCol + q * D;
       if (kind == kEvRescale) {
         // the MMA thread committed o_done (phase c) after issuing P.V number `tile` - 1 (for a
@@ -662,36 +714,93 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         const int row_g = tile * 128 + row;
         const Seq S = seq_of<VL>(bh, p);
         const bool valid = row_g < S.N;
-        const long long orow = S.bc * p.o_sb + S.h * p.o_sh + static_cast<long long>(S.q0 + row_g) * p.o_sn;
+        // A tile leaves through the stage buffers and the TMA store (rows past the tensor's end
+        // are clipped by the copy); only the last tile of a packed sequence, whose rows past the
+        // sequence's end belong to the next sequence, is written row by row instead.
+        const bool staged = !VL || tile * 128 + 128 <= S.N;
+        if (staged) {
+          const long long lse_first = S.lse0 + tile * 128;
+          const bool lse_bulk = p.lse != nullptr && tile * 128 + 128 <= S.N && (lse_first & 3) == 0;
+          if (p.lse != nullptr && !lse_bulk && valid) p.lse[S.lse0 + row_g] = lse2 * kLn2;
+          const int sw = (row >> 1) & 3;  // 64-byte swizzle: 16-byte chunk c of row r sits at c ^ ((r >> 1) & 3)
 #pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t r[32];
-          tmem_ld_32cols(tO + 32 * cc, r);
-          tmem_ld_wait(r);
-          if (!valid) continue;
-          if (p.o_fp32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + 32 * cc);
+          for (int cc = 0; cc < D / 32 && ok; ++cc) {
+            uint32_t r[32];
+            tmem_ld_32cols(tO + 32 * cc, r);
+            tmem_ld_wait(r);
+            if (cc == D / 32 - 1) {
+              // O is in registers: the next unit's first P.V may overwrite it in TMEM
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) bar_arrive(&o_free[q]);
+            }
+            if (p.o_fp32) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
-                                   __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + orow + 32 * cc);
+              for (int h2 = 0; h2 < 2; ++h2) {
+                if (!(ok = stage_acquire())) break;
+                uint8_t* dst = stage + (stc & 1u) * C::kStageBytes + row * 64;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv, __uint_as_float(r[8 * i + 1]) * inv);
-              w.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv);
-              w.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv);
-              w.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv);
-              dst[i] = w;
+                for (int i = 0; i < 4; ++i)
+                  *reinterpret_cast<float4*>(dst + ((i ^ sw) << 4)) =
+                      make_float4(__uint_as_float(r[16 * h2 + 4 * i]) * inv, __uint_as_float(r[16 * h2 + 4 * i + 1]) * inv,
+                                  __uint_as_float(r[16 * h2 + 4 * i + 2]) * inv,
+                                  __uint_as_float(r[16 * h2 + 4 * i + 3]) * inv);
+                const bool with_lse = lse_bulk && cc == 0 && h2 == 0;
+                if (with_lse) lse_stage[(stc & 1u) * 128 + row] = lse2 * kLn2;
+                stage_release(32 * cc + 16 * h2, S.q0 + tile * 128, S.h, S.bc, with_lse, lse_first);
+              }
+            } else {
+              if (!(ok = stage_acquire())) break;
+              uint8_t* dst = stage + (stc & 1u) * C::kStageBytes + row * 64;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv, __uint_as_float(r[8 * i + 1]) * inv);
+                w.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv);
+                w.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv);
+                w.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv);
+                *reinterpret_cast<uint4*>(dst + ((i ^ sw) << 4)) = w;
+              }
+              const bool with_lse = lse_bulk && cc == 0;
+              if (with_lse) lse_stage[(stc & 1u) * 128 + row] = lse2 * kLn2;
+              stage_release(32 * cc, S.q0 + tile * 128, S.h, S.bc, with_lse, lse_first);
             }
           }
+          if (!ok) break;
+        } else {
+          const long long orow = S.bc * p.o_sb + S.h * p.o_sh + static_cast<long long>(S.q0 + row_g) * p.o_sn;
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t r[32];
+            tmem_ld_32cols(tO + 32 * cc, r);
+            tmem_ld_wait(r);
+            if (cc == D / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) bar_arrive(&o_free[q]);
+            }
+            if (!valid) continue;
+            if (p.o_fp32) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + 32 * cc);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
+                                     __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + orow + 32 * cc);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv, __uint_as_float(r[8 * i + 1]) * inv);
+                w.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv);
+                w.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv);
+                w.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv);
+                dst[i] = w;
+              }
+            }
+          }
+          if (valid && p.lse != nullptr) p.lse[S.lse0 + row_g] = lse2 * kLn2;
         }
-        if (valid && p.lse != nullptr) p.lse[S.lse0 + row_g] = lse2 * kLn2;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) bar_arrive(&o_free[q]);
       }
     }
   } else {
@@ -902,6 +1011,24 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       const uint32_t first = it > static_cast<uint32_t>(C::kSlots) ? it - C::kSlots : 0u;
       for (uint32_t i = first; i < it; ++i) drain_wait(&full[i % C::kSlots], (i / C::kSlots) & 1u, p.status);
       if (qit > 0) drain_wait(q_full, (qit - 1u) & 1u, p.status);
+    } else if (warp == C::kEpiWarp && lane == 0) {
+      // ======================================================================== store warp
+      uint32_t stc = 0;
+      while (wait_bar(&st_full[stc & 1u], (stc >> 1) & 1u, ab)) {
+        const uint32_t b = stc & 1u;
+        const volatile int* info = stage_info + b * 8;
+        if (info[0] == 0) break;  // the correction warpgroup has finished
+        tma_store_4d(&tmO, stage + b * C::kStageBytes, info[1], info[2], info[3], info[4]);
+        if (info[5]) {
+          const long long idx = (static_cast<long long>(info[7]) << 32) | static_cast<unsigned int>(info[6]);
+          bulk_store_s2g(p.lse + idx, lse_stage + b * 128, 128 * 4);
+        }
+        bulk_commit_group();
+        bulk_wait_read_all();  // the buffer may be refilled once its store has read it
+        bar_arrive(&st_empty[b]);
+        ++stc;
+      }
+      bulk_wait_all();  // every store performed before the CTA exits
     }
   }
 
@@ -921,11 +1048,11 @@ cudaError_t set_fwd_smem_attr() {
 }
 
 template <int D, int NQ, class E, bool VL = false>
-cudaError_t launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const FwdParams& p,
-                       int num_sms, cudaStream_t stream) {
+cudaError_t launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& o,
+                       const FwdParams& p, int num_sms, cudaStream_t stream) {
   using C = FwdCfg<D, NQ, E>;
   const int grid = p.num_units < num_sms ? p.num_units : num_sms;
-  attn_fwd_kernel<D, NQ, E, VL><<<grid, C::kThreads, C::kSmemAlloc, stream>>>(q, k, v, p);
+  attn_fwd_kernel<D, NQ, E, VL><<<grid, C::kThreads, C::kSmemAlloc, stream>>>(q, k, v, o, p);
   return cudaGetLastError();
 }
 

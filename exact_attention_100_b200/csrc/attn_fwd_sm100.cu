@@ -16,18 +16,18 @@ cudaError_t setup_fwd_bf16_kernels() {
 }
 
 cudaError_t launch_attn_fwd_bf16(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                                 const FwdParams& p, int num_sms, cudaStream_t stream) {
+                                 const CUtensorMap& o, const FwdParams& p, int num_sms, cudaStream_t stream) {
   const bool vl = p.cu_q != nullptr;
   switch (d) {
     case 64:
-      return vl ? launch_fwd<64, 2, ElemBf16, true>(q, k, v, p, num_sms, stream)
-                : launch_fwd<64, 2, ElemBf16>(q, k, v, p, num_sms, stream);
+      return vl ? launch_fwd<64, 2, ElemBf16, true>(q, k, v, o, p, num_sms, stream)
+                : launch_fwd<64, 2, ElemBf16>(q, k, v, o, p, num_sms, stream);
     case 128:
-      return vl ? launch_fwd<128, 2, ElemBf16, true>(q, k, v, p, num_sms, stream)
-                : launch_fwd<128, 2, ElemBf16>(q, k, v, p, num_sms, stream);
+      return vl ? launch_fwd<128, 2, ElemBf16, true>(q, k, v, o, p, num_sms, stream)
+                : launch_fwd<128, 2, ElemBf16>(q, k, v, o, p, num_sms, stream);
     case 256:
-      return vl ? launch_fwd<256, 1, ElemBf16, true>(q, k, v, p, num_sms, stream)
-                : launch_fwd<256, 1, ElemBf16>(q, k, v, p, num_sms, stream);
+      return vl ? launch_fwd<256, 1, ElemBf16, true>(q, k, v, o, p, num_sms, stream)
+                : launch_fwd<256, 1, ElemBf16>(q, k, v, o, p, num_sms, stream);
     default:
       return cudaErrorInvalidValue;
   }

@@ -53,12 +53,14 @@ int fwd_units_per_tile_pair(int d);
 cudaError_t setup_kernels_for_current_device();
 
 // The forward kernels read Q, K and V through 4-D maps (d, rows, heads, batch) with a box of
-// 128 bytes x 128 rows x 1 x 1: any layout with d contiguous and 16-byte-aligned strides.
+// 128 bytes x 128 rows x 1 x 1, 128-byte swizzle: any layout with d contiguous and 16-byte-aligned
+// strides.  They store O through a 4-D map of the same form over O (bf16 or f32) with a box of
+// 64 bytes x 128 rows x 1 x 1 and 64-byte swizzle.
 cudaError_t launch_attn_fwd_bf16(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                                 const FwdParams& p, int num_sms, cudaStream_t stream);
+                                 const CUtensorMap& o, const FwdParams& p, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_attn_fwd_fp8(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                                const FwdParams& p, int num_sms, cudaStream_t stream);
+                                const CUtensorMap& o, const FwdParams& p, int num_sms, cudaStream_t stream);
 
 // Parameters of the backward kernels (bf16 inputs, d = 64 or 128).
 struct BwdParams {
