@@ -13,7 +13,7 @@ Entry points, by family:
 
 * forward: ``attn_fwd``, ``attn_fwd_qk`` (key length != query length), ``attn_fwd_strided``
   (any strides, e.g. sequence-major or fused QKV), ``attn_fwd_varlen`` (packed batches),
-  ``attn_fwd_noalloc`` (no device allocation);
+  ``attn_fwd_noalloc`` (no device allocation; ``attn_noalloc_status`` reads its status word);
 * FP8: ``attn_hadamard_quant``, ``attn_hadamard_quant_qkv``, ``attn_rope_hadamard_quant_qkv``
   (rotary embedding fused), ``attn_fwd_fp8``, ``attn_fwd_fp8_qk``;
 * backward: ``attn_bwd``, ``attn_bwd_qk``, ``attn_bwd_strided``, ``attn_bwd_varlen``,
@@ -21,7 +21,7 @@ Entry points, by family:
 * sequence parallelism: ``attn_merge_partials`` and the ring driver in
   :mod:`exact_attention_100_b200.ring`;
 * status: ``attn_device_status``, ``attn_status_string``, ``attn_num_kernel_launches``,
-  ``attn_selftest_wait_timeout``, ``attn_shutdown``.
+  ``attn_selftest_wait_timeout``, ``attn_noalloc_selftest_wait_timeout``, ``attn_shutdown``.
 """
 
 from __future__ import annotations
@@ -87,6 +87,10 @@ def lib() -> ctypes.CDLL:
         L.attn_selftest_wait_timeout.restype = i
         L.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
         L.attn_fwd_noalloc.restype = i
+        L.attn_noalloc_status.argtypes = [vp]
+        L.attn_noalloc_status.restype = i
+        L.attn_noalloc_selftest_wait_timeout.argtypes = [vp]
+        L.attn_noalloc_selftest_wait_timeout.restype = i
         L.attn_bwd_workspace_bytes.argtypes = [i, i, i]
         L.attn_bwd_workspace_bytes.restype = ctypes.c_ulonglong
         L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
@@ -398,6 +402,17 @@ def attn_fwd_noalloc(q, k, v, o, lse=None, scale=None, causal=False, stream=None
     _check(lib().attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, s,
                                   int(bool(causal)), ATTN_BF16, od, _stream_ptr(stream)), "attn_fwd_noalloc")
     return o, lse
+
+
+def attn_noalloc_status(stream=None) -> int:
+    """Status word of ``attn_fwd_noalloc`` on the current device (synchronises ``stream``, then
+    clears the word); allocates nothing."""
+    return int(lib().attn_noalloc_status(_stream_ptr(stream)))
+
+
+def attn_noalloc_selftest_wait_timeout(stream=None) -> None:
+    """The bounded-wait self-test aimed at the status word of ``attn_fwd_noalloc``."""
+    _check(lib().attn_noalloc_selftest_wait_timeout(_stream_ptr(stream)), "attn_noalloc_selftest_wait_timeout")
 
 
 def attn_hadamard_quant(x, signs=None, x8=None, scales=None, stream=None):

@@ -17,6 +17,11 @@
 // whatever B, H, N and d are; a call that would need more than the array holds is refused with
 // ATTN_ERR_INVALID_ARG.
 //
+// The status word is sticky: every call ORs its failures into it (a bounded wait that ran out)
+// and nothing clears it except attn_noalloc_status, which reads and clears it on a stream.  It
+// starts at zero when the library is loaded.  Calls that overlap on the GPU (different streams)
+// share the word, so a failure is reported to whichever caller reads it first.
+//
 // In host code `g_noalloc_scratch` is only a host-side stand-in for the device array: its
 // device address is obtained once per device with cudaGetSymbolAddress (with that device
 // current) during the first call on the device, and that address is what the kernel receives.
@@ -27,6 +32,7 @@
 
 #include "../../include/attn.h"
 #include "attn_kernels.h"
+#include "attn_selftest.h"
 
 namespace ea {
 cudaError_t setup_fwd_bf16_kernels();
@@ -105,6 +111,22 @@ bool encode_bf16_rows(CUtensorMap* map, const void* base, int d, int N, int H, i
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Contiguous [B, H, N, d] O (bf16 or f32) as the map of the kernel's TMA stores: box of 64 bytes
+// x 128 rows, 64-byte swizzle.
+bool encode_o_rows(CUtensorMap* map, void* base, bool f32, int d, int N, int H, int B) {
+  const cuuint64_t eb = f32 ? 4 : 2;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t row = static_cast<cuuint64_t>(d) * eb;
+  const cuuint64_t strides[3] = {row, row * static_cast<cuuint64_t>(N),
+                                 row * static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(H)};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(64 / eb), 128u, 1u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return g_encode_fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
@@ -126,13 +148,11 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
   NoAllocDevice* st = nullptr;
   int rc = noalloc_setup(&st);
   if (rc != ATTN_OK) return rc;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!encode_bf16_rows(&mq, q, d, N, H, B) || !encode_bf16_rows(&mk, k, d, N, H, B) ||
-      !encode_bf16_rows(&mv, v, d, N, H, B))
+      !encode_bf16_rows(&mv, v, d, N, H, B) || !encode_o_rows(&mo, o, o_dtype == ATTN_FP32, d, N, H, B))
     return ATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the status word must start at zero: the array keeps whatever the previous call left
-  if (cudaMemsetAsync(st->scratch, 0, kScratchNeededBytes, s) != cudaSuccess) return ATTN_ERR_CUDA;
 
   ea::FwdParams p;
   p.o = o;
@@ -158,6 +178,28 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.causal = causal;
   p.o_fp32 = o_dtype == ATTN_FP32 ? 1 : 0;
-  if (ea::launch_attn_fwd_bf16(d, mq, mk, mv, p, st->num_sms, s) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (ea::launch_attn_fwd_bf16(d, mq, mk, mv, mo, p, st->num_sms, s) != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
+}
+
+extern "C" int attn_noalloc_status(void* stream) {
+  NoAllocDevice* st = nullptr;
+  int rc = noalloc_setup(&st);
+  if (rc != ATTN_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int host = 0;  // pageable host memory: the copy completes before cudaMemcpyAsync returns or at the sync
+  if (cudaMemcpyAsync(&host, st->scratch, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (host == 0) return ATTN_OK;
+  if (cudaMemsetAsync(st->scratch, 0, sizeof(int), s) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
+  return (host & ea::kDevStatusTimeout) ? ATTN_ERR_TIMEOUT : ATTN_ERR_INVALID_ARG;
+}
+
+extern "C" int attn_noalloc_selftest_wait_timeout(void* stream) {
+  NoAllocDevice* st = nullptr;
+  int rc = noalloc_setup(&st);
+  if (rc != ATTN_OK) return rc;
+  return ea::launch_wait_selftest(st->scratch, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK
+                                                                                              : ATTN_ERR_CUDA;
 }

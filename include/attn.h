@@ -332,15 +332,34 @@ int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, 
  * a call needing more than the array holds would be refused with ATTN_ERR_INVALID_ARG.
  *   - The first call on each device does a one-time set-up (device address of the array,
  *     kernel attributes); make that first call before any stream capture.
- *   - Every call shares the array: each call clears the status word on `stream` before its
- *     kernel runs, and calls that overlap on the GPU (different streams) race on it.
- *   - A bounded wait that runs out inside such a call is recorded only in that static word;
- *     attn_device_status() does not report it (use attn_fwd when that report is needed).
+ *   - Every call shares the array.  Its status word is sticky: a call ORs into it the failures
+ *     of its kernel (a bounded wait that ran out), and only attn_noalloc_status reads and
+ *     clears it.  Calls that overlap on the GPU (different streams) race on the word: a
+ *     failure is reported to whichever caller reads it first.
+ *   - attn_device_status() does not see these calls; attn_noalloc_status() does.
  *   - Calls through this entry point are not counted by attn_num_kernel_launches().
  */
 int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                      int B, int H, int N, int d, float scale, int causal,
                      int dtype, int o_dtype, void* stream);
+
+/*
+ * attn_noalloc_status -- synchronises `stream`, returns the status word of attn_fwd_noalloc
+ * (the static array on the current device) and clears it; allocates nothing.  The pages have no
+ * counterpart.  ATTN_OK if no call since the last read reported a problem; ATTN_ERR_TIMEOUT if
+ * a bounded wait inside one ran out (that call's O and LSE are undefined; the context stays
+ * usable); ATTN_ERR_CUDA if the copy or the synchronisation failed.  Like attn_fwd_noalloc, its
+ * first call on a device does the one-time set-up.
+ */
+int attn_noalloc_status(void* stream);
+
+/*
+ * attn_noalloc_selftest_wait_timeout -- attn_selftest_wait_timeout pointed at the status word
+ * of attn_fwd_noalloc: one thread waits on an mbarrier that nothing arrives at, gives up after
+ * the bound (2 s) and records a timeout there; the next attn_noalloc_status(stream) returns
+ * ATTN_ERR_TIMEOUT.  Allocates nothing.  Returns ATTN_OK once the kernel is enqueued.
+ */
+int attn_noalloc_selftest_wait_timeout(void* stream);
 
 /*
  * attn_device_status -- synchronises `stream`, returns the current device's status word and
