@@ -10,9 +10,8 @@
 //
 // Roles (warp specialisation, "FlashAttention-3", section "异步搬运与异步计算"):
 //   warps 0..4*NQ-1   softmax warpgroup q = warp/4: one thread per S row (= TMEM lane)
-//   next 4 warps      correction warpgroup: serves events from the MMA thread -- a lazy O
-//                     rescale before a P.V, or the epilogue of a finished Q tile (O / l into
-//                     shared-memory stage buffers, LSE)
+//   next 4 warps      correction warpgroup: the epilogue of a finished Q tile (O / l into
+//                     shared-memory stage buffers, LSE), on events from the MMA thread
 //   next warp         MMA issuer (one thread issues every tcgen05.mma)
 //   next warp         TMA producer (one thread; Q tiles and a ring of K/V slots)
 //   next warp         store warp (one thread): TMA stores of the staged O slices and bulk
@@ -31,10 +30,11 @@
 // bf16 or E4M3) overwrites the first columns of its S buffer; O_q at [256 + D*q, +D).
 //
 // Lazy rescale: a row's reference max m moves only when a block max exceeds it by more than
-// Elem::kTau (base-2 units).  The softmax thread rescales l itself and flags the rows whose O
-// must be multiplied by alpha = 2^(m_old - m_new); only then does the MMA thread ask the
-// correction warpgroup to rescale O before the next P.V.  O and l always refer to the same m,
-// so O / l is exact, and p <= 2^kTau.
+// Elem::kTau (base-2 units).  The softmax thread then multiplies l, and its row of O in TMEM,
+// by alpha = 2^(m_old - m_new) itself, before it hands P over: the P.V of the previous block,
+// the last MMA that wrote O, has completed by then (with two Q tiles it was issued before S of
+// this block, and one thread issues every MMA in order; with one tile the thread waits on
+// pv_done), and the next P.V waits for this P.  O and l always refer to the same m, so O / l is exact, and p <= 2^kTau.
 //
 // Softmax arithmetic per block: one TMEM load of the whole row, eight independent max chains,
 // x = s * c - m with packed f32x2 FMAs, p = 2^x on the special-function unit for most pairs
@@ -99,14 +99,12 @@ struct FwdCfg {
   static constexpr int kStageOff = kRingOff + kSlots * kTileBytes;
   static constexpr int kLseStageOff = kStageOff + 2 * kStageBytes;
   static constexpr int kBarOff = kLseStageOff + 2 * 128 * 4;
-  // full[kSlots], empty[kSlots], q_full, q_empty, s_full[kSBufs], p_full[kSBufs], o_corr[NQ],
+  // full[kSlots], empty[kSlots], q_full, q_empty, s_full[kSBufs], p_full[kSBufs], pv_done[NQ],
   // o_done[NQ], o_free[NQ], ev_full[kEvents], ev_empty[kEvents], drain, st_full[2], st_empty[2]
   static constexpr int kNumBars = 2 * kSlots + 2 + 2 * kSBufs + 3 * NQ + 2 * kEvents + 1 + 4;
-  static constexpr int kAlphaOff = kBarOff + ((kNumBars * 8 + 15) / 16) * 16;
-  static constexpr int kRowMOff = kAlphaOff + NQ * 2 * 128 * 4;
+  static constexpr int kRowMOff = kBarOff + ((kNumBars * 8 + 15) / 16) * 16;
   static constexpr int kRowLOff = kRowMOff + NQ * 2 * 128 * 4;
-  static constexpr int kFlagOff = kRowLOff + NQ * 2 * 128 * 4;  // [NQ][2] int, one byte per warp
-  static constexpr int kEventOff = kFlagOff + 16;               // [kEvents][4] int
+  static constexpr int kEventOff = kRowLOff + NQ * 2 * 128 * 4;  // [kEvents][4] int
   static constexpr int kStageInfoOff = kEventOff + kEvents * 16;  // [2][8] int: what a stage holds
   static constexpr int kMiscOff = kStageInfoOff + 2 * 8 * 4;
   // packed batches: sorted sequence keys [kSchedSeqs] and the unit prefix [kSchedRounds + 1]
@@ -123,7 +121,7 @@ struct FwdCfg {
   static_assert(NQ != 2 || (2 * kRegSoftmax + kRegCorr + kRegOther) * 128 == 65536, "register split");
 };
 
-enum : int { kEvRescale = 0, kEvEpilogue = 1, kEvEnd = 2 };
+enum : int { kEvEpilogue = 1, kEvEnd = 2 };
 
 // The sequence of one (batch entry, head) pair.  Fixed-length batches take every field from
 // the parameters; packed variable-length batches (VL) read the sequence's row range from the
@@ -356,8 +354,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
   uint64_t* q_empty = q_full + 1;
   uint64_t* s_full = q_empty + 1;          // [kSBufs] S ready in TMEM
   uint64_t* p_full = s_full + C::kSBufs;   // [kSBufs] P ready in TMEM (softmax warps)
-  uint64_t* o_corr = p_full + C::kSBufs;   // [NQ] O rescaled (correction warps)
-  uint64_t* o_done = o_corr + NQ;          // [NQ] a P.V finished (commit)
+  uint64_t* pv_done = p_full + C::kSBufs;  // [NQ] one completion per P.V of the tile (commit, NQ = 1)
+  uint64_t* o_done = pv_done + NQ;         // [NQ] the last P.V of a tile finished (commit)
   uint64_t* o_free = o_done + NQ;          // [NQ] epilogue finished reading O (correction warps)
   uint64_t* ev_full = o_free + NQ;         // [kEvents] event posted (MMA thread)
   uint64_t* ev_empty = ev_full + C::kEvents;  // [kEvents] event taken (correction warps)
@@ -367,12 +365,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
   uint8_t* stage = smem + C::kStageOff;                                   // [2][128 rows][64 B]
   float* lse_stage = reinterpret_cast<float*>(smem + C::kLseStageOff);    // [2][128]
   volatile int* stage_info = reinterpret_cast<volatile int*>(smem + C::kStageInfoOff);  // [2][8]
-  float* alpha_s = reinterpret_cast<float*>(smem + C::kAlphaOff);  // [NQ][2][128]
   // [NQ][2][128], slot = parity of the tile's unit count: a tile with a single K/V block writes
   // the next unit's values before the previous epilogue has necessarily read its own
   float* row_m = reinterpret_cast<float*>(smem + C::kRowMOff);     // base-2 LSE
   float* row_l = reinterpret_cast<float*>(smem + C::kRowLOff);     // divisor of O
-  volatile int* flags = reinterpret_cast<volatile int*>(smem + C::kFlagOff);    // [NQ][2]
   volatile int* events = reinterpret_cast<volatile int*>(smem + C::kEventOff);  // [kEvents][4]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
@@ -389,7 +385,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       bar_init(&p_full[b], 4);  // one arrive per softmax warp
     }
     for (int q = 0; q < NQ; ++q) {
-      bar_init(&o_corr[q], 4);
+      bar_init(&pv_done[q], 1);
       bar_init(&o_done[q], 1);
       bar_init(&o_free[q], 4);
     }
@@ -611,19 +607,34 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         tmem_st_32cols(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
         if constexpr (!E::kFp8) tmem_st_32cols(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
         tmem_st_wait();
-        const uint32_t slot = sit & 1u;
-        alpha_s[(q * 2 + slot) * 128 + row] = alpha;
-        const bool need_rescale = __any_sync(0xffffffffu, alpha != 1.f) && j > 0;
+        if (__any_sync(0xffffffffu, alpha != 1.f) && j > 0) {
+          // the reference max moved: O *= alpha for this warp's rows, once the previous block's
+          // P.V has landed.  With two Q tiles it has (it was issued before S of this block); with
+          // one, S of this block goes in first, so wait for completion number sit of pv_done.
+          if constexpr (NQ == 1) {
+            ok = warp_all(wait_bar(&pv_done[q], (sit - 1u) & 1u, ab));
+            if (!ok) break;
+          }
+          tc_fence_after();
+          const uint32_t tO = lane_base + C::kOCol + q * D;
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld_32cols(tO + 32 * cc, o);
+            tmem_ld_wait(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st_32cols(tO + 32 * cc, o);
+          }
+          tmem_st_wait();
+        }
         if (j == n - 1) {
           row_m[(q * 2 + (uit & 1u)) * 128 + row] = m + lg2_approx(l);
           row_l[(q * 2 + (uit & 1u)) * 128 + row] = l * l_div;
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          reinterpret_cast<volatile uint8_t*>(flags + q * 2 + slot)[quarter] = need_rescale ? 1 : 0;
-          bar_arrive(&p_full[sbuf]);
-        }
+        if (lane == 0) bar_arrive(&p_full[sbuf]);
         ++sit;
       }
       ++uit;
@@ -681,29 +692,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         break;
       }
       const uint32_t tO = tmem + lane_off + C::kOCol + q * D;
-      if (kind == kEvRescale) {
-        // the MMA thread committed o_done (phase c) after issuing P.V number `tile` - 1 (for a
-        // rescale the event's last field carries the P.V number): that P.V must land first
-        ok = warp_all(wait_bar(&o_done[q], c & 1u, ab));
-        if (!ok) break;
-        tc_fence_after();
-        const float alpha = alpha_s[(q * 2 + (static_cast<uint32_t>(tile) & 1u)) * 128 + row];
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t r[32];
-            tmem_ld_32cols(tO + 32 * cc, r);
-            tmem_ld_wait(r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st_32cols(tO + 32 * cc, r);
-          }
-          tmem_st_wait();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) bar_arrive(&o_corr[q]);
-      } else {
+      {
         // epilogue: the MMA thread committed o_done (phase c) after the tile's last P.V
         ok = warp_all(wait_bar(&o_done[q], c & 1u, ab));
         if (!ok) break;
@@ -812,10 +801,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       const uint32_t q_base = smem_addr(smem + C::kQOff);
       const uint32_t ring_base = smem_addr(smem + C::kRingOff);
       uint32_t it = 0, qit = 0, sc = 0, ev = 0;
-      // per tile: P.V issued, rescale requests (o_corr phases), units (o_free phases), o_done commits
-      uint32_t pc[NQ], rc[NQ], uc[NQ], od[NQ];
+      // per tile: P.V issued, units (o_free phases), o_done commits
+      uint32_t pc[NQ], uc[NQ], od[NQ];
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) pc[q] = rc[q] = uc[q] = od[q] = 0;
+      for (int q = 0; q < NQ; ++q) pc[q] = uc[q] = od[q] = 0;
 
       auto slot_of = [&](uint32_t idx) { return idx % C::kSlots; };
       // TMA-filled shared memory read by the tensor core stays in the async proxy: the wait alone
@@ -871,16 +860,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
           // P.V 0 overwrites O: the previous unit's epilogue of this tile must be done with it
           if (!wait_bar(&o_free[q], (uc[q] & 1u) ^ 1u, ab)) return false;
           ++uc[q];
-        } else if (flags[q * 2 + (pc[q] & 1u)] != 0) {
-          // o_done is committed only when the correction warpgroup needs it: the commit covers
-          // every MMA issued so far, P.V number pc[q]-1 included
-          tc_commit(&o_done[q]);
-          if (!push_event(kEvRescale, q, od[q]++, 0, static_cast<int>(pc[q]), 0)) return false;
-          if (!wait_bar(&o_corr[q], rc[q] & 1u, ab)) return false;
-          ++rc[q];
         }
         tc_fence_after();
         issue_pv(q, vslot, buf, j > 0);
+        if constexpr (NQ == 1) tc_commit(&pv_done[q]);  // a lazy rescale of the next block waits for it
         if (j == n_q - 1) {
           // uc[q] was counted at j == 0 of this unit: the softmax wrote slot (uc[q] - 1) & 1
           tc_commit(&o_done[q]);
