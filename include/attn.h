@@ -210,10 +210,11 @@ int attn_rope_hadamard_quant_qkv(const void* q, const void* k, const void* v, vo
  *   q_scale, k_scale, v_scale   [B, H, ceil(N/128)] float32 block scales, device.
  *   o              [B, H, N, d] of o_dtype (ATTN_BF16 or ATTN_FP32), device, written.
  *   lse            [B, H, N] float32 or NULL, as for attn_fwd.
- *   d              must be 128.
+ *   d              128 or 256 (64: ATTN_ERR_UNSUPPORTED).
  *   scale, causal, stream   as for attn_fwd.
  * Arithmetic: E4M3 products accumulated in float32; the Q/K block scales are folded into the
- * softmax scale of each tile pair; P is scaled by 2^(8-tau) * s_v(block) / max_block s_v and
+ * softmax scale of each tile pair; P is scaled by 2^(8-tau) * s_v(block) / max_block s_v (tau = 6,
+ * the lazy-rescale threshold in base 2, so the scaled P stays <= 256 < 448) and
  * rounded to E4M3 before the P.V product; O is divided by l and rescaled at the end.
  */
 int attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
