@@ -442,7 +442,7 @@ int fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale
   int rc = check_common(B, H, Nq, scale, causal, o_dtype);
   if (rc != ATTN_OK) return rc;
   if (Nk <= 0 || !units_fit(B, H, Nq)) return ATTN_ERR_INVALID_ARG;
-  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   DeviceState* st = nullptr;
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
@@ -454,7 +454,7 @@ int fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale
       !encode_o_map(&mo, o, o_dtype, d, Nq, H, B, s.sn, s.sh, s.sb))
     return ATTN_ERR_CUDA;
   ea::FwdParams p;
-  fill_params(p, o, lse, st->status, B, H, Nq, Nk, 2, scale, causal, o_dtype);
+  fill_params(p, o, lse, st->status, B, H, Nq, Nk, ea::fwd_units_per_tile_pair(d), scale, causal, o_dtype);
   p.o_sb = s.sb;
   p.o_sh = s.sh;
   p.o_sn = s.sn;

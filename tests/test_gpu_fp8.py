@@ -46,9 +46,9 @@ def _quantise(q, k, v, signs):
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("n", [1, 127, 300, 1024])
 @pytest.mark.parametrize("use_signs", [True, False])
-def test_against_oracle_on_dequantised_inputs(causal, n, use_signs):
-    d = 128
-    q, k, v = normal_qkv(1, 2, n, d, seed=n, outlier_frac=1e-3)
+@pytest.mark.parametrize("d", [128, 256])
+def test_against_oracle_on_dequantised_inputs(causal, n, use_signs, d):
+    q, k, v = normal_qkv(1, 2, n, d, seed=n + d, outlier_frac=1e-3)
     signs = hadamard_signs(d) if use_signs else None
     q8, qs, k8, ks, v8, vs = _quantise(q, k, v, signs)
     o, lse = ea.attn_fwd_fp8(q8, k8, v8, qs, ks, vs, causal=causal, o_dtype=torch.float32)
@@ -68,8 +68,13 @@ def test_against_oracle_on_dequantised_inputs(causal, n, use_signs):
     assert lrel.max() <= 1e-3, lrel.max()
 
 
-def test_fp8_workload_rmse_with_and_without_hadamard():
-    B, H, N, d = 2, 16, 8192, 128
+@pytest.mark.parametrize("B,H,N,d", [(2, 16, 8192, 128), (2, 8, 8192, 256)])
+def test_fp8_workload_rmse_with_and_without_hadamard(B, H, N, d):
+    """The FP8 workload (d = 128, the configuration the 3e-2 bar is set on, with and without the
+    transform) and the same token count at d = 256 (the sweep's H = 2048 / d).  At d = 256 the
+    bar holds on the transformed path; without the transform the error of quantising the
+    outlier inputs alone is already about 2.3e-2 (the float64 oracle on the dequantised inputs,
+    exact P), so there the test only requires that the transform lowers the error."""
     q, k, v = normal_qkv(B, H, N, d, seed=0, outlier_frac=1e-3)
     rng = np.random.default_rng(3)
     rows = [(int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(N))) for _ in range(48)]
@@ -83,18 +88,20 @@ def test_fp8_workload_rmse_with_and_without_hadamard():
             o_ref, _ = attention_ref(q[b, h, i:i + 1], k[b, h], v[b, h], 1 / math.sqrt(d), False)
             err.append(o[b, h, i].cpu().numpy().astype(np.float64) - o_ref[0])
         rmse[use] = float(np.sqrt(np.mean(np.square(err))))
-    assert rmse[True] <= 3e-2 and rmse[False] <= 3e-2, rmse
+    assert rmse[True] <= 3e-2, rmse
+    if d == 128:
+        assert rmse[False] <= 3e-2, rmse
     assert rmse[True] < rmse[False], rmse
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("nq,nk", [(128, 300), (300, 128), (1, 513), (513, 1), (640, 130)])
-def test_fp8_qk_against_oracle_on_dequantised_inputs(nq, nk, causal):
+@pytest.mark.parametrize("nq,nk,d", [(128, 300, 128), (300, 128, 128), (1, 513, 128), (513, 1, 128), (640, 130, 128),
+                                     (300, 700, 256), (513, 129, 256)])
+def test_fp8_qk_against_oracle_on_dequantised_inputs(nq, nk, d, causal):
     """attn_fwd_fp8_qk: key length different from the query length (bottom-right causal); the
     same bars as the equal-length case on rows that see a key, O = 0 and LSE = -inf on rows
     that see none."""
     from exact_attention_100_b200.inputs import normal_qkv_lengths
-    d = 128
     q, k, v = normal_qkv_lengths(1, 2, nq, nk, d, seed=nq + nk)
     q8, qs, k8, ks, v8, vs = _quantise(q, k, v, hadamard_signs(d))
     o, lse = ea.attn_fwd_fp8_qk(q8, k8, v8, qs, ks, vs, causal=causal, o_dtype=torch.float32)
