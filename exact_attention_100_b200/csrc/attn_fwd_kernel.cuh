@@ -22,7 +22,8 @@
 // Overlap ("FlashAttention-3", sections "Ping-pong 调度" and "同一个 warpgroup 内部也能再叠一层";
 // "Flash Attention V3 解析", section 3.2.3):
 //   NQ = 2: per K/V block j the MMA order is PV0(j), S0(j+1), PV1(j), S1(j+1): the tensor core
-//           runs one tile's GEMMs while the other tile's softmax runs.
+//           runs one tile's GEMMs while the other tile's softmax runs.  On a unit's last block
+//           S0(0) of the next unit goes in before PV1, so units overlap too.
 //   NQ = 1: S is double-buffered in TMEM and S(j+1) is issued before PV(j), so the softmax of
 //           block j+1 overlaps P.V of block j.
 //
@@ -878,6 +879,31 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       };
 
       bool ok = true;
+      // Two Q tiles: on a unit's last step, once tile 0 has had its last P.V, S0(0) of the next
+      // unit goes in before tile 1's last P.V if that unit's Q and K_0 have already landed, so
+      // that tile 0's softmax of the next unit overlaps the end of this one.  (Its Q was
+      // requested when this unit's last S went in; K_0 needs one ring slot.)  Only tests the
+      // barriers, never waits: a late load must not hold back tile 1's last P.V.
+      bool s0_early = false;
+      auto issue_next_s0 = [&](int k) {
+        for (int k2 = k + 1;; ++k2) {
+          const int u2 = unit_index(k2);
+          if (u2 >= num_units) return false;
+          const Unit U2 = decode_unit<NQ, VL>(u2, p, sched);
+          if constexpr (VL) {
+            if (!U2.present) continue;
+          }
+          if (U2.n_max == 0 || U2.n[0] == 0) return false;
+          // `it` is the next unit's K_0
+          if (!bar_test_wait(smem_addr(q_full), qit & 1u) ||
+              !bar_test_wait(smem_addr(&full[slot_of(it)]), (it / C::kSlots) & 1u))
+            return false;
+          ++qit;
+          issue_s(0, slot_of(it), 0);
+          tc_commit(&s_full[0]);
+          return true;
+        }
+      };
       for (int k = 0; ok; ++k) {
         const int u = unit_index(k);
         if (u >= num_units) break;
@@ -887,21 +913,24 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         }
         const uint32_t base = it;  // ring index of K_0; K_j = base + 2j, V_j = base + 2j + 1
         it += 2u * U.n_max;
-        ok = wait_bar(q_full, qit & 1u, ab);
-        ++qit;
-        if (!ok) break;
+        if (!s0_early) {  // (an early S0 already waited for this unit's Q and K_0)
+          ok = wait_bar(q_full, qit & 1u, ab);
+          ++qit;
+          if (!ok) break;
+        }
         if (U.n_max == 0) {  // no tile of the unit sees a key: nothing to compute, Q is free again
           tc_commit(q_empty);
           continue;
         }
-        if (!(ok = wait_loaded(base))) break;
+        if (!s0_early && !(ok = wait_loaded(base))) break;
         if constexpr (NQ == 2) {
 #pragma unroll
           for (int q = 0; q < NQ; ++q)
-            if (U.n[q] > 0) {
+            if (U.n[q] > 0 && !(q == 0 && s0_early)) {
               issue_s(q, slot_of(base), q);
               tc_commit(&s_full[q]);
             }
+          s0_early = false;
           tc_commit(&empty[slot_of(base)]);
           if (U.n_max == 1) tc_commit(q_empty);
           for (int j = 0; j < U.n_max && ok; ++j) {
@@ -917,6 +946,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
                 issue_s(0, slot_of(ki), 0);
                 tc_commit(&s_full[0]);
               }
+            } else if (j < U.n[1]) {
+              s0_early = issue_next_s0(k);
             }
             if (j < U.n[1] && !(ok = pv_step(1, j, U.n[1], U.bh, U.tile0, slot_of(vi), 1))) break;
             tc_commit(&empty[slot_of(vi)]);
