@@ -401,7 +401,7 @@ def run_ours(args):
     bwd = bwd_section(args, dev, rank) if not args.no_bwd else None
     varlen = varlen_section(args, dev, rank) if not args.no_varlen else None
     ring = ring_section(args, dev, rank) if not args.no_ring else None
-    sweep = sweep_section(args, dev) if not args.no_sweep else None
+    sweep = sweep_section(args, dev, uuid) if not args.no_sweep else None
     barrier()
     if rank == 0:
         peaks = load_peaks()
@@ -751,7 +751,7 @@ SWEEP_DS = (64, 128, 256)
 SWEEP_NS = (512, 1024, 2048, 4096, 8192, 16384)
 
 
-def sweep_section(args, dev):
+def sweep_section(args, dev, uuid=None):
     """The head-dim x length sweep (16384 tokens per head-batch: B = 16384/N, H = 2048/d, causal and
     not) and the B=4 H=16 N=2048 d=128 configuration, each timed like the headline (3 warm-ups,
     then the mean of 10 calls with a cold L2).  Inputs are iid N(0,1) drawn by torch on the device
@@ -765,6 +765,9 @@ def sweep_section(args, dev):
     g = torch.Generator(device=dev).manual_seed(1)
     points = [("C4", d, N, 16384 // N, 2048 // d) for d in SWEEP_DS for N in SWEEP_NS] + [("C2", 128, 2048, 4, 16)]
     out = []
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    t_begin = time.time()
     for (cfg, d, N, B, H) in points:
         q, k, v = (torch.randn(B, H, N, d, device=dev, generator=g).to(torch.bfloat16) for _ in range(3))
         o = torch.empty_like(q)
@@ -784,9 +787,13 @@ def sweep_section(args, dev):
             out.append({"config": cfg, "d": d, "N": N, "B": B, "H": H,
                         "causal": causal, "ms": round(ms, 5), "tflops": round(tf, 1), "frac": round(tf / burst, 4)})
         del q, k, v, o, lse
+    t_end = time.time()
     assert ea.attn_device_status() == ea.ATTN_OK
     return {"points": out, "peak_tflops": burst, "peak_source": peaks["source"],
-            "timing": "3 warm-ups, mean of 10 calls, 256 MiB buffer written between calls"}
+            "timing": "3 warm-ups, mean of 10 calls, 256 MiB buffer written between calls",
+            "clocks": sampler.stop(t_begin, t_end),
+            "clocks_note": "the whole sweep runs back to back after the other sections; a median SM clock below "
+                           "the maximum with sw_power_cap means its longer points ran power-capped"}
 
 
 def run_sweep(args):
