@@ -880,29 +880,38 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
 
       bool ok = true;
       // Two Q tiles: on a unit's last step, once tile 0 has had its last P.V, S0(0) of the next
-      // unit goes in before tile 1's last P.V if that unit's Q and K_0 have already landed, so
+      // unit goes in before tile 1's last P.V as soon as that unit's Q and K_0 have landed, so
       // that tile 0's softmax of the next unit overlaps the end of this one.  (Its Q was
-      // requested when this unit's last S went in; K_0 needs one ring slot.)  Only tests the
-      // barriers, never waits: a late load must not hold back tile 1's last P.V.
+      // requested when this unit's last S went in; K_0 needs one ring slot.)  The MMA thread
+      // polls both events: whichever comes first goes first, so a late load never holds back
+      // tile 1's last P.V.  Returns whether S0 was issued.
       bool s0_early = false;
       auto issue_next_s0 = [&](int k) {
-        for (int k2 = k + 1;; ++k2) {
+        int k2 = k + 1;
+        Unit U2;
+        for (;; ++k2) {
           const int u2 = unit_index(k2);
           if (u2 >= num_units) return false;
-          const Unit U2 = decode_unit<NQ, VL>(u2, p, sched);
+          U2 = decode_unit<NQ, VL>(u2, p, sched);
           if constexpr (VL) {
             if (!U2.present) continue;
           }
-          if (U2.n_max == 0 || U2.n[0] == 0) return false;
-          // `it` is the next unit's K_0
-          if (!bar_test_wait(smem_addr(q_full), qit & 1u) ||
-              !bar_test_wait(smem_addr(&full[slot_of(it)]), (it / C::kSlots) & 1u))
-            return false;
-          ++qit;
-          issue_s(0, slot_of(it), 0);
-          tc_commit(&s_full[0]);
-          return true;
+          break;
         }
+        if (U2.n_max == 0 || U2.n[0] == 0) return false;
+        // `it` is the next unit's K_0; P1 of this step completes p_full[1] phase pc[1] & 1
+        const uint32_t a_q = smem_addr(q_full), a_k = smem_addr(&full[slot_of(it)]), a_p = smem_addr(&p_full[1]);
+        const uint32_t ph_q = qit & 1u, ph_k = (it / C::kSlots) & 1u, ph_p = pc[1] & 1u;
+        const unsigned long long t0 = global_timer_ns();
+        for (uint32_t n = 0;; ++n) {
+          if (bar_test_wait(a_q, ph_q) && bar_test_wait(a_k, ph_k)) break;
+          if (bar_test_wait(a_p, ph_p)) return false;
+          if ((n & 15u) == 15u && (*ab.flag || global_timer_ns() - t0 > kWaitLimitNs)) return false;
+        }
+        ++qit;
+        issue_s(0, slot_of(it), 0);
+        tc_commit(&s_full[0]);
+        return true;
       };
       for (int k = 0; ok; ++k) {
         const int u = unit_index(k);
