@@ -524,6 +524,32 @@ def fp8_section(args, dev, rank):
                              "vs_unrotated": rope_ms / pre_ms, "peak_source": peaks["source"],
                              "note": "Q and K rotated (frequency-major tables [64, 8192] float32, L2-resident "
                                      "after the first read), then H D and E4M3; V quantised as it is"}
+
+    # the same launch reading Q, K, V as head views of one fused [B, N, 3, H, d] projection
+    fused = torch.empty((B, N, 3, H, d), dtype=torch.bfloat16, device=dev)
+    views = [fused[:, :, j].transpose(1, 2) for j in range(3)]
+    for view, x in zip(views, (q, k, v)):
+        view.copy_(x)
+
+    def pre_strided():
+        ea.attn_hadamard_quant_qkv_strided(views[0], views[1], views[2], signs, outs=outs, stream=stream)
+
+    for _ in range(3):
+        pre_strided()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        pre_strided()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    st_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    sgbs = pre_bytes / (st_ms * 1e-3) / 1e9
+    out["prekernel_strided"] = {"ms_3_tensors": st_ms, "achieved_gbs": sgbs, "frac": sgbs / float(peaks["hbm_gbs"]),
+                                "vs_contiguous": st_ms / pre_ms, "bytes_per_call": pre_bytes,
+                                "note": "Q, K, V read as head views of one fused [B, N, 3, H, d] bf16 buffer "
+                                        "(attn_hadamard_quant_qkv_strided); contiguous E4M3 outputs"}
+    del fused, views
     try:
         o = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
         lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
@@ -697,12 +723,35 @@ def varlen_section(args, dev, rank):
     flops = sum(attn_flops(1, H, n, d, causal) for n in lens)
     peaks = load_peaks()
     tf = flops / (ms * 1e-3) / 1e12
+    # the backward of the same packed batch (bf16 gradients, dO iid N(0,1) by torch)
+    dout = torch.randn(q.shape, generator=torch.Generator(device=dev).manual_seed(3), device=dev).to(torch.bfloat16)
+    g = [torch.empty_like(q) for _ in range(3)]
+    ws = torch.empty(ea.attn_bwd_workspace_bytes(len(lens), H, max(lens)) // 4, dtype=torch.float32, device=dev)
+
+    def bstep():
+        ea.attn_bwd_varlen(q, k, v, o, lse, dout, cu_q, cu_k, max(lens), max(lens), dq=g[0], dk=g[1], dv=g[2],
+                           workspace=ws, causal=causal, stream=stream)
+
+    for _ in range(3):
+        bstep()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        bstep()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+    bms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    btf = 2.5 * flops / (bms * 1e-3) / 1e12
     return {"workload": f"bf16 packed varlen fwd, {len(lens)} sequences of {w['lo']}..{w['hi']} tokens "
                         f"(total {w['total']}), H={H} d={d} causal",
             "lengths": lens, "ms": ms, "achieved_tflops": tf, "peak_tflops": float(peaks["bf16_tflops"]),
             "frac": tf / float(peaks["bf16_tflops"]), "bound": "tensor", "flops_per_call": flops,
             "flops_note": "sum over sequences of 4 H d N^2 / 2 (causal), as the headline counts",
-            "peak_source": peaks["source"]}
+            "peak_source": peaks["source"],
+            "bwd": {"ms": bms, "achieved_tflops": btf, "frac": btf / float(peaks["bf16_tflops"]),
+                    "flops_note": "2.5 x the forward count (five products), bf16 gradients, 3 launches"}}
 
 
 def bwd_section(args, dev, rank):

@@ -77,10 +77,14 @@ def lib() -> ctypes.CDLL:
         L.attn_rope_hadamard_quant_qkv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
         L.attn_rope_hadamard_quant_qkv.restype = i
         L.attn_hadamard_quant_qkv.restype = i
+        L.attn_hadamard_quant_qkv_strided.argtypes = [vp] * 10 + [i, i, i, i, vp, vp]
+        L.attn_hadamard_quant_qkv_strided.restype = i
         L.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
         L.attn_fwd_fp8.restype = i
         L.attn_fwd_fp8_qk.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
         L.attn_fwd_fp8_qk.restype = i
+        L.attn_fwd_fp8_strided.argtypes = [vp] * 8 + [i, i, i, i, i, vp, f, i, i, vp]
+        L.attn_fwd_fp8_strided.restype = i
         L.attn_merge_partials.argtypes = [vp, vp, vp, vp, ctypes.c_longlong, i, i, vp]
         L.attn_merge_partials.restype = i
         L.attn_selftest_wait_timeout.argtypes = [vp]
@@ -450,6 +454,29 @@ def attn_hadamard_quant_qkv(q, k, v, signs, outs=None, stream=None):
     return outs
 
 
+def attn_hadamard_quant_qkv_strided(q, k, v, signs, outs=None, stream=None):
+    """attn_hadamard_quant_qkv on logical [B, H, N, d] bf16 views with any strides whose last one
+    is 1 (e.g. the head views of one fused [B, N, 3, H, d] projection), without a copy.  The
+    outputs are contiguous, bit-identical to attn_hadamard_quant_qkv on contiguous copies.
+    Returns ``(q8, k8, v8, q_scale, k_scale, v_scale)``; ``outs`` may supply them."""
+    import torch
+    B, H, N, d = _dims(q)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or t.stride(-1) != 1 or t.shape != q.shape:
+            raise ValueError("q, k, v must be bf16 of one shape with a contiguous last dimension")
+    nb = (N + 127) // 128
+    if outs is None:
+        outs = tuple(torch.empty(q.shape, dtype=torch.uint8, device=q.device) for _ in range(3)) + \
+            tuple(torch.empty((B, H, nb), dtype=torch.float32, device=q.device) for _ in range(3))
+    q8, k8, v8, qs, ks, vs = outs
+    strides = (ctypes.c_longlong * 9)(*[int(x) for t in (q, k, v) for x in t.stride()[:3]])
+    _check(lib().attn_hadamard_quant_qkv_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs),
+                                                 _ptr(ks), _ptr(vs), _ptr(signs), B, H, N, d,
+                                                 ctypes.cast(strides, ctypes.c_void_p), _stream_ptr(stream)),
+           "attn_hadamard_quant_qkv_strided")
+    return outs
+
+
 def attn_rope_hadamard_quant_qkv(q, k, v, signs, cos, sin, outs=None, stream=None):
     """attn_hadamard_quant_qkv with Q and K first rotated by the rotary tables ``cos``, ``sin``
     (frequency-major [d/2, n_pos] float32 cuda tensors, n_pos >= N; row n of each sequence uses
@@ -511,6 +538,35 @@ def attn_fwd_fp8_qk(q8, k8, v8, q_scale, k_scale, v_scale, o=None, lse=None, sca
     _check(lib().attn_fwd_fp8_qk(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
                                  _ptr(o), _ptr(lse), B, H, Nq, Nk, d, s, int(bool(causal)), od, _stream_ptr(stream)),
            "attn_fwd_fp8_qk")
+    return o, lse
+
+
+def attn_fwd_fp8_strided(q8, k8, v8, q_scale, k_scale, v_scale, o=None, lse=None, scale=None, causal=False,
+                        o_dtype=None, stream=None):
+    """attn_fwd_fp8_qk on logical [B, H, N, d] uint8 (E4M3) views and an output ``o`` with any
+    strides whose last one is 1 (E4M3 strides multiples of 16, O strides multiples of 8), e.g. O
+    written straight into a sequence-major [B, N, H, d] buffer.  The scales stay contiguous
+    [B, H, ceil(N/128)].  ``o`` defaults to a contiguous tensor.  Returns ``(o, lse)``."""
+    import torch
+    B, H, Nq, d = _dims(q8)
+    Nk = int(k8.shape[2])
+    if tuple(k8.shape) != (B, H, Nk, d) or v8.shape != k8.shape:
+        raise ValueError("k8 and v8 must be [B, H, Nk, d] with q8's B, H, d")
+    for t in (q8, k8, v8):
+        if t.dtype != torch.uint8 or t.stride(-1) != 1:
+            raise ValueError("q8, k8, v8 must be uint8 with a contiguous last dimension")
+    if o is None:
+        o = torch.empty((B, H, Nq, d), dtype=o_dtype or torch.bfloat16, device=q8.device)
+    if tuple(o.shape) != (B, H, Nq, d) or o.stride(-1) != 1:
+        raise ValueError("o must be [B, H, Nq, d] with a contiguous last dimension")
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q8.device)
+    strides = (ctypes.c_longlong * 12)(*[int(x) for t in (q8, k8, v8, o) for x in t.stride()[:3]])
+    od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_fwd_fp8_strided(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
+                                      _ptr(o), _ptr(lse), B, H, Nq, Nk, d, ctypes.cast(strides, ctypes.c_void_p), s,
+                                      int(bool(causal)), od, _stream_ptr(stream)), "attn_fwd_fp8_strided")
     return o, lse
 
 

@@ -74,20 +74,6 @@ int device_state(DeviceState** out) {
   return ATTN_OK;
 }
 
-// 3-D tiled map over a contiguous [BH, N, row_bytes/elem] tensor: box = 128 bytes x 128 rows
-// x 1 head, 128-byte swizzle, zero fill outside the tensor.
-bool encode_rows_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N,
-                     int BH) {
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem_bytes,
-                                 static_cast<cuuint64_t>(d) * elem_bytes * static_cast<cuuint64_t>(N)};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes), 128u, 1u};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  return g_encode(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // 4-D tiled map for the forward kernels: dims (d, rows, heads, batch) with the caller's element
 // strides of a row, a head and a batch entry (d contiguous); box = 128 bytes x 128 rows x 1 x 1,
 // 128-byte swizzle, zero fill past the last row.
@@ -123,8 +109,9 @@ bool encode_o_map(CUtensorMap* map, void* base, int o_dtype, int d, int N, int H
 }
 
 // Element strides (batch, head, row) of one [B, H, N, d] tensor; the forward's maps and its O
-// stores take any strides that are positive multiples of 8 elements below 2^36.  A stride of a
-// dimension of extent 1 is never used to address anything and is replaced by 8.
+// stores take any strides that are positive multiples of 16 bytes (8 bf16 elements, 16 E4M3
+// codes) below 2^36 elements.  A stride of a dimension of extent 1 is never used to address
+// anything and is replaced by that multiple.
 struct Strides {
   long long sb, sh, sn;
 };
@@ -134,12 +121,12 @@ Strides contiguous_strides(int H, int N, int d) {
   return {sh * H, sh, sn};
 }
 
-bool canonical_strides(const long long* s, int B, int H, int N, Strides* out) {
+bool canonical_strides(const long long* s, int B, int H, int N, Strides* out, long long align = 8) {
   long long v[3] = {s[0], s[1], s[2]};
   const int ext[3] = {B, H, N};
   for (int i = 0; i < 3; ++i) {
-    if (ext[i] == 1) v[i] = 8;
-    if (v[i] <= 0 || (v[i] & 7) != 0 || v[i] >= (1ll << 36)) return false;
+    if (ext[i] == 1) v[i] = align;
+    if (v[i] <= 0 || v[i] % align != 0 || v[i] >= (1ll << 36)) return false;
   }
   *out = {v[0], v[1], v[2]};
   return true;
@@ -361,11 +348,12 @@ int attn_hadamard_quant(const void* x, void* x8, float* scales, const signed cha
   int rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
   const float post = signs ? static_cast<float>(1.0 / std::sqrt(static_cast<double>(d))) : 1.0f;
+  const Strides c = contiguous_strides(H, N, d);
   CUtensorMap mx;
-  if (!encode_rows_map(&mx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H)) return ATTN_ERR_CUDA;
+  if (!encode_fwd_map(&mx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, H, B, c.sn, c.sh, c.sb)) return ATTN_ERR_CUDA;
   uint8_t* out = static_cast<uint8_t*>(x8);
   const int transform = signs != nullptr ? 1 : 0;
-  if (ea::launch_hadamard_quant(&mx, 1, &out, &scales, &post, &transform, signs, B * H, N, d, nullptr, nullptr,
+  if (ea::launch_hadamard_quant(&mx, 1, &out, &scales, &post, &transform, signs, B * H, H, N, d, nullptr, nullptr,
                                 nullptr, 0, st->num_sms, st->status,
                                static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
@@ -377,10 +365,11 @@ int attn_hadamard_quant(const void* x, void* x8, float* scales, const signed cha
 
 namespace {
 
-// attn_hadamard_quant_qkv and attn_rope_hadamard_quant_qkv (cos/sin NULL: no rotation).
+// attn_hadamard_quant_qkv, attn_hadamard_quant_qkv_strided and attn_rope_hadamard_quant_qkv
+// (cos/sin NULL: no rotation; st3 NULL: contiguous inputs, else their element strides).
 int hq_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8, float* q_scale, float* k_scale,
            float* v_scale, const signed char* signs, const float* cos, const float* sin, int n_pos, int B, int H, int N,
-           int d, void* stream) {
+           int d, const Strides* st3, void* stream) {
   const void* in[3] = {q, k, v};
   void* out[3] = {q8, k8, v8};
   float* sc[3] = {q_scale, k_scale, v_scale};
@@ -395,14 +384,18 @@ int hq_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void
   int rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
   CUtensorMap maps[3];
-  for (int t = 0; t < 3; ++t)
-    if (!encode_rows_map(&maps[t], in[t], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H)) return ATTN_ERR_CUDA;
+  const Strides c = contiguous_strides(H, N, d);
+  for (int t = 0; t < 3; ++t) {
+    const Strides& st = st3 ? st3[t] : c;
+    if (!encode_fwd_map(&maps[t], in[t], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, H, B, st.sn, st.sh, st.sb))
+      return ATTN_ERR_CUDA;
+  }
   const float rsd = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
   uint8_t* o8[3] = {static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8), static_cast<uint8_t*>(v8)};
   const float post[3] = {rsd, rsd, 1.0f};
   const int transform[3] = {1, 1, 0};
   const int rope[3] = {1, 1, 0};  // Q and K rotated, V not
-  if (ea::launch_hadamard_quant(maps, 3, o8, sc, post, transform, signs, B * H, N, d, cos ? rope : nullptr, cos, sin,
+  if (ea::launch_hadamard_quant(maps, 3, o8, sc, post, transform, signs, B * H, H, N, d, cos ? rope : nullptr, cos, sin,
                                 n_pos, st->num_sms, st->status, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
@@ -416,7 +409,18 @@ extern "C" {
 int attn_hadamard_quant_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8,
                             float* q_scale, float* k_scale, float* v_scale, const signed char* signs, int B, int H,
                             int N, int d, void* stream) {
-  return hq_qkv(q, k, v, q8, k8, v8, q_scale, k_scale, v_scale, signs, nullptr, nullptr, 0, B, H, N, d, stream);
+  return hq_qkv(q, k, v, q8, k8, v8, q_scale, k_scale, v_scale, signs, nullptr, nullptr, 0, B, H, N, d, nullptr,
+                stream);
+}
+
+int attn_hadamard_quant_qkv_strided(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8,
+                                    float* q_scale, float* k_scale, float* v_scale, const signed char* signs, int B,
+                                    int H, int N, int d, const long long* strides, void* stream) {
+  if (strides == nullptr || B <= 0 || H <= 0 || N <= 0) return ATTN_ERR_INVALID_ARG;
+  Strides st3[3];
+  for (int t = 0; t < 3; ++t)
+    if (!canonical_strides(strides + 3 * t, B, H, N, &st3[t])) return ATTN_ERR_INVALID_ARG;
+  return hq_qkv(q, k, v, q8, k8, v8, q_scale, k_scale, v_scale, signs, nullptr, nullptr, 0, B, H, N, d, st3, stream);
 }
 
 int attn_rope_hadamard_quant_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8,
@@ -424,17 +428,18 @@ int attn_rope_hadamard_quant_qkv(const void* q, const void* k, const void* v, vo
                                  const float* cos, const float* sin, int n_pos, int B, int H, int N, int d,
                                  void* stream) {
   if (!cos || !sin || !aligned16(cos) || !aligned16(sin) || n_pos < N) return ATTN_ERR_INVALID_ARG;
-  return hq_qkv(q, k, v, q8, k8, v8, q_scale, k_scale, v_scale, signs, cos, sin, n_pos, B, H, N, d, stream);
+  return hq_qkv(q, k, v, q8, k8, v8, q_scale, k_scale, v_scale, signs, cos, sin, n_pos, B, H, N, d, nullptr, stream);
 }
 
 }  // extern "C"
 
 namespace {
 
-// attn_fwd_fp8 and attn_fwd_fp8_qk: E4M3 Q [B, H, Nq, d], K and V [B, H, Nk, d], contiguous.
+// attn_fwd_fp8, attn_fwd_fp8_qk and attn_fwd_fp8_strided: E4M3 Q [B, H, Nq, d], K and V
+// [B, H, Nk, d]; st4 (NULL: contiguous) the element strides of q8, k8, v8 and o.
 int fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
-            const float* v_scale, void* o, float* lse, int B, int H, int Nq, int Nk, int d, float scale, int causal,
-            int o_dtype, void* stream) {
+            const float* v_scale, void* o, float* lse, int B, int H, int Nq, int Nk, int d, const Strides* st4,
+            float scale, int causal, int o_dtype, void* stream) {
   if (!q8 || !k8 || !v8 || !q_scale || !k_scale || !v_scale || !o) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || (lse && !aligned16(lse)) ||
       !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(v_scale))
@@ -446,18 +451,19 @@ int fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale
   DeviceState* st = nullptr;
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
-  const Strides s = contiguous_strides(H, Nq, d), sk = contiguous_strides(H, Nk, d);
+  const Strides cq = contiguous_strides(H, Nq, d), ck = contiguous_strides(H, Nk, d);
+  const Strides sq = st4 ? st4[0] : cq, sk = st4 ? st4[1] : ck, sv = st4 ? st4[2] : ck, so = st4 ? st4[3] : cq;
   CUtensorMap mq, mk, mv, mo;
-  if (!encode_fwd_map(&mq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Nq, H, B, s.sn, s.sh, s.sb) ||
+  if (!encode_fwd_map(&mq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Nq, H, B, sq.sn, sq.sh, sq.sb) ||
       !encode_fwd_map(&mk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Nk, H, B, sk.sn, sk.sh, sk.sb) ||
-      !encode_fwd_map(&mv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Nk, H, B, sk.sn, sk.sh, sk.sb) ||
-      !encode_o_map(&mo, o, o_dtype, d, Nq, H, B, s.sn, s.sh, s.sb))
+      !encode_fwd_map(&mv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Nk, H, B, sv.sn, sv.sh, sv.sb) ||
+      !encode_o_map(&mo, o, o_dtype, d, Nq, H, B, so.sn, so.sh, so.sb))
     return ATTN_ERR_CUDA;
   ea::FwdParams p;
   fill_params(p, o, lse, st->status, B, H, Nq, Nk, ea::fwd_units_per_tile_pair(d), scale, causal, o_dtype);
-  p.o_sb = s.sb;
-  p.o_sh = s.sh;
-  p.o_sn = s.sn;
+  p.o_sb = so.sb;
+  p.o_sh = so.sh;
+  p.o_sn = so.sn;
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.v_scale = v_scale;
@@ -474,13 +480,28 @@ extern "C" {
 int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
                  const float* v_scale, void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
                  int o_dtype, void* stream) {
-  return fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, N, d, scale, causal, o_dtype, stream);
+  return fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, N, d, nullptr, scale, causal, o_dtype,
+                 stream);
 }
 
 int attn_fwd_fp8_qk(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
                     const float* v_scale, void* o, float* lse, int B, int H, int Nq, int Nk, int d, float scale,
                     int causal, int o_dtype, void* stream) {
-  return fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, Nq, Nk, d, scale, causal, o_dtype, stream);
+  return fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, Nq, Nk, d, nullptr, scale, causal, o_dtype,
+                 stream);
+}
+
+int attn_fwd_fp8_strided(const void* q8, const void* k8, const void* v8, const float* q_scale,
+                         const float* k_scale, const float* v_scale, void* o, float* lse, int B, int H, int Nq,
+                         int Nk, int d, const long long* strides, float scale, int causal, int o_dtype,
+                         void* stream) {
+  if (strides == nullptr || B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0) return ATTN_ERR_INVALID_ARG;
+  Strides st4[4];
+  for (int t = 0; t < 4; ++t)
+    if (!canonical_strides(strides + 3 * t, B, H, t == 1 || t == 2 ? Nk : Nq, &st4[t], t < 3 ? 16 : 8))
+      return ATTN_ERR_INVALID_ARG;
+  return fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, Nq, Nk, d, st4, scale, causal, o_dtype,
+                 stream);
 }
 
 unsigned long long attn_bwd_workspace_bytes(int B, int H, int N) {

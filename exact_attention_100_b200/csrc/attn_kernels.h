@@ -105,16 +105,17 @@ cudaError_t setup_bwd_kernels();
 cudaError_t launch_attn_bwd(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                             const CUtensorMap& dout, const BwdParams& p, int num_sms, cudaStream_t stream);
 
-// Hadamard + per-block E4M3 quantisation of 1..3 tensors of one shape [BH, N, d] in one launch:
-// tm[t] is a 3-D tiled map over tensor t (bf16, box 64 x 128 x 1, 128-byte swizzle); x8[t] its
-// E4M3 output, scales[t] its [BH, ceil(N/128)] block scales, post[t] the factor on the stored
-// scale, transform[t] != 0 to apply H_d D (signs: d entries +-1).  rope (NULL: none) marks
+// Hadamard + per-block E4M3 quantisation of 1..3 tensors of one shape [B, H, N, d] in one launch:
+// tm[t] is a 4-D tiled map (d, rows, heads, batch) over tensor t with its own strides (bf16, box
+// 64 x 128 x 1 x 1, 128-byte swizzle); x8[t] its contiguous E4M3 output, scales[t] its
+// [BH, ceil(N/128)] block scales, post[t] the factor on the stored scale, transform[t] != 0 to
+// apply H_d D (signs: d entries +-1).  rope (NULL: none) marks
 // the tensors whose rows are first rotated with the frequency-major [d/2, n_pos] float32 tables
 // cos and sin (n_pos >= N).
 cudaError_t launch_hadamard_quant(const CUtensorMap* tm, int ntensors, uint8_t* const* x8, float* const* scales,
-                                  const float* post, const int* transform, const signed char* signs, int BH, int N,
-                                  int d, const int* rope, const float* cos, const float* sin, int n_pos, int num_sms,
-                                  int* status, cudaStream_t stream);
+                                  const float* post, const int* transform, const signed char* signs, int BH, int H,
+                                  int N, int d, const int* rope, const float* cos, const float* sin, int n_pos,
+                                  int num_sms, int* status, cudaStream_t stream);
 
 // Sets the pre-kernel's shared-memory attributes on the current device.
 cudaError_t setup_hadamard_quant_kernels();

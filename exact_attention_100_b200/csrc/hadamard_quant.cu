@@ -98,6 +98,7 @@ struct HqJob {
   const float* sin;
   int n_pos;
   int blocks_per_tensor;
+  int H;              // heads: batch*head bh = b * H + h reaches the maps as (h, b)
 };
 
 template <int D, bool ROPE>
@@ -149,7 +150,8 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
     bar_arrive_expect_tx(&bar[buf], C::kBufBytes);
 #pragma unroll
     for (int bx = 0; bx < C::kBoxes; ++bx)
-      tma_load_3d(smem + buf * C::kBufBytes + bx * 16384, tm, &bar[buf], bx * 64, blk * 128, bh);
+      tma_load_4d(smem + buf * C::kBufBytes + bx * 16384, tm, &bar[buf], bx * 64, blk * 128, bh % job.H,
+                  bh / job.H);
   };
 
   // two blocks in flight: block i of this CTA goes to buffer i % 2, and the load of block i + 2
@@ -408,9 +410,9 @@ cudaError_t setup_hadamard_quant_kernels() {
 }
 
 cudaError_t launch_hadamard_quant(const CUtensorMap* tm, int ntensors, uint8_t* const* x8, float* const* scales,
-                                  const float* post, const int* transform, const signed char* signs, int BH, int N,
-                                  int d, const int* rope, const float* cos, const float* sin, int n_pos, int num_sms,
-                                  int* status, cudaStream_t stream) {
+                                  const float* post, const int* transform, const signed char* signs, int BH, int H,
+                                  int N, int d, const int* rope, const float* cos, const float* sin, int n_pos,
+                                  int num_sms, int* status, cudaStream_t stream) {
   if (ntensors < 1 || ntensors > 3) return cudaErrorInvalidValue;
   const bool with_rope = rope != nullptr;
   if (with_rope && (cos == nullptr || sin == nullptr)) return cudaErrorInvalidValue;
@@ -425,6 +427,7 @@ cudaError_t launch_hadamard_quant(const CUtensorMap* tm, int ntensors, uint8_t* 
   }
   job.cos = cos;
   job.sin = sin;
+  job.H = H;
   job.n_pos = n_pos;
   switch (d) {
     case 64:

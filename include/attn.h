@@ -181,6 +181,25 @@ int attn_hadamard_quant_qkv(const void* q, const void* k, const void* v, void* q
                             int B, int H, int N, int d, void* stream);
 
 /*
+ * attn_hadamard_quant_qkv_strided -- attn_hadamard_quant_qkv reading Q, K and V laid out with
+ * arbitrary strides (e.g. the head views of one fused [B, N, 3, H, d] projection), without a
+ * transpose copy.
+ *
+ *   q, k, v     logical [B, H, N, d] bf16 tensors, device (read): element (b, h, n, c) of tensor
+ *               t at base_t + b*sb_t + h*sh_t + n*sn_t + c elements (d contiguous).
+ *   strides     HOST pointer to 9 int64 values, read during the call and not kept: {sb, sh, sn}
+ *               for q, then k and v, in elements, with the rules of attn_fwd_strided (positive
+ *               multiples of 8 below 2^36; the stride of an extent-1 dimension is ignored).
+ *   q8, k8, v8, q_scale, k_scale, v_scale   contiguous outputs as for attn_hadamard_quant_qkv.
+ * Each output is bit-identical to attn_hadamard_quant_qkv on contiguous copies of the inputs;
+ * a bad stride returns ATTN_ERR_INVALID_ARG.  Other arguments and errors as there.
+ */
+int attn_hadamard_quant_qkv_strided(const void* q, const void* k, const void* v, void* q8, void* k8,
+                                    void* v8, float* q_scale, float* k_scale, float* v_scale,
+                                    const signed char* signs, int B, int H, int N, int d,
+                                    const long long* strides, void* stream);
+
+/*
  * attn_rope_hadamard_quant_qkv -- attn_hadamard_quant_qkv with the rotary position embedding of
  * Q and K fused in front of the transform ("FlashAttention-3", section "为什么 Hadamard 适合放到
  * 内核里": the transform fuses with RoPE, another bandwidth-bound step; the pages do not define
@@ -234,6 +253,26 @@ int attn_fwd_fp8_qk(const void* q8, const void* k8, const void* v8,
                     const float* q_scale, const float* k_scale, const float* v_scale,
                     void* o, float* lse, int B, int H, int Nq, int Nk, int d, float scale,
                     int causal, int o_dtype, void* stream);
+
+/*
+ * attn_fwd_fp8_strided -- attn_fwd_fp8_qk on E4M3 inputs and an output laid out with arbitrary
+ * strides (e.g. O written straight into a sequence-major [B, Nq, H, d] buffer).
+ *
+ *   q8, k8, v8, o   logical [B, H, N, d] tensors (N = Nq for q8 and o, Nk for k8 and v8):
+ *                   element (b, h, n, c) at base + b*sb + h*sh + n*sn + c elements.
+ *   strides     HOST pointer to 12 int64 values, read during the call and not kept: {sb, sh, sn}
+ *               for q8, k8, v8 and o, in elements, below 2^36; those of q8, k8, v8 positive
+ *               multiples of 16, those of o positive multiples of 8 (16-byte rows for the
+ *               tensor-memory-access unit); the stride of an extent-1 dimension is ignored.
+ *               o must not overlap the inputs.
+ *   q_scale, k_scale, v_scale, lse   contiguous, as for attn_fwd_fp8_qk.
+ * Results are bit-identical to attn_fwd_fp8_qk on contiguous copies; a bad stride returns
+ * ATTN_ERR_INVALID_ARG.  Other arguments, arithmetic and errors as for attn_fwd_fp8_qk.
+ */
+int attn_fwd_fp8_strided(const void* q8, const void* k8, const void* v8,
+                         const float* q_scale, const float* k_scale, const float* v_scale,
+                         void* o, float* lse, int B, int H, int Nq, int Nk, int d,
+                         const long long* strides, float scale, int causal, int o_dtype, void* stream);
 
 /*
  * attn_bwd_workspace_bytes -- size of the float32 workspace attn_bwd needs:

@@ -35,7 +35,8 @@ def test_header_declares_the_boundary():
                             "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv", "attn_bwd_strided",
                             "attn_bwd_varlen", "attn_fwd_fp8_qk", "attn_merge_partials",
                             "attn_selftest_wait_timeout", "attn_noalloc_status",
-                            "attn_noalloc_selftest_wait_timeout"])
+                            "attn_noalloc_selftest_wait_timeout", "attn_hadamard_quant_qkv_strided",
+                            "attn_fwd_fp8_strided"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -297,6 +298,63 @@ def test_fwd_fp8_qk_rejects_bad_arguments(L):
     assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
 
 
+def test_hadamard_quant_qkv_strided_rejects_bad_arguments(L):
+    f = L.attn_hadamard_quant_qkv_strided
+    B, H, N, d = 2, 4, 300, 128
+    # the head views of one fused [B, N, 3, H, d] projection
+    good = [N * 3 * H * d, d, 3 * H * d] * 3
+    ok = [P, P, P, P2, P2, P2, P2, P2, P2, P, B, H, N, d, _strides(good), NULL]
+    a = list(ok)
+    a[14] = NULL
+    assert f(*a) == ea.ATTN_ERR_INVALID_ARG
+    for i in range(10):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for pos, val in [(0, 0), (1, 4), (2, -8), (5, 12), (8, 1 << 36)]:
+        bad = list(good)
+        bad[pos] = val
+        a = list(ok)
+        a[14] = _strides(bad)
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (pos, val)
+    for idx, val in [(10, 0), (11, 0), (12, 0)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+    a = list(ok)
+    a[13] = 32
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+
+
+def test_fwd_fp8_strided_rejects_bad_arguments(L):
+    f = L.attn_fwd_fp8_strided
+    B, H, Nq, Nk, d = 2, 4, 128, 300, 128
+    # contiguous codes, O sequence-major [B, Nq, H, d]
+    good = [H * Nq * d, Nq * d, d, H * Nk * d, Nk * d, d, H * Nk * d, Nk * d, d, Nq * H * d, d, H * d]
+    ok = [P, P, P, P2, P2, P2, P2, NULL, B, H, Nq, Nk, d, _strides(good), 0.1, 1, 0, NULL]
+    a = list(ok)
+    a[13] = NULL
+    assert f(*a) == ea.ATTN_ERR_INVALID_ARG
+    for i in range(7):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    # code strides must be multiples of 16 elements (16 bytes), O strides multiples of 8
+    for pos, val in [(0, 8), (2, 8), (4, 24), (8, 0), (9, 4), (11, -8), (10, 1 << 36)]:
+        bad = list(good)
+        bad[pos] = val
+        a = list(ok)
+        a[13] = _strides(bad)
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (pos, val)
+    for idx, val in [(8, 0), (10, 0), (11, 0), (14, 0.0), (15, 2), (16, 7)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+    a = list(ok)
+    a[12] = 64
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+
+
 def test_merge_partials_rejects_bad_arguments(L):
     f = L.attn_merge_partials
     ok = [P, P, P2, P2, 1000, 128, 0, NULL]
@@ -376,5 +434,5 @@ def test_python_binding_has_same_names():
                  "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided",
                  "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv", "attn_bwd_strided", "attn_bwd_varlen",
                  "attn_fwd_fp8_qk", "attn_merge_partials", "attn_selftest_wait_timeout", "attn_noalloc_status",
-                 "attn_noalloc_selftest_wait_timeout"]:
+                 "attn_noalloc_selftest_wait_timeout", "attn_hadamard_quant_qkv_strided", "attn_fwd_fp8_strided"]:
         assert callable(getattr(ea, name)), name

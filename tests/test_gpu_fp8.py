@@ -130,3 +130,41 @@ def test_fp8_qk_equal_lengths_is_attn_fwd_fp8():
     b = ea.attn_fwd_fp8_qk(q8, k8, v8, qs, ks, vs, causal=True)
     torch.cuda.synchronize()
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,H,nq,nk,d", [(2, 3, 300, 513, 128), (1, 2, 257, 257, 256), (1, 1, 1, 130, 128)])
+def test_fp8_strided_sequence_major_matches_contiguous(B, H, nq, nk, d, causal):
+    """attn_fwd_fp8_strided on E4M3 codes held as head views of padded sequence-major buffers,
+    writing O into a padded sequence-major [B, Nq, H, d] buffer: O and LSE are bit-identical to
+    attn_fwd_fp8_qk on the contiguous codes, the padding is untouched, and O is within the E4M3
+    bounds of the oracle on the dequantised inputs."""
+    q, _, _ = normal_qkv(B, H, nq, d, seed=nq + d, outlier_frac=1e-3)
+    _, k, v = normal_qkv(B, H, nk, d, seed=nk + 3 * d, outlier_frac=1e-3)
+    q8, qs, k8, ks, v8, vs = _quantise(q, k, v, hadamard_signs(d))
+    ref_o, ref_lse = ea.attn_fwd_fp8_qk(q8, k8, v8, qs, ks, vs, causal=causal, o_dtype=torch.float32)
+
+    def seq_major(x8):
+        b, h, n, dd = x8.shape
+        buf = torch.zeros((b, n, h, dd + 16), dtype=torch.uint8, device="cuda")
+        view = buf[..., :dd].transpose(1, 2)
+        view.copy_(x8)
+        return view
+
+    o_buf = torch.full((B, nq, H, d + 8), float("nan"), dtype=torch.float32, device="cuda")
+    o_view = o_buf[..., :d].transpose(1, 2)
+    o, lse = ea.attn_fwd_fp8_strided(seq_major(q8), seq_major(k8), seq_major(v8), qs, ks, vs, o=o_view,
+                                     causal=causal)
+    torch.cuda.synchronize()
+    assert torch.equal(o.contiguous(), ref_o) and torch.equal(lse, ref_lse)
+    # the padding columns of the output buffer are not written
+    assert torch.isnan(o_buf[..., d:]).all()
+    qd = dequant_ref(q8.cpu().numpy(), qs.cpu().numpy())
+    kd = dequant_ref(k8.cpu().numpy(), ks.cpu().numpy())
+    vd = dequant_ref(v8.cpu().numpy(), vs.cpu().numpy())
+    o_ref, lse_ref = attention_ref(qd, kd, vd, 1 / math.sqrt(d), causal)
+    og = o.cpu().numpy().astype(np.float64)
+    seen = np.isfinite(lse_ref)
+    err = og[seen] - o_ref[seen]
+    assert float(np.sqrt(np.mean(err ** 2))) <= 1e-2
+    assert np.abs(err).max() <= (2.0 ** -4 + 1e-2) * np.abs(vd).max()

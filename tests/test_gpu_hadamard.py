@@ -75,3 +75,30 @@ def test_qkv_launch_matches_oracle(d, n):
         rc, rs = hadamard_quant_ref(x, s)
         np.testing.assert_array_equal(sc.cpu().numpy(), rs)
         np.testing.assert_array_equal(c8.cpu().numpy(), rc)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("B,H,n", [(2, 3, 300), (1, 1, 1), (1, 4, 1024)])
+def test_strided_qkv_launch_on_a_fused_projection(d, B, H, n):
+    """attn_hadamard_quant_qkv_strided on the head views of one fused [B, N, 3, H, d] buffer with
+    a padded row (8 spare elements): the codes and scales are the oracle's and bit-identical to
+    attn_hadamard_quant_qkv on contiguous copies."""
+    q, k, v = normal_qkv(B, H, n, d, seed=n + 11 * d, outlier_frac=1e-3)
+    signs = hadamard_signs(d)
+    s = torch.from_numpy(signs).cuda()
+    fused = torch.zeros((B, n, 3 * H * d + 8), dtype=torch.bfloat16, device="cuda")
+    views = []
+    for j, x in enumerate((q, k, v)):
+        view = fused[:, :, j * H * d:(j + 1) * H * d].view(B, n, H, d).transpose(1, 2)
+        view.copy_(torch.from_numpy(x).to(torch.bfloat16).cuda())
+        views.append(view)
+    assert not views[0].is_contiguous() or (H == 1 and n == 1)
+    outs = ea.attn_hadamard_quant_qkv_strided(*views, s)
+    ref = ea.attn_hadamard_quant_qkv(*[t.contiguous() for t in views], s)
+    torch.cuda.synchronize()
+    for a, b in zip(outs, ref):
+        assert torch.equal(a, b)
+    for x, sg, c8, sc in ((q, signs, outs[0], outs[3]), (k, signs, outs[1], outs[4]), (v, None, outs[2], outs[5])):
+        rc, rs = hadamard_quant_ref(x, sg)
+        np.testing.assert_array_equal(sc.cpu().numpy(), rs)
+        np.testing.assert_array_equal(c8.cpu().numpy(), rc)
