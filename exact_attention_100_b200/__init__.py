@@ -95,6 +95,8 @@ def lib() -> ctypes.CDLL:
         L.attn_noalloc_status.restype = i
         L.attn_noalloc_selftest_wait_timeout.argtypes = [vp]
         L.attn_noalloc_selftest_wait_timeout.restype = i
+        L.attn_fwd_schedule.argtypes = [i, i, i, i, i, i, i, i, vp, ctypes.c_longlong, vp]
+        L.attn_fwd_schedule.restype = i
         L.attn_bwd_workspace_bytes.argtypes = [i, i, i]
         L.attn_bwd_workspace_bytes.restype = ctypes.c_ulonglong
         L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
@@ -568,6 +570,31 @@ def attn_fwd_fp8_strided(q8, k8, v8, q_scale, k_scale, v_scale, o=None, lse=None
                                       _ptr(o), _ptr(lse), B, H, Nq, Nk, d, ctypes.cast(strides, ctypes.c_void_p), s,
                                       int(bool(causal)), od, _stream_ptr(stream)), "attn_fwd_fp8_strided")
     return o, lse
+
+
+def attn_fwd_schedule(B, H, Nq, Nk, d, causal=False, fp8=False, num_ctas=148):
+    """The forward kernels' work lists for a fixed-length launch (host only, no CUDA call).
+
+    Returns ``None`` if the launch keeps the kernels' round-robin order, else a list with, for
+    each CTA, the unit ids it computes in order (unit u: batch*head ``u % (B*H)``, round
+    ``u // (B*H)``, see ``attn_fwd_schedule`` in ``include/attn.h``)."""
+    need = ctypes.c_longlong(0)
+    dt = ATTN_E4M3 if fp8 else ATTN_BF16
+    _check(lib().attn_fwd_schedule(B, H, Nq, Nk, d, int(bool(causal)), dt, num_ctas, None, 0, ctypes.byref(need)),
+           "attn_fwd_schedule")
+    if need.value == 0:
+        return None
+    buf = (ctypes.c_int * need.value)()
+    _check(lib().attn_fwd_schedule(B, H, Nq, Nk, d, int(bool(causal)), dt, num_ctas, ctypes.cast(buf, ctypes.c_void_p),
+                                   need.value, ctypes.byref(need)), "attn_fwd_schedule")
+    t = list(buf)
+    grid = len(t) - 1 - _units(B, H, Nq, d)  # the table is [grid + 1 offsets][units]
+    return [t[grid + 1 + t[b]: grid + 1 + t[b + 1]] for b in range(grid)]
+
+
+def _units(B, H, Nq, d):
+    tiles = 1 if d == 256 else 2
+    return B * H * (((Nq + 127) // 128 + tiles - 1) // tiles)
 
 
 def attn_merge_partials(o_acc, lse_acc, o_part, lse_part, stream=None):

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <vector>
 
 #include "../../include/attn.h"
 #include "attn_kernels.h"
@@ -155,6 +156,7 @@ void fill_params(ea::FwdParams& p, void* o, float* lse, int* status, int B, int 
   p.cu_q = p.cu_k = nullptr;
   p.total_q = p.total_k = 0;
   p.vl_sched = 0;
+  p.unit_tab = nullptr;
   p.N = N;
   p.BH = B * H;
   p.H = H;
@@ -251,6 +253,8 @@ int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.o_sb = so.sb;
   p.o_sh = so.sh;
   p.o_sn = so.sn;
+  p.unit_tab = ea::fwd_unit_table(p, ea::fwd_units_per_tile_pair(d), d, 2, ea::fwd_grid(p, st->num_sms),
+                                  static_cast<cudaStream_t>(stream));
   if (ea::launch_attn_fwd_bf16(d, mq, mk, mv, mo, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
@@ -467,6 +471,8 @@ int fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.v_scale = v_scale;
+  p.unit_tab = ea::fwd_unit_table(p, ea::fwd_units_per_tile_pair(d), d, 1, ea::fwd_grid(p, st->num_sms),
+                                  static_cast<cudaStream_t>(stream));
   if (ea::launch_attn_fwd_fp8(d, mq, mk, mv, mo, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(1);
@@ -502,6 +508,26 @@ int attn_fwd_fp8_strided(const void* q8, const void* k8, const void* v8, const f
       return ATTN_ERR_INVALID_ARG;
   return fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, Nq, Nk, d, st4, scale, causal, o_dtype,
                  stream);
+}
+
+int attn_fwd_schedule(int B, int H, int Nq, int Nk, int d, int causal, int dtype, int num_ctas, int* out,
+                      long long cap, long long* needed) {
+  if (needed == nullptr || cap < 0 || (cap > 0 && out == nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || num_ctas <= 0 || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 0x7FFFFFFFLL || !units_fit(B, H, Nq)) return ATTN_ERR_INVALID_ARG;
+  if (dtype != ATTN_BF16 && dtype != ATTN_E4M3) return dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  if (dtype == ATTN_E4M3 && d == 64) return ATTN_ERR_UNSUPPORTED;
+  const int tiles = ea::fwd_units_per_tile_pair(d);
+  ea::FwdParams p;
+  fill_params(p, nullptr, nullptr, nullptr, B, H, Nq, Nk, tiles, 1.0f, causal, ATTN_BF16);
+  std::vector<int> t;
+  *needed = 0;
+  if (!ea::fwd_unit_schedule(p, tiles, d, dtype == ATTN_E4M3 ? 1 : 2, ea::fwd_grid(p, num_ctas), &t)) return ATTN_OK;
+  *needed = static_cast<long long>(t.size());
+  if (static_cast<long long>(t.size()) <= cap)
+    for (size_t i = 0; i < t.size(); ++i) out[i] = t[i];
+  return ATTN_OK;
 }
 
 unsigned long long attn_bwd_workspace_bytes(int B, int H, int N) {
@@ -673,6 +699,7 @@ void attn_shutdown(void) {
     st = DeviceState{};
   }
   if (have_dev) cudaSetDevice(cur);
+  ea::free_unit_tables();
 }
 
 }  // extern "C"

@@ -235,8 +235,14 @@ __device__ __forceinline__ Unit decode_unit(int u, const FwdParams& p, const int
   return U;
 }
 
-// k-th unit of this CTA: round-robin over CTAs, alternating direction every round.
-__device__ __forceinline__ int unit_index(int k) {
+// k-th unit of this CTA: from the host's work lists (tab: [gridDim.x + 1] offsets, then unit
+// ids), or else round-robin over CTAs, alternating direction every round.  Past the end of its
+// list a CTA gets a value >= num_units.
+__device__ __forceinline__ int unit_index(int k, const int* tab) {
+  if (tab != nullptr) {
+    const int i = __ldg(tab + blockIdx.x) + k;
+    return i < __ldg(tab + blockIdx.x + 1) ? __ldg(tab + gridDim.x + 1 + i) : 0x7FFFFFFF;
+  }
   const int g = gridDim.x;
   return k * g + ((k & 1) ? (g - 1 - (int)blockIdx.x) : (int)blockIdx.x);
 }
@@ -509,7 +515,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
     uint32_t uit = 0;  // units this warpgroup's tile took part in
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int u = unit_index(k);
+      const int u = unit_index(k, p.unit_tab);
       if (u >= num_units) break;
       const Unit U = decode_unit<NQ, VL>(u, p, sched);
       const Seq& S = U.s;
@@ -890,7 +896,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         int k2 = k + 1;
         Unit U2;
         for (;; ++k2) {
-          const int u2 = unit_index(k2);
+          const int u2 = unit_index(k2, p.unit_tab);
           if (u2 >= num_units) return false;
           U2 = decode_unit<NQ, VL>(u2, p, sched);
           if constexpr (VL) {
@@ -914,7 +920,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         return true;
       };
       for (int k = 0; ok; ++k) {
-        const int u = unit_index(k);
+        const int u = unit_index(k, p.unit_tab);
         if (u >= num_units) break;
         const Unit U = decode_unit<NQ, VL>(u, p, sched);
         if constexpr (VL) {
@@ -1002,7 +1008,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       uint32_t it = 0, qit = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int u = unit_index(k);
+        const int u = unit_index(k, p.unit_tab);
         if (u >= num_units) break;
         const Unit U = decode_unit<NQ, VL>(u, p, sched);
         const Seq& S = U.s;
@@ -1078,7 +1084,7 @@ template <int D, int NQ, class E, bool VL = false>
 cudaError_t launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& o,
                        const FwdParams& p, int num_sms, cudaStream_t stream) {
   using C = FwdCfg<D, NQ, E>;
-  const int grid = p.num_units < num_sms ? p.num_units : num_sms;
+  const int grid = fwd_grid(p, num_sms);
   attn_fwd_kernel<D, NQ, E, VL><<<grid, C::kThreads, C::kSmemAlloc, stream>>>(q, k, v, o, p);
   return cudaGetLastError();
 }

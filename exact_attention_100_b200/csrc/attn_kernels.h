@@ -4,6 +4,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <vector>
+
 namespace ea {
 
 // Device status word bits (OR-ed into the library's per-device status word).
@@ -44,7 +46,25 @@ struct FwdParams {
   // packed batches with B <= 1024 and n_pairs <= 1023: every CTA sorts the sequences by their
   // number of tile pairs and deals out only the units that exist, longest first
   int vl_sched;
+  // fixed-length batches: per-CTA work lists from fwd_unit_schedule in device memory, or
+  // nullptr for the kernel's round-robin order
+  const int* unit_tab;
 };
+
+// CTAs of a persistent forward launch: one per SM, or one per unit if there are fewer.
+int fwd_grid(const FwdParams& p, int num_sms);
+
+// Work lists of the forward kernels for the fixed-length launch p on `grid` CTAs, nq Q tiles per
+// unit, head dim d, elem_bytes per K/V element: out = [grid + 1 list offsets][num_units unit
+// ids]; CTA b computes the units out[grid + 1 + i], i in [out[b], out[b + 1]), in that order.
+// Returns false (out untouched) for launches left to the round-robin order (packed batches,
+// more than 2^20 units).
+bool fwd_unit_schedule(const FwdParams& p, int nq, int d, int elem_bytes, int grid, std::vector<int>* out);
+
+// The table of fwd_unit_schedule in device memory on the current device, built on the first
+// launch of a shape and cached until free_unit_tables (nullptr: round-robin order).
+const int* fwd_unit_table(const FwdParams& p, int nq, int d, int elem_bytes, int grid, cudaStream_t stream);
+void free_unit_tables();
 
 // Q tiles of 128 rows handled together by one unit of the bf16 kernel for head dim d.
 int fwd_units_per_tile_pair(int d);

@@ -162,6 +162,7 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
   p.cu_q = p.cu_k = nullptr;
   p.total_q = p.total_k = 0;
   p.vl_sched = 0;
+  p.unit_tab = nullptr;  // the round-robin order: a table would need device memory
   p.N = N;
   p.BH = B * H;
   p.H = H;

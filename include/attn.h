@@ -24,8 +24,9 @@
  *     enqueued asynchronously; the call returns once it is enqueued.
  *   - Arguments are checked before any CUDA call; a bad argument returns an error status and
  *     enqueues nothing.  No entry point allocates memory per call.  The library keeps one small
- *     per-device workspace (a device status word), created on first use and released by
- *     attn_shutdown().
+ *     per-device workspace (a device status word), created on first use, and the forward's
+ *     per-shape work lists (attn_fwd_schedule), created on the first launch of a shape; both
+ *     are released by attn_shutdown().
  *   - Calls on the same device may come from several host threads; the library's per-device
  *     set-up is guarded by a mutex.
  *   - Errors of the device-side work itself (a bounded wait inside a kernel that ran out) are
@@ -273,6 +274,35 @@ int attn_fwd_fp8_strided(const void* q8, const void* k8, const void* v8,
                          const float* q_scale, const float* k_scale, const float* v_scale,
                          void* o, float* lse, int B, int H, int Nq, int Nk, int d,
                          const long long* strides, float scale, int causal, int o_dtype, void* stream);
+
+/*
+ * attn_fwd_schedule -- the work lists the persistent forward kernels follow for a fixed-length
+ * launch (introspection: every forward entry point builds them itself).  Host only: no CUDA
+ * call is made.
+ *
+ * A unit is one (batch*head, group of Q tiles): unit u covers bh = u % (B*H) and the Q tiles
+ * [t0, t0 + T) with T = 2 (d = 64, 128) or 1 (d = 256), r = u / (B*H), and t0 = T * r, or
+ * T * (n_pairs - 1 - r) when causal (n_pairs = ceil(ceil(Nq / 128) / T)).  The units are
+ * ordered longest first within groups of heads (the K and V of a group fit a 64 MB share of the
+ * 126 MB L2, unless that leaves fewer than two units per CTA in a group) and dealt by greedy list
+ * scheduling under a cost of K/V blocks per unit ("FlashAttention-2/3", FA-2 improvement 3:
+ * parallelism over the sequence; longest first balances causal units of unequal length).
+ *
+ *   B, H, Nq, Nk, d, causal   the launch, as for attn_fwd_qk.
+ *   dtype       ATTN_BF16 (attn_fwd*) or ATTN_E4M3 (attn_fwd_fp8*: K/V elements of one byte).
+ *   num_ctas    the persistent grid: the device's SM count (fewer if there are fewer units).
+ *   out, cap    host int32 array of cap entries, written if cap >= *needed: [num_ctas + 1]
+ *               list offsets, then the unit ids; CTA b computes out[num_ctas + 1 + i] for i in
+ *               [out[b], out[b + 1]), in that order.
+ *   needed      host: entries of the table, or 0 if the launch keeps the kernels' round-robin
+ *               order (more than 2^20 units; packed batches always do).
+ * Returns ATTN_OK, ATTN_ERR_INVALID_ARG or ATTN_ERR_UNSUPPORTED as the forward call would.
+ * The tables are built on the first launch of a shape (one allocation and one synchronous copy)
+ * and kept until attn_shutdown; a launch inside a stream capture of a shape not seen before,
+ * and attn_fwd_noalloc, use the round-robin order, with identical results.
+ */
+int attn_fwd_schedule(int B, int H, int Nq, int Nk, int d, int causal, int dtype, int num_ctas,
+                      int* out, long long cap, long long* needed);
 
 /*
  * attn_bwd_workspace_bytes -- size of the float32 workspace attn_bwd needs:

@@ -36,7 +36,7 @@ def test_header_declares_the_boundary():
                             "attn_bwd_varlen", "attn_fwd_fp8_qk", "attn_merge_partials",
                             "attn_selftest_wait_timeout", "attn_noalloc_status",
                             "attn_noalloc_selftest_wait_timeout", "attn_hadamard_quant_qkv_strided",
-                            "attn_fwd_fp8_strided"])
+                            "attn_fwd_fp8_strided", "attn_fwd_schedule"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -434,5 +434,6 @@ def test_python_binding_has_same_names():
                  "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_qk", "attn_bwd_qk", "attn_fwd_strided",
                  "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv", "attn_bwd_strided", "attn_bwd_varlen",
                  "attn_fwd_fp8_qk", "attn_merge_partials", "attn_selftest_wait_timeout", "attn_noalloc_status",
-                 "attn_noalloc_selftest_wait_timeout", "attn_hadamard_quant_qkv_strided", "attn_fwd_fp8_strided"]:
+                 "attn_noalloc_selftest_wait_timeout", "attn_hadamard_quant_qkv_strided", "attn_fwd_fp8_strided",
+                 "attn_fwd_schedule"]:
         assert callable(getattr(ea, name)), name

@@ -60,6 +60,24 @@ def test_noalloc_matches_oracle_and_attn_fwd_on_two_calls(B, H, N, d, causal, o_
         assert ((lse - lse_ref).abs() / lse_ref.abs()).max().item() <= LSE_REL, call
 
 
+@pytest.mark.parametrize("B,H,N,d", [(2, 16, 8192, 128), (1, 32, 4096, 64), (2, 4, 2000, 256)])
+def test_work_lists_do_not_change_results(B, H, N, d):
+    """attn_fwd follows the host-built work lists (attn_fwd_schedule), attn_fwd_noalloc the
+    round-robin order: every unit is computed the same way whichever CTA takes it, so O and LSE
+    are bit-identical (causal, where the two orders differ most)."""
+    ea_build.build()
+    assert ea.attn_fwd_schedule(B, H, N, N, d, causal=True) is not None
+    g = torch.Generator(device="cuda").manual_seed(N + d)
+    q, k, v = (torch.randn(B, H, N, d, device="cuda", generator=g).to(torch.bfloat16) for _ in range(3))
+    o_ref, lse_ref = ea.attn_fwd(q, k, v, causal=True)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    assert _call_noalloc(q, k, v, o, lse, True) == ea.ATTN_OK
+    torch.cuda.synchronize()
+    assert ea.attn_noalloc_status() == ea.ATTN_OK and ea.attn_device_status() == ea.ATTN_OK
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+
+
 def test_noalloc_status_reports_a_timeout_once():
     """A bounded wait that runs out, recorded in the static status word (the self-test kernel
     waits on a barrier that nothing arrives at, for 2 s), is reported by attn_noalloc_status,
