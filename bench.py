@@ -744,6 +744,28 @@ def varlen_section(args, dev, rank):
     assert ea.attn_device_status() == ea.ATTN_OK
     bms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
     btf = 2.5 * flops / (bms * 1e-3) / 1e12
+    # the E4M3 forward of the same packed batch: codes and per-sequence block scales from the
+    # packed pre-kernel (Q, K through H D), then attn_fwd_fp8_varlen
+    from exact_attention_100_b200.inputs import hadamard_signs
+    signs = torch.from_numpy(hadamard_signs(d)).to(dev)
+    q8s = ea.attn_hadamard_quant_qkv_varlen(q, k, v, signs, cu_q, cu_k, max(lens), max(lens))
+    o8 = torch.empty_like(q)
+
+    def fstep():
+        ea.attn_fwd_fp8_varlen(*q8s, cu_q, cu_k, max(lens), max(lens), o=o8, lse=lse, causal=causal, stream=stream)
+
+    for _ in range(3):
+        fstep()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        fstep()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+    fms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    ftf = flops / (fms * 1e-3) / 1e12
     return {"workload": f"bf16 packed varlen fwd, {len(lens)} sequences of {w['lo']}..{w['hi']} tokens "
                         f"(total {w['total']}), H={H} d={d} causal",
             "lengths": lens, "ms": ms, "achieved_tflops": tf, "peak_tflops": float(peaks["bf16_tflops"]),
@@ -751,7 +773,11 @@ def varlen_section(args, dev, rank):
             "flops_note": "sum over sequences of 4 H d N^2 / 2 (causal), as the headline counts",
             "peak_source": peaks["source"],
             "bwd": {"ms": bms, "achieved_tflops": btf, "frac": btf / float(peaks["bf16_tflops"]),
-                    "flops_note": "2.5 x the forward count (five products), bf16 gradients, 3 launches"}}
+                    "flops_note": "2.5 x the forward count (five products), bf16 gradients, 3 launches"},
+            "fp8_fwd": {"ms": fms, "achieved_tflops": ftf, "vs_bf16": ms / fms,
+                        "note": "attn_fwd_fp8_varlen on the same batch (E4M3 codes and per-sequence "
+                                "128-row block scales from attn_hadamard_quant_qkv_varlen; the "
+                                "pre-kernel is not in the timed region), bf16 O"}}
 
 
 def bwd_section(args, dev, rank):

@@ -85,6 +85,10 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_fp8_qk.restype = i
         L.attn_fwd_fp8_strided.argtypes = [vp] * 8 + [i, i, i, i, i, vp, f, i, i, vp]
         L.attn_fwd_fp8_strided.restype = i
+        L.attn_hadamard_quant_qkv_varlen.argtypes = [vp] * 12 + [i] * 7 + [vp, vp]
+        L.attn_hadamard_quant_qkv_varlen.restype = i
+        L.attn_fwd_fp8_varlen.argtypes = [vp] * 10 + [i] * 7 + [f, i, i, vp]
+        L.attn_fwd_fp8_varlen.restype = i
         L.attn_merge_partials.argtypes = [vp, vp, vp, vp, ctypes.c_longlong, i, i, vp]
         L.attn_merge_partials.restype = i
         L.attn_selftest_wait_timeout.argtypes = [vp]
@@ -595,6 +599,79 @@ def attn_fwd_schedule(B, H, Nq, Nk, d, causal=False, fp8=False, num_ctas=148):
 def _units(B, H, Nq, d):
     tiles = 1 if d == 256 else 2
     return B * H * (((Nq + 127) // 128 + tiles - 1) // tiles)
+
+
+def _check_cu(cu_seqlens_q, cu_seqlens_k):
+    import torch
+    for c in (cu_seqlens_q, cu_seqlens_k):
+        if c.dtype != torch.int32 or c.dim() != 1 or not c.is_contiguous() or not c.is_cuda:
+            raise ValueError("cu_seqlens must be contiguous int32 cuda tensors")
+    if cu_seqlens_k.shape != cu_seqlens_q.shape:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B + 1 entries")
+    return int(cu_seqlens_q.shape[0]) - 1
+
+
+def attn_hadamard_quant_qkv_varlen(q, k, v, signs, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                                   outs=None, stream=None):
+    """Packed batch: ``q`` [total_q, H, d], ``k``, ``v`` [total_k, H, d] bf16 (row and head strides
+    free, last dimension contiguous) quantised per 128-row block of each sequence.  Returns
+    ``(q8, k8, v8, q_scale, k_scale, v_scale)``: codes [total, H, d] uint8 and scales
+    [B, H, ceil(max_seqlen / 128)] float32."""
+    import torch
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape:
+        raise ValueError("q must be [total_q, H, d], k and v [total_k, H, d]")
+    total_q, H, d = (int(x) for x in q.shape)
+    total_k = int(k.shape[0])
+    if (int(k.shape[1]), int(k.shape[2])) != (H, d):
+        raise ValueError("k and v must have q's H and d")
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or t.stride(-1) != 1:
+            raise ValueError("q, k, v must be bf16 with a contiguous last dimension")
+    B = _check_cu(cu_seqlens_q, cu_seqlens_k)
+    nbq, nbk = (int(max_seqlen_q) + 127) // 128, (int(max_seqlen_k) + 127) // 128
+    if outs is None:
+        dev = q.device
+        outs = (torch.empty((total_q, H, d), dtype=torch.uint8, device=dev),
+                torch.empty((total_k, H, d), dtype=torch.uint8, device=dev),
+                torch.empty((total_k, H, d), dtype=torch.uint8, device=dev),
+                torch.empty((B, H, nbq), dtype=torch.float32, device=dev),
+                torch.empty((B, H, nbk), dtype=torch.float32, device=dev),
+                torch.empty((B, H, nbk), dtype=torch.float32, device=dev))
+    q8, k8, v8, qs, ks, vs = outs
+    strides = (ctypes.c_longlong * 6)(*[int(x) for t in (q, k, v) for x in t.stride()[:2]])
+    _check(lib().attn_hadamard_quant_qkv_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs),
+                                                _ptr(ks), _ptr(vs), _ptr(signs), _ptr(cu_seqlens_q),
+                                                _ptr(cu_seqlens_k), B, H, total_q, total_k, int(max_seqlen_q),
+                                                int(max_seqlen_k), d, ctypes.cast(strides, ctypes.c_void_p),
+                                                _stream_ptr(stream)), "attn_hadamard_quant_qkv_varlen")
+    return outs
+
+
+def attn_fwd_fp8_varlen(q8, k8, v8, q_scale, k_scale, v_scale, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                        max_seqlen_k, o=None, lse=None, scale=None, causal=False, o_dtype=None, stream=None):
+    """The E4M3 forward over a packed batch (codes and scales from
+    :func:`attn_hadamard_quant_qkv_varlen`, with the same offsets and longest lengths).
+    Returns ``(o [total_q, H, d], lse [H, total_q])``."""
+    import torch
+    total_q, H, d = (int(x) for x in q8.shape)
+    total_k = int(k8.shape[0])
+    for t in (q8, k8, v8):
+        if t.dtype != torch.uint8 or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError("q8, k8, v8 must be contiguous uint8 [total, H, d]")
+    B = _check_cu(cu_seqlens_q, cu_seqlens_k)
+    if o is None:
+        o = torch.empty((total_q, H, d), dtype=o_dtype or torch.bfloat16, device=q8.device)
+    if tuple(o.shape) != (total_q, H, d) or not o.is_contiguous():
+        raise ValueError("o must be a contiguous [total_q, H, d] tensor")
+    if lse is None:
+        lse = torch.empty((H, total_q), dtype=torch.float32, device=q8.device)
+    od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_fwd_fp8_varlen(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
+                                     _ptr(o), _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, H, total_q,
+                                     total_k, int(max_seqlen_q), int(max_seqlen_k), d, s, int(bool(causal)), od,
+                                     _stream_ptr(stream)), "attn_fwd_fp8_varlen")
+    return o, lse
 
 
 def attn_merge_partials(o_acc, lse_acc, o_part, lse_part, stream=None):

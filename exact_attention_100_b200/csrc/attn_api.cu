@@ -157,6 +157,7 @@ void fill_params(ea::FwdParams& p, void* o, float* lse, int* status, int B, int 
   p.total_q = p.total_k = 0;
   p.vl_sched = 0;
   p.unit_tab = nullptr;
+  p.max_nk = Nk;
   p.N = N;
   p.BH = B * H;
   p.H = H;
@@ -166,6 +167,7 @@ void fill_params(ea::FwdParams& p, void* o, float* lse, int* status, int B, int 
   p.n_blocks = (N + 127) / 128;
   p.Nk = Nk;
   p.nbk = (Nk + 127) / 128;
+  p.kv_sstride = p.nbk;
   p.off = Nk - N;
   p.n_pairs = (p.n_blocks + q_tiles - 1) / q_tiles;
   p.num_units = p.BH * p.n_pairs;
@@ -427,6 +429,55 @@ int attn_hadamard_quant_qkv_strided(const void* q, const void* k, const void* v,
   return hq_qkv(q, k, v, q8, k8, v8, q_scale, k_scale, v_scale, signs, nullptr, nullptr, 0, B, H, N, d, st3, stream);
 }
 
+int attn_hadamard_quant_qkv_varlen(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8,
+                                   float* q_scale, float* k_scale, float* v_scale, const signed char* signs,
+                                   const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H, int total_q,
+                                   int total_k, int max_seqlen_q, int max_seqlen_k, int d, const long long* strides,
+                                   void* stream) {
+  const void* in[3] = {q, k, v};
+  void* out[3] = {q8, k8, v8};
+  float* sc[3] = {q_scale, k_scale, v_scale};
+  for (int t = 0; t < 3; ++t) {
+    if (!in[t] || !out[t] || !sc[t]) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(in[t]) || !aligned16(out[t]) || !aligned16(sc[t])) return ATTN_ERR_INVALID_ARG;
+  }
+  if (!signs || !aligned16(signs) || !cu_seqlens_q || !cu_seqlens_k || !strides) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || static_cast<long long>(B) * H > 0x7FFFFFFFLL) return ATTN_ERR_INVALID_ARG;
+  constexpr int kMaxRows = 0x7FFFFFFF - (1 << 20);  // row coordinates (offset + 128 * block) stay inside int
+  const int tot[3] = {total_q, total_k, total_k};
+  const int mx[3] = {max_seqlen_q, max_seqlen_k, max_seqlen_k};
+  long long units = 0;
+  Strides st3[3];
+  for (int t = 0; t < 3; ++t) {
+    if (tot[t] <= 0 || tot[t] > kMaxRows || mx[t] <= 0 || mx[t] > kMaxRows) return ATTN_ERR_INVALID_ARG;
+    units += static_cast<long long>(B) * H * ((mx[t] + 127) / 128);
+    const long long s3[3] = {8, strides[2 * t + 1], strides[2 * t]};  // {batch (unused), head, row}
+    if (!canonical_strides(s3, 1, H, tot[t], &st3[t])) return ATTN_ERR_INVALID_ARG;
+  }
+  if (units > 0x7FFFFFFFLL - 65536) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  CUtensorMap maps[3];
+  for (int t = 0; t < 3; ++t)
+    if (!encode_fwd_map(&maps[t], in[t], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, tot[t], H, 1, st3[t].sn, st3[t].sh,
+                        st3[t].sb))
+      return ATTN_ERR_CUDA;
+  const float rsd = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  uint8_t* o8[3] = {static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8), static_cast<uint8_t*>(v8)};
+  const float post[3] = {rsd, rsd, 1.0f};
+  const int transform[3] = {1, 1, 0};
+  const int* cu[3] = {cu_seqlens_q, cu_seqlens_k, cu_seqlens_k};
+  if (ea::launch_hadamard_quant_varlen(maps, 3, o8, sc, post, transform, signs, B, H, cu, tot, mx, d, st->num_sms,
+                                       st->status, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return ATTN_OK;
+}
+
 int attn_rope_hadamard_quant_qkv(const void* q, const void* k, const void* v, void* q8, void* k8, void* v8,
                                  float* q_scale, float* k_scale, float* v_scale, const signed char* signs,
                                  const float* cos, const float* sin, int n_pos, int B, int H, int N, int d,
@@ -508,6 +559,58 @@ int attn_fwd_fp8_strided(const void* q8, const void* k8, const void* v8, const f
       return ATTN_ERR_INVALID_ARG;
   return fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, Nq, Nk, d, st4, scale, causal, o_dtype,
                  stream);
+}
+
+int attn_fwd_fp8_varlen(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
+                        const float* v_scale, void* o, float* lse, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                        int B, int H, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                        float scale, int causal, int o_dtype, void* stream) {
+  if (!q8 || !k8 || !v8 || !q_scale || !k_scale || !v_scale || !o || !cu_seqlens_q || !cu_seqlens_k)
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || (lse && !aligned16(lse)) ||
+      !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(v_scale) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
+    return ATTN_ERR_INVALID_ARG;
+  int rc = check_common(B, H, max_seqlen_q, scale, causal, o_dtype);
+  if (rc != ATTN_OK) return rc;
+  constexpr int kMaxRows = 0x7FFFFFFF - (1 << 20);
+  if (total_q <= 0 || total_k <= 0 || total_q > kMaxRows || total_k > kMaxRows || max_seqlen_q > kMaxRows ||
+      max_seqlen_k <= 0 || max_seqlen_k > kMaxRows)
+    return ATTN_ERR_INVALID_ARG;
+  if (!units_fit(B, H, max_seqlen_q)) return ATTN_ERR_INVALID_ARG;
+  if (d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  // [total, H, d] contiguous: row stride H*d, head stride d
+  const long long sn = static_cast<long long>(H) * d;
+  CUtensorMap mq, mk, mv, mo;
+  if (!encode_fwd_map(&mq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, total_q, H, 1, sn, d, 16) ||
+      !encode_fwd_map(&mk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, total_k, H, 1, sn, d, 16) ||
+      !encode_fwd_map(&mv, v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, total_k, H, 1, sn, d, 16) ||
+      !encode_o_map(&mo, o, o_dtype, d, total_q, H, 1, sn, d, 8))
+    return ATTN_ERR_CUDA;
+  ea::FwdParams p;
+  // sized for B sequences of max_seqlen_q queries each; shorter ones skip the surplus units
+  fill_params(p, o, lse, st->status, B, H, max_seqlen_q, total_k, ea::fwd_units_per_tile_pair(d), scale, causal,
+              o_dtype);
+  p.o_sb = 0;
+  p.o_sh = d;
+  p.o_sn = sn;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  p.vl_sched = (B <= 1024 && p.n_pairs <= 1023) ? 1 : 0;
+  p.kv_sstride = (max_seqlen_k + 127) / 128;
+  p.max_nk = max_seqlen_k;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  if (ea::launch_attn_fwd_fp8(d, mq, mk, mv, mo, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  g_launches.fetch_add(1);
+  return ATTN_OK;
 }
 
 int attn_fwd_schedule(int B, int H, int Nq, int Nk, int d, int causal, int dtype, int num_ctas, int* out,

@@ -161,7 +161,8 @@ __device__ __forceinline__ Seq seq_of(int bh, const FwdParams& p) {
     int k0 = __ldg(p.cu_k + b), k1 = __ldg(p.cu_k + b + 1);
     // p.N is the longest query length the launch was sized for; a sequence that breaks a
     // bound is treated as empty (nothing read or written for it) and reported
-    if (!(0 <= q0 && q0 <= q1 && q1 <= p.total_q && q1 - q0 <= p.N && 0 <= k0 && k0 <= k1 && k1 <= p.total_k)) {
+    if (!(0 <= q0 && q0 <= q1 && q1 <= p.total_q && q1 - q0 <= p.N && 0 <= k0 && k0 <= k1 && k1 <= p.total_k &&
+          k1 - k0 <= p.max_nk)) {
       s.bad = true;
       q0 = q1 = k0 = k1 = 0;
     }
@@ -550,10 +551,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       if constexpr (E::kFp8) {
         // the Q block scale folds into c; P is stored as p * kPScale * s_v(j) / max_j s_v(j)
         c_base *= __ldg(p.q_scale + static_cast<size_t>(U.bh) * nb + U.tile0 + q);
-        ks = p.k_scale + static_cast<size_t>(U.bh) * p.nbk;
-        vs = p.v_scale + static_cast<size_t>(U.bh) * p.nbk;
+        ks = p.k_scale + static_cast<size_t>(U.bh) * p.kv_sstride;
+        vs = p.v_scale + static_cast<size_t>(U.bh) * p.kv_sstride;
         float vmax = 0.f;
-        for (int b = lane; b < p.nbk; b += 32) vmax = fmaxf(vmax, __ldg(vs + b));
+        for (int b = lane; b < S.nbk; b += 32) vmax = fmaxf(vmax, __ldg(vs + b));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
         ps_log2_base = lg2_approx(E::kPScale / vmax);

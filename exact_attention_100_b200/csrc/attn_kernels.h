@@ -49,6 +49,11 @@ struct FwdParams {
   // fixed-length batches: per-CTA work lists from fwd_unit_schedule in device memory, or
   // nullptr for the kernel's round-robin order
   const int* unit_tab;
+  // E4M3: blocks per (batch, head) row of k_scale and v_scale (nbk; for packed batches
+  // ceil(max_nk / 128)); packed batches: the longest key sequence allowed (longer ones are
+  // reported as bad offsets)
+  int kv_sstride;
+  int max_nk;
 };
 
 // CTAs of a persistent forward launch: one per SM, or one per unit if there are fewer.
@@ -136,6 +141,14 @@ cudaError_t launch_hadamard_quant(const CUtensorMap* tm, int ntensors, uint8_t* 
                                   const float* post, const int* transform, const signed char* signs, int BH, int H,
                                   int N, int d, const int* rope, const float* cos, const float* sin, int n_pos,
                                   int num_sms, int* status, cudaStream_t stream);
+
+// The same for packed batches: tensor t is [total[t], H, d] (tm[t] a 4-D map (d, rows, heads, 1)),
+// sequence b owning rows cu[t][b] .. cu[t][b+1]-1 (device offsets), quantised in 128-row blocks
+// of each sequence; x8[t] is [total[t], H, d] contiguous, scales[t] [B, H, ceil(max_len[t]/128)].
+cudaError_t launch_hadamard_quant_varlen(const CUtensorMap* tm, int ntensors, uint8_t* const* x8, float* const* scales,
+                                         const float* post, const int* transform, const signed char* signs, int B,
+                                         int H, const int* const* cu, const int* total, const int* max_len, int d,
+                                         int num_sms, int* status, cudaStream_t stream);
 
 // Sets the pre-kernel's shared-memory attributes on the current device.
 cudaError_t setup_hadamard_quant_kernels();

@@ -172,6 +172,8 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
   p.n_blocks = (N + 127) / 128;
   p.Nk = N;
   p.nbk = p.n_blocks;
+  p.kv_sstride = p.nbk;
+  p.max_nk = N;
   p.off = 0;
   const int tiles = ea::fwd_units_per_tile_pair(d);
   p.n_pairs = (p.n_blocks + tiles - 1) / tiles;

@@ -25,6 +25,13 @@
 // so that the 32 rows of a warp read one contiguous 128-byte line per frequency (row-major
 // tables cost each warp load 32 lines and made the kernel L1-bound).  For d = 256 the partner
 // coordinate sits two lanes away.
+//
+// Packed batches (VL): tensor t holds B sequences of different lengths, rows cu_t[b] ..
+// cu_t[b+1]-1 of a [total_t, H, d] tensor, and is quantised in 128-row blocks of each sequence,
+// so that a block never mixes two sequences: a block's rows past its sequence's end (the next
+// sequence's rows, which the TMA box reads) count as zero and are not written.  Block j of
+// sequence b, head h has scale [b, h, j] of a [B, H, ceil(max_len_t / 128)] array; blocks past a
+// sequence's end are skipped (their barrier phase completes without a load).
 
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -99,9 +106,40 @@ struct HqJob {
   int n_pos;
   int blocks_per_tensor;
   int H;              // heads: batch*head bh = b * H + h reaches the maps as (h, b)
+  // packed batches (VL kernels): per tensor the B + 1 row offsets, the rows of the tensor, the
+  // scale blocks per (sequence, head) = ceil(longest sequence / 128), and the first unit
+  const int* cu[3];
+  int total[3];
+  int nbmax[3];
+  int unit0[4];
 };
 
-template <int D, bool ROPE>
+// One 128-row block of a packed tensor: sequence row range and where its scale goes.
+struct VlBlock {
+  int t, bh, j;   // tensor, b * H + h, block of the sequence
+  int row0;       // first row of the block in the [total, H, d] tensor
+  int rows;       // rows of the block inside the sequence (0: past its end, or bad offsets)
+  bool bad;       // offsets out of order, outside the tensor or longer than nbmax blocks
+};
+
+__device__ __forceinline__ VlBlock vl_block(int u, const HqJob& job) {
+  VlBlock r;
+  r.t = u < job.unit0[1] ? 0 : (u < job.unit0[2] ? 1 : 2);
+  const int rem = u - (r.t == 0 ? 0 : (r.t == 1 ? job.unit0[1] : job.unit0[2]));
+  const int nbm = r.t == 0 ? job.nbmax[0] : (r.t == 1 ? job.nbmax[1] : job.nbmax[2]);
+  const int* cu = r.t == 0 ? job.cu[0] : (r.t == 1 ? job.cu[1] : job.cu[2]);
+  const int total = r.t == 0 ? job.total[0] : (r.t == 1 ? job.total[1] : job.total[2]);
+  r.j = rem % nbm;
+  r.bh = rem / nbm;
+  const int b = r.bh / job.H;
+  const int s0 = __ldg(cu + b), s1 = __ldg(cu + b + 1);
+  r.bad = !(0 <= s0 && s0 <= s1 && s1 <= total && (s1 - s0 + 127) / 128 <= nbm);
+  r.row0 = s0 + r.j * 128;
+  r.rows = r.bad ? 0 : min(128, max(0, s1 - r.row0));
+  return r;
+}
+
+template <int D, bool ROPE, bool VL>
 __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCtasPerSm)
     hadamard_quant_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
                           const __grid_constant__ CUtensorMap tm2, const HqJob job,
@@ -142,16 +180,30 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
   __syncthreads();
 
   auto issue = [&](int u, int buf) {
-    const int t = u / job.blocks_per_tensor;
-    const int b = u - t * job.blocks_per_tensor;
-    const int blk = b % n_blocks;
-    const int bh = b / n_blocks;
-    const CUtensorMap* tm = t == 0 ? &tm0 : (t == 1 ? &tm1 : &tm2);
-    bar_arrive_expect_tx(&bar[buf], C::kBufBytes);
+    if constexpr (VL) {
+      // packed tensors are [total, H, d]: the maps are (d, rows, heads, 1)
+      const VlBlock vb = vl_block(u, job);
+      if (vb.rows == 0) {  // past the sequence's end: complete the phase without a load
+        bar_arrive(&bar[buf]);
+        return;
+      }
+      const CUtensorMap* tm = vb.t == 0 ? &tm0 : (vb.t == 1 ? &tm1 : &tm2);
+      bar_arrive_expect_tx(&bar[buf], C::kBufBytes);
 #pragma unroll
-    for (int bx = 0; bx < C::kBoxes; ++bx)
-      tma_load_4d(smem + buf * C::kBufBytes + bx * 16384, tm, &bar[buf], bx * 64, blk * 128, bh % job.H,
-                  bh / job.H);
+      for (int bx = 0; bx < C::kBoxes; ++bx)
+        tma_load_4d(smem + buf * C::kBufBytes + bx * 16384, tm, &bar[buf], bx * 64, vb.row0, vb.bh % job.H, 0);
+    } else {
+      const int t = u / job.blocks_per_tensor;
+      const int b = u - t * job.blocks_per_tensor;
+      const int blk = b % n_blocks;
+      const int bh = b / n_blocks;
+      const CUtensorMap* tm = t == 0 ? &tm0 : (t == 1 ? &tm1 : &tm2);
+      bar_arrive_expect_tx(&bar[buf], C::kBufBytes);
+#pragma unroll
+      for (int bx = 0; bx < C::kBoxes; ++bx)
+        tma_load_4d(smem + buf * C::kBufBytes + bx * 16384, tm, &bar[buf], bx * 64, blk * 128, bh % job.H,
+                    bh / job.H);
+    }
   };
 
   // two blocks in flight: block i of this CTA goes to buffer i % 2, and the load of block i + 2
@@ -165,10 +217,29 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
     const int buf = it & 1;
     thread_wait(&bar[buf], (it >> 1) & 1, &abort_s, status);
 
-    const int t = u / job.blocks_per_tensor;
-    const int b = u - t * job.blocks_per_tensor;
-    const int blk = b % n_blocks;
-    const int bh = b / n_blocks;
+    int t, blk, bh, rows_valid = 128;
+    long long vl_row0 = 0;
+    if constexpr (VL) {
+      const VlBlock vb = vl_block(u, job);
+      if (vb.bad && tid == 0 && vb.j == 0) atomicOr(status, kDevStatusBadSeqlens);
+      if (vb.rows == 0) {
+        // nothing loaded, nothing written; the CTA still meets at the barrier every block has
+        __syncthreads();
+        if (abort_s) break;
+        if (tid == 0 && u + 2 * static_cast<int>(gridDim.x) < total_blocks) issue(u + 2 * gridDim.x, buf);
+        continue;
+      }
+      t = vb.t;
+      blk = vb.j;
+      bh = vb.bh;
+      rows_valid = vb.rows;
+      vl_row0 = vb.row0;
+    } else {
+      t = u / job.blocks_per_tensor;
+      const int b = u - t * job.blocks_per_tensor;
+      blk = b % n_blocks;
+      bh = b / n_blocks;
+    }
     // explicit selects keep the parameter block out of local memory
     const bool transform = (t == 0 ? job.transform[0] : (t == 1 ? job.transform[1] : job.transform[2])) != 0;
     const uint8_t* sb = smem + buf * C::kBufBytes;
@@ -311,6 +382,13 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
       }
     }
 
+    if constexpr (VL) {
+      // rows of the next sequence inside the box: zero (the transform of a zero row is zero)
+      if (row >= rows_valid) {
+#pragma unroll
+        for (int e = 0; e < kE; ++e) v[e] = 0.f;
+      }
+    }
     // block amax: four chains in the thread, then the lanes, then the warps
     float am[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -332,11 +410,14 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
     const float post = t == 0 ? job.post[0] : (t == 1 ? job.post[1] : job.post[2]);
     const float s_u = fmaxf(__fdiv_rn(amax, 448.f), 1.17549435e-38f);
     const float rcp = __frcp_rn(s_u);
-    if (tid == 0) scales[static_cast<size_t>(bh) * n_blocks + blk] = __fmul_rn(s_u, post);
+    const int nbs = VL ? (t == 0 ? job.nbmax[0] : (t == 1 ? job.nbmax[1] : job.nbmax[2])) : n_blocks;
+    if (tid == 0) scales[static_cast<size_t>(bh) * nbs + blk] = __fmul_rn(s_u, post);
 
     const int grow = blk * 128 + row;
-    if (grow < N) {
-      uint8_t* out = x8 + (static_cast<size_t>(bh) * N + grow) * D + part * kE;
+    if (VL ? row < rows_valid : grow < N) {
+      // contiguous outputs: [BH, N, d], or [total, H, d] for packed tensors
+      uint8_t* out = VL ? x8 + ((vl_row0 + row) * job.H + bh % job.H) * D + part * kE
+                        : x8 + (static_cast<size_t>(bh) * N + grow) * D + part * kE;
 #pragma unroll
       for (int c = 0; c < kE / 16; ++c) {
         uint32_t w[4];
@@ -374,19 +455,30 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
   }
 }
 
-template <int D, bool ROPE>
+template <int D, bool ROPE, bool VL = false>
 static cudaError_t launch_hq(const CUtensorMap* tm, int ntensors, const HqJob& job0, const signed char* signs, int BH,
                              int N, int num_sms, int* status, cudaStream_t stream) {
   using C = HqCfg<D, ROPE>;
   const int n_blocks = (N + 127) / 128;
-  const long long per = static_cast<long long>(BH) * n_blocks;
-  const long long total = per * ntensors;
-  if (total > 0x7FFFFFFFLL - 65536) return cudaErrorInvalidValue;  // u + 2 * grid stays an int
   HqJob job = job0;
-  job.blocks_per_tensor = static_cast<int>(per);
+  long long total = 0;
+  if constexpr (VL) {
+    // units: every (sequence, head, block up to the longest sequence's) of each tensor
+    for (int t = 0; t < 3; ++t) {
+      job.unit0[t] = static_cast<int>(t < ntensors ? total : 0x7FFFFFFF);
+      if (t < ntensors) total += static_cast<long long>(BH) * job.nbmax[t];
+      if (total > 0x7FFFFFFFLL - 65536) return cudaErrorInvalidValue;
+    }
+    job.unit0[3] = static_cast<int>(total);
+  } else {
+    const long long per = static_cast<long long>(BH) * n_blocks;
+    total = per * ntensors;
+    if (total > 0x7FFFFFFFLL - 65536) return cudaErrorInvalidValue;  // u + 2 * grid stays an int
+    job.blocks_per_tensor = static_cast<int>(per);
+  }
   const long long cap = static_cast<long long>(num_sms) * C::kCtasPerSm;
   const int grid = static_cast<int>(total < cap ? total : cap);
-  hadamard_quant_kernel<D, ROPE><<<grid, C::kThreads, 2 * C::kBufBytes + 1024, stream>>>(
+  hadamard_quant_kernel<D, ROPE, VL><<<grid, C::kThreads, 2 * C::kBufBytes + 1024, stream>>>(
       tm[0], tm[ntensors > 1 ? 1 : 0], tm[ntensors > 2 ? 2 : 0], job, signs, N, n_blocks, static_cast<int>(total),
       status);
   return cudaGetLastError();
@@ -394,12 +486,46 @@ static cudaError_t launch_hq(const CUtensorMap* tm, int ntensors, const HqJob& j
 
 template <int D>
 static cudaError_t set_hq_attr() {
-  cudaError_t e = cudaFuncSetAttribute(hadamard_quant_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       2 * HqCfg<D>::kBufBytes + 1024);
+  cudaError_t e = cudaFuncSetAttribute(hadamard_quant_kernel<D, false, false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * HqCfg<D>::kBufBytes + 1024);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(hadamard_quant_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(hadamard_quant_kernel<D, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              2 * HqCfg<D, true>::kBufBytes + 1024);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(hadamard_quant_kernel<D, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             2 * HqCfg<D>::kBufBytes + 1024);
   return e;
+}
+
+cudaError_t launch_hadamard_quant_varlen(const CUtensorMap* tm, int ntensors, uint8_t* const* x8, float* const* scales,
+                                         const float* post, const int* transform, const signed char* signs, int B,
+                                         int H, const int* const* cu, const int* total, const int* max_len, int d,
+                                         int num_sms, int* status, cudaStream_t stream) {
+  if (ntensors < 1 || ntensors > 3) return cudaErrorInvalidValue;
+  HqJob job{};
+  for (int t = 0; t < 3; ++t) {
+    const int s = t < ntensors ? t : 0;
+    job.x8[t] = x8[s];
+    job.scales[t] = scales[s];
+    job.post[t] = post[s];
+    job.transform[t] = transform[s];
+    job.cu[t] = cu[s];
+    job.total[t] = total[s];
+    job.nbmax[t] = (max_len[s] + 127) / 128;
+    if (job.nbmax[t] < 1) return cudaErrorInvalidValue;
+  }
+  job.H = H;
+  const int BH = B * H;
+  switch (d) {
+    case 64:
+      return launch_hq<64, false, true>(tm, ntensors, job, signs, BH, 0, num_sms, status, stream);
+    case 128:
+      return launch_hq<128, false, true>(tm, ntensors, job, signs, BH, 0, num_sms, status, stream);
+    case 256:
+      return launch_hq<256, false, true>(tm, ntensors, job, signs, BH, 0, num_sms, status, stream);
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t setup_hadamard_quant_kernels() {

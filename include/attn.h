@@ -201,6 +201,38 @@ int attn_hadamard_quant_qkv_strided(const void* q, const void* k, const void* v,
                                     const long long* strides, void* stream);
 
 /*
+ * attn_hadamard_quant_qkv_varlen -- attn_hadamard_quant_qkv for a packed batch of B sequences of
+ * different lengths (the layout of attn_fwd_varlen), quantised in 128-row blocks of each
+ * sequence, so that no block (and no scale) mixes two sequences.
+ *
+ *   q           [total_q, H, d] bf16, device (read): sequence b owns rows cu_seqlens_q[b] ..
+ *               cu_seqlens_q[b+1]-1.
+ *   k, v        [total_k, H, d] bf16, device (read): sequence b owns rows cu_seqlens_k[b] .. [b+1]-1.
+ *   strides     HOST pointer to 6 int64 values: {row stride, head stride} for q, k, v, in
+ *               elements, with the rules of attn_fwd_varlen (the head dimension is contiguous).
+ *   q8          [total_q, H, d] E4M3 bytes, contiguous, device (written for the rows of each sequence).
+ *   k8, v8      [total_k, H, d] E4M3 bytes, contiguous, device (written likewise).
+ *   q_scale     [B, H, ceil(max_seqlen_q / 128)] float32, device: entry [b, h, j] is the scale
+ *               of rows 128j .. 128j+127 of sequence b (entries past a sequence's last block are
+ *               not written).
+ *   k_scale, v_scale   [B, H, ceil(max_seqlen_k / 128)] float32, device, likewise.
+ *   cu_seqlens_q, cu_seqlens_k   DEVICE int32 arrays of B + 1 offsets, as for attn_fwd_varlen.
+ *   max_seqlen_q, max_seqlen_k   >= every query / key length: they size the scale arrays.
+ *   signs, d    as for attn_hadamard_quant_qkv (Q and K transformed, V not).
+ * For each sequence, codes and scales are bit-identical to attn_hadamard_quant_qkv on that
+ * sequence alone.  A block's rows past its sequence's end (the next sequence's rows) count as
+ * zero for its scale and are not written.  A sequence whose offsets break their rules (or that
+ * is longer than its max_seqlen) is skipped and reported by attn_device_status() as
+ * ATTN_ERR_INVALID_ARG.  Other errors as for attn_hadamard_quant_qkv.
+ */
+int attn_hadamard_quant_qkv_varlen(const void* q, const void* k, const void* v, void* q8, void* k8,
+                                   void* v8, float* q_scale, float* k_scale, float* v_scale,
+                                   const signed char* signs, const int* cu_seqlens_q,
+                                   const int* cu_seqlens_k, int B, int H, int total_q, int total_k,
+                                   int max_seqlen_q, int max_seqlen_k, int d, const long long* strides,
+                                   void* stream);
+
+/*
  * attn_rope_hadamard_quant_qkv -- attn_hadamard_quant_qkv with the rotary position embedding of
  * Q and K fused in front of the transform ("FlashAttention-3", section "为什么 Hadamard 适合放到
  * 内核里": the transform fuses with RoPE, another bandwidth-bound step; the pages do not define
@@ -303,6 +335,32 @@ int attn_fwd_fp8_strided(const void* q8, const void* k8, const void* v8,
  */
 int attn_fwd_schedule(int B, int H, int Nq, int Nk, int d, int causal, int dtype, int num_ctas,
                       int* out, long long cap, long long* needed);
+
+/*
+ * attn_fwd_fp8_varlen -- attn_fwd_fp8 over a packed batch of B sequences of different lengths,
+ * each an independent problem, on the outputs of attn_hadamard_quant_qkv_varlen.
+ *
+ *   q8          [total_q, H, d] E4M3 bytes, contiguous, device; sequence b owns rows
+ *               cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1.
+ *   k8, v8      [total_k, H, d] E4M3 bytes, contiguous, device; rows cu_seqlens_k[b] .. [b+1]-1.
+ *   q_scale     [B, H, ceil(max_seqlen_q / 128)] float32 per-sequence block scales, device.
+ *   k_scale, v_scale   [B, H, ceil(max_seqlen_k / 128)] float32, device.
+ *   o           [total_q, H, d] of o_dtype, contiguous, device, written for every row of every
+ *               sequence.
+ *   lse         [H, total_q] float32 or NULL.
+ *   cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k   as for attn_hadamard_quant_qkv_varlen
+ *               (the same values: they index the scales).
+ *   d           128 or 256.
+ * Per sequence: bit-identical to attn_fwd_fp8_qk on that sequence's codes and scales alone
+ * (causal alignment, rows with no visible key, arithmetic).  Offsets that break the rules of
+ * attn_fwd_varlen, or a key sequence longer than max_seqlen_k, skip that sequence and are
+ * reported by attn_device_status() as ATTN_ERR_INVALID_ARG.  Errors otherwise as attn_fwd_fp8.
+ */
+int attn_fwd_fp8_varlen(const void* q8, const void* k8, const void* v8,
+                        const float* q_scale, const float* k_scale, const float* v_scale,
+                        void* o, float* lse, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                        int B, int H, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                        int d, float scale, int causal, int o_dtype, void* stream);
 
 /*
  * attn_bwd_workspace_bytes -- size of the float32 workspace attn_bwd needs:

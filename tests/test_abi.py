@@ -36,7 +36,8 @@ def test_header_declares_the_boundary():
                             "attn_bwd_varlen", "attn_fwd_fp8_qk", "attn_merge_partials",
                             "attn_selftest_wait_timeout", "attn_noalloc_status",
                             "attn_noalloc_selftest_wait_timeout", "attn_hadamard_quant_qkv_strided",
-                            "attn_fwd_fp8_strided", "attn_fwd_schedule"])
+                            "attn_fwd_fp8_strided", "attn_fwd_schedule", "attn_hadamard_quant_qkv_varlen",
+                            "attn_fwd_fp8_varlen"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -355,6 +356,55 @@ def test_fwd_fp8_strided_rejects_bad_arguments(L):
     assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
 
 
+def test_hadamard_quant_qkv_varlen_rejects_bad_arguments(L):
+    f = L.attn_hadamard_quant_qkv_varlen
+    H, d = 4, 128
+    good = [H * d, d] * 3
+    ok = [P, P, P, P2, P2, P2, P2, P2, P2, P, P, P, 3, H, 1000, 900, 500, 400, d, _strides(good), NULL]
+    for i in range(12):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    a = list(ok)
+    a[19] = NULL
+    assert f(*a) == ea.ATTN_ERR_INVALID_ARG
+    a = list(ok)
+    a[10] = ctypes.c_void_p(0x10002)  # offsets not 4-byte aligned
+    assert f(*a) == ea.ATTN_ERR_INVALID_ARG
+    for idx, val in [(12, 0), (13, 0), (14, 0), (15, -1), (16, 0), (17, 0), (14, 0x7FFFFFFF)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+    bad = list(good)
+    bad[0] = 12
+    a = list(ok)
+    a[19] = _strides(bad)
+    assert f(*a) == ea.ATTN_ERR_INVALID_ARG
+    a = list(ok)
+    a[18] = 96
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+
+
+def test_fwd_fp8_varlen_rejects_bad_arguments(L):
+    f = L.attn_fwd_fp8_varlen
+    ok = [P, P, P, P2, P2, P2, P, NULL, P, P, 3, 4, 1000, 900, 500, 400, 128, 0.1, 1, 0, NULL]
+    for i in range(7):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for i in (8, 9):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for idx, val in [(10, 0), (11, 0), (12, 0), (13, 0), (14, 0), (15, 0), (17, 0.0), (18, 2), (19, 9)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+    a = list(ok)
+    a[16] = 64
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+
+
 def test_merge_partials_rejects_bad_arguments(L):
     f = L.attn_merge_partials
     ok = [P, P, P2, P2, 1000, 128, 0, NULL]
@@ -435,5 +485,5 @@ def test_python_binding_has_same_names():
                  "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv", "attn_bwd_strided", "attn_bwd_varlen",
                  "attn_fwd_fp8_qk", "attn_merge_partials", "attn_selftest_wait_timeout", "attn_noalloc_status",
                  "attn_noalloc_selftest_wait_timeout", "attn_hadamard_quant_qkv_strided", "attn_fwd_fp8_strided",
-                 "attn_fwd_schedule"]:
+                 "attn_fwd_schedule", "attn_hadamard_quant_qkv_varlen", "attn_fwd_fp8_varlen"]:
         assert callable(getattr(ea, name)), name
