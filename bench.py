@@ -596,19 +596,21 @@ def fp8_section(args, dev, rank):
         ms16 = float(np.mean([a.elapsed_time(b) for a, b in evs]))
         out["forward"]["bf16_same_shape"] = {"ms": ms16, "achieved_tflops": fl / (ms16 * 1e-3) / 1e12,
                                              "fp8_speedup": ms16 / ms8}
-        out["forward_d256"] = fp8_d256_section(dev, rank, steps, flush, fp8_peak)
+        out["forward_d256"] = fp8_other_d_section(dev, rank, steps, flush, fp8_peak, d=256)
+        out["forward_d64"] = fp8_other_d_section(dev, rank, steps, flush, fp8_peak, d=64)
     except Exception as e:  # the E4M3 forward reports unsupported until it is built
         out["forward"] = {"unavailable": str(e)}
     return out
 
 
-def fp8_d256_section(dev, rank, steps, flush, fp8_peak):
-    """The E4M3 forward at d = 256 on the same token count (B=2 H=8 N=8192, non-causal, the
-    outlier recipe, Hadamard on Q and K), and the bf16 kernel on the same unquantised inputs."""
+def fp8_other_d_section(dev, rank, steps, flush, fp8_peak, d=256):
+    """The E4M3 forward at another head dim on the same token count (B=2 H=2048/d N=8192,
+    non-causal, the outlier recipe, Hadamard on Q and K), and the bf16 kernel on the same
+    unquantised inputs."""
     import torch
     import exact_attention_100_b200 as ea
     from exact_attention_100_b200.inputs import normal_qkv, hadamard_signs
-    B, H, N, d = 2, 8, 8192, 256
+    B, H, N = 2, 2048 // d, 8192
     qn, kn, vn = normal_qkv(B, H, N, d, seed=rank, outlier_frac=1e-3)
     q, k, v = (torch.from_numpy(a).to(torch.bfloat16).to(dev) for a in (qn, kn, vn))
     q8 = ea.attn_hadamard_quant_qkv(q, k, v, torch.from_numpy(hadamard_signs(d)).to(dev))
@@ -632,7 +634,7 @@ def fp8_d256_section(dev, rank, steps, flush, fp8_peak):
     ms16 = timed(lambda: ea.attn_fwd(q, k, v, o=o, lse=lse, causal=False, stream=stream))
     fl = attn_flops(B, H, N, d, False)
     assert ea.attn_device_status() == ea.ATTN_OK
-    return {"workload": "B=2 H=8 N=8192 d=256 non-causal, 0.1% N(0,10^2) outliers, seeded signs", "ms": ms8,
+    return {"workload": f"B=2 H={H} N=8192 d={d} non-causal, 0.1% N(0,10^2) outliers, seeded signs", "ms": ms8,
             "achieved_tflops": fl / (ms8 * 1e-3) / 1e12, "frac": fl / (ms8 * 1e-3) / 1e12 / fp8_peak,
             "bf16_same_shape_ms": ms16, "fp8_speedup": ms16 / ms8}
 

@@ -77,18 +77,20 @@ int device_state(DeviceState** out) {
 
 // 4-D tiled map for the forward kernels: dims (d, rows, heads, batch) with the caller's element
 // strides of a row, a head and a batch entry (d contiguous); box = 128 bytes x 128 rows x 1 x 1,
-// 128-byte swizzle, zero fill past the last row.
+// 128-byte swizzle (64 bytes and 64-byte swizzle where a row has only 64 bytes: E4M3 at d = 64),
+// zero fill past the last row.
 bool encode_fwd_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N, int H,
                     int B, long long sn, long long sh, long long sb) {
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(B)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(sn) * elem_bytes, static_cast<cuuint64_t>(sh) * elem_bytes,
                                  static_cast<cuuint64_t>(sb) * elem_bytes};
-  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), 128u, 1u, 1u};
+  const int box_row = d * elem_bytes < 128 ? d * elem_bytes : 128;
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(box_row / elem_bytes), 128u, 1u, 1u};
   const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   return g_encode(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+                  box_row == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 4-D tiled map over O for the forward's TMA stores: dims (d, rows, heads, batch), the caller's
@@ -502,7 +504,7 @@ int fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale
   int rc = check_common(B, H, Nq, scale, causal, o_dtype);
   if (rc != ATTN_OK) return rc;
   if (Nk <= 0 || !units_fit(B, H, Nq)) return ATTN_ERR_INVALID_ARG;
-  if (d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   DeviceState* st = nullptr;
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
@@ -578,7 +580,7 @@ int attn_fwd_fp8_varlen(const void* q8, const void* k8, const void* v8, const fl
       max_seqlen_k <= 0 || max_seqlen_k > kMaxRows)
     return ATTN_ERR_INVALID_ARG;
   if (!units_fit(B, H, max_seqlen_q)) return ATTN_ERR_INVALID_ARG;
-  if (d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   DeviceState* st = nullptr;
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
@@ -620,7 +622,6 @@ int attn_fwd_schedule(int B, int H, int Nq, int Nk, int d, int causal, int dtype
   if (static_cast<long long>(B) * H > 0x7FFFFFFFLL || !units_fit(B, H, Nq)) return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_BF16 && dtype != ATTN_E4M3) return dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
-  if (dtype == ATTN_E4M3 && d == 64) return ATTN_ERR_UNSUPPORTED;
   const int tiles = ea::fwd_units_per_tile_pair(d);
   ea::FwdParams p;
   fill_params(p, nullptr, nullptr, nullptr, B, H, Nq, Nk, tiles, 1.0f, causal, ATTN_BF16);

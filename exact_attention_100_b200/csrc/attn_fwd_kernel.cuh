@@ -82,8 +82,11 @@ constexpr int kVlSchedSeqs = 1024, kVlSchedRounds = 1023;
 
 template <int D, int NQ, class E>
 struct FwdCfg {
-  static constexpr int kBoxBytes = 128 * 128;                 // one TMA box: 128 rows x 128 bytes
-  static constexpr int kBoxes = D * E::kBytes / 128;
+  // one TMA box: 128 rows x 128 bytes (128-byte swizzle), or x 64 bytes (64-byte swizzle) where
+  // a row has only 64 bytes (E4M3, d = 64)
+  static constexpr int kBoxRow = D * E::kBytes < 128 ? D * E::kBytes : 128;
+  static constexpr int kBoxBytes = 128 * kBoxRow;
+  static constexpr int kBoxes = D * E::kBytes / kBoxRow;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;       // 128 rows x D elements
   // K/V ring: as many slots as 192 KB hold besides Q, at most 8 (2 for bf16 d = 256)
   static constexpr int kSlots = (196608 - NQ * kTileBytes) / kTileBytes > 8 ? 8
@@ -825,13 +828,18 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
       auto wait_loaded = [&](uint32_t idx) {
         return wait_bar(&full[idx % C::kSlots], (idx / C::kSlots) & 1u, ab);
       };
+      // operand descriptors for the tiles' swizzle: 8-row atoms of 8 * kBoxRow bytes
+      auto sdesc = [](uint32_t addr, uint32_t lbo) {
+        return C::kBoxRow == 128 ? make_sdesc_sw128(addr, lbo, 1024) : make_sdesc_sw64(addr, lbo, 512);
+      };
       auto issue_s = [&](int q, uint32_t slot, uint32_t buf) {
         const uint32_t d = tmem + buf * 128;
+        constexpr int kStepsPerBox = C::kBoxRow / 32;  // 32-byte K steps inside a row of a box
 #pragma unroll
         for (int kk = 0; kk < D * E::kBytes / 32; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-          const uint64_t a = make_sdesc_sw128(q_base + q * C::kTileBytes + off, 16, 1024);
-          const uint64_t b = make_sdesc_sw128(ring_base + slot * C::kTileBytes + off, 16, 1024);
+          const uint32_t off = (kk / kStepsPerBox) * C::kBoxBytes + (kk % kStepsPerBox) * 32;
+          const uint64_t a = sdesc(q_base + q * C::kTileBytes + off, 16);
+          const uint64_t b = sdesc(ring_base + slot * C::kTileBytes + off, 16);
           if constexpr (E::kFp8)
             mma_f8_ss(d, a, b, kIdS, kk > 0 ? 1u : 0u);
           else
@@ -844,7 +852,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
         for (int kk = 0; kk < 128 / E::kKeysPerMma; ++kk) {
           const uint32_t a = tmem + buf * 128 + kk * 8;  // kKeysPerMma keys of P = 8 columns
           const uint64_t b =
-              make_sdesc_sw128(ring_base + slot * C::kTileBytes + kk * E::kKeysPerMma * 128, C::kBoxBytes, 1024);
+              sdesc(ring_base + slot * C::kTileBytes + kk * E::kKeysPerMma * C::kBoxRow, C::kBoxBytes);
           if constexpr (E::kFp8)
             mma_f8_ts(d, a, b, kIdPV, (acc || kk > 0) ? 1u : 0u);
           else
@@ -1024,7 +1032,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
 #pragma unroll
           for (int b = 0; b < C::kBoxes; ++b)
             tma_load_4d(smem + C::kQOff + q * C::kTileBytes + b * C::kBoxBytes, &tmQ, q_full,
-                        b * (128 / E::kBytes), S.q0 + (U.tile0 + q) * 128, S.h, S.bc);
+                        b * (C::kBoxRow / E::kBytes), S.q0 + (U.tile0 + q) * 128, S.h, S.bc);
         ++qit;
         for (int j = 0; j < U.n_max && ok; ++j) {
 #pragma unroll
@@ -1035,8 +1043,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, E>::kThreads, 1)
             uint8_t* dst = smem + C::kRingOff + s * C::kTileBytes;
 #pragma unroll
             for (int b = 0; b < C::kBoxes; ++b)
-              tma_load_4d(dst + b * C::kBoxBytes, kv ? &tmV : &tmK, &full[s], b * (128 / E::kBytes), S.k0 + j * 128,
-                          S.h, S.bc);
+              tma_load_4d(dst + b * C::kBoxBytes, kv ? &tmV : &tmK, &full[s], b * (C::kBoxRow / E::kBytes),
+                          S.k0 + j * 128, S.h, S.bc);
             ++it;
           }
         }

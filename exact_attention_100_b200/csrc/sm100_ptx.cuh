@@ -262,6 +262,17 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lb
   return d;
 }
 
+// The same for a 64-byte-swizzled operand (layout 4): rows of 64 bytes, 8-row atoms of 512 bytes
+// (16-byte chunk c of row r at c ^ ((r >> 1) & 3), the TMA's 64-byte swizzle); SBO = 512 when packed.
+__device__ __forceinline__ uint64_t make_sdesc_sw64(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= 4ull << 61;
+  return d;
+}
+
 // ---------------------------------------------------------------------------------------------
 // tcgen05: TMEM <-> registers.  Warp w of the CTA reaches TMEM lanes 32*(w%4) .. 32*(w%4)+31;
 // with the 32x32b shape thread t of the warp holds lane 32*(w%4)+t and .xN gives it N

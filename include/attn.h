@@ -262,7 +262,8 @@ int attn_rope_hadamard_quant_qkv(const void* q, const void* k, const void* v, vo
  *   q_scale, k_scale, v_scale   [B, H, ceil(N/128)] float32 block scales, device.
  *   o              [B, H, N, d] of o_dtype (ATTN_BF16 or ATTN_FP32), device, written.
  *   lse            [B, H, N] float32 or NULL, as for attn_fwd.
- *   d              128 or 256 (64: ATTN_ERR_UNSUPPORTED).
+ *   d              64, 128 or 256 (at d = 64 the E4M3 rows are 64 bytes: 64-byte TMA boxes
+ *                  and swizzle).
  *   scale, causal, stream   as for attn_fwd.
  * Arithmetic: E4M3 products accumulated in float32; the Q/K block scales are folded into the
  * softmax scale of each tile pair; P is scaled by 2^(8-tau) * s_v(block) / max_block s_v (tau = 6,
@@ -350,7 +351,7 @@ int attn_fwd_schedule(int B, int H, int Nq, int Nk, int d, int causal, int dtype
  *   lse         [H, total_q] float32 or NULL.
  *   cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k   as for attn_hadamard_quant_qkv_varlen
  *               (the same values: they index the scales).
- *   d           128 or 256.
+ *   d           64, 128 or 256.
  * Per sequence: bit-identical to attn_fwd_fp8_qk on that sequence's codes and scales alone
  * (causal alignment, rows with no visible key, arithmetic).  Offsets that break the rules of
  * attn_fwd_varlen, or a key sequence longer than max_seqlen_k, skip that sequence and are

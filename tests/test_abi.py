@@ -111,7 +111,7 @@ def test_fwd_fp8_rejects_bad_arguments(L):
         a[i] = NULL
         assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
     a = list(ok)
-    a[11] = 64
+    a[11] = 96
     assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
     a = list(ok)
     a[12] = -0.5
@@ -295,7 +295,7 @@ def test_fwd_fp8_qk_rejects_bad_arguments(L):
         a[idx] = val
         assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
     a = list(ok)
-    a[12] = 64
+    a[12] = 96
     assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
 
 
@@ -352,7 +352,7 @@ def test_fwd_fp8_strided_rejects_bad_arguments(L):
         a[idx] = val
         assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
     a = list(ok)
-    a[12] = 64
+    a[12] = 96
     assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
 
 
@@ -401,7 +401,7 @@ def test_fwd_fp8_varlen_rejects_bad_arguments(L):
         a[idx] = val
         assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
     a = list(ok)
-    a[16] = 64
+    a[16] = 96
     assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
 
 

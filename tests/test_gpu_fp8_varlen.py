@@ -110,7 +110,7 @@ def _check_forward(lq, lk, H, d, causal, seed, o_dtype=torch.float32, oracle_hea
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_forward_per_sequence_matches_fixed_length_and_oracle(d, causal):
     # ragged lengths, an empty key sequence, a single row, Nq != Nk both ways
     lq = [300, 1, 128, 513, 7, 257, 0]

@@ -122,4 +122,4 @@ def test_huge_launch_keeps_round_robin_and_bad_arguments():
     with pytest.raises(RuntimeError):
         ea.attn_fwd_schedule(0, 1, 128, 128, 128)
     with pytest.raises(RuntimeError):
-        ea.attn_fwd_schedule(1, 1, 128, 128, 64, fp8=True)
+        ea.attn_fwd_schedule(1, 1, 128, 128, 96, fp8=True)
