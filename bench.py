@@ -70,7 +70,7 @@ def load_peaks():
         return dict(FALLBACK_PEAKS)
 
 
-FWD_SOURCES = ("attn_fwd_kernel.cuh", "attn_fwd_sm100.cu", "attn_kernels.h", "sm100_ptx.cuh")
+FWD_SOURCES = ("attn_fwd_kernel.cuh", "attn_fwd_sm100.cu", "attn_kernels.h", "sm100_ptx.cuh", "unit_table.cu")
 
 
 def kernel_source_hash(names=FWD_SOURCES):
@@ -1032,6 +1032,17 @@ def run_profile_case(args):
         cu_q, cu_k = torch.from_numpy(cq).to(dev), torch.from_numpy(ck).to(dev)
         for _ in range(args.reps):
             ea.attn_fwd_varlen(pq, pk, pv, cu_q, cu_k, max(lens), causal=bool(causal))
+    elif args.profile_case == "fp8_varlen":
+        # the bench's packed batch through the packed pre-kernel and the packed E4M3 forward
+        from exact_attention_100_b200.inputs import normal_qkv_packed
+        w = VARLEN_WORKLOAD
+        lens = varlen_lengths(w["total"], w["lo"], w["hi"], w["seed"])
+        qn, kn, vn, cq, ck = normal_qkv_packed(lens, lens, H, d, seed=w["seed"])
+        pq, pk, pv = (torch.from_numpy(a).to(torch.bfloat16).to(dev) for a in (qn, kn, vn))
+        cu_q, cu_k = torch.from_numpy(cq).to(dev), torch.from_numpy(ck).to(dev)
+        outs = ea.attn_hadamard_quant_qkv_varlen(pq, pk, pv, signs, cu_q, cu_k, max(lens), max(lens))
+        for _ in range(args.reps):
+            ea.attn_fwd_fp8_varlen(*outs, cu_q, cu_k, max(lens), max(lens), causal=bool(causal))
     elif args.profile_case == "bwd":
         o, lse = ea.attn_fwd(q, k, v, causal=bool(causal))
         do = torch.randn_like(q)
@@ -1066,7 +1077,7 @@ def main():
     ap.add_argument("--no-ring", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="leave the head-dim x length sweep out of the line")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv", "hq_rope", "varlen", "bwd", "merge"], default=None,
+    ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv", "hq_rope", "varlen", "fp8_varlen", "bwd", "merge"], default=None,
                     help="run --reps untimed calls of one entry point (for an ncu capture) and exit")
     ap.add_argument("--shape", type=int, nargs=5, default=[2, 16, 8192, 128, 1], metavar=("B", "H", "N", "d", "CAUSAL"))
     ap.add_argument("--reps", type=int, default=3)

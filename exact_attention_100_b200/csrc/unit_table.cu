@@ -30,7 +30,7 @@ namespace ea {
 
 namespace {
 
-constexpr long long kGroupKvBytes = 64ll << 20;  // K and V of the heads whose units run together
+constexpr long long kGroupKvBytes = 32ll << 20;  // K and V of the heads whose units run together
 constexpr long long kMaxTableUnits = 1ll << 20;  // larger launches keep the round-robin order
 constexpr size_t kMaxTables = 4096;              // cached shapes per process; later ones too
 constexpr int kUnitOverhead = 2;                 // fixed cost of a unit (fill, epilogue), in blocks

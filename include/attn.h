@@ -316,7 +316,7 @@ int attn_fwd_fp8_strided(const void* q8, const void* k8, const void* v8,
  * A unit is one (batch*head, group of Q tiles): unit u covers bh = u % (B*H) and the Q tiles
  * [t0, t0 + T) with T = 2 (d = 64, 128) or 1 (d = 256), r = u / (B*H), and t0 = T * r, or
  * T * (n_pairs - 1 - r) when causal (n_pairs = ceil(ceil(Nq / 128) / T)).  The units are
- * ordered longest first within groups of heads (the K and V of a group fit a 64 MB share of the
+ * ordered longest first within groups of heads (the K and V of a group fit a 32 MB share of the
  * 126 MB L2, unless that leaves fewer than two units per CTA in a group) and dealt by greedy list
  * scheduling under a cost of K/V blocks per unit ("FlashAttention-2/3", FA-2 improvement 3:
  * parallelism over the sequence; longest first balances causal units of unequal length).

@@ -83,7 +83,7 @@ def _group_size(B, H, Nq, Nk, d, elem=2, num_ctas=148):
     P = math.ceil(math.ceil(Nq / 128) / _tiles(d))
     g = min(num_ctas, BH * P)
     kv = 2 * Nk * d * elem
-    G = min(BH, max(max(1, (64 << 20) // kv), math.ceil(2 * g / P)))
+    G = min(BH, max(max(1, (32 << 20) // kv), math.ceil(2 * g / P)))
     n_groups = math.ceil(BH / G)
     return math.ceil(BH / n_groups)
 
@@ -96,7 +96,7 @@ def _group_of(l, B, H, Nq, Nk, d):
 @pytest.mark.parametrize("B,H,Nq,Nk,d,causal", SHAPES)
 def test_first_units_share_one_group_of_heads(B, H, Nq, Nk, d, causal):
     """Every CTA's first unit lies in the first group of heads when that group has at least as
-    many units as there are CTAs; the group's K and V fit 64 MB unless fewer heads would leave
+    many units as there are CTAs; the group's K and V fit 32 MB unless fewer heads would leave
     fewer than two units per CTA."""
     lists = ea.attn_fwd_schedule(B, H, Nq, Nk, d, causal=causal)
     BH = B * H
@@ -104,7 +104,7 @@ def test_first_units_share_one_group_of_heads(B, H, Nq, Nk, d, causal):
     G = _group_size(B, H, Nq, Nk, d)
     if G * P >= len(lists):
         assert {l[0] % BH for l in lists} <= set(range(G))
-    if 2 * Nk * d * 2 * G > (64 << 20):
+    if 2 * Nk * d * 2 * G > (32 << 20):
         assert G * P <= 2 * len(lists) + P or G == 1
 
 
