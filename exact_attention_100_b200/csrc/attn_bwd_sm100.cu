@@ -516,6 +516,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         tc_commit(st_s);
         mma_abt<D>(tmem + 128, v_base, q_at(qc) + C::kTileBytes);       // dP^T = V dO^T
         tc_commit(st_dp);
+        // K and V are read only by S^T and dP^T: once the unit's last pair has been issued, their
+        // completion frees the buffer, so the next unit's K and V load during this unit's last
+        // block and epilogue
+        if (i0 + 1 >= nb) tc_commit(kv_empty);
         for (int i = i0; i < nb && ok; ++i, ++qc) {
           const uint32_t q_base = q_at(qc);
           const uint32_t do_base = q_base + C::kTileBytes;
@@ -541,11 +545,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           if (next) {
             mma_abt<D>(tmem + 128, v_base, q_at(qc + 1) + C::kTileBytes);
             tc_commit(st_dp);
+            if (i + 2 >= nb) tc_commit(kv_empty);  // that was the unit's last dP^T
           }
         }
         if (!ok) break;
         tc_commit(dkv_done);
-        tc_commit(kv_empty);
         ++uc;
       }
       tc_commit(drain_bar);
@@ -834,6 +838,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         mma_abt<D>(tmem + 128, do_base, v_addr(vb0));
         tc_commit(dp_full);
         tc_commit(&vempty[vb0 % C::kVSlots]);
+        // Q and dO are read only by S and dP: once the unit's last pair has been issued, their
+        // completion frees the buffer for the next unit's Q and dO (dQ reads dS and K)
+        if (n == 1) tc_commit(qdo_empty);
         for (int j = 0; j < n && ok; ++j, ++sc) {
           const bool next = j + 1 < n;
           if (next) {
@@ -853,13 +860,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
             mma_abt<D>(tmem + 128, do_base, v_addr(vb0 + j + 1));
             tc_commit(dp_full);
             tc_commit(&vempty[(vb0 + j + 1) % C::kVSlots]);
+            if (j + 2 == n) tc_commit(qdo_empty);  // that was the unit's last dP
           }
         }
         if (!ok) break;
         if (!(ok = issue_dq(n - 1, sc - 1))) break;
         if (!ok) break;
         tc_commit(dq_done);
-        tc_commit(qdo_empty);
         ++uc;
       }
       tc_commit(drain_bar);
