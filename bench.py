@@ -816,12 +816,36 @@ def bwd_section(args, dev, rank):
     flops = 2.5 * attn_flops(B, H, N, d, causal)  # dV, dP, dS-recompute S, dK, dQ: five N x N x d products
     peaks = load_peaks()
     tf = flops / (ms * 1e-3) / 1e12
-    return {"workload": "bf16 attention bwd B=2 H=16 N=8192 d=128 causal (dQ, dK, dV from O, LSE, dO)",
-            "ms": ms, "achieved_tflops": tf, "peak_tflops": float(peaks["bf16_tflops"]),
-            "frac": tf / float(peaks["bf16_tflops"]), "bound": "tensor",
-            "flops_per_call": flops, "flops_note": "algorithmic 2.5 x forward (five products); the kernels "
-                                                 "recompute S and dP a second time for dQ",
-            "launches_per_call": 3, "peak_source": peaks["source"]}
+    out = {"workload": "bf16 attention bwd B=2 H=16 N=8192 d=128 causal (dQ, dK, dV from O, LSE, dO)",
+           "ms": ms, "achieved_tflops": tf, "peak_tflops": float(peaks["bf16_tflops"]),
+           "frac": tf / float(peaks["bf16_tflops"]), "bound": "tensor",
+           "flops_per_call": flops, "flops_note": "algorithmic 2.5 x forward (five products); attn_bwd "
+                                                "recomputes S and dP a second time for dQ",
+           "launches_per_call": 3, "peak_source": peaks["source"]}
+    # the same gradients with dS kept in the workspace (attn_bwd_ds: five products, 2.2 GB)
+    ws_ds = torch.empty(ea.attn_bwd_ds_workspace_bytes(B, H, N, causal), dtype=torch.uint8, device=dev)
+
+    def step_ds():
+        ea.attn_bwd_ds(q, k, v, o, lse, do, dq, dk, dv, ws_ds, causal=causal, stream=stream)
+
+    for _ in range(3):
+        step_ds()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        step_ds()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+    ms_ds = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    tf_ds = flops / (ms_ds * 1e-3) / 1e12
+    out["ds"] = {"ms": ms_ds, "achieved_tflops": tf_ds, "frac": tf_ds / float(peaks["bf16_tflops"]),
+                 "workspace_bytes": int(ws_ds.numel()), "vs_recompute": ms / ms_ds,
+                 "note": "attn_bwd_ds: the dK/dV kernel stores each bf16 dS tile, a third kernel streams "
+                         "them with K through the tensor cores for dQ (no recomputation)"}
+    del ws_ds
+    return out
 
 
 SWEEP_DS = (64, 128, 256)
@@ -1048,6 +1072,11 @@ def run_profile_case(args):
         do = torch.randn_like(q)
         for _ in range(args.reps):
             ea.attn_bwd(q, k, v, o, lse, do, causal=bool(causal))
+    elif args.profile_case == "bwd_ds":
+        o, lse = ea.attn_fwd(q, k, v, causal=bool(causal))
+        do = torch.randn_like(q)
+        for _ in range(args.reps):
+            ea.attn_bwd_ds(q, k, v, o, lse, do, causal=bool(causal))
     else:
         outs = None
         for _ in range(args.reps):
@@ -1077,7 +1106,7 @@ def main():
     ap.add_argument("--no-ring", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="leave the head-dim x length sweep out of the line")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv", "hq_rope", "varlen", "fp8_varlen", "bwd", "merge"], default=None,
+    ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv", "hq_rope", "varlen", "fp8_varlen", "bwd", "bwd_ds", "merge"], default=None,
                     help="run --reps untimed calls of one entry point (for an ncu capture) and exit")
     ap.add_argument("--shape", type=int, nargs=5, default=[2, 16, 8192, 128, 1], metavar=("B", "H", "N", "d", "CAUSAL"))
     ap.add_argument("--reps", type=int, default=3)

@@ -103,6 +103,10 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_schedule.restype = i
         L.attn_bwd_workspace_bytes.argtypes = [i, i, i]
         L.attn_bwd_workspace_bytes.restype = ctypes.c_ulonglong
+        L.attn_bwd_ds_workspace_bytes.argtypes = [i, i, i, i]
+        L.attn_bwd_ds_workspace_bytes.restype = ctypes.c_ulonglong
+        L.attn_bwd_ds.argtypes = [vp] * 10 + [i, i, i, i, f, i, i, vp]
+        L.attn_bwd_ds.restype = i
         L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
         L.attn_bwd.restype = i
         L.attn_bwd_qk.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
@@ -205,6 +209,39 @@ def attn_bwd(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None, s
     _check(lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
                           _ptr(workspace), B, H, N, d, s, int(bool(causal)), gcode, _stream_ptr(stream)),
            "attn_bwd")
+    return dq, dk, dv
+
+
+def attn_bwd_ds_workspace_bytes(B, H, N, causal):
+    """Bytes of the workspace :func:`attn_bwd_ds` needs (0 if the shape has too many tiles)."""
+    return int(lib().attn_bwd_ds_workspace_bytes(B, H, N, int(bool(causal))))
+
+
+def attn_bwd_ds(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None, scale=None, causal=False,
+                g_dtype=None, stream=None):
+    """attn_bwd with the dS tiles kept in the workspace: dQ is formed from the stored dS instead
+    of recomputing S and dP (five products instead of seven), for
+    ``attn_bwd_ds_workspace_bytes(B, H, N, causal)`` bytes of workspace (a uint8 tensor) instead
+    of attn_bwd_workspace_bytes.  Arguments and results otherwise as :func:`attn_bwd`."""
+    import torch
+    B, H, N, d = _dims(q)
+    for t in (q, k, v, o, dout):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError("q, k, v, o, dout must be contiguous bf16 tensors of one shape")
+    gd = g_dtype or (dq.dtype if dq is not None else torch.bfloat16)
+    dq = dq if dq is not None else torch.empty(q.shape, dtype=gd, device=q.device)
+    dk = dk if dk is not None else torch.empty(q.shape, dtype=gd, device=q.device)
+    dv = dv if dv is not None else torch.empty(q.shape, dtype=gd, device=q.device)
+    if workspace is None:
+        nbytes = attn_bwd_ds_workspace_bytes(B, H, N, causal)
+        if nbytes == 0:
+            raise ValueError("too many dS tiles for this shape: use attn_bwd")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
+    s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
+    _check(lib().attn_bwd_ds(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                             _ptr(dv), _ptr(workspace), B, H, N, d, s, int(bool(causal)), gcode,
+                             _stream_ptr(stream)), "attn_bwd_ds")
     return dq, dk, dv
 
 

@@ -653,9 +653,22 @@ struct Packed {
 
 // attn_bwd, attn_bwd_qk, attn_bwd_strided and attn_bwd_varlen.  st8: element strides of q, k, v,
 // o, dout, dq, dk, dv.  Fixed-length batches: Nq, Nk are the lengths; packed ones: the longest.
+// Bytes of the dS-mode workspace: D and LSE * log2 e (padded rows), rounded up to 1024, then the
+// bf16 dS^T tiles of every (batch, head): n_b (n_b + 1) / 2 causal, n_b^2 otherwise, 32 KB each.
+// 0 if a size is not positive or the tiles cannot be indexed with int.
+unsigned long long bwd_ds_workspace_bytes(int B, int H, int N, int causal) {
+  if (B <= 0 || H <= 0 || N <= 0 || (causal != 0 && causal != 1)) return 0ull;
+  const unsigned long long bh = static_cast<unsigned long long>(B) * static_cast<unsigned long long>(H);
+  const unsigned long long nb = (static_cast<unsigned long long>(N) + 127ull) / 128ull;
+  const unsigned long long tiles = causal ? nb * (nb + 1ull) / 2ull : nb * nb;
+  if (bh * tiles >= 0x7FFFFFFFull) return 0ull;
+  const unsigned long long head = (2ull * bh * nb * 128ull * 4ull + 1023ull) / 1024ull * 1024ull;
+  return head + bh * tiles * 128ull * 128ull * 2ull;
+}
+
 int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
              void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk, int d, const Strides* st8,
-             const Packed* pk, float scale, int causal, int g_dtype, void* stream) {
+             const Packed* pk, float scale, int causal, int g_dtype, void* stream, bool ds_mode = false) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
@@ -712,6 +725,19 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const v
   p.cu_k = pk ? pk->cu_k : nullptr;
   p.total_q = pk ? pk->total_q : 0;
   p.total_k = pk ? pk->total_k : 0;
+  p.ds = nullptr;
+  p.ds_tiles = 0;
+  if (ds_mode) {
+    // the dS^T tiles follow D and LSE in the workspace (bwd_ds_workspace_bytes)
+    const long long nb = n_blocks;
+    p.ds_tiles = causal ? nb * (nb + 1) / 2 : nb * nb;
+    const size_t head = (2ull * static_cast<size_t>(p.BH) * p.n_pad * 4ull + 1023ull) / 1024ull * 1024ull;
+    p.ds = static_cast<uint8_t*>(workspace) + head;
+    if (ea::launch_attn_bwd_ds(d, mq, mk, mv, mdo, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    g_launches.fetch_add(3);
+    return ATTN_OK;
+  }
   if (ea::launch_attn_bwd(d, mq, mk, mv, mdo, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
   g_launches.fetch_add(3);
@@ -721,6 +747,22 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const v
 }  // namespace
 
 extern "C" {
+
+unsigned long long attn_bwd_ds_workspace_bytes(int B, int H, int N, int causal) {
+  return bwd_ds_workspace_bytes(B, H, N, causal);
+}
+
+int attn_bwd_ds(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                void* dq, void* dk, void* dv, void* workspace, int B, int H, int N, int d, float scale, int causal,
+                int g_dtype, void* stream) {
+  if (B <= 0 || H <= 0 || N <= 0 || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (bwd_ds_workspace_bytes(B, H, N, causal) == 0ull) return ATTN_ERR_INVALID_ARG;  // too many tiles for int
+  const Strides s = contiguous_strides(H, N, d);
+  const Strides st8[8] = {s, s, s, s, s, s, s, s};
+  return bwd_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, N, N, d, st8, nullptr, scale, causal, g_dtype,
+                  stream, true);
+}
 
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
              void* dq, void* dk, void* dv, void* workspace, int B, int H, int N, int d, float scale, int causal,

@@ -322,7 +322,7 @@ struct DkdvCfg : BwdCfg<D> {
   static_assert(256 + 2 * D <= 512, "TMEM budget");
 };
 
-template <int D, bool VL>
+template <int D, bool VL, bool DS = false>
 __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -457,6 +457,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         ok = warp_all(wait_bar(st_dp, qc & 1u, ab));
         if (!ok) break;
         tc_fence_after();
+        // dS mode: tile (i, kb) of the workspace, stored chunk-major (16-byte chunk j of query
+        // columns [8j, 8j + 8) for all 128 key rows, then chunk j + 1), so that a warp's store of
+        // one chunk writes 512 contiguous bytes; the layout is the tensor core's non-swizzled
+        // MN-major operand layout, which the dQ pass copies into shared memory as it is
+        uint8_t* ds_tile = nullptr;
+        if constexpr (DS) {
+          const long long tile = static_cast<long long>(U.bh) * p.ds_tiles +
+                                 (p.causal ? static_cast<long long>(i) * (i + 1) / 2 + kb
+                                           : static_cast<long long>(i) * nb + kb);
+          ds_tile = static_cast<uint8_t*>(p.ds) + tile * (128 * 128 * 2) + row * 16;
+        }
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t dp[32];
@@ -473,11 +484,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
             dk[t] = pack_bf16x2(y0, y1);
           }
           tmem_st_16cols(lane_base + 128 + 64 * h + 16 * c, dk);
+          if constexpr (DS) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)  // chunk 8h + 4c + v4: queries 64h + 32c + 8 v4 .. + 8
+              *reinterpret_cast<uint4*>(ds_tile + (8 * h + 4 * c + v4) * 2048) =
+                  make_uint4(dk[4 * v4], dk[4 * v4 + 1], dk[4 * v4 + 2], dk[4 * v4 + 3]);
+          }
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) bar_arrive(dst_full);
+
       }
       if (!ok) break;
       // epilogue: dV and scale * dK of this key block
@@ -922,6 +940,188 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ dQ from stored dS (dS mode)
+// Unit u: query block i of head bh (causal: longest first) and its key blocks kb = 0 .. n-1,
+// streamed through a ring of slots that each hold the bf16 dS^T tile (i, kb) written by the dK/dV
+// kernel (one 32 KB bulk copy: it is stored in the non-swizzled MN-major operand layout) and the
+// K tile kb (TMA): dQ_i += dS(i, kb) K_kb on the tensor cores, A = dS read MN-major (queries
+// contiguous in 16-byte chunks), B = K read MN-major (d contiguous, 128-byte swizzle).  No S, P or dP is
+// recomputed: five products in all instead of seven.  dQ is double-buffered in TMEM (2 x D
+// columns) so that one unit's epilogue overlaps the next unit's products.  Roles: warps 0-3 the
+// epilogue (one TMEM lane quarter each), warp 4 lane 0 the MMA issuer, warp 5 lane 0 the TMA
+// producer.  Fixed-length batches, equal query and key lengths.
+template <int D>
+struct DqDsCfg {
+  static constexpr int kDsBytes = 128 * 128 * 2;             // one dS^T tile (chunk-major)
+  static constexpr int kKBytes = BwdCfg<D>::kTileBytes;      // one K tile
+  static constexpr int kSlotBytes = kDsBytes + kKBytes;
+  static constexpr int kSlots = 3;
+  static constexpr int kThreads = 192;
+  static constexpr int kMmaWarp = 4;
+  static constexpr int kLoadWarp = 5;
+  static constexpr int kBarOff = kSlots * kSlotBytes;
+  // full[kSlots], empty[kSlots], dq_done[2], dq_free[2], drain
+  static constexpr int kNumBars = 2 * kSlots + 5;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kMiscOff + 16;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;
+  static constexpr uint32_t kTmemCols = 2 * D;
+  // M = 128 queries, N = D, K = 16 keys per instruction; A and B both MN-major
+  static constexpr uint32_t kIdQ = make_idesc(128, D, 1, true) | (1u << 15);
+  static_assert(kSmemAlloc <= 232448, "shared memory budget");
+};
+
+// dS-mode dQ unit u: head bh, query block i, n key blocks, and its first tile's index
+struct DsUnit {
+  int bh, i, n;
+  long long tile0;
+};
+__device__ __forceinline__ DsUnit ds_unit(int u, const BwdParams& p) {
+  DsUnit U;
+  U.bh = u % p.BH;
+  const int r = u / p.BH;
+  U.i = p.causal ? p.n_blocks - 1 - r : r;
+  U.n = p.causal ? U.i + 1 : p.n_blocks;
+  U.tile0 = static_cast<long long>(U.bh) * p.ds_tiles +
+            (p.causal ? static_cast<long long>(U.i) * (U.i + 1) / 2 : static_cast<long long>(U.i) * p.n_blocks);
+  return U;
+}
+
+template <int D>
+__global__ void __launch_bounds__(DqDsCfg<D>::kThreads, 1)
+    bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tmK, const BwdParams p) {
+  using C = DqDsCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* full = bars;
+  uint64_t* empty = full + C::kSlots;
+  uint64_t* dq_done = empty + C::kSlots;
+  uint64_t* dq_free = dq_done + 2;
+  uint64_t* drain_bar = dq_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kSlots; ++s) {
+      bar_init(&full[s], 1);
+      bar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      bar_init(&dq_done[b], 1);
+      bar_init(&dq_free[b], 4);
+    }
+    bar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == C::kLoadWarp && lane == 0) {
+    prefetch_tensor_map(&tmK);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const AbortState ab{abort_flag, p.status};
+  const int num_units = p.BH * p.n_blocks;
+
+  if (warp < 4) {
+    // ================================================================ epilogue: scale * dQ
+    const int row = warp * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    uint32_t uc = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int u = unit_of(k);
+      if (u >= num_units) break;
+      const DsUnit U = ds_unit(u, p);
+      const uint32_t buf = uc & 1u;
+      ok = warp_all(wait_bar(&dq_done[buf], (uc >> 1) & 1u, ab));
+      if (!ok) break;
+      tc_fence_after();
+      const int b = U.bh / p.H, h = U.bh - b * p.H;
+      const int q_g = U.i * 128 + row;
+      const size_t off_q = static_cast<size_t>(b * p.dq_sb + h * p.dq_sh + static_cast<long long>(q_g) * p.dq_sn);
+      store_row<D>(lane_base + buf * D, p.dq, off_q, p.scale, p.g_fp32 != 0, q_g < p.N);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) bar_arrive(&dq_free[buf]);
+      ++uc;
+    }
+  } else if (warp == C::kMmaWarp) {
+    if (lane == 0) {
+      // ================================================================== MMA issuer
+      const uint32_t ring = smem_addr(smem);
+      uint32_t it = 0, uc = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int u = unit_of(k);
+        if (u >= num_units) break;
+        const DsUnit U = ds_unit(u, p);
+        const uint32_t buf = uc & 1u;
+        // the epilogue of the unit before last must be done reading this dQ buffer
+        if (!(ok = wait_bar(&dq_free[buf], ((uc >> 1) & 1u) ^ 1u, ab))) break;
+        tc_fence_after();
+        for (int j = 0; j < U.n && ok; ++j, ++it) {
+          const uint32_t s = it % C::kSlots;
+          // TMA-filled shared memory read by the tensor core: the wait alone orders it
+          if (!(ok = wait_bar(&full[s], (it / C::kSlots) & 1u, ab))) break;
+          const uint32_t a_base = ring + s * C::kSlotBytes;
+          const uint32_t b_base = a_base + C::kDsBytes;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_f16_ss(tmem + buf * D, make_sdesc_mn_noswz(a_base + kk * 256, 2048, 128),
+                       make_sdesc_sw128(b_base + kk * 16 * 128, BwdCfg<D>::kBoxBytes, 1024), C::kIdQ,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(&dq_done[buf]);
+        ++uc;
+      }
+      tc_commit(drain_bar);
+      drain(drain_bar, 0, p.status);
+    }
+  } else {
+    if (lane == 0) {
+      // =============================================================== TMA producer
+      uint32_t it = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int u = unit_of(k);
+        if (u >= num_units) break;
+        const DsUnit U = ds_unit(u, p);
+        const int b = U.bh / p.H, h = U.bh - b * p.H;
+        for (int j = 0; j < U.n && ok; ++j, ++it) {
+          const uint32_t s = it % C::kSlots;
+          if (!(ok = wait_bar(&empty[s], ((it / C::kSlots) & 1u) ^ 1u, ab))) break;
+          uint8_t* dst = smem + s * C::kSlotBytes;
+          bar_arrive_expect_tx(&full[s], C::kSlotBytes);
+          bulk_load_g2s(dst, static_cast<const uint8_t*>(p.ds) + (U.tile0 + j) * C::kDsBytes, C::kDsBytes, &full[s]);
+          load_tile<D>(dst + C::kDsBytes, &tmK, &full[s], j * 128, h, b);
+        }
+      }
+      // every issued copy lands before the CTA can exit
+      const uint32_t first = it > static_cast<uint32_t>(C::kSlots) ? it - C::kSlots : 0u;
+      for (uint32_t i = first; i < it; ++i) drain(&full[i % C::kSlots], (i / C::kSlots) & 1u, p.status);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
 template <int D, bool VL>
 cudaError_t setup_d() {
   cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, VL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -929,7 +1129,36 @@ cudaError_t setup_d() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(bwd_dq_kernel<D, VL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              DqCfg<D>::kSmemAlloc);
+  if constexpr (!VL) {
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               DkdvCfg<D>::kSmemAlloc);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_dq_ds_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               DqDsCfg<D>::kSmemAlloc);
+  }
   return e;
+}
+
+template <int D>
+cudaError_t launch_d_ds(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& dout,
+                        const BwdParams& p, int num_sms, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(p.BH) * p.n_pad;
+  const long long threads = rows * (D / 16);
+  const long long blocks = (threads + 255) / 256;
+  if (blocks > 0x7FFFFFFFLL || p.ds == nullptr || p.cu_q != nullptr) return cudaErrorInvalidValue;
+  bwd_prep_kernel<D, false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int kv_units = p.BH * p.nbk;
+  const int kv_grid = kv_units < num_sms ? kv_units : num_sms;
+  bwd_dkdv_kernel<D, false, true><<<kv_grid, BwdCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(q, k, v, dout, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int q_units = p.BH * p.n_blocks;
+  const int q_grid = q_units < num_sms ? q_units : num_sms;
+  bwd_dq_ds_kernel<D><<<q_grid, DqDsCfg<D>::kThreads, DqDsCfg<D>::kSmemAlloc, stream>>>(k, p);
+  return cudaGetLastError();
 }
 
 template <int D, bool VL>
@@ -973,6 +1202,19 @@ cudaError_t launch_attn_bwd(int d, const CUtensorMap& q, const CUtensorMap& k, c
     case 128:
       return vl ? launch_d<128, true>(q, k, v, dout, p, num_sms, stream)
                 : launch_d<128, false>(q, k, v, dout, p, num_sms, stream);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_attn_bwd_ds(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                               const CUtensorMap& dout, const BwdParams& p, int num_sms,
+                               cudaStream_t stream) {
+  switch (d) {
+    case 64:
+      return launch_d_ds<64>(q, k, v, dout, p, num_sms, stream);
+    case 128:
+      return launch_d_ds<128>(q, k, v, dout, p, num_sms, stream);
     default:
       return cudaErrorInvalidValue;
   }

@@ -122,6 +122,12 @@ struct BwdParams {
   const int* cu_k;
   int total_q;
   int total_k;
+  // dS mode (ds == nullptr: dQ recomputes S and dP): the dK/dV kernel also writes its bf16 dS^T
+  // tiles to ds, [BH][ds_tiles] tiles of 32 KB, tile (i, kb) of query block i and key block kb
+  // at i (i + 1) / 2 + kb (causal) or i * n_blocks + kb, each [16 chunks of 8 queries][128 key
+  // rows][8 queries], and dQ is formed from them; fixed-length batches, equal lengths
+  void* ds;
+  long long ds_tiles;
 };
 
 cudaError_t setup_bwd_kernels();
@@ -129,6 +135,12 @@ cudaError_t setup_bwd_kernels();
 // forward (p.cu_q selects the packed-batch kernels).
 cudaError_t launch_attn_bwd(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                             const CUtensorMap& dout, const BwdParams& p, int num_sms, cudaStream_t stream);
+
+// The dS mode: D and LSE * log2 e, then dK/dV writing the dS^T tiles, then dQ = scale dS K
+// streamed from them (each 32 KB tile stored chunk-major: 16-byte chunks of 8 queries for the
+// 128 key rows, chunk after chunk, the tensor core's non-swizzled MN-major operand layout).
+cudaError_t launch_attn_bwd_ds(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                               const CUtensorMap& dout, const BwdParams& p, int num_sms, cudaStream_t stream);
 
 // Hadamard + per-block E4M3 quantisation of 1..3 tensors of one shape [B, H, N, d] in one launch:
 // tm[t] is a 4-D tiled map (d, rows, heads, batch) over tensor t with its own strides (bf16, box

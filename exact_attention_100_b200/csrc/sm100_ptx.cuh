@@ -273,6 +273,18 @@ __device__ __forceinline__ uint64_t make_sdesc_sw64(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// The same without swizzle (layout 0), for an MN-major operand stored as "core matrices" of 8
+// K-rows x 16 bytes (8 consecutive MN elements per row, the 8 rows 16 bytes apart, 128 bytes in
+// all): `mn_stride` = byte distance between core matrices adjacent along MN (stride byte offset
+// field), `k_stride` = between core matrices adjacent along K (leading byte offset field).
+__device__ __forceinline__ uint64_t make_sdesc_mn_noswz(uint32_t saddr, uint32_t mn_stride, uint32_t k_stride) {
+  uint64_t d = static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((k_stride >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((mn_stride >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  return d;
+}
+
 // ---------------------------------------------------------------------------------------------
 // tcgen05: TMEM <-> registers.  Warp w of the CTA reaches TMEM lanes 32*(w%4) .. 32*(w%4)+31;
 // with the 32x32b shape thread t of the warp holds lane 32*(w%4)+t and .xN gives it N

@@ -407,6 +407,33 @@ int attn_bwd_qk(const void* q, const void* k, const void* v, const void* o, cons
                 void* stream);
 
 /*
+ * attn_bwd_ds_workspace_bytes -- size of the workspace attn_bwd_ds needs: the float32 rows of
+ * attn_bwd_workspace_bytes (rounded up to 1024 bytes), then one bf16 128 x 128 tile of dS per
+ * (batch, head, query block, visible key block): B * H * n (n + 1) / 2 tiles causal, B * H * n^2
+ * otherwise, n = ceil(N / 128), 32 KB each (2.2 GB at B=2 H=16 N=8192 causal).  Returns 0 if a
+ * size is not positive or there are 2^31 - 1 tiles or more.
+ */
+unsigned long long attn_bwd_ds_workspace_bytes(int B, int H, int N, int causal);
+
+/*
+ * attn_bwd_ds -- attn_bwd that keeps dS instead of recomputing it: the dK/dV kernel writes each
+ * bf16 dS tile (the one its dK product uses) into the workspace, and a third kernel streams them
+ * with the K tiles through the tensor cores, dQ = scale dS K ("Flash Attention V3 解析", section
+ * 4.2: dQ accumulates over the key blocks; here in a fixed order, without atomics).  Five
+ * products instead of attn_bwd's seven, for O(N^2) workspace.
+ *
+ *   workspace   device, 16-byte aligned, attn_bwd_ds_workspace_bytes(B, H, N, causal) bytes;
+ *               owned by the caller and overwritten.
+ *   Other arguments as for attn_bwd (d 64 or 128, equal query and key lengths, contiguous).
+ * dK and dV are bit-identical to attn_bwd's; dQ agrees with it within the rounding of the two
+ * ways of forming dS (the bounds of attn_bwd hold for both).  Deterministic.  Returns
+ * ATTN_ERR_INVALID_ARG also when attn_bwd_ds_workspace_bytes would return 0.
+ */
+int attn_bwd_ds(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                int B, int H, int N, int d, float scale, int causal, int g_dtype, void* stream);
+
+/*
  * attn_bwd_strided -- attn_bwd_qk on tensors laid out with arbitrary strides (the backward of
  * attn_fwd_strided).
  *

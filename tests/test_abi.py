@@ -37,7 +37,7 @@ def test_header_declares_the_boundary():
                             "attn_selftest_wait_timeout", "attn_noalloc_status",
                             "attn_noalloc_selftest_wait_timeout", "attn_hadamard_quant_qkv_strided",
                             "attn_fwd_fp8_strided", "attn_fwd_schedule", "attn_hadamard_quant_qkv_varlen",
-                            "attn_fwd_fp8_varlen"])
+                            "attn_fwd_fp8_varlen", "attn_bwd_ds_workspace_bytes", "attn_bwd_ds"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -441,6 +441,38 @@ def test_bwd_workspace_bytes(L):
     assert L.attn_bwd_workspace_bytes(1, 1, -5) == 0
 
 
+def test_bwd_ds_workspace_bytes(L):
+    f = L.attn_bwd_ds_workspace_bytes
+    nb = 64
+    head = (2 * 32 * nb * 128 * 4 + 1023) // 1024 * 1024
+    assert f(2, 16, 8192, 1) == head + 32 * (nb * (nb + 1) // 2) * 32768
+    assert f(2, 16, 8192, 0) == head + 32 * nb * nb * 32768
+    assert f(1, 1, 1, 1) == 1024 + 32768
+    for a in [(0, 1, 128, 0), (1, 0, 128, 0), (1, 1, 0, 0), (1, 1, 128, 2)]:
+        assert f(*a) == 0, a
+    # 2^31 - 1 tiles or more cannot be addressed by the dQ pass's tensor map
+    assert f(1, 1 << 20, 1 << 14, 0) == 0
+
+
+def test_bwd_ds_rejects_bad_arguments(L):
+    f = L.attn_bwd_ds
+    ok = [P, P, P, P, P, P2, P, P, P, P, 1, 2, 256, 128, 0.1, 1, 0, NULL]
+    for i in range(10):
+        a = list(ok)
+        a[i] = NULL
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for idx, val in [(10, 0), (11, 0), (12, 0), (14, 0.0), (15, 2), (16, 7)]:
+        a = list(ok)
+        a[idx] = val
+        assert f(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+    a = list(ok)
+    a[13] = 256
+    assert f(*a) == ea.ATTN_ERR_UNSUPPORTED
+    a = list(ok)
+    a[11], a[12], a[15] = 1 << 20, 1 << 14, 0  # too many dS tiles
+    assert f(*a) == ea.ATTN_ERR_INVALID_ARG
+
+
 def test_bwd_rejects_bad_arguments(L):
     f = L.attn_bwd
     ok = [P, P, P, P, P, P2, P2, P2, P2, P2, 1, 1, 128, 128, 0.1, 0, 0, NULL]
@@ -485,5 +517,6 @@ def test_python_binding_has_same_names():
                  "attn_fwd_varlen", "attn_rope_hadamard_quant_qkv", "attn_bwd_strided", "attn_bwd_varlen",
                  "attn_fwd_fp8_qk", "attn_merge_partials", "attn_selftest_wait_timeout", "attn_noalloc_status",
                  "attn_noalloc_selftest_wait_timeout", "attn_hadamard_quant_qkv_strided", "attn_fwd_fp8_strided",
-                 "attn_fwd_schedule", "attn_hadamard_quant_qkv_varlen", "attn_fwd_fp8_varlen"]:
+                 "attn_fwd_schedule", "attn_hadamard_quant_qkv_varlen", "attn_fwd_fp8_varlen",
+                 "attn_bwd_ds_workspace_bytes", "attn_bwd_ds"]:
         assert callable(getattr(ea, name)), name
