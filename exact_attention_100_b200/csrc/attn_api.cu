@@ -727,12 +727,19 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const v
   p.total_k = pk ? pk->total_k : 0;
   p.ds = nullptr;
   p.ds_tiles = 0;
+  p.kv_tab = p.q_tab = nullptr;
   if (ds_mode) {
     // the dS^T tiles follow D and LSE in the workspace (bwd_ds_workspace_bytes)
     const long long nb = n_blocks;
     p.ds_tiles = causal ? nb * (nb + 1) / 2 : nb * nb;
     const size_t head = (2ull * static_cast<size_t>(p.BH) * p.n_pad * 4ull + 1023ull) / 1024ull * 1024ull;
     p.ds = static_cast<uint8_t*>(workspace) + head;
+    // work lists: the units of groups of heads whose streamed tensors fit L2 run together
+    const int kv_units = p.BH * p.nbk, q_units = p.BH * p.n_blocks;
+    p.kv_tab = ea::bwd_unit_table(p, 1, d, kv_units < st->num_sms ? kv_units : st->num_sms,
+                                  static_cast<cudaStream_t>(stream));
+    p.q_tab = ea::bwd_unit_table(p, 2, d, q_units < st->num_sms ? q_units : st->num_sms,
+                                 static_cast<cudaStream_t>(stream));
     if (ea::launch_attn_bwd_ds(d, mq, mk, mv, mdo, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
       return ATTN_ERR_CUDA;
     g_launches.fetch_add(3);

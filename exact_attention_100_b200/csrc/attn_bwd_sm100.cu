@@ -233,6 +233,16 @@ __device__ __forceinline__ int unit_of(int k) {
   return k * g + ((k & 1) ? (g - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x));
 }
 
+// k-th unit of this CTA from a host-built work list (tab: [gridDim.x + 1] offsets, then unit
+// ids), or the round-robin order without one; past the end of the list a value >= every unit.
+__device__ __forceinline__ int unit_of(int k, const int* tab) {
+  if (tab != nullptr) {
+    const int i = __ldg(tab + blockIdx.x) + k;
+    return i < __ldg(tab + blockIdx.x + 1) ? __ldg(tab + gridDim.x + 1 + i) : 0x7FFFFFFF;
+  }
+  return unit_of(k);
+}
+
 // dK/dV unit u: key block kb of head bh and the first query block i0 that sees any of its keys
 // (causal, bottom-right: query r sees key c iff c <= r + off); i0 >= n_blocks: no query does.
 // `present`: the block lies inside its sequence (always, unless packed).
@@ -389,7 +399,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     uint32_t qc = 0, uit = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int u = unit_of(k);
+      const int u = unit_of(k, p.kv_tab);
       if (u >= num_units) break;
       const KvUnit U = kv_unit<VL>(u, p);
       if constexpr (VL) {
@@ -518,7 +528,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       uint32_t qc = 0, uc = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int u = unit_of(k);
+        const int u = unit_of(k, p.kv_tab);
         if (u >= num_units) break;
         const KvUnit U = kv_unit<VL>(u, p);
         if constexpr (VL) {
@@ -579,7 +589,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       uint32_t qc = 0, uc = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int u = unit_of(k);
+        const int u = unit_of(k, p.kv_tab);
         if (u >= num_units) break;
         const KvUnit U = kv_unit<VL>(u, p);
         if constexpr (VL) {
@@ -1038,7 +1048,7 @@ __global__ void __launch_bounds__(DqDsCfg<D>::kThreads, 1)
     uint32_t uc = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int u = unit_of(k);
+      const int u = unit_of(k, p.q_tab);
       if (u >= num_units) break;
       const DsUnit U = ds_unit(u, p);
       const uint32_t buf = uc & 1u;
@@ -1061,7 +1071,7 @@ __global__ void __launch_bounds__(DqDsCfg<D>::kThreads, 1)
       uint32_t it = 0, uc = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int u = unit_of(k);
+        const int u = unit_of(k, p.q_tab);
         if (u >= num_units) break;
         const DsUnit U = ds_unit(u, p);
         const uint32_t buf = uc & 1u;
@@ -1094,7 +1104,7 @@ __global__ void __launch_bounds__(DqDsCfg<D>::kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int u = unit_of(k);
+        const int u = unit_of(k, p.q_tab);
         if (u >= num_units) break;
         const DsUnit U = ds_unit(u, p);
         const int b = U.bh / p.H, h = U.bh - b * p.H;

@@ -128,7 +128,18 @@ struct BwdParams {
   // rows][8 queries], and dQ is formed from them; fixed-length batches, equal lengths
   void* ds;
   long long ds_tiles;
+  // dS mode: per-CTA work lists of the dK/dV kernel and of the dQ pass (bwd_unit_table), or
+  // nullptr for the round-robin order
+  const int* kv_tab;
+  const int* q_tab;
 };
+
+// Work lists of the backward's dK/dV kernel (kind 1: units u = kb * BH + bh) or of the dQ pass
+// from stored dS (kind 2: units u = r * BH + bh, query block n_blocks - 1 - r causal, else r),
+// in the form of fwd_unit_schedule: longest first within groups of heads whose streamed tensors
+// (Q and dO, or K) fit 32 MB, dealt by greedy list scheduling; fixed-length batches only.
+bool bwd_unit_schedule(const BwdParams& p, int kind, int d, int grid, std::vector<int>* out);
+const int* bwd_unit_table(const BwdParams& p, int kind, int d, int grid, cudaStream_t stream);
 
 cudaError_t setup_bwd_kernels();
 // D and LSE*log2e into the workspace, then dK/dV and dQ; q/k/v/dout are 4-D maps as for the
