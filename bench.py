@@ -783,7 +783,9 @@ def varlen_section(args, dev, rank):
 
 
 def bwd_section(args, dev, rank):
-    """Times attn_bwd on the headline workload (device-resident inputs, bf16 gradients)."""
+    """Times the backward on the headline workload (device-resident inputs, bf16 gradients):
+    attn_bwd_ds (dS kept in a 2.2 GB workspace, five products) as the line's figure, and
+    attn_bwd (dQ recomputes S and dP, a 2 MB workspace) beside it."""
     import torch
     import exact_attention_100_b200 as ea
     from exact_attention_100_b200.inputs import normal_qkv, normal_dout
@@ -795,55 +797,40 @@ def bwd_section(args, dev, rank):
     stream = torch.cuda.current_stream()
     o, lse = ea.attn_fwd(q, k, v, causal=causal, stream=stream)
     dq, dk, dv = (torch.empty_like(q) for _ in range(3))
-    ws = torch.empty(ea.attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device=dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-
-    def step():
-        ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal=causal, stream=stream)
-
-    for _ in range(3):
-        step()
     steps = max(3, min(args.steps, 50))
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    for i in range(steps):
-        flush.fill_(float(i))
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    assert ea.attn_device_status() == ea.ATTN_OK
-    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
-    flops = 2.5 * attn_flops(B, H, N, d, causal)  # dV, dP, dS-recompute S, dK, dQ: five N x N x d products
-    peaks = load_peaks()
-    tf = flops / (ms * 1e-3) / 1e12
-    out = {"workload": "bf16 attention bwd B=2 H=16 N=8192 d=128 causal (dQ, dK, dV from O, LSE, dO)",
-           "ms": ms, "achieved_tflops": tf, "peak_tflops": float(peaks["bf16_tflops"]),
-           "frac": tf / float(peaks["bf16_tflops"]), "bound": "tensor",
-           "flops_per_call": flops, "flops_note": "algorithmic 2.5 x forward (five products); attn_bwd "
-                                                "recomputes S and dP a second time for dQ",
-           "launches_per_call": 3, "peak_source": peaks["source"]}
-    # the same gradients with dS kept in the workspace (attn_bwd_ds: five products, 2.2 GB)
+
+    def timed(step):
+        for _ in range(3):
+            step()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(float(i))
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        assert ea.attn_device_status() == ea.ATTN_OK
+        return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+    ws = torch.empty(ea.attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device=dev)
+    ms_rc = timed(lambda: ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal=causal, stream=stream))
     ws_ds = torch.empty(ea.attn_bwd_ds_workspace_bytes(B, H, N, causal), dtype=torch.uint8, device=dev)
-
-    def step_ds():
-        ea.attn_bwd_ds(q, k, v, o, lse, do, dq, dk, dv, ws_ds, causal=causal, stream=stream)
-
-    for _ in range(3):
-        step_ds()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    for i in range(steps):
-        flush.fill_(float(i))
-        evs[i][0].record(stream)
-        step_ds()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    assert ea.attn_device_status() == ea.ATTN_OK
-    ms_ds = float(np.mean([a.elapsed_time(b) for a, b in evs]))
-    tf_ds = flops / (ms_ds * 1e-3) / 1e12
-    out["ds"] = {"ms": ms_ds, "achieved_tflops": tf_ds, "frac": tf_ds / float(peaks["bf16_tflops"]),
-                 "workspace_bytes": int(ws_ds.numel()), "vs_recompute": ms / ms_ds,
-                 "note": "attn_bwd_ds: the dK/dV kernel stores each bf16 dS tile, a third kernel streams "
-                         "them with K through the tensor cores for dQ (no recomputation)"}
+    ms = timed(lambda: ea.attn_bwd_ds(q, k, v, o, lse, do, dq, dk, dv, ws_ds, causal=causal, stream=stream))
+    flops = 2.5 * attn_flops(B, H, N, d, causal)  # dV, dP, S, dK, dQ: five N x N x d products
+    peaks = load_peaks()
+    tf, tf_rc = flops / (ms * 1e-3) / 1e12, flops / (ms_rc * 1e-3) / 1e12
+    out = {"workload": "bf16 attention bwd B=2 H=16 N=8192 d=128 causal (dQ, dK, dV from O, LSE, dO)",
+           "entry_point": "attn_bwd_ds", "ms": ms, "achieved_tflops": tf,
+           "peak_tflops": float(peaks["bf16_tflops"]), "frac": tf / float(peaks["bf16_tflops"]), "bound": "tensor",
+           "flops_per_call": flops, "flops_note": "algorithmic 2.5 x forward (five products)",
+           "workspace_bytes": int(ws_ds.numel()), "launches_per_call": 3, "peak_source": peaks["source"],
+           "note": "attn_bwd_ds: the dK/dV kernel stores each bf16 dS tile, a third kernel streams them with K "
+                   "through the tensor cores for dQ (no recomputation)",
+           "recompute": {"entry_point": "attn_bwd", "ms": ms_rc, "achieved_tflops": tf_rc,
+                         "frac": tf_rc / float(peaks["bf16_tflops"]), "workspace_bytes": int(ws.numel() * 4),
+                         "note": "dQ recomputes S and dP: seven products on the tensor cores"},
+           "ds_vs_recompute": ms_rc / ms}
     del ws_ds
     return out
 
