@@ -63,6 +63,34 @@ class _Emulated:
 
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("world", [1, 2, 4])
+def test_ring_driver_zigzag_on_one_gpu(world, causal):
+    """The zig-zag layout with the library's kernels, each rank emulated on one GPU: rank r holds
+    chunks r and 2W - 1 - r of 2W; its rows of the whole-sequence result within the bf16 bars."""
+    from exact_attention_100_b200.ring import zigzag_chunks
+    B, H, N, d = 1, 2, 1024, 128
+    q, k, v = normal_qkv(B, H, N, d, seed=10 + world)
+    tq, tk, tv = (torch.from_numpy(a).to(torch.bfloat16).cuda() for a in (q, k, v))
+    c = N // (2 * world)
+    rows = [np.r_[a * c:(a + 1) * c, b * c:(b + 1) * c] for a, b in (zigzag_chunks(r, world) for r in range(world))]
+    idx = [torch.from_numpy(r).cuda() for r in rows]
+    held = [(tk[:, :, i].contiguous(), tv[:, :, i].contiguous()) for i in idx]
+    bufs = [torch.stack([torch.stack([kk[:, :, :c], vv[:, :, :c]]), torch.stack([kk[:, :, c:], vv[:, :, c:]])])
+            for kk, vv in held]
+    scale = 1.0 / math.sqrt(d)
+    o_ref, lse_ref = attention_ref(q, k, v, scale, causal)
+    for r in range(world):
+        o, lse = ring_attention_fwd(tq[:, :, idx[r]].contiguous(), held[r][0], held[r][1], causal=causal,
+                                    scale=scale, rank=r, world=world, exchange=_Emulated(bufs, r), layout="zigzag")
+        torch.cuda.synchronize()
+        assert ea.attn_device_status() == ea.ATTN_OK
+        err = np.abs(o.double().cpu().numpy() - o_ref[:, :, rows[r]])
+        assert err.max() <= O_MAX_ABS and err.mean() <= O_MEAN_ABS, (r, err.max())
+        rel = np.abs(lse.double().cpu().numpy() - lse_ref[:, :, rows[r]]) / np.abs(lse_ref[:, :, rows[r]])
+        assert rel.max() <= LSE_REL, (r, rel.max())
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("world", [1, 2, 4])
 def test_ring_driver_on_one_gpu(world, causal):
     B, H, N, d = 1, 2, 1024, 128
     q, k, v = normal_qkv(B, H, N, d, seed=world)
