@@ -746,6 +746,27 @@ def varlen_section(args, dev, rank):
     assert ea.attn_device_status() == ea.ATTN_OK
     bms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
     btf = 2.5 * flops / (bms * 1e-3) / 1e12
+    # the same backward with dS kept in the workspace (attn_bwd_varlen_ds)
+    ws_ds = torch.empty(ea.attn_bwd_varlen_ds_workspace_bytes(len(lens), H, max(lens), max(lens)), dtype=torch.uint8,
+                        device=dev)
+
+    def dsstep():
+        ea.attn_bwd_varlen_ds(q, k, v, o, lse, dout, cu_q, cu_k, max(lens), max(lens), dq=g[0], dk=g[1], dv=g[2],
+                              workspace=ws_ds, causal=causal, stream=stream)
+
+    for _ in range(3):
+        dsstep()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        dsstep()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+    dms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    dtf = 2.5 * flops / (dms * 1e-3) / 1e12
+    del ws_ds
     # the E4M3 forward of the same packed batch: codes and per-sequence block scales from the
     # packed pre-kernel (Q, K through H D), then attn_fwd_fp8_varlen
     from exact_attention_100_b200.inputs import hadamard_signs
@@ -774,8 +795,11 @@ def varlen_section(args, dev, rank):
             "frac": tf / float(peaks["bf16_tflops"]), "bound": "tensor", "flops_per_call": flops,
             "flops_note": "sum over sequences of 4 H d N^2 / 2 (causal), as the headline counts",
             "peak_source": peaks["source"],
-            "bwd": {"ms": bms, "achieved_tflops": btf, "frac": btf / float(peaks["bf16_tflops"]),
-                    "flops_note": "2.5 x the forward count (five products), bf16 gradients, 3 launches"},
+            "bwd": {"entry_point": "attn_bwd_varlen_ds", "ms": dms, "achieved_tflops": dtf,
+                    "frac": dtf / float(peaks["bf16_tflops"]),
+                    "flops_note": "2.5 x the forward count (five products), bf16 gradients, 3 launches",
+                    "recompute": {"entry_point": "attn_bwd_varlen", "ms": bms, "achieved_tflops": btf,
+                                  "frac": btf / float(peaks["bf16_tflops"])}},
             "fp8_fwd": {"ms": fms, "achieved_tflops": ftf, "vs_bf16": ms / fms,
                         "note": "attn_fwd_fp8_varlen on the same batch (E4M3 codes and per-sequence "
                                 "128-row block scales from attn_hadamard_quant_qkv_varlen; the "

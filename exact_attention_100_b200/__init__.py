@@ -71,6 +71,10 @@ def lib() -> ctypes.CDLL:
         L.attn_bwd_strided.restype = i
         L.attn_bwd_varlen.argtypes = [vp] * 12 + [i, i, i, i, i, i, i, vp, f, i, i, vp]
         L.attn_bwd_varlen.restype = i
+        L.attn_bwd_varlen_ds.argtypes = [vp] * 12 + [i, i, i, i, i, i, i, vp, f, i, i, vp]
+        L.attn_bwd_varlen_ds.restype = i
+        L.attn_bwd_varlen_ds_workspace_bytes.argtypes = [i, i, i, i]
+        L.attn_bwd_varlen_ds_workspace_bytes.restype = ctypes.c_ulonglong
         L.attn_hadamard_quant.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
         L.attn_hadamard_quant.restype = i
         L.attn_hadamard_quant_qkv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
@@ -399,6 +403,25 @@ def attn_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqle
     """The backward of :func:`attn_fwd_varlen`: ``q``, ``o``, ``dout`` [total_q, H, d], ``k``, ``v``
     [total_k, H, d] (bf16, row and head strides free, last dimension contiguous), ``lse``
     [H, total_q].  Returns ``(dq, dk, dv)``."""
+    return _bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, dq, dk, dv,
+                       workspace, scale, causal, g_dtype, stream, False)
+
+
+def attn_bwd_varlen_ds_workspace_bytes(B, H, max_seqlen_q, max_seqlen_k):
+    """Bytes of the workspace :func:`attn_bwd_varlen_ds` needs (0 if too many tiles)."""
+    return int(lib().attn_bwd_varlen_ds_workspace_bytes(B, H, int(max_seqlen_q), int(max_seqlen_k)))
+
+
+def attn_bwd_varlen_ds(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, dq=None,
+                       dk=None, dv=None, workspace=None, scale=None, causal=False, g_dtype=None, stream=None):
+    """:func:`attn_bwd_varlen` with the dS tiles kept in the workspace (a uint8 tensor of
+    :func:`attn_bwd_varlen_ds_workspace_bytes` bytes), as :func:`attn_bwd_ds` for fixed lengths."""
+    return _bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, dq, dk, dv,
+                       workspace, scale, causal, g_dtype, stream, True)
+
+
+def _bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, dq, dk, dv,
+                workspace, scale, causal, g_dtype, stream, ds):
     import torch
     if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape or o.shape != q.shape or dout.shape != q.shape:
         raise ValueError("expected q, o, dout [total_q, H, d] and k, v [total_k, H, d]")
@@ -426,15 +449,20 @@ def attn_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqle
             raise ValueError("gradients must have their input's shape and a contiguous last dimension")
     mq = min(int(max_seqlen_q), total_q)
     if workspace is None:
-        workspace = torch.empty(attn_bwd_workspace_bytes(B, H, mq) // 4, dtype=torch.float32, device=q.device)
+        if ds:
+            nbytes = attn_bwd_varlen_ds_workspace_bytes(B, H, int(max_seqlen_q), int(max_seqlen_k))
+            if nbytes == 0:
+                raise ValueError("too many dS tiles for this batch: use attn_bwd_varlen")
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+        else:
+            workspace = torch.empty(attn_bwd_workspace_bytes(B, H, mq) // 4, dtype=torch.float32, device=q.device)
     strides = (ctypes.c_longlong * 16)(*[int(x) for t in (q, k, v, o, dout, dq, dk, dv) for x in t.stride()[:2]])
     gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
-    _check(lib().attn_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
-                                 _ptr(dv), _ptr(workspace), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, H, total_q,
-                                 total_k, int(max_seqlen_q), int(max_seqlen_k), d,
-                                 ctypes.cast(strides, ctypes.c_void_p), s, int(bool(causal)), gcode,
-                                 _stream_ptr(stream)), "attn_bwd_varlen")
+    fn, name = (lib().attn_bwd_varlen_ds, "attn_bwd_varlen_ds") if ds else (lib().attn_bwd_varlen, "attn_bwd_varlen")
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+              _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, H, total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), d,
+              ctypes.cast(strides, ctypes.c_void_p), s, int(bool(causal)), gcode, _stream_ptr(stream)), name)
     return dq, dk, dv
 
 

@@ -656,6 +656,18 @@ struct Packed {
 // Bytes of the dS-mode workspace: D and LSE * log2 e (padded rows), rounded up to 1024, then the
 // bf16 dS^T tiles of every (batch, head): n_b (n_b + 1) / 2 causal, n_b^2 otherwise, 32 KB each.
 // 0 if a size is not positive or the tiles cannot be indexed with int.
+// The same for packed batches: a rectangle of ceil(max_q / 128) x ceil(max_k / 128) tiles per
+// (sequence, head).
+unsigned long long bwd_varlen_ds_workspace_bytes(int B, int H, int max_q, int max_k) {
+  if (B <= 0 || H <= 0 || max_q <= 0 || max_k <= 0) return 0ull;
+  const unsigned long long bh = static_cast<unsigned long long>(B) * static_cast<unsigned long long>(H);
+  const unsigned long long nb = (static_cast<unsigned long long>(max_q) + 127ull) / 128ull;
+  const unsigned long long nbk = (static_cast<unsigned long long>(max_k) + 127ull) / 128ull;
+  if (bh * nb * nbk >= 0x7FFFFFFFull) return 0ull;
+  const unsigned long long head = (2ull * bh * nb * 128ull * 4ull + 1023ull) / 1024ull * 1024ull;
+  return head + bh * nb * nbk * 128ull * 128ull * 2ull;
+}
+
 unsigned long long bwd_ds_workspace_bytes(int B, int H, int N, int causal) {
   if (B <= 0 || H <= 0 || N <= 0 || (causal != 0 && causal != 1)) return 0ull;
   const unsigned long long bh = static_cast<unsigned long long>(B) * static_cast<unsigned long long>(H);
@@ -727,19 +739,31 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const v
   p.total_k = pk ? pk->total_k : 0;
   p.ds = nullptr;
   p.ds_tiles = 0;
+  p.ds_rect = 0;
+  p.ds_nbk = 0;
   p.kv_tab = p.q_tab = nullptr;
   if (ds_mode) {
-    // the dS^T tiles follow D and LSE in the workspace (bwd_ds_workspace_bytes)
+    // the dS^T tiles follow D and LSE in the workspace (bwd_ds_workspace_bytes): a triangle or a
+    // square of tiles per (batch, head); packed batches: a rectangle of n_blocks x nbk tiles per
+    // (sequence, head), whatever each sequence's lengths
     const long long nb = n_blocks;
-    p.ds_tiles = causal ? nb * (nb + 1) / 2 : nb * nb;
+    if (pk != nullptr) {
+      p.ds_rect = 1;
+      p.ds_nbk = static_cast<int>(nbk);
+      p.ds_tiles = nb * nbk;
+    } else {
+      p.ds_tiles = causal ? nb * (nb + 1) / 2 : nb * nb;
+    }
     const size_t head = (2ull * static_cast<size_t>(p.BH) * p.n_pad * 4ull + 1023ull) / 1024ull * 1024ull;
     p.ds = static_cast<uint8_t*>(workspace) + head;
-    // work lists: the units of groups of heads whose streamed tensors fit L2 run together
-    const int kv_units = p.BH * p.nbk, q_units = p.BH * p.n_blocks;
-    p.kv_tab = ea::bwd_unit_table(p, 1, d, kv_units < st->num_sms ? kv_units : st->num_sms,
-                                  static_cast<cudaStream_t>(stream));
-    p.q_tab = ea::bwd_unit_table(p, 2, d, q_units < st->num_sms ? q_units : st->num_sms,
-                                 static_cast<cudaStream_t>(stream));
+    if (pk == nullptr) {
+      // work lists: the units of groups of heads whose streamed tensors fit L2 run together
+      const int kv_units = p.BH * p.nbk, q_units = p.BH * p.n_blocks;
+      p.kv_tab = ea::bwd_unit_table(p, 1, d, kv_units < st->num_sms ? kv_units : st->num_sms,
+                                    static_cast<cudaStream_t>(stream));
+      p.q_tab = ea::bwd_unit_table(p, 2, d, q_units < st->num_sms ? q_units : st->num_sms,
+                                   static_cast<cudaStream_t>(stream));
+    }
     if (ea::launch_attn_bwd_ds(d, mq, mk, mv, mdo, p, st->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
       return ATTN_ERR_CUDA;
     g_launches.fetch_add(3);
@@ -824,6 +848,35 @@ int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, 
   const Packed pk{cu_seqlens_q, cu_seqlens_k, total_q, total_k};
   return bwd_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, max_seqlen_q, max_seqlen_k, d, st8, &pk, scale,
                   causal, g_dtype, stream);
+}
+
+unsigned long long attn_bwd_varlen_ds_workspace_bytes(int B, int H, int max_seqlen_q, int max_seqlen_k) {
+  return bwd_varlen_ds_workspace_bytes(B, H, max_seqlen_q, max_seqlen_k);
+}
+
+int attn_bwd_varlen_ds(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                       void* dq, void* dk, void* dv, void* workspace, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                       int B, int H, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                       const long long* strides, float scale, int causal, int g_dtype, void* stream) {
+  if (!cu_seqlens_q || !cu_seqlens_k || !strides || B <= 0 || H <= 0) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
+    return ATTN_ERR_INVALID_ARG;
+  constexpr int kMaxRows = 0x7FFFFFFF - (1 << 20);
+  if (total_q <= 0 || total_k <= 0 || total_q > kMaxRows || total_k > kMaxRows || max_seqlen_q <= 0 ||
+      max_seqlen_k <= 0 || max_seqlen_q > kMaxRows || max_seqlen_k > kMaxRows)
+    return ATTN_ERR_INVALID_ARG;
+  if (bwd_varlen_ds_workspace_bytes(B, H, max_seqlen_q, max_seqlen_k) == 0ull) return ATTN_ERR_INVALID_ARG;
+  if (max_seqlen_q > total_q) max_seqlen_q = total_q;  // no sequence is longer than its tensor
+  if (max_seqlen_k > total_k) max_seqlen_k = total_k;
+  Strides st8[8];
+  for (int t = 0; t < 8; ++t) {
+    const bool key_side = t == 1 || t == 2 || t == 6 || t == 7;
+    const long long s3[3] = {8, strides[2 * t + 1], strides[2 * t]};  // {batch (unused), head, row}
+    if (!canonical_strides(s3, 1, H, key_side ? total_k : total_q, &st8[t])) return ATTN_ERR_INVALID_ARG;
+  }
+  const Packed pk{cu_seqlens_q, cu_seqlens_k, total_q, total_k};
+  return bwd_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, max_seqlen_q, max_seqlen_k, d, st8, &pk, scale,
+                  causal, g_dtype, stream, true);
 }
 
 int attn_device_status(void* stream) {

@@ -243,6 +243,13 @@ __device__ __forceinline__ int unit_of(int k, const int* tab) {
   return unit_of(k);
 }
 
+// dS mode: index of tile (query block i, key block kb) of batch*head bh in the workspace
+__device__ __forceinline__ long long ds_tile_index(const BwdParams& p, int bh, int i, int kb) {
+  const long long base = static_cast<long long>(bh) * p.ds_tiles;
+  if (p.ds_rect) return base + static_cast<long long>(i) * p.ds_nbk + kb;
+  return base + (p.causal ? static_cast<long long>(i) * (i + 1) / 2 + kb : static_cast<long long>(i) * p.n_blocks + kb);
+}
+
 // dK/dV unit u: key block kb of head bh and the first query block i0 that sees any of its keys
 // (causal, bottom-right: query r sees key c iff c <= r + off); i0 >= n_blocks: no query does.
 // `present`: the block lies inside its sequence (always, unless packed).
@@ -471,13 +478,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         // columns [8j, 8j + 8) for all 128 key rows, then chunk j + 1), so that a warp's store of
         // one chunk writes 512 contiguous bytes; the layout is the tensor core's non-swizzled
         // MN-major operand layout, which the dQ pass copies into shared memory as it is
+        // A key row past the sequence end stores zeros: the dQ pass multiplies the tile by a K tile
+        // whose rows there are the next sequence's keys (packed) or TMA's zero fill, and a finite
+        // zero keeps both out of dQ (an unmasked score of such a row need not even be finite).
         uint8_t* ds_tile = nullptr;
-        if constexpr (DS) {
-          const long long tile = static_cast<long long>(U.bh) * p.ds_tiles +
-                                 (p.causal ? static_cast<long long>(i) * (i + 1) / 2 + kb
-                                           : static_cast<long long>(i) * nb + kb);
-          ds_tile = static_cast<uint8_t*>(p.ds) + tile * (128 * 128 * 2) + row * 16;
-        }
+        [[maybe_unused]] const bool ds_keep = key_g < S.Nk;
+        if constexpr (DS) ds_tile = static_cast<uint8_t*>(p.ds) + ds_tile_index(p, U.bh, i, kb) * (128 * 128 * 2) + row * 16;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t dp[32];
@@ -498,7 +504,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4)  // chunk 8h + 4c + v4: queries 64h + 32c + 8 v4 .. + 8
               *reinterpret_cast<uint4*>(ds_tile + (8 * h + 4 * c + v4) * 2048) =
-                  make_uint4(dk[4 * v4], dk[4 * v4 + 1], dk[4 * v4 + 2], dk[4 * v4 + 3]);
+                  ds_keep ? make_uint4(dk[4 * v4], dk[4 * v4 + 1], dk[4 * v4 + 2], dk[4 * v4 + 3])
+                          : make_uint4(0u, 0u, 0u, 0u);
           }
         }
         tmem_st_wait();
@@ -981,23 +988,7 @@ struct DqDsCfg {
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
 };
 
-// dS-mode dQ unit u: head bh, query block i, n key blocks, and its first tile's index
-struct DsUnit {
-  int bh, i, n;
-  long long tile0;
-};
-__device__ __forceinline__ DsUnit ds_unit(int u, const BwdParams& p) {
-  DsUnit U;
-  U.bh = u % p.BH;
-  const int r = u / p.BH;
-  U.i = p.causal ? p.n_blocks - 1 - r : r;
-  U.n = p.causal ? U.i + 1 : p.n_blocks;
-  U.tile0 = static_cast<long long>(U.bh) * p.ds_tiles +
-            (p.causal ? static_cast<long long>(U.i) * (U.i + 1) / 2 : static_cast<long long>(U.i) * p.n_blocks);
-  return U;
-}
-
-template <int D>
+template <int D, bool VL>
 __global__ void __launch_bounds__(DqDsCfg<D>::kThreads, 1)
     bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tmK, const BwdParams p) {
   using C = DqDsCfg<D>;
@@ -1050,15 +1041,23 @@ __global__ void __launch_bounds__(DqDsCfg<D>::kThreads, 1)
     for (int k = 0; ok; ++k) {
       const int u = unit_of(k, p.q_tab);
       if (u >= num_units) break;
-      const DsUnit U = ds_unit(u, p);
+      const QUnit U = q_unit<VL>(u, p);
+      if constexpr (VL) {
+        if (!U.present) continue;  // past its sequence's queries: every role skips it
+      }
+      const BSeq& S = U.S;
+      const int q_g = U.qb * 128 + row;
+      const size_t off_q = static_cast<size_t>(S.bc * p.dq_sb + S.h * p.dq_sh +
+                                               (S.q0 + static_cast<long long>(q_g)) * p.dq_sn);
+      if (U.n == 0) {  // these queries see no key: dQ = 0 (no products, no TMEM buffer)
+        if (q_g < S.N) zero_row<D>(p.dq, off_q, p.g_fp32 != 0);
+        continue;
+      }
       const uint32_t buf = uc & 1u;
       ok = warp_all(wait_bar(&dq_done[buf], (uc >> 1) & 1u, ab));
       if (!ok) break;
       tc_fence_after();
-      const int b = U.bh / p.H, h = U.bh - b * p.H;
-      const int q_g = U.i * 128 + row;
-      const size_t off_q = static_cast<size_t>(b * p.dq_sb + h * p.dq_sh + static_cast<long long>(q_g) * p.dq_sn);
-      store_row<D>(lane_base + buf * D, p.dq, off_q, p.scale, p.g_fp32 != 0, q_g < p.N);
+      store_row<D>(lane_base + buf * D, p.dq, off_q, p.scale, p.g_fp32 != 0, q_g < S.N);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) bar_arrive(&dq_free[buf]);
@@ -1073,7 +1072,11 @@ __global__ void __launch_bounds__(DqDsCfg<D>::kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int u = unit_of(k, p.q_tab);
         if (u >= num_units) break;
-        const DsUnit U = ds_unit(u, p);
+        const QUnit U = q_unit<VL>(u, p);
+        if constexpr (VL) {
+          if (!U.present) continue;
+        }
+        if (U.n == 0) continue;
         const uint32_t buf = uc & 1u;
         // the epilogue of the unit before last must be done reading this dQ buffer
         if (!(ok = wait_bar(&dq_free[buf], ((uc >> 1) & 1u) ^ 1u, ab))) break;
@@ -1106,15 +1109,19 @@ __global__ void __launch_bounds__(DqDsCfg<D>::kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int u = unit_of(k, p.q_tab);
         if (u >= num_units) break;
-        const DsUnit U = ds_unit(u, p);
-        const int b = U.bh / p.H, h = U.bh - b * p.H;
+        const QUnit U = q_unit<VL>(u, p);
+        if constexpr (VL) {
+          if (!U.present) continue;
+        }
+        const BSeq& S = U.S;
         for (int j = 0; j < U.n && ok; ++j, ++it) {
           const uint32_t s = it % C::kSlots;
           if (!(ok = wait_bar(&empty[s], ((it / C::kSlots) & 1u) ^ 1u, ab))) break;
           uint8_t* dst = smem + s * C::kSlotBytes;
           bar_arrive_expect_tx(&full[s], C::kSlotBytes);
-          bulk_load_g2s(dst, static_cast<const uint8_t*>(p.ds) + (U.tile0 + j) * C::kDsBytes, C::kDsBytes, &full[s]);
-          load_tile<D>(dst + C::kDsBytes, &tmK, &full[s], j * 128, h, b);
+          bulk_load_g2s(dst, static_cast<const uint8_t*>(p.ds) + ds_tile_index(p, U.bh, U.qb, j) * C::kDsBytes,
+                        C::kDsBytes, &full[s]);
+          load_tile<D>(dst + C::kDsBytes, &tmK, &full[s], S.k0 + j * 128, S.h, S.bc);
         }
       }
       // every issued copy lands before the CTA can exit
@@ -1139,35 +1146,33 @@ cudaError_t setup_d() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(bwd_dq_kernel<D, VL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              DqCfg<D>::kSmemAlloc);
-  if constexpr (!VL) {
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DkdvCfg<D>::kSmemAlloc);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(bwd_dq_ds_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DqDsCfg<D>::kSmemAlloc);
-  }
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, VL, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DkdvCfg<D>::kSmemAlloc);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(bwd_dq_ds_kernel<D, VL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DqDsCfg<D>::kSmemAlloc);
   return e;
 }
 
-template <int D>
+template <int D, bool VL>
 cudaError_t launch_d_ds(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& dout,
                         const BwdParams& p, int num_sms, cudaStream_t stream) {
   const long long rows = static_cast<long long>(p.BH) * p.n_pad;
   const long long threads = rows * (D / 16);
   const long long blocks = (threads + 255) / 256;
-  if (blocks > 0x7FFFFFFFLL || p.ds == nullptr || p.cu_q != nullptr) return cudaErrorInvalidValue;
-  bwd_prep_kernel<D, false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  if (blocks > 0x7FFFFFFFLL || p.ds == nullptr || (p.cu_q != nullptr) != VL) return cudaErrorInvalidValue;
+  bwd_prep_kernel<D, VL><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int kv_units = p.BH * p.nbk;
   const int kv_grid = kv_units < num_sms ? kv_units : num_sms;
-  bwd_dkdv_kernel<D, false, true><<<kv_grid, BwdCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(q, k, v, dout, p);
+  bwd_dkdv_kernel<D, VL, true><<<kv_grid, BwdCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(q, k, v, dout, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int q_units = p.BH * p.n_blocks;
   const int q_grid = q_units < num_sms ? q_units : num_sms;
-  bwd_dq_ds_kernel<D><<<q_grid, DqDsCfg<D>::kThreads, DqDsCfg<D>::kSmemAlloc, stream>>>(k, p);
+  bwd_dq_ds_kernel<D, VL><<<q_grid, DqDsCfg<D>::kThreads, DqDsCfg<D>::kSmemAlloc, stream>>>(k, p);
   return cudaGetLastError();
 }
 
@@ -1220,11 +1225,14 @@ cudaError_t launch_attn_bwd(int d, const CUtensorMap& q, const CUtensorMap& k, c
 cudaError_t launch_attn_bwd_ds(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                                const CUtensorMap& dout, const BwdParams& p, int num_sms,
                                cudaStream_t stream) {
+  const bool vl = p.cu_q != nullptr;
   switch (d) {
     case 64:
-      return launch_d_ds<64>(q, k, v, dout, p, num_sms, stream);
+      return vl ? launch_d_ds<64, true>(q, k, v, dout, p, num_sms, stream)
+                : launch_d_ds<64, false>(q, k, v, dout, p, num_sms, stream);
     case 128:
-      return launch_d_ds<128>(q, k, v, dout, p, num_sms, stream);
+      return vl ? launch_d_ds<128, true>(q, k, v, dout, p, num_sms, stream)
+                : launch_d_ds<128, false>(q, k, v, dout, p, num_sms, stream);
     default:
       return cudaErrorInvalidValue;
   }

@@ -128,6 +128,10 @@ struct BwdParams {
   // rows][8 queries], and dQ is formed from them; fixed-length batches, equal lengths
   void* ds;
   long long ds_tiles;
+  // packed batches: tiles indexed i * ds_nbk + kb per (sequence, head), ds_tiles = n_blocks *
+  // ds_nbk (ds_rect = 1), for any per-sequence lengths
+  int ds_rect;
+  int ds_nbk;
   // dS mode: per-CTA work lists of the dK/dV kernel and of the dQ pass (bwd_unit_table), or
   // nullptr for the round-robin order
   const int* kv_tab;

@@ -475,6 +475,29 @@ int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, 
                     const long long* strides, float scale, int causal, int g_dtype, void* stream);
 
 /*
+ * attn_bwd_varlen_ds_workspace_bytes -- size of the workspace attn_bwd_varlen_ds needs: the
+ * float32 rows of attn_bwd_workspace_bytes(B, H, max_seqlen_q) rounded up to 1024 bytes, then
+ * B * H * ceil(max_seqlen_q / 128) * ceil(max_seqlen_k / 128) bf16 tiles of 32 KB (a rectangle
+ * per sequence and head, whatever the sequences' lengths; only the visible tiles are written).
+ * Returns 0 if a size is not positive or there are 2^31 - 1 tiles or more.
+ */
+unsigned long long attn_bwd_varlen_ds_workspace_bytes(int B, int H, int max_seqlen_q, int max_seqlen_k);
+
+/*
+ * attn_bwd_varlen_ds -- attn_bwd_varlen that keeps dS in the workspace and forms dQ from it, as
+ * attn_bwd_ds does for fixed lengths (five products instead of seven).
+ *   workspace   device, 16-byte aligned, attn_bwd_varlen_ds_workspace_bytes(B, H, max_seqlen_q,
+ *               max_seqlen_k) bytes; owned by the caller and overwritten.
+ * Other arguments, offsets rules and their reporting as for attn_bwd_varlen.  dK and dV are
+ * bit-identical to attn_bwd_varlen's; the bounds of attn_bwd hold for every sequence.
+ */
+int attn_bwd_varlen_ds(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                       const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                       const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H,
+                       int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                       const long long* strides, float scale, int causal, int g_dtype, void* stream);
+
+/*
  * attn_fwd_noalloc -- attn_fwd for callers that cannot allocate device memory.  The pages have
  * no counterpart; it exists for this library's users.
  *

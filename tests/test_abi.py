@@ -37,7 +37,8 @@ def test_header_declares_the_boundary():
                             "attn_selftest_wait_timeout", "attn_noalloc_status",
                             "attn_noalloc_selftest_wait_timeout", "attn_hadamard_quant_qkv_strided",
                             "attn_fwd_fp8_strided", "attn_fwd_schedule", "attn_hadamard_quant_qkv_varlen",
-                            "attn_fwd_fp8_varlen", "attn_bwd_ds_workspace_bytes", "attn_bwd_ds"])
+                            "attn_fwd_fp8_varlen", "attn_bwd_ds_workspace_bytes", "attn_bwd_ds",
+                            "attn_bwd_varlen_ds_workspace_bytes", "attn_bwd_varlen_ds"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -473,6 +474,29 @@ def test_bwd_ds_rejects_bad_arguments(L):
     assert f(*a) == ea.ATTN_ERR_INVALID_ARG
 
 
+def test_bwd_varlen_ds_workspace_bytes_and_rejections(L):
+    f = L.attn_bwd_varlen_ds_workspace_bytes
+    head = (2 * 128 * 27 * 128 * 4 + 1023) // 1024 * 1024
+    assert f(8, 16, 3369, 3369) == head + 128 * 27 * 27 * 32768
+    assert f(1, 1, 1, 300) == 1024 + 3 * 32768
+    for a in [(0, 1, 1, 1), (1, 0, 1, 1), (1, 1, 0, 1), (1, 1, 1, 0)]:
+        assert f(*a) == 0, a
+    g = L.attn_bwd_varlen_ds
+    good = [16 * 128, 128] * 8
+    ok = [P, P, P, P, P, P2, P, P, P, P, P, P, 3, 16, 1000, 900, 500, 400, 128, _strides(good), 0.1, 1, 0, NULL]
+    for i in range(12):
+        a = list(ok)
+        a[i] = NULL
+        assert g(*a) == ea.ATTN_ERR_INVALID_ARG, i
+    for idx, val in [(12, 0), (13, 0), (14, 0), (15, 0), (16, 0), (17, 0), (20, 0.0), (21, 2)]:
+        a = list(ok)
+        a[idx] = val
+        assert g(*a) == ea.ATTN_ERR_INVALID_ARG, (idx, val)
+    a = list(ok)
+    a[18] = 256
+    assert g(*a) == ea.ATTN_ERR_UNSUPPORTED
+
+
 def test_bwd_rejects_bad_arguments(L):
     f = L.attn_bwd
     ok = [P, P, P, P, P, P2, P2, P2, P2, P2, 1, 1, 128, 128, 0.1, 0, 0, NULL]
@@ -518,5 +542,6 @@ def test_python_binding_has_same_names():
                  "attn_fwd_fp8_qk", "attn_merge_partials", "attn_selftest_wait_timeout", "attn_noalloc_status",
                  "attn_noalloc_selftest_wait_timeout", "attn_hadamard_quant_qkv_strided", "attn_fwd_fp8_strided",
                  "attn_fwd_schedule", "attn_hadamard_quant_qkv_varlen", "attn_fwd_fp8_varlen",
-                 "attn_bwd_ds_workspace_bytes", "attn_bwd_ds"]:
+                 "attn_bwd_ds_workspace_bytes", "attn_bwd_ds", "attn_bwd_varlen_ds_workspace_bytes",
+                 "attn_bwd_varlen_ds"]:
         assert callable(getattr(ea, name)), name

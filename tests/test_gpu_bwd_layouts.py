@@ -73,7 +73,7 @@ def test_strided_gradients_into_a_fused_buffer():
         assert torch.equal(a, b)
 
 
-def _packed_run(lq, lk, H, d, causal, seed, layout="plain"):
+def _packed_run(lq, lk, H, d, causal, seed, layout="plain", ds=False):
     q, k, v, cq, ck = normal_qkv_packed(lq, lk, H, d, seed=seed)
     do = np.random.default_rng(seed + 100).standard_normal(q.shape).astype(np.float32)
     from exact_attention_100_b200.inputs import round_to_bf16
@@ -87,10 +87,16 @@ def _packed_run(lq, lk, H, d, causal, seed, layout="plain"):
     tcq, tck = torch.from_numpy(cq).cuda(), torch.from_numpy(ck).cuda()
     scale = 1.0 / math.sqrt(d)
     o, lse = ea.attn_fwd_varlen(tq, tk, tv, tcq, tck, max(lq), scale=scale, causal=causal)
-    grads = ea.attn_bwd_varlen(tq, tk, tv, o, lse, tdo, tcq, tck, max(lq), max(lk), scale=scale, causal=causal,
-                               g_dtype=torch.float32)
+    bwd = ea.attn_bwd_varlen_ds if ds else ea.attn_bwd_varlen
+    grads = bwd(tq, tk, tv, o, lse, tdo, tcq, tck, max(lq), max(lk), scale=scale, causal=causal, g_dtype=torch.float32)
     torch.cuda.synchronize()
     assert ea.attn_device_status() == ea.ATTN_OK
+    if ds:
+        # dK and dV come from the same dK/dV arithmetic as attn_bwd_varlen: the same bits
+        ref = ea.attn_bwd_varlen(tq, tk, tv, o, lse, tdo, tcq, tck, max(lq), max(lk), scale=scale, causal=causal,
+                                 g_dtype=torch.float32)
+        torch.cuda.synchronize()
+        assert torch.equal(grads[1], ref[1]) and torch.equal(grads[2], ref[2])
     return (q, k, v, do, cq, ck, scale), (tq, tk, tv, tdo, o, lse), [g.cpu().numpy() for g in grads]
 
 
@@ -167,6 +173,41 @@ def test_packed_bench_batch_two_heads(causal):
             refs = attention_bwd_chunked_ref(qs, ks, vs, dos, scale, causal)
             o_ref, _ = attention_ref(qs, ks, vs, scale, causal)
             _check_grads([t(g) for g in grads], refs, _bounds(qs, ks, vs, dos, o_ref, scale, causal))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_packed_ds_matches_oracle(d, causal):
+    """attn_bwd_varlen_ds (dS kept in the workspace): the same bound per sequence, dK and dV the
+    bits of attn_bwd_varlen."""
+    lq = [300, 1, 129, 128, 513, 127]
+    inputs, _, grads = _packed_run(lq, lq, 2, d, causal, seed=15, ds=True)
+    _check_packed(inputs, grads, causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_packed_ds_lengths_differ_per_sequence(causal):
+    lq = [200, 0, 64, 700, 130, 5]
+    lk = [90, 17, 0, 260, 600, 1]
+    inputs, _, grads = _packed_run(lq, lk, 2, 128, causal, seed=16, ds=True)
+    _check_packed(inputs, grads, causal)
+
+
+def test_packed_ds_bench_batch_two_heads():
+    """The bench's packed workload through attn_bwd_varlen_ds, causal: every sequence of heads 0
+    and 15 against the float64 oracle under the derived bound."""
+    from bench import VARLEN_WORKLOAD, varlen_lengths
+    w = VARLEN_WORKLOAD
+    lens = varlen_lengths(w["total"], w["lo"], w["hi"], w["seed"])
+    (q, k, v, do, cq, ck, scale), _, grads = _packed_run(lens, lens, w["H"], w["d"], True, seed=w["seed"], ds=True)
+    for h in (0, w["H"] - 1):
+        for b in range(len(lens)):
+            q0, q1 = int(cq[b]), int(cq[b + 1])
+            t = lambda x: x[q0:q1, h][None, None]
+            qs, ks, vs, dos = t(q), t(k), t(v), t(do)
+            refs = attention_bwd_chunked_ref(qs, ks, vs, dos, scale, True)
+            o_ref, _ = attention_ref(qs, ks, vs, scale, True)
+            _check_grads([t(g) for g in grads], refs, _bounds(qs, ks, vs, dos, o_ref, scale, True))
 
 
 def test_packed_bad_offsets_are_reported():
