@@ -455,6 +455,369 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Rotary embedding + transform + quantisation for d = 64 and 128 (d = 256 keeps the kernel above).
+//
+// One thread holds a whole row, so that the rotation (coordinates i and i + d/2) and every
+// butterfly stage stay inside the thread, in the textbook stage order.  The 128 x d/2 slice of
+// each table that a 128-row block needs is staged once per position block in shared memory,
+// position-major with its 16-byte chunks permuted so that the 8 rows of a quarter warp read
+// distinct banks; the units are ordered position block first, so that one staged slice serves
+// every head and tensor at those positions (the tables are read from DRAM once).  A CTA works on
+// kSlots blocks at a time, one 128-thread slot each, with its own TMA buffers, barrier phases and
+// named barrier; with one buffer per slot (d = 128, where a row takes the registers of two) the
+// next block's load is issued as soon as the slot has unpacked the current one.
+//
+// Rounding is that of the oracle's composition: products and the sum of the rotation each
+// rounded, the sign flips of D exact and applied to the rotated values, each butterfly rounded
+// once.  A packed f32x2 multiply is fused by the assembler into a following packed add or sub
+// even with .rn, so the rotation's products are packed fmas with a run-time -0.0 addend.
+template <int D>
+struct HqRopeCfg {
+  static constexpr int kSlots = D == 128 ? 3 : 4;
+  static constexpr int kBufs = D == 128 ? 1 : 2;     // TMA buffers per slot
+  static constexpr int kThreads = 128 * kSlots;
+  static constexpr int kBufBytes = 128 * D * 2;      // one bf16 block
+  static constexpr int kTabBytes = 128 * (D / 2) * 4;  // one table slice, float32
+  static constexpr int kSmem = 2 * kTabBytes + kSlots * kBufs * kBufBytes + 1024;
+};
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// (a0, a1) *= (b0, b1), each lane rounded once, as a packed fma whose addend z is -0.0 known
+// only at run time (x + (-0) = x for every x, zeros included); an fma's result is never fused
+// into another operation
+__device__ __forceinline__ void mul2r(float& a0, float& a1, float b0, float b1, float z) {
+  asm("{\n\t.reg .b64 ra, rb, rz;\n\tmov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %3};\n\t"
+      "mov.b64 rz, {%4, %4};\n\tfma.rn.f32x2 ra, ra, rb, rz;\n\tmov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1) : "f"(b0), "f"(b1), "f"(z));
+}
+
+// bounded wait that reports whether the phase completed
+__device__ __forceinline__ bool slot_wait(uint64_t* bar, uint32_t parity, volatile int* abort_s, int* status) {
+  const uint32_t a = smem_addr(bar);
+  if (bar_try_wait(a, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  while (!bar_try_wait(a, parity)) {
+    if (*abort_s || global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_s = 1;
+      atomicOr(status, kDevStatusTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// The units of slot `slot` in the CTA's range [lo, hi): the range is cut at multiples of P (the
+// units of one position block) into segments, and slot s takes units a + s, a + s + S, ... of
+// segment [a, b).  slot_first: the slot's first unit at or after segment start `a`, or hi.
+__device__ __forceinline__ int slot_first(int a, int hi, int P, int slot) {
+  while (a < hi) {
+    const int b = min(hi, (a / P + 1) * P);
+    if (a + slot < b) return a + slot;
+    a = b;
+  }
+  return hi;
+}
+template <int S>
+__device__ __forceinline__ int slot_next(int u, int hi, int P, int slot) {
+  const int b = min(hi, (u / P + 1) * P);
+  return u + S < b ? u + S : slot_first(b, hi, P, slot);
+}
+
+template <int D>
+__global__ void __launch_bounds__(HqRopeCfg<D>::kThreads, 1)
+    hq_rope_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
+                   const __grid_constant__ CUtensorMap tm2, const HqJob job, const signed char* __restrict__ signs,
+                   int N, int n_blocks, int BH, int ntensors, int* status) {
+  using C = HqRopeCfg<D>;
+  constexpr int S = C::kSlots;
+  constexpr int NB = C::kBufs;
+  constexpr int kBoxes = D / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  float* const tab_c = reinterpret_cast<float*>(smem);
+  float* const tab_s = reinterpret_cast<float*>(smem + C::kTabBytes);
+  uint8_t* const bufs = smem + 2 * C::kTabBytes;
+  __shared__ __align__(8) uint64_t bar[S][NB];
+  __shared__ float warp_max[S][2][4];
+  __shared__ int abort_s[S];
+  __shared__ __align__(16) float fsig[D];  // the signs of D as +-1.0f
+  __shared__ float zero_s;                 // -0.0f, read back as an opaque value
+
+  const int tid = threadIdx.x;
+  const int slot = tid >> 7;
+  const int row = tid & 127;  // row of the block
+  const int lane = tid & 31;
+  const int swarp = row >> 5;  // warp within the slot
+
+  if (tid == 0) {
+    // one thread initialises every slot's barriers, so that its fence publishes them all to
+    // the TMA unit
+    for (int i = 0; i < S; ++i) {
+      for (int j = 0; j < NB; ++j) bar_init(&bar[i][j], 1);
+      abort_s[i] = 0;
+    }
+    zero_s = -0.0f;
+    fence_barrier_init();
+    prefetch_tensor_map(&tm0);
+    prefetch_tensor_map(&tm1);
+    prefetch_tensor_map(&tm2);
+  }
+  for (int i = tid; i < D; i += C::kThreads) fsig[i] = (signs != nullptr && __ldg(signs + i) == -1) ? -1.f : 1.f;
+  __syncthreads();
+  const float zneg = *static_cast<volatile float*>(&zero_s);
+
+  const int P = ntensors * BH;  // units of one position block: (tensor, batch*head)
+  const long long U = static_cast<long long>(n_blocks) * P;
+  const int lo = static_cast<int>(U * blockIdx.x / gridDim.x);
+  const int hi = static_cast<int>(U * (blockIdx.x + 1) / gridDim.x);
+  const bool producer = row == 0;
+  uint64_t* const sbar = bar[slot];
+  uint8_t* const sbuf = bufs + slot * NB * C::kBufBytes;
+  volatile int* const sabort = &abort_s[slot];
+
+  auto issue = [&](int u, int buf) {
+    const int blk = u / P;
+    const int rem = u - blk * P;
+    const int t = rem / BH;
+    const int bh = rem - t * BH;
+    const CUtensorMap* tm = t == 0 ? &tm0 : (t == 1 ? &tm1 : &tm2);
+    bar_arrive_expect_tx(&sbar[buf], C::kBufBytes);
+#pragma unroll
+    for (int bx = 0; bx < kBoxes; ++bx)
+      tma_load_4d(sbuf + buf * C::kBufBytes + bx * 16384, tm, &sbar[buf], bx * 64, blk * 128, bh % job.H, bh / job.H);
+  };
+
+  int pre = hi;    // producer: the next unit to load
+  int issued = 0;  // producer: loads issued, and waits of its own that completed
+  int waited = 0;
+  if (producer) {
+    pre = slot_first(lo, hi, P, slot);
+    for (int j = 0; j < NB && pre < hi; ++j) {
+      issue(pre, j);
+      ++issued;
+      pre = slot_next<S>(pre, hi, P, slot);
+    }
+  }
+
+  int k = 0;  // units of this slot so far
+  for (int a = lo; a < hi;) {
+    const int blk = a / P;
+    const int b = min(hi, (blk + 1) * P);
+    const int t_first = (a - blk * P) / BH, t_last = (b - 1 - blk * P) / BH;
+    bool need = false;
+    for (int t = t_first; t <= t_last; ++t) need |= (t == 0 ? job.rope[0] : (t == 1 ? job.rope[1] : job.rope[2])) != 0;
+    __syncthreads();  // every slot is done with the previous slice
+    if (need) {
+      // the slice of this position block (rows past the sequence end take the last position's
+      // entries; their values are zero), every load of the thread in flight before its stores
+      constexpr int kRowsPer = C::kThreads / 128;
+      constexpr int kPer = (D / 2 + kRowsPer - 1) / kRowsPer;
+      const size_t np = static_cast<size_t>(job.n_pos);
+      const int pos = min(blk * 128 + row, N - 1);
+      float cv[kPer], sv[kPer];
+#pragma unroll
+      for (int m = 0; m < kPer; ++m) {
+        const int i = slot + m * kRowsPer;
+        if (i < D / 2) {
+          cv[m] = __ldg(job.cos + i * np + pos);
+          sv[m] = __ldg(job.sin + i * np + pos);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < kPer; ++m) {
+        const int i = slot + m * kRowsPer;
+        if (i < D / 2) {
+          const int ch = i >> 2;
+          const int idx = row * (D / 2) + ((ch ^ ((row + (ch >> 3)) & 7)) << 2) + (i & 3);
+          tab_c[idx] = cv[m];
+          tab_s[idx] = sv[m];
+        }
+      }
+    }
+    __syncthreads();
+
+    for (int u = a + slot; u < b; u += S, ++k) {
+      const int buf = NB == 1 ? 0 : (k & 1);
+      const uint32_t parity = NB == 1 ? (k & 1) : ((k >> 1) & 1);
+      const int rem = u - blk * P;
+      const int t = rem / BH;
+      const int bh = rem - t * BH;
+      if (!*sabort) {
+        const bool ok = slot_wait(&sbar[buf], parity, sabort, status);
+        if (producer && ok) ++waited;
+      }
+      const bool rotate = (t == 0 ? job.rope[0] : (t == 1 ? job.rope[1] : job.rope[2])) != 0;
+      const bool transform = (t == 0 ? job.transform[0] : (t == 1 ? job.transform[1] : job.transform[2])) != 0;
+      const uint8_t* sb = sbuf + buf * C::kBufBytes;
+
+      // v[c] = coordinate c of the row
+      float v[D];
+#pragma unroll
+      for (int c8 = 0; c8 < D / 8; ++c8) {
+        const int e0 = 8 * c8;
+        const uint4 w = *reinterpret_cast<const uint4*>(sb + (e0 >> 6) * 16384 + row * 128 +
+                                                        ((((e0 & 63) >> 3) ^ (row & 7)) << 4));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          v[e0 + 2 * m] = __uint_as_float(ws[m] << 16);
+          v[e0 + 2 * m + 1] = __uint_as_float(ws[m] & 0xFFFF0000u);
+        }
+      }
+      if constexpr (NB == 1) {
+        // the slot has read its buffer: load the next block into it
+        named_bar_sync(1 + slot, 128);
+        if (!*sabort && producer && pre < hi) {
+          issue(pre, 0);
+          ++issued;
+          pre = slot_next<S>(pre, hi, P, slot);
+        }
+      }
+      if (rotate) {
+        // (x_i, x_{i+d/2}) -> (x_i c - x_{i+d/2} s, x_{i+d/2} c + x_i s), frequency i
+#pragma unroll
+        for (int q = 0; q < D / 8; ++q) {
+          const int idx = row * (D / 2) + ((q ^ ((row + (q >> 3)) & 7)) << 2);
+          const float4 c4 = *reinterpret_cast<const float4*>(tab_c + idx);
+          const float4 s4 = *reinterpret_cast<const float4*>(tab_s + idx);
+          const float cs[4] = {c4.x, c4.y, c4.z, c4.w};
+          const float sn[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+          for (int m = 0; m < 4; m += 2) {
+            const int j = 4 * q + m;
+            float al0 = v[j], al1 = v[j + 1], bl0 = v[D / 2 + j], bl1 = v[D / 2 + j + 1];
+            float ah0 = bl0, ah1 = bl1, bh0 = al0, bh1 = al1;
+            mul2r(al0, al1, cs[m], cs[m + 1], zneg);  // x_lo c
+            mul2r(bl0, bl1, sn[m], sn[m + 1], zneg);  // x_hi s
+            mul2r(ah0, ah1, cs[m], cs[m + 1], zneg);  // x_hi c
+            mul2r(bh0, bh1, sn[m], sn[m + 1], zneg);  // x_lo s
+            sub2(al0, al1, bl0, bl1);
+            add2(ah0, ah1, bh0, bh1);
+            v[j] = al0;
+            v[j + 1] = al1;
+            v[D / 2 + j] = ah0;
+            v[D / 2 + j + 1] = ah1;
+          }
+        }
+      }
+      if (transform) {
+        // D (exact sign flips) fused with the stride-1 butterflies: (s_e x_e) +- s_{e+1} x_{e+1}
+#pragma unroll
+        for (int q = 0; q < D / 4; ++q) {
+          const float4 sg = *reinterpret_cast<const float4*>(fsig + 4 * q);
+          const float sgs[4] = {sg.x, sg.y, sg.z, sg.w};
+#pragma unroll
+          for (int m = 0; m < 4; m += 2) {
+            const int e = 4 * q + m;
+            const float x = v[e] * sgs[m];
+            const float y = v[e + 1];
+            v[e] = fmaf(sgs[m + 1], y, x);
+            v[e + 1] = fmaf(-sgs[m + 1], y, x);
+          }
+        }
+        // strides 2 .. d/2 on register pairs (e, e+1): a packed add and a packed sub make two
+        // butterflies
+#pragma unroll
+        for (int h = 2; h < D; h <<= 1) {
+#pragma unroll
+          for (int e = 0; e < D; e += 2) {
+            if ((e & h) == 0) {
+              float s0 = v[e], s1 = v[e + 1], d0 = v[e], d1 = v[e + 1];
+              add2(s0, s1, v[e + h], v[e + h + 1]);
+              sub2(d0, d1, v[e + h], v[e + h + 1]);
+              v[e] = s0;
+              v[e + 1] = s1;
+              v[e + h] = d0;
+              v[e + h + 1] = d1;
+            }
+          }
+        }
+      }
+
+      float am[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < D; ++e) am[e & 3] = fmaxf(am[e & 3], fabsf(v[e]));
+      float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      if (lane == 0) warp_max[slot][k & 1][swarp] = amax;
+      // every warp of the slot has posted its maximum (and, with two buffers, read buffer `buf`)
+      named_bar_sync(1 + slot, 128);
+      if (*sabort) continue;
+      if constexpr (NB == 2) {
+        if (producer && pre < hi) {
+          issue(pre, buf);
+          ++issued;
+          pre = slot_next<S>(pre, hi, P, slot);
+        }
+      }
+      amax = fmaxf(fmaxf(warp_max[slot][k & 1][0], warp_max[slot][k & 1][1]),
+                   fmaxf(warp_max[slot][k & 1][2], warp_max[slot][k & 1][3]));
+
+      uint8_t* const x8 = t == 0 ? job.x8[0] : (t == 1 ? job.x8[1] : job.x8[2]);
+      float* const scales = t == 0 ? job.scales[0] : (t == 1 ? job.scales[1] : job.scales[2]);
+      const float post = t == 0 ? job.post[0] : (t == 1 ? job.post[1] : job.post[2]);
+      const float s_u = fmaxf(__fdiv_rn(amax, 448.f), 1.17549435e-38f);
+      const float rcp = __frcp_rn(s_u);
+      if (producer) scales[static_cast<size_t>(bh) * n_blocks + blk] = __fmul_rn(s_u, post);
+      const int grow = blk * 128 + row;
+      if (grow < N) {
+        uint8_t* const out = x8 + (static_cast<size_t>(bh) * N + grow) * D;
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t w[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int e = 16 * c + 4 * m;
+            float a0 = v[e], a1 = v[e + 1], a2 = v[e + 2], a3 = v[e + 3];
+            mul2(a0, a1, rcp);
+            mul2(a2, a3, rcp);
+            const __nv_fp8x2_storage_t l = __nv_cvt_float2_to_fp8x2(make_float2(a0, a1), __NV_SATFINITE, __NV_E4M3);
+            const __nv_fp8x2_storage_t h = __nv_cvt_float2_to_fp8x2(make_float2(a2, a3), __NV_SATFINITE, __NV_E4M3);
+            w[m] = static_cast<uint32_t>(l) | (static_cast<uint32_t>(h) << 16);
+          }
+          *reinterpret_cast<uint4*>(out + 16 * c) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+    a = b;
+  }
+  // no TMA copy may still be in flight when the CTA exits: after an abort, the slot's loads from
+  // its first unwaited one on may not have landed
+  if (producer) {
+    for (int i = waited; i < issued; ++i) {
+      const uint32_t ad = smem_addr(&sbar[NB == 1 ? 0 : (i & 1)]);
+      const uint32_t par = NB == 1 ? (i & 1) : ((i >> 1) & 1);
+      const unsigned long long t0 = global_timer_ns();
+      while (!bar_try_wait(ad, par)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          atomicOr(status, kDevStatusTimeout);
+          break;
+        }
+      }
+    }
+  }
+}
+
+template <int D>
+static cudaError_t launch_hq_rope(const CUtensorMap* tm, int ntensors, const HqJob& job0, const signed char* signs,
+                                  int BH, int N, int num_sms, int* status, cudaStream_t stream) {
+  using C = HqRopeCfg<D>;
+  const int n_blocks = (N + 127) / 128;
+  const long long total = static_cast<long long>(BH) * n_blocks * ntensors;
+  if (total > 0x7FFFFFFFLL - 65536) return cudaErrorInvalidValue;
+  const long long want = (total + C::kSlots - 1) / C::kSlots;
+  const int grid = static_cast<int>(want < num_sms ? want : num_sms);
+  hq_rope_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tm[0], tm[ntensors > 1 ? 1 : 0],
+                                                             tm[ntensors > 2 ? 2 : 0], job0, signs, N, n_blocks, BH,
+                                                             ntensors, status);
+  return cudaGetLastError();
+}
+
 template <int D, bool ROPE, bool VL = false>
 static cudaError_t launch_hq(const CUtensorMap* tm, int ntensors, const HqJob& job0, const signed char* signs, int BH,
                              int N, int num_sms, int* status, cudaStream_t stream) {
@@ -488,9 +851,13 @@ template <int D>
 static cudaError_t set_hq_attr() {
   cudaError_t e = cudaFuncSetAttribute(hadamard_quant_kernel<D, false, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * HqCfg<D>::kBufBytes + 1024);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(hadamard_quant_kernel<D, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             2 * HqCfg<D, true>::kBufBytes + 1024);
+  if (e == cudaSuccess) {
+    if constexpr (D == 256)
+      e = cudaFuncSetAttribute(hadamard_quant_kernel<D, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               2 * HqCfg<D, true>::kBufBytes + 1024);
+    else
+      e = cudaFuncSetAttribute(hq_rope_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, HqRopeCfg<D>::kSmem);
+  }
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(hadamard_quant_kernel<D, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              2 * HqCfg<D>::kBufBytes + 1024);
@@ -557,10 +924,10 @@ cudaError_t launch_hadamard_quant(const CUtensorMap* tm, int ntensors, uint8_t* 
   job.n_pos = n_pos;
   switch (d) {
     case 64:
-      return with_rope ? launch_hq<64, true>(tm, ntensors, job, signs, BH, N, num_sms, status, stream)
+      return with_rope ? launch_hq_rope<64>(tm, ntensors, job, signs, BH, N, num_sms, status, stream)
                        : launch_hq<64, false>(tm, ntensors, job, signs, BH, N, num_sms, status, stream);
     case 128:
-      return with_rope ? launch_hq<128, true>(tm, ntensors, job, signs, BH, N, num_sms, status, stream)
+      return with_rope ? launch_hq_rope<128>(tm, ntensors, job, signs, BH, N, num_sms, status, stream)
                        : launch_hq<128, false>(tm, ntensors, job, signs, BH, N, num_sms, status, stream);
     case 256:
       return with_rope ? launch_hq<256, true>(tm, ntensors, job, signs, BH, N, num_sms, status, stream)
