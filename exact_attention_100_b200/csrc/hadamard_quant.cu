@@ -466,7 +466,9 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
 // every head and tensor at those positions (the tables are read from DRAM once).  A CTA works on
 // kSlots blocks at a time, one 128-thread slot each, with its own TMA buffers, barrier phases and
 // named barrier; with one buffer per slot (d = 128, where a row takes the registers of two) the
-// next block's load is issued as soon as the slot has unpacked the current one.
+// next block's load is issued as soon as the slot has unpacked the current one.  A warp's codes go
+// through shared memory (rows permuted in 16-byte chunks), so that each store instruction writes
+// 512 contiguous bytes of the output instead of one 16-byte piece of 32 rows.
 //
 // Rounding is that of the oracle's composition: products and the sum of the rotation each
 // rounded, the sign flips of D exact and applied to the rotated values, each butterfly rounded
@@ -479,7 +481,8 @@ struct HqRopeCfg {
   static constexpr int kThreads = 128 * kSlots;
   static constexpr int kBufBytes = 128 * D * 2;      // one bf16 block
   static constexpr int kTabBytes = 128 * (D / 2) * 4;  // one table slice, float32
-  static constexpr int kSmem = 2 * kTabBytes + kSlots * kBufs * kBufBytes + 1024;
+  static constexpr int kOutBytes = 128 * D;          // one block of codes, staged per warp for the store
+  static constexpr int kSmem = 2 * kTabBytes + kSlots * (kBufs * kBufBytes + kOutBytes) + 1024;
 };
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
@@ -541,6 +544,7 @@ __global__ void __launch_bounds__(HqRopeCfg<D>::kThreads, 1)
   float* const tab_c = reinterpret_cast<float*>(smem);
   float* const tab_s = reinterpret_cast<float*>(smem + C::kTabBytes);
   uint8_t* const bufs = smem + 2 * C::kTabBytes;
+  uint8_t* const outs = bufs + S * NB * C::kBufBytes;
   __shared__ __align__(8) uint64_t bar[S][NB];
   __shared__ float warp_max[S][2][4];
   __shared__ int abort_s[S];
@@ -639,6 +643,17 @@ __global__ void __launch_bounds__(HqRopeCfg<D>::kThreads, 1)
       }
     }
     __syncthreads();
+    if (b < hi) {
+      // bring the next position block's slice into L2 while this one is worked on
+      const int pos0 = (blk + 1) * 128;
+      const size_t np = static_cast<size_t>(job.n_pos);
+      for (int l = tid; l < 2 * (D / 2) * 4; l += C::kThreads) {
+        const int i = (l >> 2) % (D / 2), j = l & 3;
+        const float* tb = l < (D / 2) * 4 ? job.cos : job.sin;
+        if (pos0 + 32 * j < job.n_pos)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(tb + i * np + pos0 + 32 * j));
+      }
+    }
 
     for (int u = a + slot; u < b; u += S, ++k) {
       const int buf = NB == 1 ? 0 : (k & 1);
@@ -764,11 +779,14 @@ __global__ void __launch_bounds__(HqRopeCfg<D>::kThreads, 1)
       const float s_u = fmaxf(__fdiv_rn(amax, 448.f), 1.17549435e-38f);
       const float rcp = __frcp_rn(s_u);
       if (producer) scales[static_cast<size_t>(bh) * n_blocks + blk] = __fmul_rn(s_u, post);
-      const int grow = blk * 128 + row;
-      if (grow < N) {
-        uint8_t* const out = x8 + (static_cast<size_t>(bh) * N + grow) * D;
+      {
+        // the warp's 32 rows of codes: row r at r * D, 16-byte chunk c at chunk c ^ ((r / G) % CPR),
+        // G rows per 128-byte line, CPR chunks per row (conflict-free writes and reads)
+        constexpr int CPR = D / 16;
+        constexpr int G = 128 / D;
+        uint8_t* const ws = outs + (slot * 4 + swarp) * (32 * D);
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
+        for (int c = 0; c < CPR; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
@@ -780,8 +798,19 @@ __global__ void __launch_bounds__(HqRopeCfg<D>::kThreads, 1)
             const __nv_fp8x2_storage_t h = __nv_cvt_float2_to_fp8x2(make_float2(a2, a3), __NV_SATFINITE, __NV_E4M3);
             w[m] = static_cast<uint32_t>(l) | (static_cast<uint32_t>(h) << 16);
           }
-          *reinterpret_cast<uint4*>(out + 16 * c) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(ws + lane * D + ((c ^ ((lane / G) % CPR)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
+        __syncwarp();
+        const int row0 = blk * 128 + swarp * 32;  // sequence row of the warp's first row
+        uint8_t* const gout = x8 + (static_cast<size_t>(bh) * N + row0) * D;
+#pragma unroll
+        for (int i = 0; i < 32 * D / 512; ++i) {
+          const int rr = i * (512 / D) + lane / CPR;
+          const int c = lane % CPR;
+          const uint4 val = *reinterpret_cast<const uint4*>(ws + rr * D + ((c ^ ((rr / G) % CPR)) << 4));
+          if (row0 + rr < N) *reinterpret_cast<uint4*>(gout + 512 * i + 16 * lane) = val;
+        }
+        __syncwarp();
       }
     }
     a = b;
