@@ -45,6 +45,24 @@ def test_bit_exact_against_oracle(B, H, N, d):
     np.testing.assert_array_equal(v8, rc)
 
 
+@pytest.mark.parametrize("B,H,N,d", [(1, 4, 8192, 128), (1, 1, 20000, 64)])
+def test_bit_exact_where_blocks_of_a_cta_span_positions(B, H, N, d):
+    """Sizes at which most CTAs of the d = 64/128 kernel work on blocks of two position blocks,
+    so that the staged table slice is replaced mid-range (and the next one prefetched); the
+    second has a ragged last block and more table rows than positions."""
+    q, k, v = normal_qkv(B, H, N, d, seed=N + d + H, outlier_frac=1e-3)
+    signs = hadamard_signs(d)
+    cos, sin = rope_tables(N + 5, d)
+    q8, k8, v8, qs, ks, vs = _run(q, k, v, signs, cos, sin)
+    for got, x in (((q8, qs), q), ((k8, ks), k)):
+        rc, rs = hadamard_quant_ref(rope_ref(x, cos, sin).astype(np.float64), signs)
+        np.testing.assert_array_equal(got[1], rs)
+        np.testing.assert_array_equal(got[0], rc)
+    rc, rs = hadamard_quant_ref(v, None)
+    np.testing.assert_array_equal(vs, rs)
+    np.testing.assert_array_equal(v8, rc)
+
+
 def test_identity_tables_give_the_unrotated_preprocessing():
     """cos = 1, sin = 0 at every position: the same bits as attn_hadamard_quant_qkv."""
     B, H, N, d = 2, 2, 260, 128
