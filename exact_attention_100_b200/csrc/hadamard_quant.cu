@@ -17,14 +17,14 @@
 // codes are E4M3(y * (1/s_u)) (round to nearest even, saturating); the stored dequantisation
 // scale is s_u * post_scale (post_scale = 1/sqrt(d) with the transform, 1 without).
 //
-// With ROPE, the tensors marked for it are first given the rotary position embedding the same
-// page names as a bandwidth-bound step to fuse with the transform: coordinates i and i + d/2 of
-// row n are rotated by the angle whose cosine and sine the caller's tables hold at [i, n],
-// in float32 with each product and the sum rounded (no fused multiply-add); then D (an exact
-// sign flip) and the butterflies run on the rotated float32 row.  The tables are frequency-major
-// so that the 32 rows of a warp read one contiguous 128-byte line per frequency (row-major
-// tables cost each warp load 32 lines and made the kernel L1-bound).  For d = 256 the partner
-// coordinate sits two lanes away.
+// With ROPE (d = 256; d = 64 and 128 have hq_rope_kernel below), the tensors marked for it are
+// first given the rotary position embedding the same page names as a bandwidth-bound step to
+// fuse with the transform: coordinates i and i + d/2 of row n are rotated by the angle whose
+// cosine and sine the caller's tables hold at [i, n], in float32 with each product and the sum
+// rounded (no fused multiply-add); then D (an exact sign flip) and the butterflies run on the
+// rotated float32 row.  The tables are frequency-major so that the 32 rows of a warp read one
+// contiguous 128-byte line per frequency (row-major tables cost each warp load 32 lines and made
+// the kernel L1-bound).  Four lanes hold a row; the partner coordinate sits two lanes away.
 //
 // Packed batches (VL): tensor t holds B sequences of different lengths, rows cu_t[b] ..
 // cu_t[b+1]-1 of a [total_t, H, d] tensor, and is quantised in 128-row blocks of each sequence,
@@ -84,6 +84,7 @@ __device__ __forceinline__ void thread_wait(uint64_t* bar, uint32_t parity, vola
 
 template <int D, bool ROPE = false>
 struct HqCfg {
+  static_assert(!ROPE || D == 256, "the rotary embedding at d = 64 and 128 is hq_rope_kernel");
   // elements of a row held by one thread: at most 64 with the rotary embedding, whose table
   // loads need registers to be in flight (a whole d = 128 row per thread left too few)
   static constexpr int kElems = (D == 256 || ROPE) ? 64 : D;
@@ -91,7 +92,7 @@ struct HqCfg {
   static constexpr int kThreads = 128 * kThreadsPerRow;
   static constexpr int kBoxes = D / 64;             // 128-byte TMA boxes per row
   static constexpr int kBufBytes = 128 * D * 2;
-  static constexpr int kCtasPerSm = D == 256 ? 1 : (D == 128 ? (ROPE ? 2 : 3) : 5);
+  static constexpr int kCtasPerSm = D == 256 ? 1 : (D == 128 ? 3 : 5);
 };
 
 // Up to three tensors of one shape in one launch (Q and K with the transform, V without).
@@ -319,17 +320,7 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
       // rows past the sequence end hold zeros (TMA fill): any table row leaves them zero
       const int pos = min(blk * 128 + row, N - 1);
       const size_t np = static_cast<size_t>(job.n_pos);
-      if constexpr (C::kThreadsPerRow == 1) {
-        const float* cr = job.cos + pos;
-        const float* sr = job.sin + pos;
-#pragma unroll
-        for (int i = 0; i < D / 2; ++i) {
-          const float c = __ldg(cr + i * np), s = __ldg(sr + i * np);
-          const float a = v[i], b = v[i + D / 2];
-          v[i] = __fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s));
-          v[i + D / 2] = __fadd_rn(__fmul_rn(b, c), __fmul_rn(a, s));
-        }
-      } else {
+      if constexpr (ROPE) {  // (d = 256: four lanes per row)
         // the lower half of the parts holds coordinates 0 .. D/2-1, the upper half their
         // partners D/2 .. D-1, kThreadsPerRow/2 lanes away
         constexpr int kHalf = C::kThreadsPerRow / 2;
