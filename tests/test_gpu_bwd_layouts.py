@@ -210,7 +210,8 @@ def test_packed_ds_bench_batch_two_heads():
             _check_grads([t(g) for g in grads], refs, _bounds(qs, ks, vs, dos, o_ref, scale, True))
 
 
-def test_packed_bad_offsets_are_reported():
+@pytest.mark.parametrize("ds", [False, True])
+def test_packed_bad_offsets_are_reported(ds):
     lq = [300, 200, 250]
     q, k, v, cq, ck = normal_qkv_packed(lq, lq, 2, 64, seed=8)
     tq, tk, tv = (torch.from_numpy(a).to(torch.bfloat16).cuda() for a in (q, k, v))
@@ -221,6 +222,7 @@ def test_packed_bad_offsets_are_reported():
     bad = tcq.clone()
     bad[2] = 100  # sequence 1 decreasing, sequence 2 longer than max_seqlen_q
     dq = torch.full(tq.shape, float("nan"), dtype=torch.float32, device="cuda")
-    ea.attn_bwd_varlen(tq, tk, tv, o, lse, torch.ones_like(tq), bad, tck, 300, 300, dq=dq, causal=True)
+    bwd = ea.attn_bwd_varlen_ds if ds else ea.attn_bwd_varlen
+    bwd(tq, tk, tv, o, lse, torch.ones_like(tq), bad, tck, 300, 300, dq=dq, causal=True)
     assert ea.attn_device_status() == ea.ATTN_ERR_INVALID_ARG
     assert not torch.isnan(dq[:300]).any() and torch.isnan(dq[300:]).all()
