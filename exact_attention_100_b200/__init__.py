@@ -188,6 +188,20 @@ def attn_bwd_workspace_bytes(B: int, H: int, N: int) -> int:
     return int(lib().attn_bwd_workspace_bytes(int(B), int(H), int(N)))
 
 
+def _workspace(workspace, nbytes, device, name):
+    """The caller's workspace checked against the ``nbytes`` the call needs (the C entry points
+    take no size and would write past a smaller buffer), or a new one of that size."""
+    import torch
+    if workspace is None:
+        return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError(f"{name}: the workspace must be a contiguous cuda tensor")
+    if workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"{name}: the workspace has {workspace.numel() * workspace.element_size()} bytes, "
+                         f"{nbytes} are needed")
+    return workspace
+
+
 def attn_bwd(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None, scale=None, causal=False,
              g_dtype=None, stream=None):
     """(dQ, dK, dV) of attn_fwd for the upstream gradient ``dout``.
@@ -206,8 +220,7 @@ def attn_bwd(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None, s
     dq = dq if dq is not None else torch.empty(q.shape, dtype=gd, device=q.device)
     dk = dk if dk is not None else torch.empty(q.shape, dtype=gd, device=q.device)
     dv = dv if dv is not None else torch.empty(q.shape, dtype=gd, device=q.device)
-    if workspace is None:
-        workspace = torch.empty(attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device=q.device)
+    workspace = _workspace(workspace, attn_bwd_workspace_bytes(B, H, N), q.device, "attn_bwd")
     gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
     _check(lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
@@ -236,11 +249,10 @@ def attn_bwd_ds(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None
     dq = dq if dq is not None else torch.empty(q.shape, dtype=gd, device=q.device)
     dk = dk if dk is not None else torch.empty(q.shape, dtype=gd, device=q.device)
     dv = dv if dv is not None else torch.empty(q.shape, dtype=gd, device=q.device)
-    if workspace is None:
-        nbytes = attn_bwd_ds_workspace_bytes(B, H, N, causal)
-        if nbytes == 0:
-            raise ValueError("too many dS tiles for this shape: use attn_bwd")
-        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    nbytes = attn_bwd_ds_workspace_bytes(B, H, N, causal)
+    if nbytes == 0:
+        raise ValueError("too many dS tiles for this shape: use attn_bwd")
+    workspace = _workspace(workspace, nbytes, q.device, "attn_bwd_ds")
     gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
     _check(lib().attn_bwd_ds(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
@@ -355,8 +367,7 @@ def attn_bwd_qk(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None
     dq = dq if dq is not None else torch.empty(q.shape, dtype=gd, device=q.device)
     dk = dk if dk is not None else torch.empty(k.shape, dtype=gd, device=q.device)
     dv = dv if dv is not None else torch.empty(k.shape, dtype=gd, device=q.device)
-    if workspace is None:
-        workspace = torch.empty(attn_bwd_workspace_bytes(B, H, Nq) // 4, dtype=torch.float32, device=q.device)
+    workspace = _workspace(workspace, attn_bwd_workspace_bytes(B, H, Nq), q.device, "attn_bwd")
     gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
     _check(lib().attn_bwd_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
@@ -387,8 +398,7 @@ def attn_bwd_strided(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace
     for g, ref in ((dq, q), (dk, k), (dv, k)):
         if g.shape != ref.shape or g.stride(-1) != 1:
             raise ValueError("gradients must have their input's shape and a contiguous last dimension")
-    if workspace is None:
-        workspace = torch.empty(attn_bwd_workspace_bytes(B, H, Nq) // 4, dtype=torch.float32, device=q.device)
+    workspace = _workspace(workspace, attn_bwd_workspace_bytes(B, H, Nq), q.device, "attn_bwd")
     strides = (ctypes.c_longlong * 24)(*[int(x) for t in (q, k, v, o, dout, dq, dk, dv) for x in t.stride()[:3]])
     gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
@@ -448,14 +458,13 @@ def _bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
         if g.shape != ref.shape or g.stride(-1) != 1:
             raise ValueError("gradients must have their input's shape and a contiguous last dimension")
     mq = min(int(max_seqlen_q), total_q)
-    if workspace is None:
-        if ds:
-            nbytes = attn_bwd_varlen_ds_workspace_bytes(B, H, int(max_seqlen_q), int(max_seqlen_k))
-            if nbytes == 0:
-                raise ValueError("too many dS tiles for this batch: use attn_bwd_varlen")
-            workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
-        else:
-            workspace = torch.empty(attn_bwd_workspace_bytes(B, H, mq) // 4, dtype=torch.float32, device=q.device)
+    if ds:
+        nbytes = attn_bwd_varlen_ds_workspace_bytes(B, H, int(max_seqlen_q), int(max_seqlen_k))
+        if nbytes == 0:
+            raise ValueError("too many dS tiles for this batch: use attn_bwd_varlen")
+    else:
+        nbytes = attn_bwd_workspace_bytes(B, H, mq)
+    workspace = _workspace(workspace, nbytes, q.device, "attn_bwd_varlen_ds" if ds else "attn_bwd_varlen")
     strides = (ctypes.c_longlong * 16)(*[int(x) for t in (q, k, v, o, dout, dq, dk, dv) for x in t.stride()[:2]])
     gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)

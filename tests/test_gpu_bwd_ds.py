@@ -100,7 +100,27 @@ def test_bwd_ds_bench_workload_whole_heads():
 def test_bwd_ds_rejects_what_attn_bwd_rejects():
     (_, (tq, tk, tv, tdo)) = _inputs(1, 1, 256, 128, seed=1)
     o, lse = ea.attn_fwd(tq, tk, tv)
-    with pytest.raises(ea.AttnError):
-        ea.attn_bwd_ds(tq, tk, tv, o, lse, tdo, workspace=torch.empty(16, dtype=torch.uint8, device="cuda")[1:])
+    nbytes = ea.attn_bwd_ds_workspace_bytes(1, 1, 256, False)
+    with pytest.raises(ea.AttnError):  # large enough, not 16-byte aligned: the library refuses it
+        ea.attn_bwd_ds(tq, tk, tv, o, lse, tdo, workspace=torch.empty(nbytes + 16, dtype=torch.uint8, device="cuda")[1:])
+    torch.cuda.synchronize()
+    assert ea.attn_device_status() == ea.ATTN_OK
+
+
+def test_workspace_smaller_than_needed_is_refused_before_any_launch():
+    """The C entry points take no workspace size; the binding checks the caller's buffer."""
+    (_, (tq, tk, tv, tdo)) = _inputs(1, 2, 300, 64, seed=2)
+    o, lse = ea.attn_fwd(tq, tk, tv, causal=True)
+    torch.cuda.synchronize()
+    launches = ea.attn_num_kernel_launches()
+    small_ds = torch.empty(ea.attn_bwd_ds_workspace_bytes(1, 2, 300, True) - 16, dtype=torch.uint8, device="cuda")
+    small = torch.empty(ea.attn_bwd_workspace_bytes(1, 2, 300) // 4 - 4, dtype=torch.float32, device="cuda")
+    with pytest.raises(ValueError):
+        ea.attn_bwd_ds(tq, tk, tv, o, lse, tdo, workspace=small_ds, causal=True)
+    with pytest.raises(ValueError):
+        ea.attn_bwd(tq, tk, tv, o, lse, tdo, workspace=small, causal=True)
+    with pytest.raises(ValueError):
+        ea.attn_bwd(tq, tk, tv, o, lse, tdo, workspace=torch.empty(1 << 20, dtype=torch.uint8), causal=True)  # host
+    assert ea.attn_num_kernel_launches() == launches
     torch.cuda.synchronize()
     assert ea.attn_device_status() == ea.ATTN_OK
