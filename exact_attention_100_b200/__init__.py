@@ -146,7 +146,43 @@ def _stream_ptr(stream):
 
 
 def _ptr(t):
-    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+    """Device pointer of a tensor on the current CUDA device (the kernels would fault on any
+    other address), or NULL for None."""
+    if t is None:
+        return ctypes.c_void_p(0)
+    import torch
+    if not t.is_cuda or t.device.index != torch.cuda.current_device():
+        raise ValueError(f"a {tuple(t.shape)} tensor is on {t.device}, not on the current CUDA device")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _out(t, shape, dtypes, what, strided=False):
+    """Checks a caller-supplied output (or scale array): the kernels write (or read) exactly
+    `shape` elements of one of `dtypes`, contiguous or, with `strided`, through the tensor's own
+    strides with a contiguous last dimension."""
+    layout_ok = t.stride(-1) == 1 if strided else t.is_contiguous()
+    if tuple(t.shape) != tuple(int(x) for x in shape) or t.dtype not in dtypes or not layout_ok:
+        names = "/".join(str(x).replace("torch.", "") for x in dtypes)
+        raise ValueError(f"{what} must be {names} of shape {tuple(int(x) for x in shape)}"
+                         f"{' with a contiguous last dimension' if strided else ', contiguous'}")
+    return t
+
+
+def _grads(dq, dk, dv, q_shape, k_shape, strided=False):
+    import torch
+    for g, shp, name in ((dq, q_shape, "dq"), (dk, k_shape, "dk"), (dv, k_shape, "dv")):
+        _out(g, shp, (torch.bfloat16, torch.float32), name, strided)
+    if not dq.dtype == dk.dtype == dv.dtype:
+        raise ValueError("dq, dk and dv must have one dtype")
+
+
+def _outs_qkv(outs, q_shape, k_shape, scale_q, scale_k):
+    import torch
+    if len(outs) != 6:
+        raise ValueError("outs must be (q8, k8, v8, q_scale, k_scale, v_scale)")
+    for t, shp, name in zip(outs, (q_shape, k_shape, k_shape, scale_q, scale_k, scale_k),
+                            ("q8", "k8", "v8", "q_scale", "k_scale", "v_scale")):
+        _out(t, shp, (torch.uint8,) if name.endswith("8") else (torch.float32,), name)
 
 
 def _check(status: int, what: str) -> None:
@@ -177,6 +213,9 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, o_dtype=None, 
         o = torch.empty(q.shape, dtype=o_dtype or torch.bfloat16, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _out(o, q.shape, (torch.bfloat16, torch.float32), "o")
+    if lse is not None:
+        _out(lse, (B, H, N), (torch.float32,), "lse")
     od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
     _check(lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, s, int(bool(causal)),
@@ -220,6 +259,8 @@ def attn_bwd(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None, s
     dq = dq if dq is not None else torch.empty(q.shape, dtype=gd, device=q.device)
     dk = dk if dk is not None else torch.empty(q.shape, dtype=gd, device=q.device)
     dv = dv if dv is not None else torch.empty(q.shape, dtype=gd, device=q.device)
+    _grads(dq, dk, dv, q.shape, q.shape)
+    _out(lse, (B, H, N), (torch.float32,), "lse")
     workspace = _workspace(workspace, attn_bwd_workspace_bytes(B, H, N), q.device, "attn_bwd")
     gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
@@ -249,6 +290,8 @@ def attn_bwd_ds(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None
     dq = dq if dq is not None else torch.empty(q.shape, dtype=gd, device=q.device)
     dk = dk if dk is not None else torch.empty(q.shape, dtype=gd, device=q.device)
     dv = dv if dv is not None else torch.empty(q.shape, dtype=gd, device=q.device)
+    _grads(dq, dk, dv, q.shape, q.shape)
+    _out(lse, (B, H, N), (torch.float32,), "lse")
     nbytes = attn_bwd_ds_workspace_bytes(B, H, N, causal)
     if nbytes == 0:
         raise ValueError("too many dS tiles for this shape: use attn_bwd")
@@ -277,6 +320,8 @@ def attn_fwd_qk(q, k, v, o=None, lse=None, scale=None, causal=False, o_dtype=Non
         o = torch.empty(q.shape, dtype=o_dtype or torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _out(o, q.shape, (torch.bfloat16, torch.float32), "o")
+    _out(lse, (B, H, Nq), (torch.float32,), "lse")
     od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
     _check(lib().attn_fwd_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d, s,
@@ -298,10 +343,10 @@ def attn_fwd_strided(q, k, v, o=None, lse=None, scale=None, causal=False, o_dtyp
             raise ValueError("q, k, v must be bf16 with a contiguous last dimension")
     if o is None:
         o = torch.empty_like(q, dtype=o_dtype or torch.bfloat16)
-    if o.shape != q.shape or o.stride(-1) != 1:
-        raise ValueError("o must be [B, H, Nq, d] with a contiguous last dimension")
+    _out(o, q.shape, (torch.bfloat16, torch.float32), "o", strided=True)
     if lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _out(lse, (B, H, Nq), (torch.float32,), "lse")
     strides = (ctypes.c_longlong * 12)(*[int(x) for t in (q, k, v, o) for x in t.stride()[:3]])
     od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
@@ -337,10 +382,10 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, o=None, l
     B = int(cu_seqlens_q.shape[0]) - 1
     if o is None:
         o = torch.empty_like(q, dtype=o_dtype or torch.bfloat16)
-    if o.shape != q.shape or o.stride(-1) != 1:
-        raise ValueError("o must be [total_q, H, d] with a contiguous last dimension")
+    _out(o, q.shape, (torch.bfloat16, torch.float32), "o", strided=True)
     if lse is None:
         lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    _out(lse, (H, total_q), (torch.float32,), "lse")
     strides = (ctypes.c_longlong * 8)(*[int(x) for t in (q, k, v, o) for x in t.stride()[:2]])
     od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
@@ -367,6 +412,8 @@ def attn_bwd_qk(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None
     dq = dq if dq is not None else torch.empty(q.shape, dtype=gd, device=q.device)
     dk = dk if dk is not None else torch.empty(k.shape, dtype=gd, device=q.device)
     dv = dv if dv is not None else torch.empty(k.shape, dtype=gd, device=q.device)
+    _grads(dq, dk, dv, q.shape, k.shape)
+    _out(lse, (B, H, Nq), (torch.float32,), "lse")
     workspace = _workspace(workspace, attn_bwd_workspace_bytes(B, H, Nq), q.device, "attn_bwd")
     gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
@@ -395,9 +442,7 @@ def attn_bwd_strided(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace
     dq = dq if dq is not None else torch.empty_like(q, dtype=gd)
     dk = dk if dk is not None else torch.empty_like(k, dtype=gd)
     dv = dv if dv is not None else torch.empty_like(v, dtype=gd)
-    for g, ref in ((dq, q), (dk, k), (dv, k)):
-        if g.shape != ref.shape or g.stride(-1) != 1:
-            raise ValueError("gradients must have their input's shape and a contiguous last dimension")
+    _grads(dq, dk, dv, q.shape, k.shape, strided=True)
     workspace = _workspace(workspace, attn_bwd_workspace_bytes(B, H, Nq), q.device, "attn_bwd")
     strides = (ctypes.c_longlong * 24)(*[int(x) for t in (q, k, v, o, dout, dq, dk, dv) for x in t.stride()[:3]])
     gcode = ATTN_FP32 if dq.dtype == torch.float32 else ATTN_BF16
@@ -454,9 +499,7 @@ def _bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
     dq = dq if dq is not None else torch.empty_like(q, dtype=gd)
     dk = dk if dk is not None else torch.empty_like(k, dtype=gd)
     dv = dv if dv is not None else torch.empty_like(v, dtype=gd)
-    for g, ref in ((dq, q), (dk, k), (dv, k)):
-        if g.shape != ref.shape or g.stride(-1) != 1:
-            raise ValueError("gradients must have their input's shape and a contiguous last dimension")
+    _grads(dq, dk, dv, q.shape, k.shape, strided=True)
     mq = min(int(max_seqlen_q), total_q)
     if ds:
         nbytes = attn_bwd_varlen_ds_workspace_bytes(B, H, int(max_seqlen_q), int(max_seqlen_k))
@@ -481,6 +524,9 @@ def attn_fwd_noalloc(q, k, v, o, lse=None, scale=None, causal=False, stream=None
     None.  The first call on a device does a one-time set-up."""
     import torch
     B, H, N, d = _dims(q)
+    _out(o, q.shape, (torch.bfloat16, torch.float32), "o")
+    if lse is not None:
+        _out(lse, (B, H, N), (torch.float32,), "lse")
     od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
     _check(lib().attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, s,
@@ -511,6 +557,8 @@ def attn_hadamard_quant(x, signs=None, x8=None, scales=None, stream=None):
         x8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty((B, H, nb), dtype=torch.float32, device=x.device)
+    _out(x8, x.shape, (torch.uint8,), "x8")
+    _out(scales, (B, H, nb), (torch.float32,), "scales")
     _check(lib().attn_hadamard_quant(_ptr(x), _ptr(x8), _ptr(scales), _ptr(signs), B, H, N, d,
                                      _stream_ptr(stream)), "attn_hadamard_quant")
     return x8, scales
@@ -527,6 +575,7 @@ def attn_hadamard_quant_qkv(q, k, v, signs, outs=None, stream=None):
     if outs is None:
         outs = tuple(torch.empty(q.shape, dtype=torch.uint8, device=q.device) for _ in range(3)) + \
             tuple(torch.empty((B, H, nb), dtype=torch.float32, device=q.device) for _ in range(3))
+    _outs_qkv(outs, q.shape, q.shape, (B, H, nb), (B, H, nb))
     q8, k8, v8, qs, ks, vs = outs
     _check(lib().attn_hadamard_quant_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs), _ptr(ks),
                                          _ptr(vs), _ptr(signs), B, H, N, d, _stream_ptr(stream)),
@@ -548,6 +597,7 @@ def attn_hadamard_quant_qkv_strided(q, k, v, signs, outs=None, stream=None):
     if outs is None:
         outs = tuple(torch.empty(q.shape, dtype=torch.uint8, device=q.device) for _ in range(3)) + \
             tuple(torch.empty((B, H, nb), dtype=torch.float32, device=q.device) for _ in range(3))
+    _outs_qkv(outs, q.shape, q.shape, (B, H, nb), (B, H, nb))
     q8, k8, v8, qs, ks, vs = outs
     strides = (ctypes.c_longlong * 9)(*[int(x) for t in (q, k, v) for x in t.stride()[:3]])
     _check(lib().attn_hadamard_quant_qkv_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs),
@@ -575,6 +625,7 @@ def attn_rope_hadamard_quant_qkv(q, k, v, signs, cos, sin, outs=None, stream=Non
     if outs is None:
         outs = tuple(torch.empty(q.shape, dtype=torch.uint8, device=q.device) for _ in range(3)) + \
             tuple(torch.empty((B, H, nb), dtype=torch.float32, device=q.device) for _ in range(3))
+    _outs_qkv(outs, q.shape, q.shape, (B, H, nb), (B, H, nb))
     q8, k8, v8, qs, ks, vs = outs
     _check(lib().attn_rope_hadamard_quant_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs),
                                               _ptr(ks), _ptr(vs), _ptr(signs), _ptr(cos), _ptr(sin),
@@ -588,10 +639,17 @@ def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o=None, lse=None, scale=
     """Attention on E4M3 inputs with per-block scales (from ``attn_hadamard_quant``)."""
     import torch
     B, H, N, d = _dims(q8)
+    nb = (N + 127) // 128
+    for t, name in ((q8, "q8"), (k8, "k8"), (v8, "v8")):
+        _out(t, (B, H, N, d), (torch.uint8,), name)
+    for t, name in ((q_scale, "q_scale"), (k_scale, "k_scale"), (v_scale, "v_scale")):
+        _out(t, (B, H, nb), (torch.float32,), name)
     if o is None:
         o = torch.empty((B, H, N, d), dtype=o_dtype or torch.bfloat16, device=q8.device)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    _out(o, (B, H, N, d), (torch.bfloat16, torch.float32), "o")
+    _out(lse, (B, H, N), (torch.float32,), "lse")
     od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
     _check(lib().attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
@@ -609,10 +667,17 @@ def attn_fwd_fp8_qk(q8, k8, v8, q_scale, k_scale, v_scale, o=None, lse=None, sca
     Nk = int(k8.shape[2])
     if tuple(k8.shape) != (B, H, Nk, d) or v8.shape != k8.shape:
         raise ValueError("k8 and v8 must be [B, H, Nk, d] with q8's B, H, d")
+    for t, name in ((q8, "q8"), (k8, "k8"), (v8, "v8")):
+        _out(t, t.shape, (torch.uint8,), name)
+    _out(q_scale, (B, H, (Nq + 127) // 128), (torch.float32,), "q_scale")
+    for t, name in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        _out(t, (B, H, (Nk + 127) // 128), (torch.float32,), name)
     if o is None:
         o = torch.empty((B, H, Nq, d), dtype=o_dtype or torch.bfloat16, device=q8.device)
     if lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q8.device)
+    _out(o, (B, H, Nq, d), (torch.bfloat16, torch.float32), "o")
+    _out(lse, (B, H, Nq), (torch.float32,), "lse")
     od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
     _check(lib().attn_fwd_fp8_qk(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
@@ -635,12 +700,15 @@ def attn_fwd_fp8_strided(q8, k8, v8, q_scale, k_scale, v_scale, o=None, lse=None
     for t in (q8, k8, v8):
         if t.dtype != torch.uint8 or t.stride(-1) != 1:
             raise ValueError("q8, k8, v8 must be uint8 with a contiguous last dimension")
+    _out(q_scale, (B, H, (Nq + 127) // 128), (torch.float32,), "q_scale")
+    for t, name in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        _out(t, (B, H, (Nk + 127) // 128), (torch.float32,), name)
     if o is None:
         o = torch.empty((B, H, Nq, d), dtype=o_dtype or torch.bfloat16, device=q8.device)
-    if tuple(o.shape) != (B, H, Nq, d) or o.stride(-1) != 1:
-        raise ValueError("o must be [B, H, Nq, d] with a contiguous last dimension")
+    _out(o, (B, H, Nq, d), (torch.bfloat16, torch.float32), "o", strided=True)
     if lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q8.device)
+    _out(lse, (B, H, Nq), (torch.float32,), "lse")
     strides = (ctypes.c_longlong * 12)(*[int(x) for t in (q8, k8, v8, o) for x in t.stride()[:3]])
     od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
@@ -711,6 +779,7 @@ def attn_hadamard_quant_qkv_varlen(q, k, v, signs, cu_seqlens_q, cu_seqlens_k, m
                 torch.empty((B, H, nbq), dtype=torch.float32, device=dev),
                 torch.empty((B, H, nbk), dtype=torch.float32, device=dev),
                 torch.empty((B, H, nbk), dtype=torch.float32, device=dev))
+    _outs_qkv(outs, (total_q, H, d), (total_k, H, d), (B, H, nbq), (B, H, nbk))
     q8, k8, v8, qs, ks, vs = outs
     strides = (ctypes.c_longlong * 6)(*[int(x) for t in (q, k, v) for x in t.stride()[:2]])
     _check(lib().attn_hadamard_quant_qkv_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs),
@@ -733,12 +802,15 @@ def attn_fwd_fp8_varlen(q8, k8, v8, q_scale, k_scale, v_scale, cu_seqlens_q, cu_
         if t.dtype != torch.uint8 or not t.is_contiguous() or t.dim() != 3:
             raise ValueError("q8, k8, v8 must be contiguous uint8 [total, H, d]")
     B = _check_cu(cu_seqlens_q, cu_seqlens_k)
+    _out(q_scale, (B, H, (int(max_seqlen_q) + 127) // 128), (torch.float32,), "q_scale")
+    for t, name in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        _out(t, (B, H, (int(max_seqlen_k) + 127) // 128), (torch.float32,), name)
     if o is None:
         o = torch.empty((total_q, H, d), dtype=o_dtype or torch.bfloat16, device=q8.device)
-    if tuple(o.shape) != (total_q, H, d) or not o.is_contiguous():
-        raise ValueError("o must be a contiguous [total_q, H, d] tensor")
+    _out(o, (total_q, H, d), (torch.bfloat16, torch.float32), "o")
     if lse is None:
         lse = torch.empty((H, total_q), dtype=torch.float32, device=q8.device)
+    _out(lse, (H, total_q), (torch.float32,), "lse")
     od = ATTN_FP32 if o.dtype == torch.float32 else ATTN_BF16
     s = float(scale) if scale is not None else 1.0 / math.sqrt(d)
     _check(lib().attn_fwd_fp8_varlen(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
