@@ -168,6 +168,14 @@ def _out(t, shape, dtypes, what, strided=False):
     return t
 
 
+def _signs(signs, d):
+    """The transform's signs: None, or d int8 entries (the kernels read d of them)."""
+    import torch
+    if signs is not None:
+        _out(signs, (d,), (torch.int8,), "signs")
+    return signs
+
+
 def _grads(dq, dk, dv, q_shape, k_shape, strided=False):
     import torch
     for g, shp, name in ((dq, q_shape, "dq"), (dk, k_shape, "dk"), (dv, k_shape, "dv")):
@@ -552,6 +560,8 @@ def attn_hadamard_quant(x, signs=None, x8=None, scales=None, stream=None):
     """
     import torch
     B, H, N, d = _dims(x)
+    if x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 tensor")
     nb = (N + 127) // 128
     if x8 is None:
         x8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
@@ -559,7 +569,7 @@ def attn_hadamard_quant(x, signs=None, x8=None, scales=None, stream=None):
         scales = torch.empty((B, H, nb), dtype=torch.float32, device=x.device)
     _out(x8, x.shape, (torch.uint8,), "x8")
     _out(scales, (B, H, nb), (torch.float32,), "scales")
-    _check(lib().attn_hadamard_quant(_ptr(x), _ptr(x8), _ptr(scales), _ptr(signs), B, H, N, d,
+    _check(lib().attn_hadamard_quant(_ptr(x), _ptr(x8), _ptr(scales), _ptr(_signs(signs, d)), B, H, N, d,
                                      _stream_ptr(stream)), "attn_hadamard_quant")
     return x8, scales
 
@@ -571,6 +581,9 @@ def attn_hadamard_quant_qkv(q, k, v, signs, outs=None, stream=None):
     """
     import torch
     B, H, N, d = _dims(q)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError("q, k, v must be contiguous bf16 tensors of one shape")
     nb = (N + 127) // 128
     if outs is None:
         outs = tuple(torch.empty(q.shape, dtype=torch.uint8, device=q.device) for _ in range(3)) + \
@@ -578,7 +591,7 @@ def attn_hadamard_quant_qkv(q, k, v, signs, outs=None, stream=None):
     _outs_qkv(outs, q.shape, q.shape, (B, H, nb), (B, H, nb))
     q8, k8, v8, qs, ks, vs = outs
     _check(lib().attn_hadamard_quant_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs), _ptr(ks),
-                                         _ptr(vs), _ptr(signs), B, H, N, d, _stream_ptr(stream)),
+                                         _ptr(vs), _ptr(_signs(signs, d)), B, H, N, d, _stream_ptr(stream)),
            "attn_hadamard_quant_qkv")
     return outs
 
@@ -601,7 +614,7 @@ def attn_hadamard_quant_qkv_strided(q, k, v, signs, outs=None, stream=None):
     q8, k8, v8, qs, ks, vs = outs
     strides = (ctypes.c_longlong * 9)(*[int(x) for t in (q, k, v) for x in t.stride()[:3]])
     _check(lib().attn_hadamard_quant_qkv_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs),
-                                                 _ptr(ks), _ptr(vs), _ptr(signs), B, H, N, d,
+                                                 _ptr(ks), _ptr(vs), _ptr(_signs(signs, d)), B, H, N, d,
                                                  ctypes.cast(strides, ctypes.c_void_p), _stream_ptr(stream)),
            "attn_hadamard_quant_qkv_strided")
     return outs
@@ -628,7 +641,7 @@ def attn_rope_hadamard_quant_qkv(q, k, v, signs, cos, sin, outs=None, stream=Non
     _outs_qkv(outs, q.shape, q.shape, (B, H, nb), (B, H, nb))
     q8, k8, v8, qs, ks, vs = outs
     _check(lib().attn_rope_hadamard_quant_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs),
-                                              _ptr(ks), _ptr(vs), _ptr(signs), _ptr(cos), _ptr(sin),
+                                              _ptr(ks), _ptr(vs), _ptr(_signs(signs, d)), _ptr(cos), _ptr(sin),
                                               int(cos.shape[1]), B, H, N, d, _stream_ptr(stream)),
            "attn_rope_hadamard_quant_qkv")
     return outs
@@ -783,7 +796,7 @@ def attn_hadamard_quant_qkv_varlen(q, k, v, signs, cu_seqlens_q, cu_seqlens_k, m
     q8, k8, v8, qs, ks, vs = outs
     strides = (ctypes.c_longlong * 6)(*[int(x) for t in (q, k, v) for x in t.stride()[:2]])
     _check(lib().attn_hadamard_quant_qkv_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs),
-                                                _ptr(ks), _ptr(vs), _ptr(signs), _ptr(cu_seqlens_q),
+                                                _ptr(ks), _ptr(vs), _ptr(_signs(signs, d)), _ptr(cu_seqlens_q),
                                                 _ptr(cu_seqlens_k), B, H, total_q, total_k, int(max_seqlen_q),
                                                 int(max_seqlen_k), d, ctypes.cast(strides, ctypes.c_void_p),
                                                 _stream_ptr(stream)), "attn_hadamard_quant_qkv_varlen")

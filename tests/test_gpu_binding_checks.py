@@ -67,3 +67,5 @@ def test_fp8_scales_and_pre_kernel_outputs():
     bad_outs = (q8, k8, v8, qs, ks, vs[:, :1].contiguous())
     _refused(lambda: ea.attn_hadamard_quant_qkv(q, k, v, signs, outs=bad_outs))
     _refused(lambda: ea.attn_hadamard_quant_qkv(q, k, v, signs, outs=(q8, k8, v8, qs, ks)))
+    _refused(lambda: ea.attn_hadamard_quant_qkv(q, k, v, signs[:32].contiguous()))  # d = 64 signs read
+    _refused(lambda: ea.attn_hadamard_quant(q.to(torch.float16), signs))
