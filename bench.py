@@ -1078,6 +1078,18 @@ def run_profile_case(args):
         outs = ea.attn_hadamard_quant_qkv_varlen(pq, pk, pv, signs, cu_q, cu_k, max(lens), max(lens))
         for _ in range(args.reps):
             ea.attn_fwd_fp8_varlen(*outs, cu_q, cu_k, max(lens), max(lens), causal=bool(causal))
+    elif args.profile_case == "varlen_bwd_ds":
+        # the bench's packed batch through the packed backward with dS kept
+        from exact_attention_100_b200.inputs import normal_qkv_packed
+        w = VARLEN_WORKLOAD
+        lens = varlen_lengths(w["total"], w["lo"], w["hi"], w["seed"])
+        qn, kn, vn, cq, ck = normal_qkv_packed(lens, lens, H, d, seed=w["seed"])
+        pq, pk, pv = (torch.from_numpy(a).to(torch.bfloat16).to(dev) for a in (qn, kn, vn))
+        cu_q, cu_k = torch.from_numpy(cq).to(dev), torch.from_numpy(ck).to(dev)
+        po, pl = ea.attn_fwd_varlen(pq, pk, pv, cu_q, cu_k, max(lens), causal=bool(causal))
+        pdo = torch.randn_like(pq)
+        for _ in range(args.reps):
+            ea.attn_bwd_varlen_ds(pq, pk, pv, po, pl, pdo, cu_q, cu_k, max(lens), max(lens), causal=bool(causal))
     elif args.profile_case == "bwd":
         o, lse = ea.attn_fwd(q, k, v, causal=bool(causal))
         do = torch.randn_like(q)
@@ -1117,7 +1129,8 @@ def main():
     ap.add_argument("--no-ring", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="leave the head-dim x length sweep out of the line")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv", "hq_rope", "varlen", "fp8_varlen", "bwd", "bwd_ds", "merge"], default=None,
+    ap.add_argument("--profile-case", choices=["fwd", "fwd_fp8", "hq_qkv", "hq_rope", "varlen", "fp8_varlen", "varlen_bwd_ds", "bwd", "bwd_ds",
+                             "merge"], default=None,
                     help="run --reps untimed calls of one entry point (for an ncu capture) and exit")
     ap.add_argument("--shape", type=int, nargs=5, default=[2, 16, 8192, 128, 1], metavar=("B", "H", "N", "d", "CAUSAL"))
     ap.add_argument("--reps", type=int, default=3)
