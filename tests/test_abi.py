@@ -545,3 +545,16 @@ def test_python_binding_has_same_names():
                  "attn_bwd_ds_workspace_bytes", "attn_bwd_ds", "attn_bwd_varlen_ds_workspace_bytes",
                  "attn_bwd_varlen_ds"]:
         assert callable(getattr(ea, name)), name
+
+
+def test_binding_refuses_host_tensors_before_any_library_call(L):
+    """A tensor in host memory would reach a kernel as a host pointer: the binding raises before
+    the call (no GPU needed to check it)."""
+    torch = pytest.importorskip("torch")
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ea.attn_fwd(q, q, q)
+    with pytest.raises(ValueError):
+        ea.attn_hadamard_quant(q)
+    with pytest.raises(ValueError):  # a wrong output dtype is refused before the pointers are taken
+        ea.attn_fwd(q, q, q, o=torch.zeros(1, 1, 128, 64, dtype=torch.uint8))
