@@ -15,7 +15,9 @@
 // textbook stage order, so every element sees the same float32 additions in the same order
 // as a plain sequential transform.  The block's largest |y| sets s_u = max(amax / 448, 2^-126);
 // codes are E4M3(y * (1/s_u)) (round to nearest even, saturating); the stored dequantisation
-// scale is s_u * post_scale (post_scale = 1/sqrt(d) with the transform, 1 without).
+// scale is s_u * post_scale (post_scale = 1/sqrt(d) with the transform, 1 without).  At
+// d = 256 the codes of a warp's 8 rows are gathered in shared memory and written 512 contiguous
+// bytes per store instruction (per-thread stores of 16-byte pieces of 8 rows took 9% longer).
 //
 // With ROPE (d = 256; d = 64 and 128 have hq_rope_kernel below), the tensors marked for it are
 // first given the rotary position embedding the same page names as a bandwidth-bound step to
@@ -93,6 +95,10 @@ struct HqCfg {
   static constexpr int kBoxes = D / 64;             // 128-byte TMA boxes per row
   static constexpr int kBufBytes = 128 * D * 2;
   static constexpr int kCtasPerSm = D == 256 ? 1 : (D == 128 ? 3 : 5);
+  // d = 256: the codes of a warp's 8 rows go through shared memory (2 KB per warp), so that
+  // every store instruction writes 512 contiguous bytes
+  static constexpr bool kStaged = kThreadsPerRow == 4;
+  static constexpr int kSmem = 2 * kBufBytes + (kStaged ? kThreads / 32 * 8 * D : 0) + 1024;
 };
 
 // Up to three tensors of one shape in one launch (Q and K with the transform, V without).
@@ -385,8 +391,8 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
 #pragma unroll
     for (int e = 0; e < kE; ++e) am[e & 3] = fmaxf(am[e & 3], fabsf(v[e]));
     float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    // non-negative, never NaN: the unsigned order of the bits is the order of the values
+    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
     if (lane == 0) warp_max[buf][warp] = amax;
     // every thread has read buffer `buf` and posted its warp maximum
     __syncthreads();
@@ -405,7 +411,41 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
     if (tid == 0) scales[static_cast<size_t>(bh) * nbs + blk] = __fmul_rn(s_u, post);
 
     const int grow = blk * 128 + row;
-    if (VL ? row < rows_valid : grow < N) {
+    if constexpr (C::kStaged && !VL) {
+      // logical 16-byte chunk ch = 4 * part + c of warp row rw at physical chunk ch ^ g, with
+      // g = 2 * (part / 2) + rw % 2: the 8 lanes of each quarter-warp access hit 8 different
+      // bank groups, for the writes (two rows, four parts) and for the reads (one row, eight chunks)
+      uint8_t* const ws = smem + 2 * C::kBufBytes + warp * (8 * D);
+      const int rw = lane >> 2;
+#pragma unroll
+      for (int c = 0; c < kE / 16; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int e = c * 16 + 4 * k;
+          float a0 = v[e], a1 = v[e + 1], a2 = v[e + 2], a3 = v[e + 3];
+          mul2(a0, a1, rcp);
+          mul2(a2, a3, rcp);
+          const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a0, a1), __NV_SATFINITE, __NV_E4M3);
+          const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(a2, a3), __NV_SATFINITE, __NV_E4M3);
+          w[k] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+        }
+        const int ch = 4 * part + c;
+        *reinterpret_cast<uint4*>(ws + rw * D + ((ch ^ (2 * (part >> 1) + (rw & 1))) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      __syncwarp();
+      const int row0 = blk * 128 + warp * 8;  // sequence row of the warp's first row
+      uint8_t* const gout = x8 + (static_cast<size_t>(bh) * N + row0) * D;
+#pragma unroll
+      for (int i = 0; i < 8 * D / 512; ++i) {
+        const int rr = 2 * i + (lane >> 4);
+        const int ch = lane & 15;
+        const uint4 val = *reinterpret_cast<const uint4*>(ws + rr * D + ((ch ^ (2 * (ch >> 3) + (rr & 1))) << 4));
+        if (row0 + rr < N) *reinterpret_cast<uint4*>(gout + 512 * i + 16 * lane) = val;
+      }
+      __syncwarp();
+    } else if (VL ? row < rows_valid : grow < N) {
       // contiguous outputs: [BH, N, d], or [total, H, d] for packed tensors
       uint8_t* out = VL ? x8 + ((vl_row0 + row) * job.H + bh % job.H) * D + part * kE
                         : x8 + (static_cast<size_t>(bh) * N + grow) * D + part * kE;
@@ -748,8 +788,8 @@ __global__ void __launch_bounds__(HqRopeCfg<D>::kThreads, 1)
 #pragma unroll
       for (int e = 0; e < D; ++e) am[e & 3] = fmaxf(am[e & 3], fabsf(v[e]));
       float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      // non-negative, never NaN: the unsigned order of the bits is the order of the values
+      amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
       if (lane == 0) warp_max[slot][k & 1][swarp] = amax;
       // every warp of the slot has posted its maximum (and, with two buffers, read buffer `buf`)
       named_bar_sync(1 + slot, 128);
@@ -861,7 +901,7 @@ static cudaError_t launch_hq(const CUtensorMap* tm, int ntensors, const HqJob& j
   }
   const long long cap = static_cast<long long>(num_sms) * C::kCtasPerSm;
   const int grid = static_cast<int>(total < cap ? total : cap);
-  hadamard_quant_kernel<D, ROPE, VL><<<grid, C::kThreads, 2 * C::kBufBytes + 1024, stream>>>(
+  hadamard_quant_kernel<D, ROPE, VL><<<grid, C::kThreads, C::kSmem, stream>>>(
       tm[0], tm[ntensors > 1 ? 1 : 0], tm[ntensors > 2 ? 2 : 0], job, signs, N, n_blocks, static_cast<int>(total),
       status);
   return cudaGetLastError();
@@ -870,17 +910,17 @@ static cudaError_t launch_hq(const CUtensorMap* tm, int ntensors, const HqJob& j
 template <int D>
 static cudaError_t set_hq_attr() {
   cudaError_t e = cudaFuncSetAttribute(hadamard_quant_kernel<D, false, false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * HqCfg<D>::kBufBytes + 1024);
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, HqCfg<D>::kSmem);
   if (e == cudaSuccess) {
     if constexpr (D == 256)
       e = cudaFuncSetAttribute(hadamard_quant_kernel<D, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               2 * HqCfg<D, true>::kBufBytes + 1024);
+                               HqCfg<D, true>::kSmem);
     else
       e = cudaFuncSetAttribute(hq_rope_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, HqRopeCfg<D>::kSmem);
   }
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(hadamard_quant_kernel<D, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             2 * HqCfg<D>::kBufBytes + 1024);
+                             HqCfg<D>::kSmem);
   return e;
 }
 
