@@ -17,7 +17,11 @@
 // codes are E4M3(y * (1/s_u)) (round to nearest even, saturating); the stored dequantisation
 // scale is s_u * post_scale (post_scale = 1/sqrt(d) with the transform, 1 without).  At
 // d = 256 the codes of a warp's 8 rows are gathered in shared memory and written 512 contiguous
-// bytes per store instruction (per-thread stores of 16-byte pieces of 8 rows took 9% longer).
+// bytes per store instruction (per-thread stores of 16-byte pieces of 8 rows took 9% longer),
+// and each of the two butterfly stages between lanes moves every value across lanes once: the
+// two lanes of a pair each keep half of the positions and receive the partner's values for
+// them (one shuffle per position instead of one per element; the launch was bound by the
+// shared-memory/shuffle crossbar, 86 -> 70 us for Q/K/V [2, 8, 8192, 256]).
 //
 // With ROPE (d = 256; d = 64 and 128 have hq_rope_kernel below), the tensors marked for it are
 // first given the rotary position embedding the same page names as a bandwidth-bound step to
@@ -250,6 +254,10 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
     // explicit selects keep the parameter block out of local memory
     const bool transform = (t == 0 ? job.transform[0] : (t == 1 ? job.transform[1] : job.transform[2])) != 0;
     const uint8_t* sb = smem + buf * C::kBufBytes;
+    // four lanes per row, transformed rows: the odd lanes hold the two halves of their part
+    // swapped (v[j] = element part * kE + (j + 32) % 64), so that the exchanges between lanes
+    // send the same registers on every lane (see the lane stages below)
+    const int sh = (C::kThreadsPerRow == 4 && transform) ? 32 * (part & 1) : 0;
 
     // this thread's kE elements of its row: element e0 = part*kE + 8c.. lives in box e0/64 at
     // 16-byte chunk ((e0 % 64) / 8) ^ (row % 8) of the row (128-byte swizzle).  With the
@@ -259,7 +267,7 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
     auto unpack_raw = [&]() {
 #pragma unroll
       for (int c = 0; c < kE / 8; ++c) {
-        const int e0 = part * kE + c * 8;
+        const int e0 = part * kE + ((c * 8 + sh) & (kE - 1));
         const uint4 w = *reinterpret_cast<const uint4*>(sb + (e0 >> 6) * 16384 + row * 128 +
                                                         ((((e0 & 63) >> 3) ^ (row & 7)) << 4));
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -274,7 +282,7 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
     auto unpack_signed_stage1 = [&]() {
 #pragma unroll
       for (int c = 0; c < kE / 8; ++c) {
-        const int e0 = part * kE + c * 8;
+        const int e0 = part * kE + ((c * 8 + sh) & (kE - 1));
         uint4 w = *reinterpret_cast<const uint4*>(sb + (e0 >> 6) * 16384 + row * 128 +
                                                   ((((e0 & 63) >> 3) ^ (row & 7)) << 4));
         const uint4 mk = *reinterpret_cast<const uint4*>(&smask[e0 / 2]);
@@ -292,8 +300,9 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
     auto later_stages = [&]() {
       // strides 2 .. kE/2 inside the thread, on register pairs (e, e+1): one packed add and one
       // packed sub make two butterflies, each lane rounding like a scalar operation
+      constexpr int kLastLocal = C::kThreadsPerRow == 4 ? kE / 2 : kE;  // handled apart below
 #pragma unroll
-      for (int h = 2; h < kE; h <<= 1) {
+      for (int h = 2; h < kLastLocal; h <<= 1) {
 #pragma unroll
         for (int e = 0; e < kE; e += 2) {
           if ((e & h) == 0) {
@@ -307,16 +316,68 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
           }
         }
       }
-      // strides kE .. D/2: the partner lane holds another part of the row; the lower part keeps
-      // v + other, the upper other - v, i.e. other + sgn * v with sgn = +-1 (exact)
+      if constexpr (C::kThreadsPerRow == 4) {
+        // Every butterfly below is fl(x + y) or fl(x - y) of its lower element x and upper
+        // element y, as an fma with multipliers +-1 (exact) and one rounding -- the value and
+        // the sign of a zero of the textbook stage.
+        // Stride 32, inside the thread; with swapped halves (odd lanes) element j sits at
+        // v[32 + j] and j + 32 at v[j]: v[j] <- s1 v[j] + v[32+j], v[32+j] <- -s1 v[32+j] + v[j].
+        const float s1 = (part & 1) ? -1.f : 1.f;
 #pragma unroll
-      for (int hl = 1; hl < C::kThreadsPerRow; hl <<= 1) {
-        const float sgn = (part & hl) != 0 ? -1.f : 1.f;
+        for (int j = 0; j < 32; j += 2) {
+          float a0 = v[j], a1 = v[j + 1], b0 = v[32 + j], b1 = v[33 + j];
+          fma2_rn(a0, a1, s1, v[32 + j], v[33 + j]);
+          fma2_rn(b0, b1, -s1, v[j], v[j + 1]);
+          v[j] = a0;
+          v[j + 1] = a1;
+          v[32 + j] = b0;
+          v[33 + j] = b1;
+        }
+        // Strides 64 and 128 between lanes.  At each, a lane pair holds the two elements of 32
+        // butterflies' worth of positions each; every lane keeps v[t], sends v[32 + t] and
+        // computes the butterflies of its kept positions with the received value r:
+        // v[t] <- b1 r + a1 v[t], v[32+t] <- b2 r + a2 v[t] (a, b = +-1 by lane).
+        // Stride 64 (lanes p, p^1; part p holds elements 64p ..): lane 0 keeps elements 0..31
+        // and sends 32..63, lane 1 keeps 96..127 and sends 64..95; sums and differences land
+        // so that the stride-128 exchange sends v[32 + t] again:
+        //   lane 0: v[t] = e(t),      v[32+t] = e(64+t)      lane 1: e(32+t),  e(96+t)
+        //   lane 2: v[t] = e(192+t),  v[32+t] = e(128+t)     lane 3: e(224+t), e(160+t)
+        {
+          const float a1 = part == 3 ? -1.f : 1.f, b1 = part == 2 ? -1.f : 1.f;
+          const float a2 = part == 1 ? -1.f : 1.f, b2 = part == 0 ? -1.f : 1.f;
 #pragma unroll
-        for (int e = 0; e < kE; e += 2) {
-          const float o0 = __shfl_xor_sync(0xffffffffu, v[e], hl);
-          const float o1 = __shfl_xor_sync(0xffffffffu, v[e + 1], hl);
-          fma2_rn(v[e], v[e + 1], sgn, o0, o1);
+          for (int t = 0; t < 32; t += 2) {
+            float r0 = __shfl_xor_sync(0xffffffffu, v[32 + t], 1);
+            float r1 = __shfl_xor_sync(0xffffffffu, v[33 + t], 1);
+            float w0 = v[t], w1 = v[t + 1], x0 = v[t], x1 = v[t + 1];
+            mul2(w0, w1, a1);
+            mul2(x0, x1, a2);
+            float q0 = r0, q1 = r1;
+            fma2_rn(r0, r1, b1, w0, w1);
+            fma2_rn(q0, q1, b2, x0, x1);
+            v[t] = r0;
+            v[t + 1] = r1;
+            v[32 + t] = q0;
+            v[33 + t] = q1;
+          }
+        }
+        // Stride 128 (lanes p, p^2): lane p ends with v[t] = e(32p + t), v[32+t] = e(128 + 32p + t)
+        {
+          const float a = part >= 2 ? -1.f : 1.f;
+#pragma unroll
+          for (int t = 0; t < 32; t += 2) {
+            const float r0 = __shfl_xor_sync(0xffffffffu, v[32 + t], 2);
+            const float r1 = __shfl_xor_sync(0xffffffffu, v[33 + t], 2);
+            float s0 = v[t], s1_ = v[t + 1], w0 = v[t], w1 = v[t + 1];
+            add2(s0, s1_, r0, r1);
+            mul2(w0, w1, a);
+            float d0 = r0, d1 = r1;
+            fma2_rn(d0, d1, -a, w0, w1);
+            v[t] = s0;
+            v[t + 1] = s1_;
+            v[32 + t] = d0;
+            v[33 + t] = d1;
+          }
         }
       }
     };
@@ -332,11 +393,14 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
         constexpr int kHalf = C::kThreadsPerRow / 2;
         const bool upper = part >= kHalf;
         const int i0 = (part % kHalf) * kE;
+        // v[e] is coordinate part * kE + (e + sh) % kE: frequency i0 + (e + sh) % kE
         const float* cr = job.cos + i0 * np + pos;
         const float* sr = job.sin + i0 * np + pos;
+        const long long lo_off = static_cast<long long>(sh) * static_cast<long long>(np);
 #pragma unroll
         for (int e = 0; e < kE; ++e) {
-          const float c = __ldg(cr + e * np), s = __ldg(sr + e * np);
+          const long long off = (e < kE / 2 ? lo_off : -lo_off) + static_cast<long long>(e) * static_cast<long long>(np);
+          const float c = __ldg(cr + off), s = __ldg(sr + off);
           const float own = v[e];
           const float other = __shfl_xor_sync(0xffffffffu, own, kHalf);
           v[e] = upper ? __fadd_rn(__fmul_rn(own, c), __fmul_rn(other, s))
@@ -347,7 +411,7 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
     auto signed_stage1 = [&]() {
 #pragma unroll
       for (int e = 0; e < kE; e += 2) {
-        const uint32_t mk = smask[(part * kE + e) / 2];
+        const uint32_t mk = smask[(part * kE + ((e + sh) & (kE - 1))) / 2];
         const float a = __uint_as_float(__float_as_uint(v[e]) ^ (mk << 16));
         const float b = __uint_as_float(__float_as_uint(v[e + 1]) ^ (mk & 0x80000000u));
         v[e] = a + b;
@@ -412,13 +476,16 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
 
     const int grow = blk * 128 + row;
     if constexpr (C::kStaged && !VL) {
-      // logical 16-byte chunk ch = 4 * part + c of warp row rw at physical chunk ch ^ g, with
-      // g = 2 * (part / 2) + rw % 2: the 8 lanes of each quarter-warp access hit 8 different
-      // bank groups, for the writes (two rows, four parts) and for the reads (one row, eight chunks)
+      // logical 16-byte chunk ch of warp row rw at physical chunk ch ^ g, g = 2 * (ch / 8) + rw % 2:
+      // the 8 lanes of each quarter-warp access hit 8 different bank groups, for the writes
+      // (two rows, four parts) and for the reads (one row, eight chunks)
       uint8_t* const ws = smem + 2 * C::kBufBytes + warp * (8 * D);
       const int rw = lane >> 2;
 #pragma unroll
       for (int c = 0; c < kE / 16; ++c) {
+        // the row's 16-byte chunk of v[16c ..]: transformed rows end the lane stages with
+        // elements 32 part .. and 128 + 32 part .., the others hold part * kE ..
+        const int ch = transform ? (c < 2 ? 2 * part + c : 8 + 2 * part + (c - 2)) : 4 * part + c;
         uint32_t w[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -430,8 +497,7 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
           const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(a2, a3), __NV_SATFINITE, __NV_E4M3);
           w[k] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
         }
-        const int ch = 4 * part + c;
-        *reinterpret_cast<uint4*>(ws + rw * D + ((ch ^ (2 * (part >> 1) + (rw & 1))) << 4)) =
+        *reinterpret_cast<uint4*>(ws + rw * D + ((ch ^ (2 * (ch >> 3) + (rw & 1))) << 4)) =
             make_uint4(w[0], w[1], w[2], w[3]);
       }
       __syncwarp();
@@ -447,10 +513,13 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
       __syncwarp();
     } else if (VL ? row < rows_valid : grow < N) {
       // contiguous outputs: [BH, N, d], or [total, H, d] for packed tensors
-      uint8_t* out = VL ? x8 + ((vl_row0 + row) * job.H + bh % job.H) * D + part * kE
-                        : x8 + (static_cast<size_t>(bh) * N + grow) * D + part * kE;
+      uint8_t* out = VL ? x8 + ((vl_row0 + row) * job.H + bh % job.H) * D
+                        : x8 + (static_cast<size_t>(bh) * N + grow) * D;
 #pragma unroll
       for (int c = 0; c < kE / 16; ++c) {
+        // the row's 16-byte chunk of v[16c ..] (four lanes per row: as in the staged stores)
+        const int ch = (C::kThreadsPerRow == 4 && transform) ? (c < 2 ? 2 * part + c : 8 + 2 * part + (c - 2))
+                                                             : part * (kE / 16) + c;
         uint32_t w[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -462,7 +531,7 @@ __global__ void __launch_bounds__(HqCfg<D, ROPE>::kThreads, HqCfg<D, ROPE>::kCta
           const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(a2, a3), __NV_SATFINITE, __NV_E4M3);
           w[k] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
         }
-        *reinterpret_cast<uint4*>(out + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(out + ch * 16) = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
   }
