@@ -51,12 +51,19 @@ def test_fp8_config_q_tensor_bit_exact():
     np.testing.assert_array_equal(codes, rc)
 
 
-def test_zero_block_and_large_values():
-    x = np.zeros((1, 1, 260, 128), dtype=np.float32)
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_zero_block_and_large_values(d):
+    """A block of zero rows (the signs of D turn them into zeros of both signs, which the
+    butterflies must carry as the sequential transform does: E4M3 keeps the sign of zero),
+    rows whose butterflies cancel exactly, a block of large values and tiny ones."""
+    x = np.zeros((1, 1, 260, d), dtype=np.float32)
     x[0, 0, 128:256] = 3.0e4
     x[0, 0, 256:, ::2] = -1.0e-30
+    x[0, 0, 10] = 1.0
+    x[0, 0, 11, ::3] = -2.0
+    x[0, 0, 12] = np.tile([1.5, -1.5], d // 2)
     x = round_to_bf16(x)
-    signs = hadamard_signs(128)
+    signs = hadamard_signs(d)
     codes, scales = _run(x, signs)
     rc, rs = hadamard_quant_ref(x.astype(np.float64), signs)
     np.testing.assert_array_equal(scales, rs)
