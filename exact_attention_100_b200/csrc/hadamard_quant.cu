@@ -9,7 +9,8 @@
 // brought into shared memory by TMA (128-byte swizzle, rows past the sequence end read as
 // zero); two blocks are in flight per CTA, the next load being issued as soon as every thread
 // has copied the current block into registers.  One thread holds a whole row (d = 64, 128) or
-// 64 elements of it (d = 256, and d = 128 with the rotary embedding; adjacent lanes): the
+// 64 elements of it (d = 256, four adjacent lanes per row, with or without the rotary
+// embedding; at d = 64 and 128 the rotary embedding has hq_rope_kernel below): the
 // unnormalised transform y = H_d (D x) runs in float32 registers with butterfly stages of
 // stride 1, 2, ..., inside a thread and the remaining strides between the lanes of a row -- the
 // textbook stage order, so every element sees the same float32 additions in the same order
@@ -91,8 +92,8 @@ __device__ __forceinline__ void thread_wait(uint64_t* bar, uint32_t parity, vola
 template <int D, bool ROPE = false>
 struct HqCfg {
   static_assert(!ROPE || D == 256, "the rotary embedding at d = 64 and 128 is hq_rope_kernel");
-  // elements of a row held by one thread: at most 64 with the rotary embedding, whose table
-  // loads need registers to be in flight (a whole d = 128 row per thread left too few)
+  // elements of a row held by one thread: the whole row at d = 64 and 128, a quarter at d = 256
+  // (ROPE implies d = 256)
   static constexpr int kElems = (D == 256 || ROPE) ? 64 : D;
   static constexpr int kThreadsPerRow = D / kElems;
   static constexpr int kThreads = 128 * kThreadsPerRow;
