@@ -61,3 +61,47 @@ def test_workload_helpers():
     lens = bench.varlen_lengths(w["total"], w["lo"], w["hi"], w["seed"])
     assert sum(lens) == w["total"] and all(0 < n <= w["hi"] for n in lens)
     assert lens == bench.varlen_lengths(w["total"], w["lo"], w["hi"], w["seed"])  # seeded
+
+
+class _DoneProcess:
+    def terminate(self):
+        pass
+
+    def wait(self):
+        return 0
+
+
+def test_clock_record_median_and_reasons(tmp_path):
+    """The clock record a line carries: the median SM clock and the throttle reasons seen
+    inside the timed window (plus a second of margin), from nvidia-smi's CSV rows as written
+    with --format=csv,noheader,nounits."""
+    sys.path.insert(0, ROOT)
+    import time
+    import bench
+    t0 = time.mktime(time.strptime("2026/12/03 12:00:00", "%Y/%m/%d %H:%M:%S"))
+    rows = [
+        # before the window: a thermal slowdown that must not be reported
+        "2026/12/03 11:59:50.100, 1200, 1965, 900.0, 0x20, Not Active, Not Active, Active, Not Active",
+        "2026/12/03 12:00:00.100, 1965, 1965, 700.5, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/03 12:00:01.100, 1890, 1965, 999.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "2026/12/03 12:00:02.100, 1965, 1965, 950.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+        "2026/12/03 12:00:30.100, 1000, 1965, 300.0, 0x8, Active, Not Active, Not Active, Not Active",
+    ]
+    s = bench.ClockSampler(None)
+    s.file.write("\n".join(rows) + "\n")
+    s.proc = _DoneProcess()
+    rec = s.stop(t0, t0 + 2.0)
+    assert rec["samples"] == 3
+    assert rec["sm_mhz"] == 1965.0 and rec["sm_max_mhz"] == 1965.0
+    assert rec["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_record_without_nvidia_smi():
+    sys.path.insert(0, ROOT)
+    import bench
+    s = bench.ClockSampler(None)
+    s.proc = None
+    rec = s.stop(0.0, 1.0)
+    assert rec["samples"] == 0 and rec["sm_mhz"] is None
+    os.unlink(s.file.name)
